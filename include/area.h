@@ -1,0 +1,253 @@
+/*
+ * libarea -- C-ABI of the AReA attention hot path on B200 (sm_100a).
+ *
+ * AReA ("Adaptive Receptive-Field Attention for Efficient High-Resolution
+ * Diffusion Transformers", arXiv 2610.17227) replaces full self-attention of a
+ * diffusion transformer above its native resolution by
+ *   Phase I  -- cross-scale coarse attention: full-resolution queries against
+ *               keys/values pooled over f x f token blocks;
+ *   Phase II -- adaptive windowed attention: shrinking windows, quadrant
+ *               splits of smooth windows (Haar DWT detail map), a Halo ring of
+ *               neighbouring keys, a global-KV bridge, and centre-weighted
+ *               blending of overlapping window outputs.
+ * Citations below name the summary pages the method is taken from:
+ *   [ai]   ai.info paper summary, "Methodology in Plain English";
+ *   [blog] gpt-diffusion.com blog, "Las dos fases de AReA" (Fase I/Fase II);
+ *   [wiki] github.com/KooroshRH/AReA wiki (overview, canvas rules).
+ *
+ * Conventions (all functions):
+ *   - Every buffer is owned by the caller and lives in device memory unless
+ *     stated otherwise.  The library allocates no device memory and keeps no
+ *     state between calls.
+ *   - Tensors are dense and contiguous.  Q, K, V, O: [B, H, N, D] with the
+ *     token index n = y * Wg + x over an Hg x Wg token grid (row-major).
+ *     Q and K arrive already rotated (RoPE is the caller's business).
+ *   - dtype: AREA_DTYPE_BF16 (storage bf16, tensor-core MMA with fp32
+ *     accumulation, D = 128 or 64) or AREA_DTYPE_F32 (storage fp32, fp32
+ *     CUDA-core arithmetic, D = 64 or 128).
+ *   - Every kernel call is asynchronous on the given stream (0 = legacy
+ *     default stream), never synchronises the host and never waits on
+ *     another CTA.  The return value reports argument validation and launch
+ *     errors only; AREA_ECUDA carries the CUDA error, see area_status_string.
+ *   - Device pointers passed to the attention calls must be 16-byte aligned.
+ */
+#ifndef AREA_H_
+#define AREA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define AREA_OK            0
+#define AREA_EINVAL        1   /* null pointer, bad size, bad enum value       */
+#define AREA_EUNSUPPORTED  2   /* dtype / head_dim / grid the library lacks    */
+#define AREA_ENOSPACE      3   /* plan or workspace buffer too small           */
+#define AREA_ECUDA         4   /* CUDA launch error (area_last_cuda_error())   */
+
+/* ---- enums ------------------------------------------------------------- */
+#define AREA_DTYPE_F32     0
+#define AREA_DTYPE_BF16    1
+
+#define AREA_POOL_MEAN     0   /* block average                                */
+#define AREA_POOL_CENTER   1   /* token (py*f + f/2, px*f + f/2)               */
+
+#define AREA_DETAIL_HH     0   /* e = HH^2                                     */
+#define AREA_DETAIL_ALL3   1   /* e = (LH^2 + HL^2) + HH^2                     */
+
+/* Returns a static, human-readable string for a status code. */
+const char* area_status_string(int status);
+/* CUDA error code of the most recent AREA_ECUDA return on this thread. */
+int area_last_cuda_error(void);
+/* Library version, e.g. "libarea 0.1.0 sm_100a". */
+const char* area_version(void);
+/*
+ * area_kernel_error -- synchronises the current device, then reports in
+ * *code whether a tensor-core kernel gave up a bounded wait since the last
+ * call (0 = none, 1 = a wait expired; that launch's output is invalid), and
+ * clears the flag.  Meant for tests and health checks, not the hot path.
+ * Errors: AREA_EINVAL (null), AREA_ECUDA.
+ */
+int area_kernel_error(int* code);
+
+/* ---- Phase I ----------------------------------------------------------- */
+
+/*
+ * area_pool_kv -- one representative key/value token per f x f block.
+ * [blog] Fase I / [ai] Phase I: keys and values are pooled to one token per
+ * f x f block, on a (Hg/f) x (Wg/f) grid.
+ *
+ *   k, v   : [B, H, Hg*Wg, D] input (dtype)
+ *   kp, vp : [B, H, (Hg/f)*(Wg/f), D] output (dtype); pooled token index
+ *            py*(Wg/f) + px.
+ *   mode   : AREA_POOL_MEAN (fp32 sum over the block, rows then columns,
+ *            divided by f*f, rounded to the output dtype) or AREA_POOL_CENTER.
+ * Errors: AREA_EINVAL if a pointer is null, a size is < 1, f does not divide
+ * Hg and Wg (the canvas rule of [wiki]: the two patch counts must share the
+ * pooling factor), or mode/dtype is unknown.  D must be a multiple of 8.
+ */
+int area_pool_kv(const void* k, const void* v, void* kp, void* vp,
+                 int B, int H, int Hg, int Wg, int D, int f, int mode,
+                 int dtype, cudaStream_t stream);
+
+/*
+ * area_coarse_attn -- Phase I cross-scale coarse attention ([ai] Phase I):
+ *   O = softmax(scale * Q Kp^T) Vp   per (b, h), text tokens absent.
+ *   q  : [B, H, N, D]; kp, vp : [B, H, Nk, D]; o : [B, H, N, D] (dtype).
+ * bf16 with D = 128 runs on the tcgen05 tensor-core kernel; every other
+ * supported combination on the CUDA-core kernel.
+ * Errors: AREA_EINVAL (null, N < 1, Nk < 1), AREA_EUNSUPPORTED (D not 64/128,
+ * unknown dtype).
+ */
+int area_coarse_attn(const void* q, const void* kp, const void* vp, void* o,
+                     int B, int H, int N, int Nk, int D, float scale,
+                     int dtype, cudaStream_t stream);
+
+/*
+ * area_full_attn -- full global attention over all N tokens, the operation
+ * AReA replaces ([ai] "Main Findings": speedups are quoted against it).
+ * Same kernels as area_coarse_attn with Nk = N.
+ */
+int area_full_attn(const void* q, const void* k, const void* v, void* o,
+                   int B, int H, int N, int D, float scale,
+                   int dtype, cudaStream_t stream);
+
+/* ---- Phase II ---------------------------------------------------------- */
+
+/*
+ * area_dwt_detail -- Haar detail energy per 2x2 token cell ([ai] Phase II:
+ * "a DWT map computed from the current hidden states measures fine detail").
+ * For cell (cy, cx) and channel c, with a = x(2cy,2cx), b = x(2cy,2cx+1),
+ * c' = x(2cy+1,2cx), d = x(2cy+1,2cx+1) widened to fp32:
+ *   HH = ((a - b) - (c' - d)) * 0.5,  LH = ((a + b) - (c' + d)) * 0.5,
+ *   HL = ((a - b) + (c' - d)) * 0.5,
+ *   e_c = HH^2 (AREA_DETAIL_HH) or (LH^2 + HL^2) + HH^2 (AREA_DETAIL_ALL3),
+ *   E = ((..((0 + e_0) + e_1)..) + e_{C-1}) * (1/C),
+ * every operation in round-to-nearest fp32 without contraction, so the map
+ * is bit-reproducible.
+ *   src    : [B, Hg*Wg, C] channels-last, src_dtype (F32 or BF16)
+ *   energy : [B, Hg/2, Wg/2] fp32 output
+ * Errors: AREA_EINVAL (null, Hg or Wg odd or < 2, C < 1, bad mode/dtype).
+ */
+int area_dwt_detail(const void* src, int src_dtype, int C, float* energy,
+                    int B, int Hg, int Wg, int mode, cudaStream_t stream);
+
+/* Configuration of one Phase II step.  jitter_seed must be 0 (no border
+ * shift).  split_thr is the mean-energy bound below which a window splits. */
+typedef struct area_plan_cfg {
+  int B;            /* batch elements (one plan each)                        */
+  int Hg, Wg;       /* token grid                                            */
+  int w;            /* scheduled window side                                 */
+  int halo;         /* Halo width h >= 0                                     */
+  int G;            /* global-KV tokens per window, 0 <= G <= 4096           */
+  float split_thr;  /* split when score < fl32(split_thr * hy * wx)          */
+  unsigned long long jitter_seed;   /* must be 0                            */
+} area_plan_cfg;
+
+/*
+ * Plan buffer layout (device memory, written by area_window_plan).  The
+ * first 256 bytes hold an int64 header; every section starts 256-byte
+ * aligned at the byte offset stored in the header.  Windows are indexed per
+ * batch element b in [0, B); "nb" = base windows per element, "nw" = 4*nb
+ * (room for a full split).
+ *   header[0]  = AREA_PLAN_MAGIC        header[1] = AREA_PLAN_VERSION
+ *   header[2..8] = B, Hg, Wg, w, halo, G, nb
+ *   header[9]  = nw
+ *   header[10+s] = byte offset of section s (AREA_PLAN_SEC_*)
+ *   header[24] = work-item capacity per element ("ni"), header[25] = N
+ * Sections:
+ *   BASE    int32 [B][nb][4]   base windows (y0, x0, hy, wx), row-major
+ *   SCORE   f32   [B][nb]      sum of token energy over the base window
+ *   SPLIT   u8    [B][nb]      1 = split into quadrants
+ *   NWIN    int32 [B]          number of final windows
+ *   WIN     int32 [B][nw][4]   final windows (y0, x0, hy, wx)
+ *   PARENT  int32 [B][nw]      base window of each final window
+ *   EXT     int32 [B][nw][4]   Halo rectangle (y0, x0, hy, wx), clipped
+ *   GCOUNT  int32 [B][nw]      G_W = min(G, N - |ext|)
+ *   GIDX    int32 [B][nw][G]   global-KV tokens in rank order, -1 padded
+ *   WSUM    f32   [B][N]       sum of tent weights over final windows
+ *   ORDER   int32 [B][N]       tokens by (energy desc, index asc)
+ *   NITEM   int32 [B+1]        work items (window, query tile) per element,
+ *                              last entry = total
+ *   ITEMS   int32 [B][ni][2]   (window, block of 256 queries) in cost order
+ *   SCRATCH                    sort and scan scratch (contents unspecified)
+ */
+#define AREA_PLAN_MAGIC    0x4145524150414c4eLL  /* "AREAPLAN" */
+#define AREA_PLAN_VERSION  1
+#define AREA_PLAN_SEC_BASE     0
+#define AREA_PLAN_SEC_SCORE    1
+#define AREA_PLAN_SEC_SPLIT    2
+#define AREA_PLAN_SEC_NWIN     3
+#define AREA_PLAN_SEC_WIN      4
+#define AREA_PLAN_SEC_PARENT   5
+#define AREA_PLAN_SEC_EXT      6
+#define AREA_PLAN_SEC_GCOUNT   7
+#define AREA_PLAN_SEC_GIDX     8
+#define AREA_PLAN_SEC_WSUM     9
+#define AREA_PLAN_SEC_ORDER    10
+#define AREA_PLAN_SEC_NITEM    11
+#define AREA_PLAN_SEC_ITEMS    12
+#define AREA_PLAN_SEC_SCRATCH  13
+#define AREA_PLAN_NSEC         14
+
+/*
+ * area_window_plan_bytes -- size of the plan buffer for cfg (host only).
+ * Errors: AREA_EINVAL (null, bad sizes, jitter_seed != 0, G > 4096).
+ */
+int area_window_plan_bytes(const area_plan_cfg* cfg, size_t* plan_bytes);
+
+/*
+ * area_window_plan -- Phase II plan on the device ([ai] Phase II, steps in
+ * the pages' order):
+ *   1. base tiling: per axis of length L, w_e = min(w, L),
+ *      n = ceil(L / w_e), start_i = floor(i (L - w_e) / (n - 1));
+ *   2. split score S = sum of token energy (token (y,x) takes the energy of
+ *      cell (y/2, x/2)), rows summed left to right then rows top to bottom,
+ *      in fp32; split iff S < fl32(split_thr * hy * wx) and hy, wx >= 2;
+ *   3. quadrants TL, TR, BL, BR, top/left halves floor(side/2);
+ *   4. Halo rectangle: the window dilated by h, clipped to the grid;
+ *   5. global-KV bridge: the first G_W = min(G, N - |ext|) tokens by
+ *      (energy desc, token index asc) that lie outside the Halo rectangle;
+ *   6. per-token sum of tent weights
+ *      t = min(y-y0+1, y0+hy-y) * min(x-x0+1, x0+wx-x) over final windows;
+ *   7. the list of (window, 256-query block) work items, costliest first.
+ *   energy : [B, Hg/2, Wg/2] fp32 from area_dwt_detail
+ *   plan   : device buffer of plan_bytes >= area_window_plan_bytes(cfg)
+ * The plan never leaves the device.  Errors: AREA_EINVAL, AREA_ENOSPACE.
+ */
+int area_window_plan(const float* energy, const area_plan_cfg* cfg,
+                     void* plan, size_t plan_bytes, cudaStream_t stream);
+
+/*
+ * area_window_attn_ws_bytes -- fp32 merge workspace for area_window_attn:
+ * B*H*Hg*Wg*D*4 bytes (host only).
+ */
+int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D,
+                              size_t* ws_bytes);
+
+/*
+ * area_window_attn -- Phase II windowed attention and centre-weighted merge
+ * ([ai] Phase II).  For every final window W of the plan:
+ *   O_W(q) = softmax(scale * q K_S^T) V_S,  S = ext(W) followed by G_W,
+ * then O(q) = sum_W t_W(q) O_W(q) / sum_W t_W(q).
+ *   q, k, v, o : [B, H, Hg*Wg, D] (dtype)
+ *   cfg, plan  : the configuration and buffer given to area_window_plan
+ *   ws         : fp32 workspace of ws_bytes >= area_window_attn_ws_bytes();
+ *                contents on entry are ignored, on exit unspecified.
+ * Errors: AREA_EINVAL, AREA_EUNSUPPORTED (D, dtype), AREA_ENOSPACE.
+ */
+int area_window_attn(const void* q, const void* k, const void* v,
+                     const area_plan_cfg* cfg, const void* plan,
+                     size_t plan_bytes, void* o, void* ws, size_t ws_bytes,
+                     int H, int D, float scale, int dtype,
+                     cudaStream_t stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* AREA_H_ */

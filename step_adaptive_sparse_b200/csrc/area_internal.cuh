@@ -1,0 +1,102 @@
+// Internal declarations shared by the libarea translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "area.h"
+
+namespace area {
+
+constexpr int kQTile = 256;          // queries per work item (two 128-row MMA tiles)
+constexpr int kMaxG = 4096;          // largest global-KV count per window
+constexpr int kMaxGrid = 1 << 15;    // largest grid side accepted (tokens)
+
+// ---------------------------------------------------------------------------
+// plan layout: computed identically by every entry point from the config
+// ---------------------------------------------------------------------------
+struct PlanLayout {
+  int64_t B, Hg, Wg, w, halo, G;
+  int64_t nby, nbx, hy, wx;     // base tiling: counts and window sides
+  int64_t nb, nw;               // base windows / final-window capacity per element
+  int64_t nitem_max;            // work-item capacity per element
+  int64_t N;                    // tokens per element
+  int64_t ntile_sort;           // 256-element tiles of the radix sort
+  int64_t off[AREA_PLAN_NSEC];  // byte offsets of the sections
+  int64_t scratch_keys_a, scratch_keys_b, scratch_vals_a, scratch_vals_b,
+          scratch_hist;         // byte offsets inside the buffer
+  int64_t total;                // bytes
+};
+
+int plan_layout(const area_plan_cfg* cfg, PlanLayout* L);
+
+// Device view of a plan (pointers into the plan buffer).
+struct PlanView {
+  int B, Hg, Wg, w, halo, G;
+  int nby, nbx, hy, wx, nb, nw, nitem_max, N;
+  int4* base;          // [B][nb]
+  float* score;        // [B][nb]
+  uint8_t* split;      // [B][nb]
+  int* nwin;           // [B]
+  int4* win;           // [B][nw]
+  int* parent;         // [B][nw]
+  int4* ext;           // [B][nw]
+  int* gcount;         // [B][nw]
+  int* gidx;           // [B][nw][G]
+  float* wsum;         // [B][N]
+  int* order;          // [B][N]
+  int* nitem;          // [B+1]
+  int2* items;         // [B][nitem_max]
+};
+
+PlanView plan_view(const PlanLayout& L, void* plan);
+
+// ---------------------------------------------------------------------------
+// small device helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float load_as_float(const float* p, int64_t i) { return p[i]; }
+__device__ __forceinline__ float load_as_float(const __nv_bfloat16* p, int64_t i) {
+  return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void store_from_float(float* p, int64_t i, float v) { p[i] = v; }
+__device__ __forceinline__ void store_from_float(__nv_bfloat16* p, int64_t i, float v) {
+  p[i] = __float2bfloat16_rn(v);
+}
+
+// Start of the i-th of n evenly spaced windows of side we on an axis of length L.
+__host__ __device__ __forceinline__ int tile_start(int i, int n, int L, int we) {
+  return n > 1 ? (int)(((int64_t)i * (L - we)) / (n - 1)) : 0;
+}
+
+// ---------------------------------------------------------------------------
+// launchers (return cudaError_t of the launch)
+// ---------------------------------------------------------------------------
+cudaError_t launch_pool_kv(const void* k, const void* v, void* kp, void* vp, int B, int H,
+                           int Hg, int Wg, int D, int f, int mode, int dtype, cudaStream_t s);
+cudaError_t launch_dwt_detail(const void* src, int src_dtype, int C, float* energy, int B,
+                              int Hg, int Wg, int mode, cudaStream_t s);
+cudaError_t launch_window_plan(const float* energy, const area_plan_cfg* cfg,
+                               const PlanLayout& L, void* plan, cudaStream_t s);
+
+// CUDA-core attention (fp32 any supported D; bf16 fallback for D = 64).
+cudaError_t launch_dense_attn_simt(const void* q, const void* k, const void* v, void* o, int B,
+                                   int H, int N, int Nk, int D, float scale, int dtype,
+                                   cudaStream_t s);
+cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v,
+                                    const PlanLayout& L, const void* plan, float* ws, int H,
+                                    int D, float scale, int dtype, cudaStream_t s);
+// Shared by both window-attention paths.
+cudaError_t launch_ws_zero(float* ws, int64_t n, cudaStream_t s);
+cudaError_t launch_window_finalize(const float* ws, const PlanLayout& L, const void* plan,
+                                   void* o, int H, int D, int dtype, cudaStream_t s);
+
+// tcgen05 tensor-core attention (bf16, D = 128).
+cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, void* o, int B,
+                                 int H, int N, int Nk, float scale, cudaStream_t s);
+cudaError_t read_and_clear_tc_error(int* code);
+cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v,
+                                  const PlanLayout& L, const void* plan, float* ws, int H,
+                                  float scale, cudaStream_t s);
+
+}  // namespace area

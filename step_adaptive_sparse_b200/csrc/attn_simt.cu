@@ -1,0 +1,247 @@
+// CUDA-core attention: the fp32 path (tiny configuration, tolerance 1e-4) and
+// the bf16 path for head_dim 64.  Same semantics as the tensor-core kernels:
+//   dense  : O = softmax(scale * Q K^T) V over all Nk keys (coarse and full
+//            attention, AReA Phase I / the speedup denominator);
+//   window : per plan work item (window W, 128-query tile), keys S = Halo
+//            rectangle of W followed by its global-KV tokens; the output of W,
+//            weighted by the tent weight of each query, is accumulated in an
+//            fp32 workspace and normalised by the per-token weight sum
+//            (AReA Phase II, centre-weighted blending of overlaps).
+// Pages: ai.info "Methodology in Plain English" (Phase I, Phase II).
+#include "area_internal.cuh"
+
+namespace area {
+namespace {
+
+constexpr int kSimtQ = 32;        // queries per block
+constexpr int kSimtTPQ = 8;       // threads per query
+constexpr int kSimtKV = 64;       // keys per shared-memory chunk
+constexpr int kSimtThreads = kSimtQ * kSimtTPQ;
+
+struct DenseRows {
+  int N, Nk;
+};
+
+template <typename T, int D, bool WINDOW>
+__global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
+    const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+    T* __restrict__ o, float* __restrict__ ws, int H, DenseRows dr, PlanView P, float scale) {
+  constexpr int DPT = D / kSimtTPQ;
+  extern __shared__ float smem[];
+  float* Ks = smem;                       // [kSimtKV][D]
+  float* Vs = smem + kSimtKV * D;         // [kSimtKV][D]
+  __shared__ int s_kvtok[kSimtKV];
+
+  const int b = blockIdx.z, h = blockIdx.y;
+  const int tid = threadIdx.x;
+  const int ql = tid / kSimtTPQ, part = tid % kSimtTPQ;
+
+  // ---- query rows and key/value set of this block
+  int N, nkv, wi = 0, r = 0;
+  int4 win = make_int4(0, 0, 0, 0), ext = make_int4(0, 0, 0, 0);
+  const int* glist = nullptr;
+  bool qvalid;
+  int qtok;
+  if (WINDOW) {
+    N = P.N;
+    const int item = blockIdx.x / (kQTile / kSimtQ);
+    const int sub = blockIdx.x % (kQTile / kSimtQ);
+    if (item >= P.nitem[b]) return;
+    const int2 it = P.items[(int64_t)b * P.nitem_max + item];
+    wi = it.x;
+    const int64_t wo = (int64_t)b * P.nw + wi;
+    win = P.win[wo];
+    ext = P.ext[wo];
+    nkv = ext.z * ext.w + P.gcount[wo];
+    glist = P.gidx + wo * P.G;
+    r = it.y * kQTile + sub * kSimtQ + ql;
+    qvalid = r < win.z * win.w;
+    qtok = qvalid ? (win.x + r / win.w) * P.Wg + win.y + r % win.w : 0;
+  } else {
+    N = dr.N;
+    nkv = dr.Nk;
+    r = blockIdx.x * kSimtQ + ql;
+    qvalid = r < N;
+    qtok = qvalid ? r : 0;
+  }
+  const int64_t bh = (int64_t)b * H + h;
+  const int Nkv_rows = WINDOW ? N : dr.Nk;  // rows of the K/V tensors per (b, h)
+  const T* qrow = q + (bh * N + qtok) * D;
+  const T* kb = k + bh * Nkv_rows * D;
+  const T* vb = v + bh * Nkv_rows * D;
+
+  float qv[DPT], acc[DPT];
+#pragma unroll
+  for (int i = 0; i < DPT; ++i) {
+    qv[i] = load_as_float(qrow, part + kSimtTPQ * i) * scale;
+    acc[i] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+
+  for (int c0 = 0; c0 < nkv; c0 += kSimtKV) {
+    const int cn = min(kSimtKV, nkv - c0);
+    if (tid < kSimtKV) {
+      int tok = 0;
+      const int j = c0 + tid;
+      if (tid < cn) {
+        if (WINDOW) {
+          const int ne = ext.z * ext.w;
+          tok = j < ne ? (ext.x + j / ext.w) * P.Wg + ext.y + j % ext.w : glist[j - ne];
+        } else {
+          tok = j;
+        }
+      }
+      s_kvtok[tid] = tok;
+    }
+    __syncthreads();
+    // cooperative load: thread -> (row, quarter of the row)
+    for (int e = tid; e < kSimtKV * 4; e += kSimtThreads) {
+      const int row = e >> 2, qd = e & 3;
+      const int64_t src = (int64_t)s_kvtok[row] * D;
+#pragma unroll 4
+      for (int d = qd * (D / 4); d < (qd + 1) * (D / 4); ++d) {
+        const bool ok = row < cn;
+        Ks[row * D + d] = ok ? load_as_float(kb, src + d) : 0.f;
+        Vs[row * D + d] = ok ? load_as_float(vb, src + d) : 0.f;
+      }
+    }
+    __syncthreads();
+    float s[kSimtKV];
+    float mc = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kSimtKV; ++j) {
+      float part_dot = 0.f;
+#pragma unroll
+      for (int i = 0; i < DPT; ++i) part_dot += qv[i] * Ks[j * D + part + kSimtTPQ * i];
+      part_dot += __shfl_xor_sync(0xffffffffu, part_dot, 1);
+      part_dot += __shfl_xor_sync(0xffffffffu, part_dot, 2);
+      part_dot += __shfl_xor_sync(0xffffffffu, part_dot, 4);
+      s[j] = j < cn ? part_dot : -INFINITY;
+      mc = fmaxf(mc, s[j]);
+    }
+    const float mn = fmaxf(m, mc);
+    const float corr = expf(m - mn);
+    l *= corr;
+#pragma unroll
+    for (int i = 0; i < DPT; ++i) acc[i] *= corr;
+#pragma unroll
+    for (int j = 0; j < kSimtKV; ++j) {
+      const float p = expf(s[j] - mn);
+      l += p;
+#pragma unroll
+      for (int i = 0; i < DPT; ++i) acc[i] += p * Vs[j * D + part + kSimtTPQ * i];
+    }
+    m = mn;
+    __syncthreads();
+  }
+  if (!qvalid) return;
+  const float inv = 1.f / l;
+  if (WINDOW) {
+    const int y = qtok / P.Wg, x = qtok % P.Wg;
+    const float t = (float)(min(y - win.x + 1, win.x + win.z - y) *
+                            min(x - win.y + 1, win.y + win.w - x));
+    float* dst = ws + (bh * N + qtok) * D;
+#pragma unroll
+    for (int i = 0; i < DPT; ++i) atomicAdd(dst + part + kSimtTPQ * i, t * acc[i] * inv);
+  } else {
+    T* dst = o + (bh * N + qtok) * D;
+#pragma unroll
+    for (int i = 0; i < DPT; ++i) store_from_float(dst, part + kSimtTPQ * i, acc[i] * inv);
+  }
+}
+
+__global__ void __launch_bounds__(256) ws_zero_kernel(float4* ws, int64_t n4) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x)
+    ws[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) window_finalize_kernel(const float4* __restrict__ ws,
+                                                              PlanView P, T* __restrict__ o,
+                                                              int H, int D) {
+  const int64_t n4 = (int64_t)P.B * H * P.N * D / 4;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = (i * 4) / D;          // (b*H + h)*N + n
+    const int n = (int)(row % P.N);
+    const int b = (int)(row / P.N / H);
+    const float inv = 1.f / P.wsum[(int64_t)b * P.N + n];
+    const float4 a = ws[i];
+    store_from_float(o, 4 * i + 0, a.x * inv);
+    store_from_float(o, 4 * i + 1, a.y * inv);
+    store_from_float(o, 4 * i + 2, a.z * inv);
+    store_from_float(o, 4 * i + 3, a.w * inv);
+  }
+}
+
+template <typename T, int D, bool WINDOW>
+cudaError_t launch_simt(dim3 grid, const void* q, const void* k, const void* v, void* o,
+                        float* ws, int H, DenseRows dr, PlanView P, float scale,
+                        cudaStream_t s) {
+  const int smem = 2 * kSimtKV * D * (int)sizeof(float);
+  auto fn = attn_simt_kernel<T, D, WINDOW>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  fn<<<grid, kSimtThreads, smem, s>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                      static_cast<const T*>(v), static_cast<T*>(o), ws, H, dr, P,
+                                      scale);
+  return cudaGetLastError();
+}
+
+int grid_cap(int64_t n, int block) {
+  int64_t g = (n + block - 1) / block;
+  const int64_t cap = 148LL * 32;
+  return (int)(g < 1 ? 1 : (g > cap ? cap : g));
+}
+
+}  // namespace
+
+cudaError_t launch_dense_attn_simt(const void* q, const void* k, const void* v, void* o, int B,
+                                   int H, int N, int Nk, int D, float scale, int dtype,
+                                   cudaStream_t s) {
+  dim3 grid((N + kSimtQ - 1) / kSimtQ, H, B);
+  DenseRows dr{N, Nk};
+  PlanView P{};
+  if (dtype == AREA_DTYPE_F32) {
+    if (D == 64) return launch_simt<float, 64, false>(grid, q, k, v, o, nullptr, H, dr, P, scale, s);
+    return launch_simt<float, 128, false>(grid, q, k, v, o, nullptr, H, dr, P, scale, s);
+  }
+  if (D == 64) return launch_simt<__nv_bfloat16, 64, false>(grid, q, k, v, o, nullptr, H, dr, P, scale, s);
+  return launch_simt<__nv_bfloat16, 128, false>(grid, q, k, v, o, nullptr, H, dr, P, scale, s);
+}
+
+cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v,
+                                    const PlanLayout& L, const void* plan, float* ws, int H,
+                                    int D, float scale, int dtype, cudaStream_t s) {
+  PlanView P = plan_view(L, const_cast<void*>(plan));
+  dim3 grid((unsigned)(L.nitem_max * (kQTile / kSimtQ)), H, (unsigned)L.B);
+  DenseRows dr{(int)L.N, (int)L.N};
+  if (dtype == AREA_DTYPE_F32) {
+    if (D == 64) return launch_simt<float, 64, true>(grid, q, k, v, nullptr, ws, H, dr, P, scale, s);
+    return launch_simt<float, 128, true>(grid, q, k, v, nullptr, ws, H, dr, P, scale, s);
+  }
+  if (D == 64) return launch_simt<__nv_bfloat16, 64, true>(grid, q, k, v, nullptr, ws, H, dr, P, scale, s);
+  return launch_simt<__nv_bfloat16, 128, true>(grid, q, k, v, nullptr, ws, H, dr, P, scale, s);
+}
+
+cudaError_t launch_ws_zero(float* ws, int64_t n, cudaStream_t s) {
+  const int64_t n4 = n / 4;
+  ws_zero_kernel<<<grid_cap(n4, 256), 256, 0, s>>>(reinterpret_cast<float4*>(ws), n4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_window_finalize(const float* ws, const PlanLayout& L, const void* plan,
+                                   void* o, int H, int D, int dtype, cudaStream_t s) {
+  PlanView P = plan_view(L, const_cast<void*>(plan));
+  const int64_t n4 = L.B * H * L.N * D / 4;
+  const int grid = grid_cap(n4, 256);
+  auto* w4 = reinterpret_cast<const float4*>(ws);
+  if (dtype == AREA_DTYPE_F32)
+    window_finalize_kernel<float><<<grid, 256, 0, s>>>(w4, P, static_cast<float*>(o), H, D);
+  else
+    window_finalize_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(w4, P, static_cast<__nv_bfloat16*>(o), H, D);
+  return cudaGetLastError();
+}
+
+}  // namespace area

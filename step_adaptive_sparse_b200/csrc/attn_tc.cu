@@ -1,0 +1,742 @@
+// tcgen05 flash attention for sm_100a (bf16 in, fp32 accumulate, head_dim 128).
+//
+// One kernel serves the three attention calls of the AReA hot path:
+//   * coarse attention (Phase I: full-resolution queries against pooled keys),
+//   * full attention (the operation AReA replaces, used for the speedup ratio),
+//   * windowed attention (Phase II: queries of a window against its Halo
+//     rectangle plus its global-KV tokens, outputs blended by tent weights).
+// Pages: ai.info "Methodology in Plain English" (Phase I, Phase II);
+// gpt-diffusion.com "Las dos fases de AReA".
+//
+// Design (one persistent CTA per SM, 384 threads):
+//   warp 0      TMA producer: Q tiles once per work unit, then a ring of K and
+//               V tiles (128 keys x 128 dims, 128B-swizzled, 32 KB each).
+//               Dense rows use tiled 2-D loads; window rows (a rectangle
+//               enumerated row-major, then the global-KV list) use gather4.
+//   warp 1      TMEM allocator and the single MMA-issuing thread.
+//   warps 4-7   softmax of query tile 0, warps 8-11 of query tile 1: each
+//               thread owns one query row (one TMEM lane).
+// TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.  P (bf16)
+// overwrites the first 64 columns of its S tile and feeds the PV MMA straight
+// from TMEM.  Online softmax rescales O in TMEM only when the running row
+// maximum grows by more than 2^8 (the final normalisation uses the same stale
+// maximum in numerator and denominator, so the result is exact).
+// Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the kernel
+// records an error code, stops issuing work and still releases its TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "area_internal.cuh"
+
+namespace area {
+
+__device__ int g_tc_error = 0;   // set on a bounded-wait expiry; read by tests
+
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kStages = 4;              // K/V ring stages of 32 KB
+constexpr int kTileBytes = 128 * 128 * 2;
+constexpr int kHalfBytes = 128 * 128;   // 128 rows x 64 bf16
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+// Shared-memory plan (offsets from a 1024-aligned base).
+constexpr int kSmemQ = 0;                              // 2 tiles x 32 KB
+constexpr int kSmemKV = 2 * kTileBytes;                // kStages x 32 KB
+constexpr int kSmemBar = kSmemKV + kStages * kTileBytes;
+constexpr int kSmemBytes = kSmemBar + 256 + 1024;      // barriers + alignment slack
+
+// barrier indices
+enum {
+  BAR_Q_FULL = 0,
+  BAR_Q_EMPTY,
+  BAR_S_FULL0, BAR_S_FULL1,
+  BAR_P_FULL0, BAR_P_FULL1,
+  BAR_O_FULL0, BAR_O_FULL1,
+  BAR_KV_FULL,                       // kStages of them
+  BAR_KV_EMPTY = BAR_KV_FULL + kStages,
+  BAR_DRAIN = BAR_KV_EMPTY + kStages,  // MMA completion before TMEM release
+  BAR_COUNT
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait for the phase of the given parity.  Returns false on expiry.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* abort_flag) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  uint32_t it = 0;
+  while (!mbar_try(bar, parity)) {
+    if ((++it & 255u) == 0) {
+      if (*(volatile int*)abort_flag) return false;
+      if (global_ns() - t0 > kWaitNs) {
+        *(volatile int*)abort_flag = 1;
+        atomicExch(&g_tc_error, 1);
+        return false;
+      }
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
+      "r"(r3)
+      : "memory");
+}
+
+// UMMA shared-memory descriptor, 128-byte swizzle, sm_100 version field.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor: fp32 accumulate, bf16 A and B, M = N = 128.
+constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) |
+                              ((128u >> 4) << 24);
+constexpr uint32_t kIdescPV = kIdescQK | (1u << 16);   // B (V) is MN-major
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                       uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+#define AREA_R32(a) "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), \
+  "=r"(a[6]), "=r"(a[7]), "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]),   \
+  "=r"(a[13]), "=r"(a[14]), "=r"(a[15]), "=r"(a[16]), "=r"(a[17]), "=r"(a[18]),            \
+  "=r"(a[19]), "=r"(a[20]), "=r"(a[21]), "=r"(a[22]), "=r"(a[23]), "=r"(a[24]),            \
+  "=r"(a[25]), "=r"(a[26]), "=r"(a[27]), "=r"(a[28]), "=r"(a[29]), "=r"(a[30]), "=r"(a[31])
+#define AREA_W32(a) "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]),       \
+  "r"(a[6]), "r"(a[7]), "r"(a[8]), "r"(a[9]), "r"(a[10]), "r"(a[11]), "r"(a[12]),          \
+  "r"(a[13]), "r"(a[14]), "r"(a[15]), "r"(a[16]), "r"(a[17]), "r"(a[18]), "r"(a[19]),      \
+  "r"(a[20]), "r"(a[21]), "r"(a[22]), "r"(a[23]), "r"(a[24]), "r"(a[25]), "r"(a[26]),      \
+  "r"(a[27]), "r"(a[28]), "r"(a[29]), "r"(a[30]), "r"(a[31])
+
+// 32 consecutive TMEM columns of this thread's lane.  The wait sits in the
+// same asm statement, so no use of the registers can be scheduled before it.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : AREA_R32(r)
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+      "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, "
+      "%27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      AREA_W32(r)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+      "%10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Work units
+// ---------------------------------------------------------------------------
+struct DenseArgs {
+  int B, H, N, Nk;
+  int units_per_head;   // ceil(N / 256)
+};
+
+struct Unit {
+  bool valid;
+  int bh;          // b*H + h
+  int b;
+  int q0;          // first query position of tile 0 (tile 1 = q0 + 128)
+  int nq;          // number of valid query positions from q0 (window: area)
+  int nkv;         // number of keys
+  int4 win, ext;   // window mode
+  const int* glist;
+};
+
+template <bool WINDOW>
+__device__ __forceinline__ Unit get_unit(int u, const DenseArgs& da, const PlanView& P, int H) {
+  Unit x;
+  x.valid = true;
+  x.glist = nullptr;
+  if (!WINDOW) {
+    x.bh = u / da.units_per_head;
+    x.b = x.bh / da.H;
+    x.q0 = (u % da.units_per_head) * 256;
+    x.nq = da.N;
+    x.nkv = da.Nk;
+    x.win = x.ext = make_int4(0, 0, 0, 0);
+  } else {
+    const int BH = P.B * H;
+    const int item = u / BH;
+    x.bh = u % BH;
+    x.b = x.bh / H;
+    if (item >= P.nitem[x.b]) {
+      x.valid = false;
+      return x;
+    }
+    const int2 it = P.items[(int64_t)x.b * P.nitem_max + item];
+    const int64_t wo = (int64_t)x.b * P.nw + it.x;
+    x.win = P.win[wo];
+    x.ext = P.ext[wo];
+    x.q0 = it.y * 256;
+    x.nq = x.win.z * x.win.w;
+    x.nkv = x.ext.z * x.ext.w + P.gcount[wo];
+    x.glist = P.gidx + wo * P.G;
+  }
+  return x;
+}
+
+// Token of the p-th key of a window unit (rectangle row-major, then global list).
+__device__ __forceinline__ int window_key_token(const Unit& x, int p, int Wg) {
+  const int ne = x.ext.z * x.ext.w;
+  if (p >= x.nkv) p = 0;
+  if (p < ne) return (x.ext.x + p / x.ext.w) * Wg + x.ext.y + p % x.ext.w;
+  return x.glist[p - ne];
+}
+
+__device__ __forceinline__ int window_query_token(const Unit& x, int p, int Wg) {
+  if (p >= x.nq) p = 0;
+  return (x.win.x + p / x.win.w) * Wg + x.win.y + p % x.win.w;
+}
+
+struct TcParams {
+  float scale_log2;
+  int H;
+  int num_units;
+  DenseArgs da;
+  PlanView P;
+  __nv_bfloat16* o;   // dense output
+  float* ws;          // window workspace
+};
+
+template <bool WINDOW>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const TcParams prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + kSmemBar;
+  __shared__ uint32_t s_tmem_base;
+  __shared__ int s_abort;
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    mbar_init(bar(BAR_Q_FULL), 1);
+    mbar_init(bar(BAR_Q_EMPTY), 1);
+    mbar_init(bar(BAR_S_FULL0), 1);
+    mbar_init(bar(BAR_S_FULL1), 1);
+    mbar_init(bar(BAR_P_FULL0), 128);
+    mbar_init(bar(BAR_P_FULL1), 128);
+    mbar_init(bar(BAR_O_FULL0), 1);
+    mbar_init(bar(BAR_O_FULL1), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(BAR_KV_FULL + s), 1);
+      mbar_init(bar(BAR_KV_EMPTY + s), 1);
+    }
+    mbar_init(bar(BAR_DRAIN), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     smem_u32(&s_tmem_base))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem_base;
+  int* abort_flag = &s_abort;
+  const int Wg = WINDOW ? prm.P.Wg : 0;
+  const int Ntok = WINDOW ? prm.P.N : prm.da.N;     // rows per (b, h) of Q
+  const int Nkrows = WINDOW ? prm.P.N : prm.da.Nk;  // rows per (b, h) of K and V
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    uint32_t kv_it = 0, unit_count = 0;
+    for (int u = blockIdx.x; u < prm.num_units; u += gridDim.x) {
+      const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H);
+      if (!x.valid) continue;
+      if (!mbar_wait(bar(BAR_Q_EMPTY), (unit_count & 1u) ^ 1u, abort_flag)) break;
+      if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL), 2 * kTileBytes);
+      __syncwarp();
+      if constexpr (!WINDOW) {
+        if (lane == 0) {
+          for (int t = 0; t < 2; ++t)
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_2d(sbase + kSmemQ + t * kTileBytes + hf * kHalfBytes, &tm_q,
+                          bar(BAR_Q_FULL), hf * 64, x.bh * Ntok + x.q0 + t * 128);
+        }
+      } else {
+        for (int t = 0; t < 2; ++t) {
+          int r[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            r[i] = x.bh * Ntok + window_query_token(x, x.q0 + t * 128 + lane * 4 + i, Wg);
+          for (int hf = 0; hf < 2; ++hf)
+            tma_gather4(sbase + kSmemQ + t * kTileBytes + hf * kHalfBytes + lane * 512, &tm_q,
+                        bar(BAR_Q_FULL), hf * 64, r[0], r[1], r[2], r[3]);
+        }
+      }
+      const int nt = (x.nkv + 127) / 128;
+      bool ok = true;
+      for (int j = 0; j < nt && ok; ++j) {
+        for (int kv = 0; kv < 2; ++kv) {       // K then V
+          const int s = (int)(kv_it % kStages);
+          if (!mbar_wait(bar(BAR_KV_EMPTY + s), ((kv_it / kStages) & 1u) ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) mbar_arrive_tx(bar(BAR_KV_FULL + s), kTileBytes);
+          __syncwarp();
+          const CUtensorMap* tm = kv ? &tm_v : &tm_k;
+          const uint32_t dst = sbase + kSmemKV + s * kTileBytes;
+          if constexpr (!WINDOW) {
+            if (lane == 0)
+              for (int hf = 0; hf < 2; ++hf)
+                tma_load_2d(dst + hf * kHalfBytes, tm, bar(BAR_KV_FULL + s), hf * 64,
+                            x.bh * Nkrows + j * 128);
+          } else {
+            int r[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              r[i] = x.bh * Nkrows + window_key_token(x, j * 128 + lane * 4 + i, Wg);
+            for (int hf = 0; hf < 2; ++hf)
+              tma_gather4(dst + hf * kHalfBytes + lane * 512, tm, bar(BAR_KV_FULL + s), hf * 64,
+                          r[0], r[1], r[2], r[3]);
+          }
+          ++kv_it;
+        }
+      }
+      if (!ok) break;
+      ++unit_count;
+    }
+    // Drain: the most recent load of every stage has landed (bounded wait).
+    int drain_abort = 0;
+    for (uint32_t k = 0; k < kStages && k < kv_it; ++k) {
+      const uint32_t it = kv_it - 1 - k;
+      mbar_wait(bar(BAR_KV_FULL + it % kStages), (it / kStages) & 1u, &drain_abort);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t kv_it = 0, unit_count = 0, s_cnt0 = 0, s_cnt1 = 0;
+      uint32_t p_cnt0 = 0, p_cnt1 = 0;
+      const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
+      const uint32_t q0s = sbase + kSmemQ, q1s = sbase + kSmemQ + kTileBytes;
+      bool ok = true;
+      auto kv_addr = [&](uint32_t it) { return sbase + kSmemKV + (it % kStages) * kTileBytes; };
+      auto qk = [&](uint32_t d, uint32_t qs, uint32_t ks) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+          mma_ss(d, sdesc(qs + off, 16, 1024), sdesc(ks + off, 16, 1024), kIdescQK, kk > 0);
+        }
+      };
+      auto pv = [&](uint32_t d, uint32_t p_tmem, uint32_t vs, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(d, p_tmem + kk * 8, sdesc(vs + kk * 2048, kHalfBytes, 1024), kIdescPV,
+                 (first && kk == 0) ? 0u : 1u);
+      };
+      for (int u = blockIdx.x; u < prm.num_units && ok; u += gridDim.x) {
+        const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H);
+        if (!x.valid) continue;
+        const int nt = (x.nkv + 127) / 128;
+        if (!(ok = mbar_wait(bar(BAR_Q_FULL), unit_count & 1u, abort_flag))) break;
+        // prologue: S(0)
+        const uint32_t k0 = kv_it;
+        if (!(ok = mbar_wait(bar(BAR_KV_FULL + k0 % kStages), (k0 / kStages) & 1u, abort_flag)))
+          break;
+        tc_fence_after();
+        qk(tS0, q0s, kv_addr(k0));
+        mma_commit(bar(BAR_S_FULL0));
+        qk(tS1, q1s, kv_addr(k0));
+        mma_commit(bar(BAR_S_FULL1));
+        mma_commit(bar(BAR_KV_EMPTY + k0 % kStages));
+        if (nt == 1) mma_commit(bar(BAR_Q_EMPTY));
+        for (int j = 0; j < nt && ok; ++j) {
+          const uint32_t vi = kv_it + 2 * j + 1;
+          const uint32_t kn = kv_it + 2 * j + 2;
+          if (!(ok = mbar_wait(bar(BAR_KV_FULL + vi % kStages), (vi / kStages) & 1u, abort_flag)))
+            break;
+          if (!(ok = mbar_wait(bar(BAR_P_FULL0), p_cnt0 & 1u, abort_flag))) break;
+          ++p_cnt0;
+          tc_fence_after();
+          pv(tO0, tS0, kv_addr(vi), j == 0);
+          if (j == nt - 1) mma_commit(bar(BAR_O_FULL0));
+          if (j + 1 < nt) {
+            if (!(ok = mbar_wait(bar(BAR_KV_FULL + kn % kStages), (kn / kStages) & 1u,
+                                 abort_flag)))
+              break;
+            tc_fence_after();
+            qk(tS0, q0s, kv_addr(kn));
+            mma_commit(bar(BAR_S_FULL0));
+          }
+          if (!(ok = mbar_wait(bar(BAR_P_FULL1), p_cnt1 & 1u, abort_flag))) break;
+          ++p_cnt1;
+          tc_fence_after();
+          pv(tO1, tS1, kv_addr(vi), j == 0);
+          if (j == nt - 1) mma_commit(bar(BAR_O_FULL1));
+          mma_commit(bar(BAR_KV_EMPTY + vi % kStages));
+          if (j + 1 < nt) {
+            qk(tS1, q1s, kv_addr(kn));
+            mma_commit(bar(BAR_S_FULL1));
+            mma_commit(bar(BAR_KV_EMPTY + kn % kStages));
+            if (j + 2 == nt) mma_commit(bar(BAR_Q_EMPTY));
+          }
+        }
+        kv_it += 2 * nt;
+        ++unit_count;
+      }
+      (void)s_cnt0;
+      (void)s_cnt1;
+      // Drain: every MMA issued by this thread has completed (bounded wait).
+      int drain_abort = 0;
+      mma_commit(bar(BAR_DRAIN));
+      mbar_wait(bar(BAR_DRAIN), 0, &drain_abort);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int qt = (warp - 4) >> 2;                  // query tile of this warpgroup
+    const int row = ((warp & 3) << 5) + lane;        // TMEM lane = query row in the tile
+    const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
+    const uint32_t tS = tmem + lane_off + (qt ? 128u : 0u);
+    const uint32_t tO = tmem + lane_off + (qt ? 384u : 256u);
+    const uint32_t bS = bar(qt ? BAR_S_FULL1 : BAR_S_FULL0);
+    const uint32_t bP = bar(qt ? BAR_P_FULL1 : BAR_P_FULL0);
+    const uint32_t bO = bar(qt ? BAR_O_FULL1 : BAR_O_FULL0);
+    uint32_t s_cnt = 0, o_cnt = 0;
+    const float sl2 = prm.scale_log2;
+    bool ok = true;
+    for (int u = blockIdx.x; u < prm.num_units && ok; u += gridDim.x) {
+      const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H);
+      if (!x.valid) continue;
+      const int nt = (x.nkv + 127) / 128;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < nt; ++j) {
+        if (!(ok = mbar_wait(bS, s_cnt & 1u, abort_flag))) break;
+        ++s_cnt;
+        tc_fence_after();
+        const int valid = min(128, x.nkv - j * 128);
+        // pass 1: row maximum over the valid keys
+        float mx = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sr[32];
+          tmem_ld32(tS + c * 32, sr);
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i < valid) mx = fmaxf(mx, __uint_as_float(sr[i]));
+        }
+        const float mnew = mx * sl2;
+        if (j == 0) {
+          m = mnew;
+        } else if (mnew > m + kRescaleThreshold) {
+          const float alpha = fast_exp2(m - mnew);
+          l *= alpha;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t orr[32];
+            tmem_ld32(tO + c * 32, orr);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+            tmem_st32(tO + c * 32, orr);
+          }
+          m = mnew;
+        }
+        // pass 2: P = exp2(S * scale * log2(e) - m) as bf16, two keys per TMEM
+        // column, written over S columns that pass 2 has already read
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sr[32];
+          tmem_ld32(tS + c * 32, sr);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float p0 = fast_exp2(fmaf(__uint_as_float(sr[i]), sl2, -m));
+            float p1 = fast_exp2(fmaf(__uint_as_float(sr[i + 1]), sl2, -m));
+            if (c * 32 + i >= valid) p0 = 0.f;
+            if (c * 32 + i + 1 >= valid) p1 = 0.f;
+            l += p0 + p1;
+            pk[i >> 1] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tS + c * 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bP);
+      }
+      if (!ok) break;
+      // epilogue
+      if (!(ok = mbar_wait(bO, o_cnt & 1u, abort_flag))) break;
+      ++o_cnt;
+      tc_fence_after();
+      const int qpos = x.q0 + qt * 128 + row;
+      const bool qvalid = qpos < x.nq;
+      const float inv = 1.f / l;
+      if constexpr (!WINDOW) {
+        __nv_bfloat16* dst = prm.o + ((int64_t)x.bh * Ntok + qpos) * 128;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(tO + c * 32, orr);
+          if (qvalid) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              uint4 w;
+              w.x = pack_bf16(__uint_as_float(orr[8 * v4 + 0]) * inv, __uint_as_float(orr[8 * v4 + 1]) * inv);
+              w.y = pack_bf16(__uint_as_float(orr[8 * v4 + 2]) * inv, __uint_as_float(orr[8 * v4 + 3]) * inv);
+              w.z = pack_bf16(__uint_as_float(orr[8 * v4 + 4]) * inv, __uint_as_float(orr[8 * v4 + 5]) * inv);
+              w.w = pack_bf16(__uint_as_float(orr[8 * v4 + 6]) * inv, __uint_as_float(orr[8 * v4 + 7]) * inv);
+              d4[v4] = w;
+            }
+          }
+        }
+      } else {
+        const int tok = window_query_token(x, qpos, Wg);
+        const int y = tok / Wg, xx = tok % Wg;
+        const float t = (float)(min(y - x.win.x + 1, x.win.x + x.win.z - y) *
+                                min(xx - x.win.y + 1, x.win.y + x.win.w - xx));
+        const float sc = t * inv;
+        float* dst = prm.ws + ((int64_t)x.bh * Ntok + tok) * 128;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(tO + c * 32, orr);
+          if (qvalid) {
+#pragma unroll
+            for (int v4 = 0; v4 < 8; ++v4)
+              red_add_v4(dst + c * 32 + 4 * v4, __uint_as_float(orr[4 * v4]) * sc,
+                         __uint_as_float(orr[4 * v4 + 1]) * sc,
+                         __uint_as_float(orr[4 * v4 + 2]) * sc,
+                         __uint_as_float(orr[4 * v4 + 3]) * sc);
+          }
+        }
+      }
+      tc_fence_before();
+    }
+  }
+  // warps 2 and 3 have no role
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 map over [rows, 128] with a box of 64 columns x box_rows rows.
+cudaError_t make_map(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {128 * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+template <bool WINDOW>
+cudaError_t launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                      const TcParams& prm, cudaStream_t s) {
+  auto fn = attn_tc_kernel<WINDOW>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int grid = prm.num_units < num_sms() ? prm.num_units : num_sms();
+  fn<<<grid > 0 ? grid : 1, kThreads, kSmemBytes, s>>>(mq, mk, mv, prm);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t read_and_clear_tc_error(int* code) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyFromSymbol(code, g_tc_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_tc_error, &zero, sizeof(int));
+}
+
+cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, void* o, int B,
+                                 int H, int N, int Nk, float scale, cudaStream_t s) {
+  CUtensorMap mq, mk, mv;
+  cudaError_t e;
+  if ((e = make_map(&mq, q, (int64_t)B * H * N, 128)) != cudaSuccess) return e;
+  if ((e = make_map(&mk, k, (int64_t)B * H * Nk, 128)) != cudaSuccess) return e;
+  if ((e = make_map(&mv, v, (int64_t)B * H * Nk, 128)) != cudaSuccess) return e;
+  TcParams prm{};
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.H = H;
+  prm.da = DenseArgs{B, H, N, Nk, (N + 255) / 256};
+  prm.num_units = B * H * prm.da.units_per_head;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  return launch_tc<false>(mq, mk, mv, prm, s);
+}
+
+cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v,
+                                  const PlanLayout& L, const void* plan, float* ws, int H,
+                                  float scale, cudaStream_t s) {
+  CUtensorMap mq, mk, mv;
+  cudaError_t e;
+  const int64_t rows = L.B * H * L.N;
+  if ((e = make_map(&mq, q, rows, 1)) != cudaSuccess) return e;
+  if ((e = make_map(&mk, k, rows, 1)) != cudaSuccess) return e;
+  if ((e = make_map(&mv, v, rows, 1)) != cudaSuccess) return e;
+  TcParams prm{};
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.H = H;
+  prm.P = plan_view(L, const_cast<void*>(plan));
+  prm.num_units = (int)(L.nitem_max * L.B * H);
+  prm.ws = ws;
+  return launch_tc<true>(mq, mk, mv, prm, s);
+}
+
+}  // namespace area

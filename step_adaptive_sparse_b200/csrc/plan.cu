@@ -1,0 +1,401 @@
+// Phase II planner on the device: base tiling, DWT-guided quadrant splits,
+// Halo rectangles, the global-KV bridge, merge-weight sums and the work list.
+//
+// Method (AReA summary pages: ai.info "Methodology in Plain English",
+// Phase II; gpt-diffusion.com "Las dos fases de AReA", Fase II): windows cover
+// the grid in an evenly spaced base tiling; windows over smooth regions of a
+// DWT detail map split into four quadrants; each window's keys are extended
+// by a Halo ring and by global-KV tokens from the rest of the image; the
+// overlapping outputs are blended with centre weights.
+//
+// Index lists, split decisions and scores are bit-exact by construction:
+// integer arithmetic, plus fp32 sums in a fixed order with explicit
+// round-to-nearest operations.  The global-KV ranking is a stable LSD radix
+// sort of the energy bits (descending), which keeps token order among ties.
+#include "area_internal.cuh"
+
+namespace area {
+
+static int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
+
+int plan_layout(const area_plan_cfg* cfg, PlanLayout* L) {
+  if (!cfg || !L) return AREA_EINVAL;
+  if (cfg->B < 1 || cfg->Hg < 2 || cfg->Wg < 2 || (cfg->Hg & 1) || (cfg->Wg & 1) ||
+      cfg->Hg > kMaxGrid || cfg->Wg > kMaxGrid || cfg->w < 1 || cfg->halo < 0 || cfg->G < 0 ||
+      cfg->G > kMaxG || cfg->jitter_seed != 0)
+    return AREA_EINVAL;
+  const int64_t N = (int64_t)cfg->Hg * cfg->Wg;
+  if (N > (int64_t(1) << 26)) return AREA_EINVAL;
+  L->B = cfg->B; L->Hg = cfg->Hg; L->Wg = cfg->Wg; L->w = cfg->w; L->halo = cfg->halo;
+  L->G = cfg->G; L->N = N;
+  L->hy = cfg->w < cfg->Hg ? cfg->w : cfg->Hg;
+  L->wx = cfg->w < cfg->Wg ? cfg->w : cfg->Wg;
+  L->nby = (cfg->Hg + L->hy - 1) / L->hy;
+  L->nbx = (cfg->Wg + L->wx - 1) / L->wx;
+  L->nb = L->nby * L->nbx;
+  L->nw = 4 * L->nb;
+  L->nitem_max = L->nb * ((L->hy * L->wx + kQTile - 1) / kQTile + 3);
+  L->ntile_sort = (N + 255) / 256;
+  const int64_t B = L->B;
+  const int64_t sizes[AREA_PLAN_NSEC] = {
+      B * L->nb * 16, B * L->nb * 4, B * L->nb, B * 4,
+      B * L->nw * 16, B * L->nw * 4, B * L->nw * 16, B * L->nw * 4,
+      B * L->nw * L->G * 4, B * N * 4, B * N * 4, (B + 1) * 4,
+      B * L->nitem_max * 8, 0};
+  int64_t off = 256;  // header
+  for (int s = 0; s < AREA_PLAN_NSEC; ++s) {
+    L->off[s] = off;
+    off = align256(off + (sizes[s] > 0 ? sizes[s] : 1));
+  }
+  // scratch of one radix sort (batch elements are sorted one after another)
+  off = L->off[AREA_PLAN_SEC_SCRATCH];
+  L->scratch_keys_a = off; off = align256(off + N * 4);
+  L->scratch_keys_b = off; off = align256(off + N * 4);
+  L->scratch_vals_a = off; off = align256(off + N * 4);
+  L->scratch_vals_b = off; off = align256(off + N * 4);
+  L->scratch_hist = off;   off = align256(off + 256 * L->ntile_sort * 4);
+  L->total = off;
+  return AREA_OK;
+}
+
+PlanView plan_view(const PlanLayout& L, void* plan) {
+  char* p = static_cast<char*>(plan);
+  PlanView v;
+  v.B = (int)L.B; v.Hg = (int)L.Hg; v.Wg = (int)L.Wg; v.w = (int)L.w; v.halo = (int)L.halo;
+  v.G = (int)L.G; v.nby = (int)L.nby; v.nbx = (int)L.nbx; v.hy = (int)L.hy; v.wx = (int)L.wx;
+  v.nb = (int)L.nb; v.nw = (int)L.nw; v.nitem_max = (int)L.nitem_max; v.N = (int)L.N;
+  v.base = reinterpret_cast<int4*>(p + L.off[AREA_PLAN_SEC_BASE]);
+  v.score = reinterpret_cast<float*>(p + L.off[AREA_PLAN_SEC_SCORE]);
+  v.split = reinterpret_cast<uint8_t*>(p + L.off[AREA_PLAN_SEC_SPLIT]);
+  v.nwin = reinterpret_cast<int*>(p + L.off[AREA_PLAN_SEC_NWIN]);
+  v.win = reinterpret_cast<int4*>(p + L.off[AREA_PLAN_SEC_WIN]);
+  v.parent = reinterpret_cast<int*>(p + L.off[AREA_PLAN_SEC_PARENT]);
+  v.ext = reinterpret_cast<int4*>(p + L.off[AREA_PLAN_SEC_EXT]);
+  v.gcount = reinterpret_cast<int*>(p + L.off[AREA_PLAN_SEC_GCOUNT]);
+  v.gidx = reinterpret_cast<int*>(p + L.off[AREA_PLAN_SEC_GIDX]);
+  v.wsum = reinterpret_cast<float*>(p + L.off[AREA_PLAN_SEC_WSUM]);
+  v.order = reinterpret_cast<int*>(p + L.off[AREA_PLAN_SEC_ORDER]);
+  v.nitem = reinterpret_cast<int*>(p + L.off[AREA_PLAN_SEC_NITEM]);
+  v.items = reinterpret_cast<int2*>(p + L.off[AREA_PLAN_SEC_ITEMS]);
+  return v;
+}
+
+namespace {
+
+struct HeaderArgs {
+  int64_t v[32];
+};
+
+__global__ void plan_header_kernel(int64_t* hdr, HeaderArgs a, int* nitem_total) {
+  const int i = threadIdx.x;
+  hdr[i] = a.v[i];
+  if (i == 0) *nitem_total = 0;
+}
+
+// Exclusive block-wide scan of one int per thread (blockDim.x multiple of 32,
+// at most 1024).  Returns the exclusive prefix; *total receives the sum.
+__device__ int block_exclusive_scan(int x, int* total) {
+  __shared__ int s_warp[33];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarp = blockDim.x >> 5;
+  int inc = x;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    int t = __shfl_up_sync(0xffffffffu, inc, d);
+    if (lane >= d) inc += t;
+  }
+  if (lane == 31) s_warp[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int wv = lane < nwarp ? s_warp[lane] : 0;
+    int wi = wv;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      int t = __shfl_up_sync(0xffffffffu, wi, d);
+      if (lane >= d) wi += t;
+    }
+    if (lane < nwarp) s_warp[lane] = wi - wv;  // exclusive warp offsets
+    if (lane == 31) s_warp[32] = wi;
+  }
+  __syncthreads();
+  const int res = s_warp[warp] + inc - x;
+  *total = s_warp[32];
+  __syncthreads();
+  return res;
+}
+
+// Split score of one base window per block.
+__global__ void __launch_bounds__(256) plan_base_kernel(const float* __restrict__ E, PlanView P,
+                                                       float thr) {
+  extern __shared__ float s_rows[];
+  const int b = blockIdx.x / P.nb, bi = blockIdx.x % P.nb;
+  const int iy = bi / P.nbx, ix = bi % P.nbx;
+  const int y0 = tile_start(iy, P.nby, P.Hg, P.hy);
+  const int x0 = tile_start(ix, P.nbx, P.Wg, P.wx);
+  const int Wc = P.Wg / 2;
+  const float* Eb = E + (int64_t)b * (P.Hg / 2) * Wc;
+  for (int y = threadIdx.x; y < P.hy; y += blockDim.x) {
+    const float* er = Eb + (int64_t)((y0 + y) >> 1) * Wc;
+    float acc = 0.f;
+    for (int x = x0; x < x0 + P.wx; ++x) acc = __fadd_rn(acc, er[x >> 1]);
+    s_rows[y] = acc;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float S = 0.f;
+    for (int y = 0; y < P.hy; ++y) S = __fadd_rn(S, s_rows[y]);
+    const float T = __fmul_rn(thr, (float)(P.hy * P.wx));
+    const bool split = P.hy >= 2 && P.wx >= 2 && S < T;
+    const int64_t o = (int64_t)b * P.nb + bi;
+    P.base[o] = make_int4(y0, x0, P.hy, P.wx);
+    P.score[o] = S;
+    P.split[o] = split ? 1 : 0;
+  }
+}
+
+__device__ __forceinline__ int4 halo_rect(int4 w, int h, int Hg, int Wg) {
+  const int ey0 = max(0, w.x - h), ex0 = max(0, w.y - h);
+  const int ey1 = min(Hg, w.x + w.z + h), ex1 = min(Wg, w.y + w.w + h);
+  return make_int4(ey0, ex0, ey1 - ey0, ex1 - ex0);
+}
+
+// Final windows, Halo rectangles, G_W and the work list of one batch element.
+__global__ void __launch_bounds__(1024) plan_windows_kernel(PlanView P) {
+  const int b = blockIdx.x;
+  const int4* base = P.base + (int64_t)b * P.nb;
+  const uint8_t* split = P.split + (int64_t)b * P.nb;
+  int4* win = P.win + (int64_t)b * P.nw;
+  int* parent = P.parent + (int64_t)b * P.nw;
+  int4* ext = P.ext + (int64_t)b * P.nw;
+  int* gcount = P.gcount + (int64_t)b * P.nw;
+  int running = 0, total;
+  for (int c0 = 0; c0 < P.nb; c0 += blockDim.x) {
+    const int i = c0 + threadIdx.x;
+    const bool valid = i < P.nb;
+    const bool sp = valid && split[i];
+    const int cnt = valid ? (sp ? 4 : 1) : 0;
+    const int at = running + block_exclusive_scan(cnt, &total);
+    if (valid) {
+      const int4 bw = base[i];
+      int4 q[4];
+      int nq = 1;
+      if (sp) {
+        const int ht = bw.z / 2, wl = bw.w / 2;
+        q[0] = make_int4(bw.x, bw.y, ht, wl);
+        q[1] = make_int4(bw.x, bw.y + wl, ht, bw.w - wl);
+        q[2] = make_int4(bw.x + ht, bw.y, bw.z - ht, wl);
+        q[3] = make_int4(bw.x + ht, bw.y + wl, bw.z - ht, bw.w - wl);
+        nq = 4;
+      } else {
+        q[0] = bw;
+      }
+      for (int j = 0; j < nq; ++j) {
+        const int4 e = halo_rect(q[j], P.halo, P.Hg, P.Wg);
+        const int64_t rest = (int64_t)P.N - (int64_t)e.z * e.w;
+        win[at + j] = q[j];
+        parent[at + j] = i;
+        ext[at + j] = e;
+        gcount[at + j] = (int)(rest < P.G ? rest : P.G);
+      }
+    }
+    running += total;
+  }
+  const int nwin = running;
+  if (threadIdx.x == 0) P.nwin[b] = nwin;
+  __syncthreads();
+  // Work items: windows whose parent kept its size first (largest KV sets),
+  // then the quadrants; within each class in window order.
+  int2* items = P.items + (int64_t)b * P.nitem_max;
+  running = 0;
+  for (int cls = 0; cls < 2; ++cls) {
+    for (int c0 = 0; c0 < nwin; c0 += blockDim.x) {
+      const int wi = c0 + threadIdx.x;
+      int nq = 0;
+      if (wi < nwin && (int)split[parent[wi]] == cls) {
+        const int4 w = win[wi];
+        nq = (w.z * w.w + kQTile - 1) / kQTile;
+      }
+      const int at = running + block_exclusive_scan(nq, &total);
+      for (int t = 0; t < nq; ++t) items[at + t] = make_int2(wi, t);
+      running += total;
+    }
+  }
+  if (threadIdx.x == 0) {
+    P.nitem[b] = running;
+    atomicAdd(P.nitem + P.B, running);
+  }
+}
+
+// ---- stable LSD radix sort of (~energy bits, token) ------------------------
+__global__ void __launch_bounds__(256) sort_init_kernel(const float* __restrict__ E, int b,
+                                                       PlanView P, uint32_t* keys, int* vals) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= P.N) return;
+  const int y = t / P.Wg, x = t % P.Wg;
+  const int Wc = P.Wg / 2;
+  const float e = E[((int64_t)b * (P.Hg / 2) + (y >> 1)) * Wc + (x >> 1)];
+  keys[t] = ~__float_as_uint(e);   // ascending order of ~bits = descending energy
+  vals[t] = t;
+}
+
+__global__ void __launch_bounds__(256) sort_hist_kernel(const uint32_t* __restrict__ keys, int n,
+                                                       int shift, uint32_t* hist, int ntile) {
+  __shared__ uint32_t s_h[256];
+  s_h[threadIdx.x] = 0;
+  __syncthreads();
+  const int i = blockIdx.x * 256 + threadIdx.x;
+  if (i < n) atomicAdd(&s_h[(keys[i] >> shift) & 255u], 1u);
+  __syncthreads();
+  hist[(int64_t)threadIdx.x * ntile + blockIdx.x] = s_h[threadIdx.x];
+}
+
+// Exclusive scan, in place, of the digit-major histogram (one block).
+__global__ void __launch_bounds__(1024) sort_scan_kernel(uint32_t* hist, int m) {
+  const int per = (m + blockDim.x - 1) / blockDim.x;
+  const int lo = threadIdx.x * per, hi = min(m, lo + per);
+  int sum = 0;
+  for (int i = lo; i < hi; ++i) sum += (int)hist[i];
+  int total;
+  int run = block_exclusive_scan(sum, &total);
+  for (int i = lo; i < hi; ++i) {
+    const int h = (int)hist[i];
+    hist[i] = (uint32_t)run;
+    run += h;
+  }
+}
+
+__global__ void __launch_bounds__(256) sort_scatter_kernel(const uint32_t* __restrict__ kin,
+                                                          const int* __restrict__ vin,
+                                                          uint32_t* kout, int* vout, int n,
+                                                          int shift, const uint32_t* hist,
+                                                          int ntile) {
+  __shared__ int s_cnt[8][257];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int j = threadIdx.x; j < 8 * 257; j += 256) (&s_cnt[0][0])[j] = 0;
+  __syncthreads();
+  const int i = blockIdx.x * 256 + threadIdx.x;
+  const bool valid = i < n;
+  const uint32_t key = valid ? kin[i] : 0u;
+  const int val = valid ? vin[i] : 0;
+  const int d = valid ? (int)((key >> shift) & 255u) : 256;
+  const unsigned peers = __match_any_sync(0xffffffffu, d);
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  if (lane == __ffs(peers) - 1) s_cnt[warp][d] = __popc(peers);
+  __syncthreads();
+  {  // exclusive prefix over warps, one digit per thread
+    const int dd = threadIdx.x;
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const int c = s_cnt[w][dd];
+      s_cnt[w][dd] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  if (valid) {
+    const int pos = (int)hist[(int64_t)d * ntile + blockIdx.x] + s_cnt[warp][d] + rank;
+    kout[pos] = key;
+    vout[pos] = val;
+  }
+}
+
+// Global-KV bridge: first G_W tokens of the ranked order outside ext(W).
+__global__ void __launch_bounds__(1024) plan_global_kernel(PlanView P) {
+  const int b = blockIdx.x / P.nw, wi = blockIdx.x % P.nw;
+  if (wi >= P.nwin[b] || P.G == 0) return;
+  const int64_t o = (int64_t)b * P.nw + wi;
+  const int4 e = P.ext[o];
+  const int gw = P.gcount[o];
+  int* out = P.gidx + o * P.G;
+  const int* order = P.order + (int64_t)b * P.N;
+  int count = 0, total;
+  for (int c0 = 0; c0 < P.N && count < gw; c0 += blockDim.x) {
+    const int p = c0 + threadIdx.x;
+    int tok = -1, flag = 0;
+    if (p < P.N) {
+      tok = order[p];
+      const int y = tok / P.Wg, x = tok % P.Wg;
+      flag = (y >= e.x && y < e.x + e.z && x >= e.y && x < e.y + e.w) ? 0 : 1;
+    }
+    const int at = count + block_exclusive_scan(flag, &total);
+    if (flag && at < gw) out[at] = tok;
+    count += total;
+  }
+  for (int j = gw + threadIdx.x; j < P.G; j += blockDim.x) out[j] = -1;
+}
+
+// Sum of tent weights per token over the final windows that contain it.
+__global__ void __launch_bounds__(256) plan_wsum_kernel(PlanView P) {
+  const int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (g >= (int64_t)P.B * P.N) return;
+  const int b = (int)(g / P.N);
+  const int t = (int)(g % P.N);
+  const int y = t / P.Wg, x = t % P.Wg;
+  int total = 0;
+  for (int iy = 0; iy < P.nby; ++iy) {
+    const int y0 = tile_start(iy, P.nby, P.Hg, P.hy);
+    if (y < y0 || y >= y0 + P.hy) continue;
+    for (int ix = 0; ix < P.nbx; ++ix) {
+      const int x0 = tile_start(ix, P.nbx, P.Wg, P.wx);
+      if (x < x0 || x >= x0 + P.wx) continue;
+      int qy0 = y0, qhy = P.hy, qx0 = x0, qwx = P.wx;
+      if (P.split[(int64_t)b * P.nb + iy * P.nbx + ix]) {
+        const int ht = P.hy / 2, wl = P.wx / 2;
+        if (y < y0 + ht) { qhy = ht; } else { qy0 = y0 + ht; qhy = P.hy - ht; }
+        if (x < x0 + wl) { qwx = wl; } else { qx0 = x0 + wl; qwx = P.wx - wl; }
+      }
+      total += min(y - qy0 + 1, qy0 + qhy - y) * min(x - qx0 + 1, qx0 + qwx - x);
+    }
+  }
+  P.wsum[g] = (float)total;
+}
+
+}  // namespace
+
+cudaError_t launch_window_plan(const float* energy, const area_plan_cfg* cfg,
+                               const PlanLayout& L, void* plan, cudaStream_t s) {
+  PlanView P = plan_view(L, plan);
+  char* base = static_cast<char*>(plan);
+  HeaderArgs h = {};
+  h.v[0] = AREA_PLAN_MAGIC; h.v[1] = AREA_PLAN_VERSION;
+  h.v[2] = L.B; h.v[3] = L.Hg; h.v[4] = L.Wg; h.v[5] = L.w; h.v[6] = L.halo; h.v[7] = L.G;
+  h.v[8] = L.nb; h.v[9] = L.nw;
+  for (int i = 0; i < AREA_PLAN_NSEC; ++i) h.v[10 + i] = L.off[i];
+  h.v[10 + AREA_PLAN_NSEC] = L.nitem_max;
+  h.v[11 + AREA_PLAN_NSEC] = L.N;
+  plan_header_kernel<<<1, 32, 0, s>>>(reinterpret_cast<int64_t*>(base), h, P.nitem + L.B);
+  const int smem = (int)(L.hy * sizeof(float));
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(plan_base_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+  }
+  plan_base_kernel<<<(unsigned)(L.B * L.nb), 256, smem, s>>>(energy, P, cfg->split_thr);
+  plan_windows_kernel<<<(unsigned)L.B, 1024, 0, s>>>(P);
+  uint32_t* ka = reinterpret_cast<uint32_t*>(base + L.scratch_keys_a);
+  uint32_t* kb = reinterpret_cast<uint32_t*>(base + L.scratch_keys_b);
+  int* va = reinterpret_cast<int*>(base + L.scratch_vals_a);
+  int* vb = reinterpret_cast<int*>(base + L.scratch_vals_b);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(base + L.scratch_hist);
+  const int n = (int)L.N, nt = (int)L.ntile_sort;
+  for (int b = 0; b < L.B; ++b) {
+    sort_init_kernel<<<nt, 256, 0, s>>>(energy, b, P, ka, va);
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 8 * pass;
+      const uint32_t* kin = (pass & 1) ? kb : ka;
+      const int* vin = (pass & 1) ? vb : va;
+      uint32_t* kout = (pass & 1) ? ka : kb;
+      int* vout = (pass == 3) ? P.order + (int64_t)b * L.N : ((pass & 1) ? va : vb);
+      sort_hist_kernel<<<nt, 256, 0, s>>>(kin, n, shift, hist, nt);
+      sort_scan_kernel<<<1, 1024, 0, s>>>(hist, 256 * nt);
+      sort_scatter_kernel<<<nt, 256, 0, s>>>(kin, vin, kout, vout, n, shift, hist, nt);
+    }
+  }
+  plan_global_kernel<<<(unsigned)(L.B * L.nw), 1024, 0, s>>>(P);
+  const int64_t ntok = L.B * L.N;
+  plan_wsum_kernel<<<(unsigned)((ntok + 255) / 256), 256, 0, s>>>(P);
+  return cudaGetLastError();
+}
+
+}  // namespace area

@@ -1,0 +1,126 @@
+"""The C-ABI library loads, exports every declared symbol, and validates its
+arguments on the host (no kernel is launched by any test in this file)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "area.h")
+
+
+@pytest.fixture(scope="module")
+def area():
+    import step_adaptive_sparse_b200 as area
+    from step_adaptive_sparse_b200 import binding
+    if not os.path.exists(binding.LIB_PATH):
+        from step_adaptive_sparse_b200.build import build
+        build()
+    area.library()
+    return area
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(area_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary_calls():
+    names = declared_functions()
+    for want in ["area_pool_kv", "area_coarse_attn", "area_full_attn", "area_dwt_detail",
+                 "area_window_plan", "area_window_plan_bytes", "area_window_attn",
+                 "area_status_string", "area_version"]:
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(area):
+    lib = area.library()
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in area.h but not exported"
+    from step_adaptive_sparse_b200 import binding
+    assert set(binding.EXPORTED) <= set(declared_functions())
+
+
+def test_version_and_status_strings(area):
+    assert "sm_100a" in area.area_version()
+    for st in range(5):
+        assert area.status_string(st).startswith("AREA_")
+    assert "unknown" in area.status_string(99)
+
+
+def test_null_and_bad_arguments_rejected_on_host(area):
+    with pytest.raises(area.AreaError) as e:
+        area.area_pool_kv(None, None, None, None, 1, 1, 4, 4, 8, 2, 0, 1)
+    assert e.value.status == area.AREA_EINVAL
+    fake = 1 << 20   # never dereferenced: validation fails first
+    cases = [
+        (lambda: area.area_pool_kv(fake, fake, fake, fake, 1, 1, 6, 4, 8, 4, 0, 1), area.AREA_EINVAL),
+        (lambda: area.area_pool_kv(fake, fake, fake, fake, 1, 1, 4, 4, 8, 2, 7, 1), area.AREA_EINVAL),
+        (lambda: area.area_pool_kv(fake, fake, fake, fake, 1, 1, 4, 4, 8, 2, 0, 5), area.AREA_EINVAL),
+        (lambda: area.area_pool_kv(fake, fake, fake, fake, 1, 1, 4, 4, 6, 2, 0, 1), area.AREA_EUNSUPPORTED),
+        (lambda: area.area_pool_kv(fake + 2, fake, fake, fake, 1, 1, 4, 4, 8, 2, 0, 1), area.AREA_EINVAL),
+        (lambda: area.area_coarse_attn(fake, fake, fake, fake, 1, 1, 16, 0, 128, 1.0, 1), area.AREA_EINVAL),
+        (lambda: area.area_coarse_attn(fake, fake, fake, fake, 1, 1, 16, 4, 96, 1.0, 1), area.AREA_EUNSUPPORTED),
+        (lambda: area.area_coarse_attn(fake, fake, fake, fake, 1, 1, 16, 4, 128, 1.0, 3), area.AREA_EUNSUPPORTED),
+        (lambda: area.area_full_attn(None, fake, fake, fake, 1, 1, 16, 128, 1.0, 1), area.AREA_EINVAL),
+        (lambda: area.area_dwt_detail(fake, 1, 16, fake, 1, 7, 8), area.AREA_EINVAL),
+        (lambda: area.area_dwt_detail(fake, 1, 0, fake, 1, 8, 8), area.AREA_EINVAL),
+        (lambda: area.area_dwt_detail(fake, 1, 4, fake, 1, 8, 8, 9), area.AREA_EINVAL),
+    ]
+    for fn, status in cases:
+        with pytest.raises(area.AreaError) as e:
+            fn()
+        assert e.value.status == status
+
+
+def test_plan_config_validation_and_sizes(area):
+    good = area.make_cfg(1, 256, 256, 64, 4, 512, 0.4)
+    n = area.area_window_plan_bytes(good)
+    assert n > 0 and n % 256 == 0
+    # plan size grows with G and with the number of windows
+    assert area.area_window_plan_bytes(area.make_cfg(1, 256, 256, 64, 4, 1024, 0.4)) > n
+    assert area.area_window_plan_bytes(area.make_cfg(1, 256, 256, 32, 4, 512, 0.4)) > n
+    assert area.area_window_plan_bytes(area.make_cfg(2, 256, 256, 64, 4, 512, 0.4)) > n
+    assert area.area_window_attn_ws_bytes(good, 24, 128) == 24 * 65536 * 128 * 4
+    for bad in [area.make_cfg(0, 256, 256, 64, 4, 512, 0.4),
+                area.make_cfg(1, 255, 256, 64, 4, 512, 0.4),
+                area.make_cfg(1, 256, 256, 0, 4, 512, 0.4),
+                area.make_cfg(1, 256, 256, 64, -1, 512, 0.4),
+                area.make_cfg(1, 256, 256, 64, 4, 5000, 0.4),
+                area.make_cfg(1, 256, 256, 64, 4, 512, 0.4, jitter_seed=7)]:
+        with pytest.raises(area.AreaError) as e:
+            area.area_window_plan_bytes(bad)
+        assert e.value.status == area.AREA_EINVAL
+
+
+def test_window_calls_reject_small_buffers_on_host(area):
+    cfg = area.make_cfg(1, 32, 32, 8, 1, 16, 0.05)
+    need = area.area_window_plan_bytes(cfg)
+    fake = 1 << 20
+    with pytest.raises(area.AreaError) as e:
+        area.area_window_plan(fake, cfg, fake, need - 256)
+    assert e.value.status == area.AREA_ENOSPACE
+    ws = area.area_window_attn_ws_bytes(cfg, 2, 64)
+    with pytest.raises(area.AreaError) as e:
+        area.area_window_attn(fake, fake, fake, cfg, fake, need, fake, fake, ws - 4, 2, 64, 0.125, 0)
+    assert e.value.status == area.AREA_ENOSPACE
+    with pytest.raises(area.AreaError) as e:
+        area.area_window_attn(fake, fake, fake, cfg, fake, need - 1, fake, fake, ws, 2, 64, 0.125, 0)
+    assert e.value.status == area.AREA_ENOSPACE
+    with pytest.raises(area.AreaError) as e:
+        area.area_window_attn(fake, fake, fake, cfg, fake + 16, need, fake, fake, ws, 2, 64, 0.125, 0)
+    assert e.value.status == area.AREA_EINVAL
+
+
+def test_binding_has_no_oracle_dependency():
+    # The product path never reaches the oracle: no module of the package
+    # imports it, and the binding fails loudly without the shared library.
+    pkg = os.path.join(ROOT, "step_adaptive_sparse_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle", text, flags=re.M), fn
+                assert "area_oracle" not in text, fn

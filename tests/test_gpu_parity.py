@@ -1,0 +1,238 @@
+"""GPU parity: the CUDA path through the C-ABI against the CPU oracle.
+
+Bars: index plans, split decisions, scores, global-KV lists, merge-weight sums
+and detail maps bit-exact; attention outputs within max-abs 2e-2 / mean-abs
+2e-3 for bf16 inputs (fp32 accumulation) and 1e-4 for fp32.  Full-size
+configurations are checked on sampled query rows: a row's output depends only
+on its own query, so the per-row comparison is exact in what it checks.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import area_oracle as ora
+from workloads import CONFIGS
+import gpu_runner as gr
+
+pytestmark = pytest.mark.gpu
+
+BIG = ["flux2048", "flux4096", "flux6144", "qwen6144x2048"]
+ALL = ["tiny"] + BIG
+
+
+def _steps(name):
+    return list(range(len(CONFIGS[name].schedule)))
+
+
+# ---------------------------------------------------------------------------
+# DWT detail map: bit-exact
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ALL)
+def test_dwt_bitexact(name):
+    cfg = CONFIGS[name]
+    _, _, _, src = gr.host_inputs(name)
+    dsrc = gr.to_dev(src, cfg.dtype)
+    for mode, mname in [(0, "hh"), (1, "all3")]:
+        got = gr.gpu_dwt(dsrc, cfg.B, cfg.Hg, cfg.Wg, cfg.C, cfg.dtype, mode).cpu().numpy()
+        want = ora.dwt_detail(src, cfg.Hg, cfg.Wg, mname)
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32)), (name, mname)
+
+
+@pytest.mark.parametrize("C,Hg,Wg,dtype", [(3, 10, 6, "fp32"), (5, 8, 14, "bf16"),
+                                           (16, 2, 2, "bf16"), (8, 34, 18, "fp32")])
+def test_dwt_odd_channels_and_small_grids(C, Hg, Wg, dtype):
+    rng = np.random.default_rng(C * 100 + Hg)
+    src = rng.standard_normal((2, Hg * Wg, C)).astype(np.float32)
+    if dtype == "bf16":
+        src = gr.to_host(gr.to_dev(src, "bf16")).astype(np.float32)
+    got = gr.gpu_dwt(gr.to_dev(src, dtype), 2, Hg, Wg, C, dtype).cpu().numpy()
+    want = ora.dwt_detail(src, Hg, Wg, "hh")
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# Planner: bit-exact at every configuration and schedule step
+# ---------------------------------------------------------------------------
+
+def _check_items(got, want, b=0):
+    nitem = int(got["nitem"][b])
+    items = got["items"][b, :nitem]
+    expect = set()
+    for i, (y0, x0, hy, wx) in enumerate(want.windows):
+        for t in range(-(-(hy * wx) // 256)):
+            expect.add((i, t))
+    assert len(items) == len(expect) and set(map(tuple, items.tolist())) == expect
+    kept = want.split[want.parent[items[:, 0]]] == 0
+    assert not np.any(np.diff(kept.astype(int)) > 0), "unsplit windows must come first"
+
+
+@pytest.mark.parametrize("name,step", [(n, s) for n in ALL for s in _steps(n)])
+def test_plan_bitexact(name, step):
+    cfg = CONFIGS[name]
+    _, _, _, src = gr.host_inputs(name)
+    E = ora.dwt_detail(src, cfg.Hg, cfg.Wg)
+    w = cfg.schedule[step]
+    want = ora.window_plan(E[0], cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
+    energy = torch.from_numpy(E).cuda()
+    _, plan, _ = gr.gpu_plan(energy, cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
+    got = gr.parse(plan)
+    gr.compare_plan(got, want)
+    Etok = ora.token_energy(E[0]).reshape(-1)
+    assert np.array_equal(got["order"][0], ora.global_rank(Etok))
+    _check_items(got, want)
+
+
+@pytest.mark.parametrize("Hg,Wg,w,h,G,thr", [
+    (16, 16, 7, 2, 5, 0.3),      # odd window side: unequal quadrants
+    (12, 20, 64, 0, 3, 0.0),     # one window covers the grid, no halo
+    (10, 14, 4, 1, 0, 9.0),      # G = 0, everything split
+    (6, 6, 2, 3, 40, 9.0),       # halo larger than the window, G > N - |ext|
+    (34, 18, 9, 1, 7, 0.25),     # ragged tiling
+])
+def test_plan_edge_cases(Hg, Wg, w, h, G, thr):
+    rng = np.random.default_rng(Hg * Wg + w)
+    E = (rng.random((2, Hg // 2, Wg // 2)) ** 2).astype(np.float32)
+    E[:, :, : max(1, Wg // 4)] = 0.0        # ties at zero energy
+    energy = torch.from_numpy(E).cuda()
+    _, plan, _ = gr.gpu_plan(energy, 2, Hg, Wg, w, h, G, thr)
+    got = gr.parse(plan)
+    for b in range(2):
+        want = ora.window_plan(E[b], Hg, Wg, w, h, G, thr)
+        gr.compare_plan(got, want, b)
+        _check_items(got, want, b)
+
+
+# ---------------------------------------------------------------------------
+# Phase I: pooling and coarse attention
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ALL)
+def test_pool_kv(name):
+    cfg = CONFIGS[name]
+    q, k, v, _ = gr.host_inputs(name)
+    dq, dk, dv, _ = gr.dev_inputs(name)
+    heads = [0, cfg.H - 1]
+    for mode, mname in [(0, "mean"), (1, "center")]:
+        kp, vp = gr.gpu_pool(dk, dv, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, cfg.f, mode, cfg.dtype)
+        for t_dev, t_host in [(kp, k), (vp, v)]:
+            got = gr.to_host(t_dev[:, heads])
+            want = ora.pool_kv(t_host[:, heads], cfg.Hg, cfg.Wg, cfg.f, mname)
+            if cfg.dtype == "bf16":   # one bf16 rounding of the output: 2^-9 relative
+                assert np.all(np.abs(got - want) <= 2.0 ** -8 * np.abs(want) * 1.0001 + 1e-30)
+            else:
+                gr.assert_close(got, want, "fp32", f"pool {name} {mname}")
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_coarse_attn(name):
+    cfg = CONFIGS[name]
+    q, k, v, _ = gr.host_inputs(name)
+    dq, dk, dv, _ = gr.dev_inputs(name)
+    kp, vp = gr.gpu_pool(dk, dv, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, cfg.f, 0, cfg.dtype)
+    o = gr.gpu_dense(dq, kp, vp, cfg.B, cfg.H, cfg.N, cfg.Nk, cfg.D, cfg.scale, cfg.dtype)
+    heads = list(range(cfg.H)) if cfg.tiny else [0, 7, cfg.H - 1]
+    rows = np.arange(cfg.N) if cfg.tiny else gr.sample_rows(cfg.N, 384, seed=1)
+    okp = ora.pool_kv(k[:, heads], cfg.Hg, cfg.Wg, cfg.f)
+    ovp = ora.pool_kv(v[:, heads], cfg.Hg, cfg.Wg, cfg.f)
+    want = ora.coarse_attn(q[:, heads], okp, ovp, cfg.scale, rows=rows)
+    got = gr.to_host(o[:, heads][:, :, torch.from_numpy(rows).cuda()])
+    gr.assert_close(got, want, cfg.dtype, f"coarse {name}")
+
+
+# ---------------------------------------------------------------------------
+# Full attention (speedup denominator)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["tiny", "flux2048", "qwen6144x2048"])
+def test_full_attn(name):
+    cfg = CONFIGS[name]
+    q, k, v, _ = gr.host_inputs(name)
+    dq, dk, dv, _ = gr.dev_inputs(name)
+    o = torch.empty_like(dq)
+    gr.area.area_full_attn(dq, dk, dv, o, cfg.B, cfg.H, cfg.N, cfg.D, cfg.scale,
+                           gr.area_dtype(cfg.dtype))
+    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H - 1]
+    rows = np.arange(cfg.N) if cfg.tiny else gr.sample_rows(cfg.N, 128, seed=2)
+    want = ora.full_attn(q[:, heads], k[:, heads], v[:, heads], cfg.scale, rows=rows)
+    got = gr.to_host(o[:, heads][:, :, torch.from_numpy(rows).cuda()])
+    gr.assert_close(got, want, cfg.dtype, f"full {name}")
+
+
+@pytest.mark.parametrize("B,H,N,Nk,D,dtype", [
+    (1, 1, 1, 1, 128, "bf16"),          # degenerate single query / key
+    (2, 3, 1000, 300, 128, "bf16"),     # ragged query and key tails
+    (1, 2, 257, 4097, 128, "bf16"),     # key count one past a tile
+    (1, 2, 300, 200, 64, "bf16"),       # head_dim 64 (CUDA-core path)
+    (2, 2, 333, 129, 64, "fp32"),
+    (1, 2, 130, 70, 128, "fp32"),
+])
+def test_dense_attn_ragged(B, H, N, Nk, D, dtype):
+    rng = np.random.default_rng(N + Nk)
+    q = rng.standard_normal((B, H, N, D)).astype(np.float32)
+    k = rng.standard_normal((B, H, Nk, D)).astype(np.float32)
+    v = rng.standard_normal((B, H, Nk, D)).astype(np.float32)
+    dq, dk, dv = gr.to_dev(q, dtype), gr.to_dev(k, dtype), gr.to_dev(v, dtype)
+    q, k, v = gr.to_host(dq), gr.to_host(dk), gr.to_host(dv)    # storage-exact values
+    scale = 1.0 / np.sqrt(D)
+    o = gr.gpu_dense(dq, dk, dv, B, H, N, Nk, D, scale, dtype)
+    gr.assert_close(gr.to_host(o), ora.coarse_attn(q, k, v, scale), dtype, "dense ragged")
+
+
+# ---------------------------------------------------------------------------
+# Phase II: windowed attention with centre-weighted merge
+# ---------------------------------------------------------------------------
+
+def _window_case(name, step, n_rows, heads):
+    cfg = CONFIGS[name]
+    q, k, v, src = gr.host_inputs(name)
+    dq, dk, dv, dsrc = gr.dev_inputs(name)
+    w = cfg.schedule[step]
+    energy = gr.gpu_dwt(dsrc, cfg.B, cfg.Hg, cfg.Wg, cfg.C, cfg.dtype)
+    pcfg, plan, nbytes = gr.gpu_plan(energy, cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G,
+                                     cfg.split_thr)
+    o = gr.gpu_window(dq, dk, dv, pcfg, plan, nbytes, cfg.H, cfg.D, cfg.scale, cfg.dtype)
+    E = ora.dwt_detail(src, cfg.Hg, cfg.Wg)
+    oplan = ora.window_plan(E[0], cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
+    gr.compare_plan(gr.parse(plan), oplan)
+    rows = np.arange(cfg.N) if n_rows is None else gr.sample_rows(cfg.N, n_rows, seed=3 + step)
+    want = ora.window_attn(q, k, v, [oplan], cfg.scale, rows=rows, heads=heads)
+    got = gr.to_host(o[:, heads][:, :, torch.from_numpy(rows).cuda()])
+    gr.assert_close(got, want, cfg.dtype, f"window {name} step {step} w={w}")
+
+
+def test_window_attn_tiny():
+    _window_case("tiny", 0, None, [0, 1])
+
+
+@pytest.mark.parametrize("name,step", [(n, s) for n in BIG for s in _steps(n)])
+def test_window_attn_big(name, step):
+    _window_case(name, step, 256, [0, CONFIGS[name].H - 1])
+
+
+@pytest.mark.parametrize("Hg,Wg,w,h,G,D,dtype,H", [
+    (16, 16, 7, 2, 5, 128, "bf16", 2),     # unequal quadrants, ragged query tiles
+    (12, 20, 64, 0, 3, 128, "bf16", 1),    # one window = full attention
+    (10, 14, 4, 1, 0, 128, "bf16", 2),     # no global KV
+    (24, 40, 12, 3, 17, 64, "bf16", 2),    # head_dim 64
+    (20, 12, 6, 1, 9, 128, "fp32", 2),     # fp32 head_dim 128
+    (64, 48, 24, 4, 130, 128, "bf16", 3),  # global list spans two key tiles
+])
+def test_window_attn_edge_cases(Hg, Wg, w, h, G, D, dtype, H):
+    rng = np.random.default_rng(Hg * 31 + Wg)
+    B = 2
+    N = Hg * Wg
+    q = rng.standard_normal((B, H, N, D)).astype(np.float32)
+    k = rng.standard_normal((B, H, N, D)).astype(np.float32)
+    v = rng.standard_normal((B, H, N, D)).astype(np.float32)
+    dq, dk, dv = gr.to_dev(q, dtype), gr.to_dev(k, dtype), gr.to_dev(v, dtype)
+    q, k, v = gr.to_host(dq), gr.to_host(dk), gr.to_host(dv)
+    E = (rng.random((B, Hg // 2, Wg // 2)) ** 3).astype(np.float32)
+    thr = float(np.median(E))
+    pcfg, plan, nbytes = gr.gpu_plan(torch.from_numpy(E).cuda(), B, Hg, Wg, w, h, G, thr)
+    scale = 1.0 / np.sqrt(D)
+    o = gr.gpu_window(dq, dk, dv, pcfg, plan, nbytes, H, D, scale, dtype)
+    plans = [ora.window_plan(E[b], Hg, Wg, w, h, G, thr) for b in range(B)]
+    for b in range(B):
+        want = ora.window_attn(q[b:b + 1], k[b:b + 1], v[b:b + 1], [plans[b]], scale)
+        gr.assert_close(gr.to_host(o[b:b + 1]), want, dtype, "window edge")

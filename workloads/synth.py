@@ -33,9 +33,12 @@ TEX_BLOCK = 16
 def round_to_bf16(x: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bf16 (ties to even), kept as float32."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32).reshape(x.shape)
+    u = x.view(np.uint32)
+    r = (u >> 16) & np.uint32(1)          # finite inputs: no uint32 overflow
+    r += np.uint32(0x7FFF)
+    r += u
+    r &= np.uint32(0xFFFF0000)
+    return r.view(np.float32).reshape(x.shape)
 
 
 def _interp_matrix(n_out: int, n_in: int) -> np.ndarray:
@@ -75,11 +78,11 @@ def _field(cfg: AreaConfig, seed: int, lead: int, ch: int) -> np.ndarray:
     g = cfg.field_grid
     grid = rng.standard_normal((lead, g, g, ch)).astype(np.float64)
     ry = _interp_matrix(cfg.Hg, g)
-    rx = _interp_matrix(cfg.Wg, g)
+    rx = _interp_matrix(cfg.Wg, g).astype(np.float32)
     out = np.empty((lead, cfg.Hg, cfg.Wg, ch), dtype=np.float32)
     for i in range(lead):
-        t = np.tensordot(ry, grid[i], axes=([1], [0]))          # [Hg, g, ch]
-        out[i] = np.einsum("xj,yjc->yxc", rx, t, optimize=True)
+        t = np.tensordot(ry, grid[i], axes=([1], [0])).astype(np.float32)   # [Hg, g, ch]
+        out[i] = np.matmul(rx[None, :, :], t)                                # [Hg, Wg, ch]
     mask = texture_mask(cfg)
     idx = np.flatnonzero(mask.reshape(-1))
     flat = out.reshape(lead, cfg.N, ch)
@@ -88,8 +91,15 @@ def _field(cfg: AreaConfig, seed: int, lead: int, ch: int) -> np.ndarray:
         return out
     if idx.size:
         flat[:, idx, :] += rng.standard_normal((lead, idx.size, ch), dtype=np.float32)
-    mean = float(np.mean(out, dtype=np.float64))
-    std = float(np.sqrt(np.mean(np.square(out, dtype=np.float64)) - mean * mean))
+    flat_all = out.reshape(-1)
+    s1 = s2 = 0.0
+    step = 1 << 24
+    for c0 in range(0, flat_all.size, step):
+        chunk = flat_all[c0:c0 + step].astype(np.float64)
+        s1 += float(chunk.sum())
+        s2 += float(np.dot(chunk, chunk))
+    mean = s1 / flat_all.size
+    std = float(np.sqrt(s2 / flat_all.size - mean * mean))
     out -= np.float32(mean)
     out *= np.float32(1.0 / std)
     if cfg.dtype == "bf16":
