@@ -1,0 +1,559 @@
+#!/usr/bin/env python
+"""Benchmark of the AReA attention hot path on B200 (libarea, sm_100a).
+
+One step = one AReA attention schedule on one synthetic FLUX.1-shaped
+6144x6144 image (384x384 tokens, 24 heads, head_dim 128, bf16):
+  8 Phase I calls   (area_pool_kv + area_coarse_attn, f = 6 -> 64x64 keys), and
+  8 Phase II calls  (area_dwt_detail + area_window_plan + area_window_attn, one
+                     per window side of the schedule 192 -> 64).
+The metric is algorithmic attention TFLOP/s: 4*D*H*(query, key) pairs the
+method defines (N*Nk per Phase I call; sum over windows of |W|*(|ext|+G_W)
+per Phase II call) divided by the step time.  Full attention over the same
+inputs is timed after the step to give the speedup ratio.
+
+Launch: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl area|reference]
+For N > 1 use torchrun; every rank runs an independent replica (the path has
+no exchange step), and the job value is the sum of the ranks' work over the
+slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "AReA attention TFLOP/s per schedule step (bf16, 1 B200)"
+DEFAULT_CONFIG = "flux6144"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work (host arithmetic on plan sizes; no kernel logic here)
+# ---------------------------------------------------------------------------
+
+def phase1_flops(cfg) -> float:
+    return 4.0 * cfg.B * cfg.H * cfg.N * cfg.Nk * cfg.D
+
+
+def full_flops(cfg) -> float:
+    return 4.0 * cfg.B * cfg.H * cfg.N * cfg.N * cfg.D
+
+
+def window_flops(plan: dict, H: int, D: int) -> float:
+    """4*D*H*sum_W |W|*(|ext W| + G_W) from a decoded device plan."""
+    tot = 0.0
+    for b in range(plan["B"]):
+        nw = int(plan["nwin"][b])
+        win = plan["win"][b, :nw].astype(np.float64)
+        ext = plan["ext"][b, :nw].astype(np.float64)
+        g = plan["gcount"][b, :nw].astype(np.float64)
+        tot += float(np.sum(win[:, 2] * win[:, 3] * (ext[:, 2] * ext[:, 3] + g)))
+    return 4.0 * D * H * tot
+
+
+def pool_bytes(cfg) -> float:
+    e = 2 if cfg.dtype == "bf16" else 4
+    return 2.0 * cfg.B * cfg.H * (cfg.N + cfg.Nk) * cfg.D * e
+
+
+def dwt_bytes(cfg) -> float:
+    e = 2 if cfg.dtype == "bf16" else 4
+    return cfg.B * cfg.N * cfg.C * e + cfg.B * (cfg.N // 4) * 4
+
+
+def plan_launches(B: int) -> int:
+    # header, base scores, windows, (sort init + 4 x (hist, scan, scatter)) per
+    # batch element, global-KV selection, weight sums
+    return 5 + 13 * B
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas; no data-path collective)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world: int, backend: str):
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+    return dist
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None:
+            dist.barrier(device_ids=[device])
+        else:
+            dist.barrier()
+
+
+def reduce_max(dist, value: float, device: str = "cpu") -> float:
+    """Max of a float over ranks (identity without a process group)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(dist, value: float, device: str = "cpu") -> float:
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self) -> dict:
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons)}
+        loaded = [x for x in sm if x > 0.5 * (smax or max(sm))] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the GPU workload
+# ---------------------------------------------------------------------------
+
+class AreaStep:
+    """Device buffers and the call sequence of one schedule step."""
+
+    def __init__(self, cfg, q, k, v, src, stream):
+        import torch
+
+        import step_adaptive_sparse_b200 as area
+        self.area, self.torch, self.cfg, self.stream = area, torch, cfg, stream
+        self.q, self.k, self.v, self.src = q, k, v, src
+        dev = q.device
+        self.dt = area.AREA_DTYPE_BF16 if cfg.dtype == "bf16" else area.AREA_DTYPE_F32
+        self.kp = torch.empty((cfg.B, cfg.H, cfg.Nk, cfg.D), dtype=q.dtype, device=dev)
+        self.vp = torch.empty_like(self.kp)
+        self.o1 = torch.empty_like(q)
+        self.o2 = torch.empty_like(q)
+        self.energy = torch.empty((cfg.B, cfg.Hg // 2, cfg.Wg // 2), dtype=torch.float32,
+                                  device=dev)
+        self.pcfg, self.plan, self.plan_bytes = [], [], []
+        wsb = 0
+        for w in cfg.schedule:
+            pc = area.make_cfg(cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
+            nb = area.area_window_plan_bytes(pc)
+            self.pcfg.append(pc)
+            self.plan.append(torch.empty(nb, dtype=torch.uint8, device=dev))
+            self.plan_bytes.append(nb)
+            wsb = max(wsb, area.area_window_attn_ws_bytes(pc, cfg.H, cfg.D))
+        self.ws = torch.empty(wsb // 4, dtype=torch.float32, device=dev)
+        self.ws_bytes = wsb
+        self.n_phase1 = len(cfg.schedule)
+        self.launches = (self.n_phase1 * 2 +
+                         len(cfg.schedule) * (1 + plan_launches(cfg.B) + 3))
+        self.calls = {"pool_kv": [], "coarse_attn": [], "dwt_detail": [], "window_plan": [],
+                      "window_attn": []}
+        self.record = False
+
+    def _ev(self):
+        return self.torch.cuda.Event(enable_timing=True)
+
+    def _timed(self, name, fn):
+        if not self.record:
+            fn()
+            return
+        a, b = self._ev(), self._ev()
+        a.record(self.stream)
+        fn()
+        b.record(self.stream)
+        self.calls[name].append((a, b))
+
+    def run(self):
+        area, cfg, s = self.area, self.cfg, self.stream
+        for _ in range(self.n_phase1):
+            self._timed("pool_kv", lambda: area.area_pool_kv(
+                self.k, self.v, self.kp, self.vp, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, cfg.f,
+                area.AREA_POOL_MEAN, self.dt, s))
+            self._timed("coarse_attn", lambda: area.area_coarse_attn(
+                self.q, self.kp, self.vp, self.o1, cfg.B, cfg.H, cfg.N, cfg.Nk, cfg.D, cfg.scale,
+                self.dt, s))
+        for i in range(len(cfg.schedule)):
+            self._timed("dwt_detail", lambda: area.area_dwt_detail(
+                self.src, self.dt, cfg.C, self.energy, cfg.B, cfg.Hg, cfg.Wg,
+                area.AREA_DETAIL_HH, s))
+            self._timed("window_plan", lambda: area.area_window_plan(
+                self.energy, self.pcfg[i], self.plan[i], self.plan_bytes[i], s))
+            self._timed("window_attn", lambda: area.area_window_attn(
+                self.q, self.k, self.v, self.pcfg[i], self.plan[i], self.plan_bytes[i],
+                self.o2, self.ws, self.ws_bytes, cfg.H, cfg.D, cfg.scale, self.dt, s))
+
+    def window_flops_per_step(self):
+        tot, per = 0.0, []
+        for p in self.plan:
+            d = self.area.parse_plan(p.cpu().numpy())
+            f = window_flops(d, self.cfg.H, self.cfg.D)
+            per.append(f)
+            tot += f
+        return tot, per
+
+    def split_fractions(self):
+        out = []
+        for p in self.plan:
+            d = self.area.parse_plan(p.cpu().numpy())
+            out.append(round(float(d["split"][0].mean()), 3))
+        return out
+
+
+def call_ms(pairs):
+    return [a.elapsed_time(b) for a, b in pairs]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return {"hbm_gbs": p.get("hbm_gbs"), "bf16_tflops": p.get("bf16_tflops"),
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def load_traffic():
+    """dram bytes per launch of the dominant kernel from a committed ncu summary."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            return json.load(fh)
+    return {}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle on a bounded sample of the same workload
+# ---------------------------------------------------------------------------
+
+def oracle_sample(cfg, q, k, v, src, budget_s: float = 15.0, rows_per_call: int = 64):
+    """Time the oracle on a sample of the step: all of the DWT map and one
+    plan per schedule step, and attention for one head on `rows_per_call`
+    query rows per call.  Returns (TFLOP/s of the sampled attention work,
+    seconds, description, threads)."""
+    from oracle import area_oracle as ora
+    t0 = time.perf_counter()
+    flops = 0.0
+    h = 0
+    rng = np.random.default_rng(0)
+    E = ora.dwt_detail(src, cfg.Hg, cfg.Wg)
+    kp = ora.pool_kv(k[:, h:h + 1], cfg.Hg, cfg.Wg, cfg.f)
+    vp = ora.pool_kv(v[:, h:h + 1], cfg.Hg, cfg.Wg, cfg.f)
+    rows = np.sort(rng.choice(cfg.N, size=rows_per_call, replace=False))
+    ora.coarse_attn(q[:, h:h + 1], kp, vp, cfg.scale, rows=rows)
+    flops += 4.0 * rows.size * cfg.Nk * cfg.D
+    done_steps = 0
+    for w in cfg.schedule:
+        if time.perf_counter() - t0 > budget_s:
+            break
+        plan = ora.window_plan(E[0], cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
+        rows = np.sort(rng.choice(cfg.N, size=rows_per_call, replace=False))
+        ora.window_attn(q, k, v, [plan], cfg.scale, rows=rows, heads=[h])
+        # pairs computed: every window containing a sampled row
+        for i, (y0, x0, hy, wx) in enumerate(plan.windows):
+            ry, rx = rows // cfg.Wg, rows % cfg.Wg
+            inside = np.sum((ry >= y0) & (ry < y0 + hy) & (rx >= x0) & (rx < x0 + wx))
+            e = plan.ext[i]
+            flops += 4.0 * cfg.D * inside * (e[2] * e[3] + plan.gcount[i])
+        done_steps += 1
+    sec = time.perf_counter() - t0
+    try:
+        threads = len(os.sched_getaffinity(0))
+    except AttributeError:
+        threads = os.cpu_count()
+    desc = (f"oracle (NumPy fp64 attention, fp32 exact-order DWT/plan) on {cfg.name}: full "
+            f"Haar map, 1 head x {rows_per_call} query rows of one Phase I call, and the plan "
+            f"plus 1 head x {rows_per_call} rows of window attention for {done_steps} of "
+            f"{len(cfg.schedule)} Phase II steps; TFLOP/s = sampled attention pairs x 4D / time")
+    return flops / sec / 1e12, sec, desc, threads
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from workloads import CONFIGS, make_detail_source, make_qkv
+    cfg = CONFIGS[args.config]
+    q, k, v = make_qkv(cfg)
+    src = make_detail_source(cfg)
+    for _ in range(args.warmup):
+        oracle_sample(cfg, q, k, v, src, budget_s=args.ref_budget / 4, rows_per_call=16)
+    vals, secs = [], []
+    desc, threads = "", 0
+    for _ in range(args.steps):
+        val, sec, desc, threads = oracle_sample(cfg, q, k, v, src, budget_s=args.ref_budget,
+                                                rows_per_call=32)
+        vals.append(val)
+        secs.append(sec)
+    value = float(np.median(vals))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * float(np.median(secs)), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "grid": [cfg.Hg, cfg.Wg], "heads": cfg.H,
+                       "head_dim": cfg.D, "batch": cfg.B, "parallelism": "replicas"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_area(args):
+    import torch
+
+    import step_adaptive_sparse_b200 as area
+    from workloads import CONFIGS, make_detail_source, make_qkv
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (libarea has no CPU path)")
+    torch.cuda.set_device(local)
+    dist = init_dist(world, "nccl")
+    dev = torch.device("cuda", local)
+    cfg = CONFIGS[args.config]
+    qh, kh, vh = make_qkv(cfg)
+    srch = make_detail_source(cfg)
+    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    # pinned host copies for the end-to-end leg
+    pin = [torch.from_numpy(x).to(tdt).pin_memory() for x in (qh, kh, vh, srch)]
+    q, k, v, src = (p.to(dev, non_blocking=False) for p in pin)
+    stream = torch.cuda.Stream(device=dev)
+    st = AreaStep(cfg, q, k, v, src, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            st.run()
+    torch.cuda.synchronize()
+    kerr = area.area_kernel_error()
+    if kerr:
+        raise SystemExit("bench.py: a tensor-core kernel gave up a bounded wait in warm-up")
+    win_flops, win_per_step = st.window_flops_per_step()
+    splits = st.split_fractions()
+    step_flops = phase1_flops(cfg) * st.n_phase1 + win_flops
+
+    # ---- timed region (device time, CUDA events on the launching stream)
+    st.record = True
+    barrier(dist, local)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        time.sleep(0.3)
+        ev0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                st.run()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(dist, local)
+    st.record = False
+    ms_local = ev0.elapsed_time(ev1)
+    ms_total = reduce_max(dist, ms_local, device=str(dev))
+    ms_step = ms_total / args.steps
+    flops_all = reduce_sum(dist, step_flops * args.steps, device=str(dev))
+    value = flops_all / (ms_total * 1e-3) / 1e12
+
+    per = {n: call_ms(p) for n, p in st.calls.items()}
+    med = {n: (float(np.median(x)) if x else None) for n, x in per.items()}
+    win_ms_steps = np.array(per["window_attn"]).reshape(args.steps, -1).mean(axis=0).tolist()
+    kerr = area.area_kernel_error()
+
+    # ---- full attention: the speedup denominator (same inputs)
+    o_full = torch.empty_like(q)
+    fe0, fe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        area.area_full_attn(q, k, v, o_full, cfg.B, cfg.H, cfg.N, cfg.D, cfg.scale, st.dt, stream)
+        fe0.record(stream)
+        for _ in range(args.full_reps):
+            area.area_full_attn(q, k, v, o_full, cfg.B, cfg.H, cfg.N, cfg.D, cfg.scale, st.dt,
+                                stream)
+        fe1.record(stream)
+    torch.cuda.synchronize()
+    full_ms = fe0.elapsed_time(fe1) / args.full_reps
+    del o_full
+
+    # ---- end to end through the C-ABI from pinned host buffers
+    out_h = torch.empty(q.shape, dtype=tdt).pin_memory()
+    h2d = sum(p.numel() * p.element_size() for p in pin)
+    d2h = out_h.numel() * out_h.element_size()
+    barrier(dist, local)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            for dst_t, src_t in zip((q, k, v, src), pin):
+                dst_t.copy_(src_t, non_blocking=True)
+            st.run()
+            out_h.copy_(st.o2, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(dist, e0.elapsed_time(e1), device=str(dev))
+    e2e_val = flops_all / (e2e_ms * 1e-3) / 1e12
+
+    # ---- roofline of the dominant kernel
+    peaks = load_peaks()
+    traffic = load_traffic()
+    n1 = st.n_phase1
+    coarse_ms = med["coarse_attn"]
+    t_coarse = coarse_ms * n1
+    t_window = float(np.sum(win_ms_steps))
+    if t_window >= t_coarse:
+        dom, dom_flops, dom_ms, dom_launches = ("window_attn", win_flops / len(cfg.schedule),
+                                                t_window / len(cfg.schedule), "3 launches")
+    else:
+        dom, dom_flops, dom_ms, dom_launches = ("coarse_attn", phase1_flops(cfg), coarse_ms,
+                                                "1 launch")
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": traffic.get(dom),
+            "kernel": dom, "per_call": dom_launches,
+            "peak_kind": f"bf16 dense, {peaks['source']} sustained",
+            "frac_of_burst_peak": achieved / peaks["bf16_tflops"]}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, sec, desc, threads = oracle_sample(cfg, qh, kh, vh, srch, budget_s=args.ref_budget)
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": desc, "seconds": sec}
+
+    clk = clocks.summary()
+    if rank == 0:
+        pool_ms, dwt_ms = med["pool_kv"], med["dwt_detail"]
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if cfg.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": cfg.name, "grid": [cfg.Hg, cfg.Wg], "tokens": cfg.N,
+                       "heads": cfg.H, "head_dim": cfg.D, "batch": cfg.B, "pool_f": cfg.f,
+                       "schedule": list(cfg.schedule), "halo": cfg.halo, "G": cfg.G,
+                       "split_thr": cfg.split_thr, "phase1_calls": n1,
+                       "phase2_calls": len(cfg.schedule),
+                       "l2": "inputs larger than L2 (0.9 GB per Q/K/V tensor)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps},
+            "gpu_launches": st.launches * args.steps,
+            "clocks": clk,
+            "kernel_error": kerr,
+            "per_call_ms": {
+                "pool_kv": pool_ms, "coarse_attn": coarse_ms, "dwt_detail": dwt_ms,
+                "window_plan": med["window_plan"], "window_attn_by_step": win_ms_steps,
+                "full_attn": full_ms},
+            "per_call_tflops": {
+                "coarse_attn": phase1_flops(cfg) / (coarse_ms * 1e-3) / 1e12,
+                "window_attn_by_step": [f / (t * 1e-3) / 1e12 for f, t in
+                                        zip(win_per_step, win_ms_steps)],
+                "full_attn": full_flops(cfg) / (full_ms * 1e-3) / 1e12},
+            "per_call_gbs": {"pool_kv": pool_bytes(cfg) / (pool_ms * 1e-3) / 1e9,
+                             "dwt_detail": dwt_bytes(cfg) / (dwt_ms * 1e-3) / 1e9,
+                             "hbm_peak_gbs": peaks["hbm_gbs"]},
+            "split_fraction_by_step": splits,
+            "speedup_vs_full_attention": (full_ms * (n1 + len(cfg.schedule))) / ms_step,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["area", "reference"], default="area")
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--full-reps", type=int, default=2)
+    ap.add_argument("--ref-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_area(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

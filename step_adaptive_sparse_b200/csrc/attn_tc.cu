@@ -18,9 +18,10 @@
 //               thread owns one query row (one TMEM lane).
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.  P (bf16)
 // overwrites the first 64 columns of its S tile and feeds the PV MMA straight
-// from TMEM.  Online softmax rescales O in TMEM only when the running row
-// maximum grows by more than 2^8 (the final normalisation uses the same stale
-// maximum in numerator and denominator, so the result is exact).
+// from TMEM.  Online softmax rescales O in TMEM only when some row of a warp
+// sees its running maximum grow by more than 2^8 (the final normalisation uses
+// the same stale maximum in numerator and denominator, so the result is exact).
+// Every branch around a .sync.aligned tcgen05 instruction is warp-uniform.
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the kernel
 // records an error code, stops issuing work and still releases its TMEM.
 #include <cuda.h>
@@ -114,6 +115,20 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* ab
     }
   }
   return true;
+}
+
+// Lane 0 waits; the outcome is broadcast so the warp stays converged.
+__device__ __forceinline__ bool warp_wait0(uint32_t bar, uint32_t parity, int* abort_flag) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Every lane waits (each acquires the barrier); the warp proceeds only if all
+// lanes saw the phase complete, so `.sync.aligned` TMEM accesses stay converged.
+__device__ __forceinline__ bool warp_wait_all(uint32_t bar, uint32_t parity, int* abort_flag) {
+  const bool ok = mbar_wait(bar, parity, abort_flag);
+  return __all_sync(0xffffffffu, ok) != 0;
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
@@ -375,7 +390,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     for (int u = blockIdx.x; u < prm.num_units; u += gridDim.x) {
       const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H);
       if (!x.valid) continue;
-      if (!mbar_wait(bar(BAR_Q_EMPTY), (unit_count & 1u) ^ 1u, abort_flag)) break;
+      if (!warp_wait0(bar(BAR_Q_EMPTY), (unit_count & 1u) ^ 1u, abort_flag)) break;
       if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL), 2 * kTileBytes);
       __syncwarp();
       if constexpr (!WINDOW) {
@@ -401,7 +416,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       for (int j = 0; j < nt && ok; ++j) {
         for (int kv = 0; kv < 2; ++kv) {       // K then V
           const int s = (int)(kv_it % kStages);
-          if (!mbar_wait(bar(BAR_KV_EMPTY + s), ((kv_it / kStages) & 1u) ^ 1u, abort_flag)) {
+          if (!warp_wait0(bar(BAR_KV_EMPTY + s), ((kv_it / kStages) & 1u) ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
@@ -433,7 +448,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     int drain_abort = 0;
     for (uint32_t k = 0; k < kStages && k < kv_it; ++k) {
       const uint32_t it = kv_it - 1 - k;
-      mbar_wait(bar(BAR_KV_FULL + it % kStages), (it / kStages) & 1u, &drain_abort);
+      warp_wait0(bar(BAR_KV_FULL + it % kStages), (it / kStages) & 1u, &drain_abort);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -534,7 +549,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const int nt = (x.nkv + 127) / 128;
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < nt; ++j) {
-        if (!(ok = mbar_wait(bS, s_cnt & 1u, abort_flag))) break;
+        if (!(ok = warp_wait_all(bS, s_cnt & 1u, abort_flag))) break;
         ++s_cnt;
         tc_fence_after();
         const int valid = min(128, x.nkv - j * 128);
@@ -548,10 +563,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           for (int i = 0; i < 32; ++i)
             if (c * 32 + i < valid) mx = fmaxf(mx, __uint_as_float(sr[i]));
         }
-        const float mnew = mx * sl2;
+        const float mnew = fmaxf(mx * sl2, m);
         if (j == 0) {
           m = mnew;
-        } else if (mnew > m + kRescaleThreshold) {
+        } else if (__any_sync(0xffffffffu, mnew > m + kRescaleThreshold)) {
+          // The decision is warp-uniform: the TMEM accesses below are
+          // .sync.aligned and must be executed by the whole warp.  Each lane
+          // rescales its own row by its own factor (1 when its max is unchanged).
           const float alpha = fast_exp2(m - mnew);
           l *= alpha;
 #pragma unroll 1
@@ -588,7 +606,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
       if (!ok) break;
       // epilogue
-      if (!(ok = mbar_wait(bO, o_cnt & 1u, abort_flag))) break;
+      if (!(ok = warp_wait_all(bO, o_cnt & 1u, abort_flag))) break;
       ++o_cnt;
       tc_fence_after();
       const int qpos = x.q0 + qt * 128 + row;

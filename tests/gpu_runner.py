@@ -32,18 +32,30 @@ def to_host(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy().astype(np.float64)
 
 
+@functools.lru_cache(maxsize=8)
+def host_src(name: str) -> np.ndarray:
+    return make_detail_source(CONFIGS[name])
+
+
 @functools.lru_cache(maxsize=1)
-def host_inputs(name: str):
-    cfg = CONFIGS[name]
-    q, k, v = make_qkv(cfg)
-    return q, k, v, make_detail_source(cfg)
+def host_qkv(name: str):
+    return make_qkv(CONFIGS[name])
 
 
-def dev_inputs(name: str):
-    cfg = CONFIGS[name]
-    q, k, v, src = host_inputs(name)
-    return (to_dev(q, cfg.dtype), to_dev(k, cfg.dtype), to_dev(v, cfg.dtype),
-            to_dev(src, cfg.dtype))
+class ConfigData:
+    """Host (storage-exact float32) and device copies of one config's inputs."""
+
+    def __init__(self, name: str):
+        cfg = CONFIGS[name]
+        self.name, self.cfg = name, cfg
+        self.q, self.k, self.v = host_qkv(name)
+        self.src = host_src(name)
+        self.dq, self.dk, self.dv = (to_dev(x, cfg.dtype) for x in (self.q, self.k, self.v))
+        self.dsrc = to_dev(self.src, cfg.dtype)
+
+    def release(self):
+        del self.dq, self.dk, self.dv, self.dsrc
+        torch.cuda.empty_cache()
 
 
 def assert_close(got: np.ndarray, want: np.ndarray, dtype: str, what: str = ""):

@@ -1,0 +1,97 @@
+"""Host logic of bench.py: work accounting and the multi-rank aggregation.
+
+The replica path has no data-path collective; the only cross-rank steps are
+the max over ranks of the device time and the sum of the work.  They are
+checked here with world-size-2 gloo process groups on the CPU.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+from oracle import area_oracle as ora
+from workloads import CONFIGS
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import datetime
+
+    import torch.distributed as dist
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        ms = [120.5, 97.25][rank]
+        work = [3.0e12, 5.0e12][rank]
+        mx = bench.reduce_max(dist, ms)
+        tot = bench.reduce_sum(dist, work)
+        bench.barrier(dist)
+        out[rank] = (mx, tot)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_reduce_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    for r in range(2):
+        mx, tot = out[r]
+        assert mx == 120.5 and tot == 8.0e12
+
+
+def test_reduce_identity_without_process_group():
+    assert bench.reduce_max(None, 3.5) == 3.5
+    assert bench.reduce_sum(None, 2.0) == 2.0
+
+
+def test_dist_env_defaults(monkeypatch):
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    assert bench.dist_env() == (0, 1, 0)
+    monkeypatch.setenv("WORLD_SIZE", "4")
+    monkeypatch.setenv("RANK", "2")
+    monkeypatch.setenv("LOCAL_RANK", "2")
+    assert bench.dist_env() == (2, 4, 2)
+
+
+def test_phase_flop_counts_match_closed_forms():
+    cfg = CONFIGS["flux4096"]
+    assert bench.phase1_flops(cfg) == 4.0 * 24 * 65536 * 4096 * 128      # 3.30 TFLOP
+    assert abs(bench.phase1_flops(cfg) / 1e12 - 3.298) < 1e-3
+    assert abs(bench.full_flops(CONFIGS["flux6144"]) / 1e12 - 267.2) < 0.1
+    # Phase I is 1/f^2 of full attention
+    assert bench.phase1_flops(cfg) * cfg.f ** 2 == bench.full_flops(cfg)
+
+
+def test_window_flops_from_plan_dict():
+    rng = np.random.default_rng(0)
+    E = rng.random((8, 8)).astype(np.float32)
+    plan = ora.window_plan(E, 16, 16, 6, 1, 5, 0.4)
+    d = {"B": 1, "nwin": np.array([plan.windows.shape[0]]), "win": plan.windows[None],
+         "ext": plan.ext[None], "gcount": plan.gcount[None]}
+    want = 0
+    for i, (y0, x0, hy, wx) in enumerate(plan.windows):
+        want += hy * wx * (len(ora.window_kv_tokens(plan, i)))
+    assert bench.window_flops(d, H=3, D=128) == 4.0 * 128 * 3 * want
+
+
+def test_plan_launch_count():
+    assert bench.plan_launches(1) == 18
+    assert bench.plan_launches(2) == 31
