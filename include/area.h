@@ -246,6 +246,37 @@ int area_window_attn(const void* q, const void* k, const void* v,
                      int H, int D, float scale, int dtype,
                      cudaStream_t stream);
 
+/*
+ * area_window_attn_noalloc -- area_window_attn for callers that cannot
+ * allocate device memory.  The paper has no counterpart: this is a library
+ * convenience, not part of the method.
+ *
+ * Some callers cannot call cudaMalloc (or any allocating routine) at the
+ * point where they run attention: code hosted by a runtime that owns every
+ * device allocation and hands out only fixed input/output buffers, or a
+ * serving loop that must not allocate once it has started.  Such a caller
+ * still passes the inputs, the plan and the output, but not the fp32 merge
+ * workspace: it lives in a static device array of 32 MiB inside the library,
+ * which every GPU that loads libarea holds until the process exits.
+ *
+ *   Arguments: as area_window_attn, without ws / ws_bytes.
+ *   Limit: B * H * Hg * Wg * D * 4 bytes must not exceed 32 MiB
+ *          (e.g. 2 heads of a 128x128 grid at D = 128); larger sizes return
+ *          AREA_ENOSPACE before anything is launched.
+ *   Set-up: the first call on a device looks up the array's device address
+ *          (cudaGetSymbolAddress, with that device current); make that first
+ *          call outside any stream capture.  It allocates nothing.
+ *   Sharing: all calls on a device use the same array.  It keeps the last
+ *          call's contents; each call clears it before use.  Calls that
+ *          overlap on the GPU (other streams, other threads) race on it and
+ *          must be serialised by the caller.
+ * Errors: AREA_EINVAL, AREA_EUNSUPPORTED, AREA_ENOSPACE, AREA_ECUDA.
+ */
+int area_window_attn_noalloc(const void* q, const void* k, const void* v,
+                             const area_plan_cfg* cfg, const void* plan,
+                             size_t plan_bytes, void* o, int H, int D,
+                             float scale, int dtype, cudaStream_t stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

@@ -66,6 +66,8 @@ _SIGS = {
     "area_window_attn_ws_bytes": (_I, [ctypes.POINTER(area_plan_cfg), _I, _I, ctypes.POINTER(_SZ)]),
     "area_window_attn": (_I, [_P, _P, _P, ctypes.POINTER(area_plan_cfg), _P, _SZ, _P, _P, _SZ,
                               _I, _I, _F, _I, _P]),
+    "area_window_attn_noalloc": (_I, [_P, _P, _P, ctypes.POINTER(area_plan_cfg), _P, _SZ, _P,
+                                      _I, _I, _F, _I, _P]),
 }
 
 
@@ -174,6 +176,16 @@ def area_window_attn(q, k, v, cfg: area_plan_cfg, plan, plan_bytes, o, ws, ws_by
     _check(_lib().area_window_attn(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(cfg), _ptr(plan),
                                    plan_bytes, _ptr(o), _ptr(ws), ws_bytes, H, D, scale, dtype,
                                    _stream(stream)), "area_window_attn")
+
+
+def area_window_attn_noalloc(q, k, v, cfg: area_plan_cfg, plan, plan_bytes, o, H, D, scale,
+                             dtype, stream=None) -> None:
+    """area_window_attn without a workspace argument, for callers that cannot
+    allocate device memory; the workspace is a 32 MiB static array of the
+    library (see include/area.h for the limit and the sharing rules)."""
+    _check(_lib().area_window_attn_noalloc(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(cfg),
+                                           _ptr(plan), plan_bytes, _ptr(o), H, D, scale, dtype,
+                                           _stream(stream)), "area_window_attn_noalloc")
 
 
 def parse_plan(buf: np.ndarray) -> dict:
