@@ -8,14 +8,14 @@
 // Pages: ai.info "Methodology in Plain English" (Phase I, Phase II);
 // gpt-diffusion.com "Las dos fases de AReA".
 //
-// Design (one persistent CTA per SM, 384 threads):
+// Design (one persistent CTA per SM, 320 threads):
 //   warp 0      TMA producer: Q tiles once per work unit, then a ring of K and
 //               V tiles (128 keys x 128 dims, 128B-swizzled, 32 KB each).
 //               Dense rows use tiled 2-D loads; window rows (a rectangle
 //               enumerated row-major, then the global-KV list) use gather4.
 //   warp 1      TMEM allocator and the single MMA-issuing thread.
-//   warps 4-7   softmax of query tile 0, warps 8-11 of query tile 1: each
-//               thread owns one query row (one TMEM lane).
+//   warps 2-5   softmax of query tile 0, warps 6-9 of query tile 1: each
+//               thread owns one query row (TMEM lane 32*(warp mod 4) + lane).
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.  P (bf16)
 // overwrites the first 64 columns of its S tile and feeds the PV MMA straight
 // from TMEM.  Online softmax rescales O in TMEM only when some row of a warp
@@ -35,7 +35,7 @@ __device__ int g_tc_error = 0;   // set on a bounded-wait expiry; read by tests
 
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 320;
 constexpr int kStages = 4;              // K/V ring stages of 32 KB
 constexpr int kTileBytes = 128 * 128 * 2;
 constexpr int kHalfBytes = 128 * 128;   // 128 rows x 64 bf16
@@ -240,6 +240,25 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
+// 128 consecutive TMEM columns of this thread's lane, loaded and waited for
+// in one statement (one round trip per S or O tile).
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x128.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, %80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, %96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, %112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, [%128];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+      : "r"(taddr)
+      : "memory");
+}
+
+// 64 consecutive TMEM columns of this thread's lane, from r[0..63].
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[128]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64};"
+      :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -294,9 +313,11 @@ __device__ __forceinline__ Unit get_unit(int u, const DenseArgs& da, const PlanV
     x.nkv = da.Nk;
     x.win = x.ext = make_int4(0, 0, 0, 0);
   } else {
-    const int BH = P.B * H;
-    const int item = u / BH;
-    x.bh = u % BH;
+    // Head-major order: consecutive units are the query blocks of one
+    // (batch, head), windows costliest first, so the CTAs in flight share a
+    // few windows' keys and values in L2.
+    const int item = u % P.nitem_max;
+    x.bh = u / P.nitem_max;
     x.b = x.bh / H;
     if (item >= P.nitem[x.b]) {
       x.valid = false;
@@ -530,9 +551,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_wait(bar(BAR_DRAIN), 0, &drain_abort);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int qt = (warp - 4) >> 2;                  // query tile of this warpgroup
+    // Warps 2-5 own query tile 0 and warps 6-9 query tile 1.  A warp may only
+    // touch the TMEM lane quarter (warp id mod 4), and each group of four
+    // consecutive warps covers all four quarters.
+    const int qt = (warp - 2) >> 2;                  // query tile of this warpgroup
     const int row = ((warp & 3) << 5) + lane;        // TMEM lane = query row in the tile
     const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
     const uint32_t tS = tmem + lane_off + (qt ? 128u : 0u);
@@ -544,34 +568,54 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const float sl2 = prm.scale_log2;
     bool ok = true;
     for (int u = blockIdx.x; u < prm.num_units && ok; u += gridDim.x) {
-      const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H);
-      if (!x.valid) continue;
-      const int nt = (x.nkv + 127) / 128;
+      int nkv;
+      {
+        const Unit x0 = get_unit<WINDOW>(u, prm.da, prm.P, prm.H);
+        if (!x0.valid) continue;
+        nkv = x0.nkv;
+      }
+      const int nt = (nkv + 127) / 128;
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < nt; ++j) {
         if (!(ok = warp_wait_all(bS, s_cnt & 1u, abort_flag))) break;
         ++s_cnt;
         tc_fence_after();
-        const int valid = min(128, x.nkv - j * 128);
-        // pass 1: row maximum over the valid keys
-        float mx = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sr[32];
-          tmem_ld32(tS + c * 32, sr);
+        const int valid = min(128, nkv - j * 128);     // warp-uniform
+        uint32_t sr[128];
+        tmem_ld128(tS, sr);
+        if (valid < 128) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c * 32 + i < valid) mx = fmaxf(mx, __uint_as_float(sr[i]));
+          for (int i = 0; i < 128; ++i)
+            if (i >= valid) sr[i] = 0xff800000u;          // -inf: no weight
         }
+        // row maximum: four independent partial maxima, then combine
+        float pm[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) pm[t] = __uint_as_float(sr[t]);
+#pragma unroll
+        for (int i = 4; i < 128; ++i) pm[i & 3] = fmaxf(pm[i & 3], __uint_as_float(sr[i]));
+        const float mx = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
         const float mnew = fmaxf(mx * sl2, m);
-        if (j == 0) {
-          m = mnew;
-        } else if (__any_sync(0xffffffffu, mnew > m + kRescaleThreshold)) {
-          // The decision is warp-uniform: the TMEM accesses below are
-          // .sync.aligned and must be executed by the whole warp.  Each lane
-          // rescales its own row by its own factor (1 when its max is unchanged).
-          const float alpha = fast_exp2(m - mnew);
-          l *= alpha;
+        // Rescale O only when some row of the warp gained more than 2^8; the
+        // decision is warp-uniform because the TMEM accesses are .sync.aligned.
+        const bool rescale = j > 0 && __any_sync(0xffffffffu, mnew > m + kRescaleThreshold);
+        const float alpha = rescale ? fast_exp2(m - mnew) : 1.f;
+        if (j == 0 || rescale) m = mnew;
+        l *= alpha;
+        // P = exp2(S * scale * log2(e) - m) as bf16, two keys per TMEM column,
+        // written over the S columns already read
+        // packed pairs go in place into sr[0..63]: slot i/2 was already read
+        float ls[2] = {0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < 128; i += 2) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sr[i]), sl2, -m));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sr[i + 1]), sl2, -m));
+          ls[(i >> 1) & 1] += p0 + p1;
+          sr[i >> 1] = pack_bf16(p0, p1);
+        }
+        l += ls[0] + ls[1];
+        tmem_st64(tS, sr);
+        if (rescale) {
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             uint32_t orr[32];
@@ -580,32 +624,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
             tmem_st32(tO + c * 32, orr);
           }
-          m = mnew;
-        }
-        // pass 2: P = exp2(S * scale * log2(e) - m) as bf16, two keys per TMEM
-        // column, written over S columns that pass 2 has already read
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sr[32];
-          tmem_ld32(tS + c * 32, sr);
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float p0 = fast_exp2(fmaf(__uint_as_float(sr[i]), sl2, -m));
-            float p1 = fast_exp2(fmaf(__uint_as_float(sr[i + 1]), sl2, -m));
-            if (c * 32 + i >= valid) p0 = 0.f;
-            if (c * 32 + i + 1 >= valid) p1 = 0.f;
-            l += p0 + p1;
-            pk[i >> 1] = pack_bf16(p0, p1);
-          }
-          tmem_st16(tS + c * 16, pk);
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bP);
       }
       if (!ok) break;
-      // epilogue
+      // epilogue (the unit is looked up again rather than kept live in
+      // registers across the key loop)
+      const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H);
       if (!(ok = warp_wait_all(bO, o_cnt & 1u, abort_flag))) break;
       ++o_cnt;
       tc_fence_after();
@@ -655,7 +682,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc_fence_before();
     }
   }
-  // warps 2 and 3 have no role
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
