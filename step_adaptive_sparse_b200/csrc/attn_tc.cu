@@ -11,8 +11,11 @@
 // Design (one persistent CTA per SM, 320 threads):
 //   warp 0      TMA producer: Q tiles once per work unit, then a ring of K and
 //               V tiles (128 keys x 128 dims, 128B-swizzled, 32 KB each).
-//               Dense rows use tiled 2-D loads; window rows (a rectangle
-//               enumerated row-major, then the global-KV list) use gather4.
+//               Dense rows use tiled 2-D loads.  Window keys are the Halo
+//               rectangle, covered by 16x8-token patches (one 3-D tiled box
+//               each, masked at the rectangle's right and bottom edges), then
+//               the global-KV list (gather4, 4 rows per lane); window queries
+//               (the rectangle enumerated row-major) use gather4.
 //   warp 1      TMEM allocator and the single MMA-issuing thread.
 //   warps 2-5   softmax of query tile 0, warps 6-9 of query tile 1: each
 //               thread owns one query row (TMEM lane 32*(warp mod 4) + lane).
@@ -41,6 +44,10 @@ constexpr int kTileBytes = 128 * 128 * 2;
 constexpr int kHalfBytes = 128 * 128;   // 128 rows x 64 bf16
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+// Window keys: the Halo rectangle is covered by patches of kPW x kPH tokens,
+// one 128-key tile each, loaded by a 3-D tiled TMA box (tokens of one grid
+// row are contiguous).  Only the global-KV list is gathered row by row.
+constexpr int kPW = 16, kPH = 8;
 
 // Shared-memory plan (offsets from a 1024-aligned base).
 constexpr int kSmemQ = 0;                              // 2 tiles x 32 KB
@@ -137,6 +144,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
 
@@ -295,7 +311,10 @@ struct Unit {
   int b;
   int q0;          // first query position of tile 0 (tile 1 = q0 + 128)
   int nq;          // number of valid query positions from q0 (window: area)
-  int nkv;         // number of keys
+  int nkv;         // dense: number of keys; window: G_W (global-KV count)
+  int nt;          // key tiles of this unit
+  int ncx;         // window: patches per row of the Halo rectangle
+  int ntr;         // window: patch tiles of the Halo rectangle
   int4 win, ext;   // window mode
   const int* glist;
 };
@@ -311,6 +330,8 @@ __device__ __forceinline__ Unit get_unit(int u, const DenseArgs& da, const PlanV
     x.q0 = (u % da.units_per_head) * 256;
     x.nq = da.N;
     x.nkv = da.Nk;
+    x.nt = (da.Nk + 127) / 128;
+    x.ncx = x.ntr = 0;
     x.win = x.ext = make_int4(0, 0, 0, 0);
   } else {
     // Head-major order: consecutive units are the query blocks of one
@@ -329,18 +350,18 @@ __device__ __forceinline__ Unit get_unit(int u, const DenseArgs& da, const PlanV
     x.ext = P.ext[wo];
     x.q0 = it.y * 256;
     x.nq = x.win.z * x.win.w;
-    x.nkv = x.ext.z * x.ext.w + P.gcount[wo];
+    x.nkv = P.gcount[wo];
+    x.ncx = (x.ext.w + kPW - 1) / kPW;
+    x.ntr = x.ncx * ((x.ext.z + kPH - 1) / kPH);
+    x.nt = x.ntr + (x.nkv + 127) / 128;
     x.glist = P.gidx + wo * P.G;
   }
   return x;
 }
 
-// Token of the p-th key of a window unit (rectangle row-major, then global list).
-__device__ __forceinline__ int window_key_token(const Unit& x, int p, int Wg) {
-  const int ne = x.ext.z * x.ext.w;
-  if (p >= x.nkv) p = 0;
-  if (p < ne) return (x.ext.x + p / x.ext.w) * Wg + x.ext.y + p % x.ext.w;
-  return x.glist[p - ne];
+// Token of the p-th global-KV key of a window unit (clamped into the list).
+__device__ __forceinline__ int window_global_token(const Unit& x, int p) {
+  return x.glist[p < x.nkv ? p : (x.nkv > 0 ? x.nkv - 1 : 0)];
 }
 
 __device__ __forceinline__ int window_query_token(const Unit& x, int p, int Wg) {
@@ -361,7 +382,8 @@ struct TcParams {
 template <bool WINDOW>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const TcParams prm) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
+               const __grid_constant__ CUtensorMap tm_vp, const TcParams prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -432,7 +454,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         bar(BAR_Q_FULL), hf * 64, r[0], r[1], r[2], r[3]);
         }
       }
-      const int nt = (x.nkv + 127) / 128;
+      const int nt = x.nt;
       bool ok = true;
       for (int j = 0; j < nt && ok; ++j) {
         for (int kv = 0; kv < 2; ++kv) {       // K then V
@@ -450,11 +472,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               for (int hf = 0; hf < 2; ++hf)
                 tma_load_2d(dst + hf * kHalfBytes, tm, bar(BAR_KV_FULL + s), hf * 64,
                             x.bh * Nkrows + j * 128);
+          } else if (j < x.ntr) {
+            // patch (px, py) of the Halo rectangle: kPH grid rows of kPW tokens
+            if (lane == 0) {
+              const CUtensorMap* tp = kv ? &tm_vp : &tm_kp;
+              const int px = j % x.ncx, py = j / x.ncx;
+              const int cx = x.ext.y + px * kPW;
+              const int cy = x.bh * prm.P.Hg + x.ext.x + py * kPH;
+              for (int hf = 0; hf < 2; ++hf)
+                tma_load_3d(dst + hf * kHalfBytes, tp, bar(BAR_KV_FULL + s), hf * 64, cx, cy);
+            }
           } else {
+            const int g0 = (j - x.ntr) * 128 + lane * 4;
             int r[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              r[i] = x.bh * Nkrows + window_key_token(x, j * 128 + lane * 4 + i, Wg);
+            for (int i = 0; i < 4; ++i) r[i] = x.bh * Nkrows + window_global_token(x, g0 + i);
             for (int hf = 0; hf < 2; ++hf)
               tma_gather4(dst + hf * kHalfBytes + lane * 512, tm, bar(BAR_KV_FULL + s), hf * 64,
                           r[0], r[1], r[2], r[3]);
@@ -496,7 +528,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       for (int u = blockIdx.x; u < prm.num_units && ok; u += gridDim.x) {
         const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H);
         if (!x.valid) continue;
-        const int nt = (x.nkv + 127) / 128;
+        const int nt = x.nt;
         if (!(ok = mbar_wait(bar(BAR_Q_FULL), unit_count & 1u, abort_flag))) break;
         // prologue: S(0)
         const uint32_t k0 = kv_it;
@@ -568,25 +600,39 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const float sl2 = prm.scale_log2;
     bool ok = true;
     for (int u = blockIdx.x; u < prm.num_units && ok; u += gridDim.x) {
-      int nkv;
+      // key-tile geometry of this unit (the rest is looked up again for the
+      // epilogue rather than kept live in registers across the key loop)
+      int nkv, nt, ntr, ncx, ew, eh;
       {
         const Unit x0 = get_unit<WINDOW>(u, prm.da, prm.P, prm.H);
         if (!x0.valid) continue;
-        nkv = x0.nkv;
+        nkv = x0.nkv; nt = x0.nt; ntr = x0.ntr; ncx = x0.ncx;
+        ew = x0.ext.w; eh = x0.ext.z;
       }
-      const int nt = (nkv + 127) / 128;
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < nt; ++j) {
         if (!(ok = warp_wait_all(bS, s_cnt & 1u, abort_flag))) break;
         ++s_cnt;
         tc_fence_after();
-        const int valid = min(128, nkv - j * 128);     // warp-uniform
         uint32_t sr[128];
         tmem_ld128(tS, sr);
-        if (valid < 128) {
+        // Key validity (warp-uniform): dense and global-KV tiles are a prefix
+        // of `valid` keys; a rectangle patch keeps columns dx < rem_x of rows
+        // dy < rem_y (key k = dy * kPW + dx).
+        if (!WINDOW || j >= ntr) {
+          const int valid = min(128, nkv - (j - ntr) * 128);
+          if (valid < 128) {
 #pragma unroll
-          for (int i = 0; i < 128; ++i)
-            if (i >= valid) sr[i] = 0xff800000u;          // -inf: no weight
+            for (int i = 0; i < 128; ++i)
+              if (i >= valid) sr[i] = 0xff800000u;        // -inf: no weight
+          }
+        } else {
+          const int rem_x = ew - (j % ncx) * kPW, rem_y = eh - (j / ncx) * kPH;
+          if (rem_x < kPW || rem_y < kPH) {
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+              if ((i % kPW) >= rem_x || (i / kPW) >= rem_y) sr[i] = 0xff800000u;
+          }
         }
         // row maximum: four independent partial maxima, then combine
         float pm[4];
@@ -720,6 +766,21 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int64_t rows, int box_row
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 3-D bf16 map over [rows_y, Wg, 128] (token-grid rows of all (b, h), grid
+// columns, head dims) with a box of 64 dims x kPW tokens x kPH grid rows.
+cudaError_t make_map_patch(CUtensorMap* m, const void* base, int64_t rows_y, int Wg) {
+  auto enc = get_encode();
+  if (!enc) return cudaErrorNotSupported;
+  cuuint64_t dims[3] = {128, (cuuint64_t)Wg, (cuuint64_t)rows_y};
+  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)Wg * 128 * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)kPW, (cuuint32_t)kPH};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 int num_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -729,12 +790,13 @@ int num_sms() {
 
 template <bool WINDOW>
 cudaError_t launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                      const TcParams& prm, cudaStream_t s) {
+                      const CUtensorMap& mkp, const CUtensorMap& mvp, const TcParams& prm,
+                      cudaStream_t s) {
   auto fn = attn_tc_kernel<WINDOW>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int grid = prm.num_units < num_sms() ? prm.num_units : num_sms();
-  fn<<<grid > 0 ? grid : 1, kThreads, kSmemBytes, s>>>(mq, mk, mv, prm);
+  fn<<<grid > 0 ? grid : 1, kThreads, kSmemBytes, s>>>(mq, mk, mv, mkp, mvp, prm);
   return cudaGetLastError();
 }
 
@@ -762,7 +824,7 @@ cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, vo
   prm.da = DenseArgs{B, H, N, Nk, (N + 255) / 256};
   prm.num_units = B * H * prm.da.units_per_head;
   prm.o = static_cast<__nv_bfloat16*>(o);
-  return launch_tc<false>(mq, mk, mv, prm, s);
+  return launch_tc<false>(mq, mk, mv, mk, mv, prm, s);   // no patch maps in dense mode
 }
 
 cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v,
@@ -774,13 +836,16 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v,
   if ((e = make_map(&mq, q, rows, 1)) != cudaSuccess) return e;
   if ((e = make_map(&mk, k, rows, 1)) != cudaSuccess) return e;
   if ((e = make_map(&mv, v, rows, 1)) != cudaSuccess) return e;
+  CUtensorMap mkp, mvp;
+  if ((e = make_map_patch(&mkp, k, L.B * H * L.Hg, (int)L.Wg)) != cudaSuccess) return e;
+  if ((e = make_map_patch(&mvp, v, L.B * H * L.Hg, (int)L.Wg)) != cudaSuccess) return e;
   TcParams prm{};
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.H = H;
   prm.P = plan_view(L, const_cast<void*>(plan));
   prm.num_units = (int)(L.nitem_max * L.B * H);
   prm.ws = ws;
-  return launch_tc<true>(mq, mk, mv, prm, s);
+  return launch_tc<true>(mq, mk, mv, mkp, mvp, prm, s);
 }
 
 }  // namespace area
