@@ -158,7 +158,7 @@ typedef struct area_plan_cfg {
  *   header[2..8] = B, Hg, Wg, w, halo, G, nb
  *   header[9]  = nw
  *   header[10+s] = byte offset of section s (AREA_PLAN_SEC_*)
- *   header[24] = work-item capacity per element ("ni"), header[25] = N
+ *   header[25] = work-item capacity per element ("ni"), header[26] = N
  * Sections:
  *   BASE    int32 [B][nb][4]   base windows (y0, x0, hy, wx), row-major
  *   SCORE   f32   [B][nb]      sum of token energy over the base window
@@ -170,6 +170,7 @@ typedef struct area_plan_cfg {
  *   GCOUNT  int32 [B][nw]      G_W = min(G, N - |ext|)
  *   GIDX    int32 [B][nw][G]   global-KV tokens in rank order, -1 padded
  *   WSUM    f32   [B][N]       sum of tent weights over final windows
+ *   COVER   int32 [B][N]       number of final windows containing the token
  *   ORDER   int32 [B][N]       tokens by (energy desc, index asc)
  *   NITEM   int32 [B+1]        work items (window, query tile) per element,
  *                              last entry = total
@@ -177,7 +178,7 @@ typedef struct area_plan_cfg {
  *   SCRATCH                    sort and scan scratch (contents unspecified)
  */
 #define AREA_PLAN_MAGIC    0x4145524150414c4eLL  /* "AREAPLAN" */
-#define AREA_PLAN_VERSION  1
+#define AREA_PLAN_VERSION  2
 #define AREA_PLAN_SEC_BASE     0
 #define AREA_PLAN_SEC_SCORE    1
 #define AREA_PLAN_SEC_SPLIT    2
@@ -191,8 +192,9 @@ typedef struct area_plan_cfg {
 #define AREA_PLAN_SEC_ORDER    10
 #define AREA_PLAN_SEC_NITEM    11
 #define AREA_PLAN_SEC_ITEMS    12
-#define AREA_PLAN_SEC_SCRATCH  13
-#define AREA_PLAN_NSEC         14
+#define AREA_PLAN_SEC_COVER    13
+#define AREA_PLAN_SEC_SCRATCH  14
+#define AREA_PLAN_NSEC         15
 
 /*
  * area_window_plan_bytes -- size of the plan buffer for cfg (host only).
@@ -213,7 +215,8 @@ int area_window_plan_bytes(const area_plan_cfg* cfg, size_t* plan_bytes);
  *   5. global-KV bridge: the first G_W = min(G, N - |ext|) tokens by
  *      (energy desc, token index asc) that lie outside the Halo rectangle;
  *   6. per-token sum of tent weights
- *      t = min(y-y0+1, y0+hy-y) * min(x-x0+1, x0+wx-x) over final windows;
+ *      t = min(y-y0+1, y0+hy-y) * min(x-x0+1, x0+wx-x) over final windows,
+ *      and the number of final windows containing the token;
  *   7. the list of (window, 256-query block) work items, costliest first.
  *   energy : [B, Hg/2, Wg/2] fp32 from area_dwt_detail
  *   plan   : device buffer of plan_bytes >= area_window_plan_bytes(cfg)

@@ -24,7 +24,7 @@ AREA_POOL_MEAN, AREA_POOL_CENTER = 0, 1
 AREA_DETAIL_HH, AREA_DETAIL_ALL3 = 0, 1
 AREA_PLAN_MAGIC = 0x4145524150414C4E
 SECTIONS = ("BASE", "SCORE", "SPLIT", "NWIN", "WIN", "PARENT", "EXT", "GCOUNT", "GIDX",
-            "WSUM", "ORDER", "NITEM", "ITEMS", "SCRATCH")
+            "WSUM", "ORDER", "NITEM", "ITEMS", "COVER", "SCRATCH")
 
 EXPORTED = ("area_status_string", "area_last_cuda_error", "area_version", "area_kernel_error",
             "area_pool_kv",
@@ -219,6 +219,7 @@ def parse_plan(buf: np.ndarray) -> dict:
            "gcount": sec("GCOUNT", np.int32, B * nw).reshape(B, nw),
            "gidx": sec("GIDX", np.int32, B * nw * G).reshape(B, nw, G),
            "wsum": sec("WSUM", np.float32, B * N).reshape(B, N),
+           "cover": sec("COVER", np.int32, B * N).reshape(B, N),
            "order": sec("ORDER", np.int32, B * N).reshape(B, N),
            "nitem": nitem,
            "items": sec("ITEMS", np.int32, B * nitem_max * 2).reshape(B, nitem_max, 2)}

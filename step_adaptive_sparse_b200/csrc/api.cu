@@ -140,12 +140,12 @@ int area_window_attn(const void* q, const void* k, const void* v, const area_pla
   if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(plan) & 255) != 0) return AREA_EINVAL;
   if (H > 65535 || L.B > 65535) return AREA_EINVAL;
   float* w = static_cast<float*>(ws);
-  cudaError_t e = area::launch_ws_zero(w, L.B * H * L.N * D, stream);
+  cudaError_t e = area::launch_ws_zero(w, L, plan, H, D, stream);
   if (e != cudaSuccess) return fail_cuda(e);
   if (dtype == AREA_DTYPE_BF16 && D == 128)
-    e = area::launch_window_attn_tc(q, k, v, L, plan, w, H, scale, stream);
+    e = area::launch_window_attn_tc(q, k, v, L, plan, o, w, H, scale, stream);
   else
-    e = area::launch_window_attn_simt(q, k, v, L, plan, w, H, D, scale, dtype, stream);
+    e = area::launch_window_attn_simt(q, k, v, L, plan, o, w, H, D, scale, dtype, stream);
   if (e != cudaSuccess) return fail_cuda(e);
   return finish(area::launch_window_finalize(w, L, plan, o, H, D, dtype, stream));
 }

@@ -45,6 +45,7 @@ struct PlanView {
   int* gcount;         // [B][nw]
   int* gidx;           // [B][nw][G]
   float* wsum;         // [B][N]
+  int* cover;          // [B][N] number of final windows containing the token
   int* order;          // [B][N]
   int* nitem;          // [B+1]
   int2* items;         // [B][nitem_max]
@@ -84,10 +85,11 @@ cudaError_t launch_dense_attn_simt(const void* q, const void* k, const void* v, 
                                    int H, int N, int Nk, int D, float scale, int dtype,
                                    cudaStream_t s);
 cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v,
-                                    const PlanLayout& L, const void* plan, float* ws, int H,
-                                    int D, float scale, int dtype, cudaStream_t s);
+                                    const PlanLayout& L, const void* plan, void* o, float* ws,
+                                    int H, int D, float scale, int dtype, cudaStream_t s);
 // Shared by both window-attention paths.
-cudaError_t launch_ws_zero(float* ws, int64_t n, cudaStream_t s);
+cudaError_t launch_ws_zero(float* ws, const PlanLayout& L, const void* plan, int H, int D,
+                           cudaStream_t s);
 cudaError_t launch_window_finalize(const float* ws, const PlanLayout& L, const void* plan,
                                    void* o, int H, int D, int dtype, cudaStream_t s);
 
@@ -96,7 +98,7 @@ cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, vo
                                  int H, int N, int Nk, float scale, cudaStream_t s);
 cudaError_t read_and_clear_tc_error(int* code);
 cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v,
-                                  const PlanLayout& L, const void* plan, float* ws, int H,
-                                  float scale, cudaStream_t s);
+                                  const PlanLayout& L, const void* plan, void* o, float* ws,
+                                  int H, float scale, cudaStream_t s);
 
 }  // namespace area

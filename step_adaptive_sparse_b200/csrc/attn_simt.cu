@@ -2,11 +2,12 @@
 // the bf16 path for head_dim 64.  Same semantics as the tensor-core kernels:
 //   dense  : O = softmax(scale * Q K^T) V over all Nk keys (coarse and full
 //            attention, AReA Phase I / the speedup denominator);
-//   window : per plan work item (window W, 128-query tile), keys S = Halo
-//            rectangle of W followed by its global-KV tokens; the output of W,
-//            weighted by the tent weight of each query, is accumulated in an
-//            fp32 workspace and normalised by the per-token weight sum
-//            (AReA Phase II, centre-weighted blending of overlaps).
+//   window : per plan work item (window W, 256-query block), keys S = Halo
+//            rectangle of W followed by its global-KV tokens.  A token inside
+//            one window only takes that window's output; a token in an overlap
+//            adds its tent-weighted share to an fp32 workspace, normalised
+//            afterwards by the per-token weight sum (AReA Phase II,
+//            centre-weighted blending of overlaps).
 // Pages: ai.info "Methodology in Plain English" (Phase I, Phase II).
 #include "area_internal.cuh"
 
@@ -137,12 +138,19 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
   if (!qvalid) return;
   const float inv = 1.f / l;
   if (WINDOW) {
-    const int y = qtok / P.Wg, x = qtok % P.Wg;
-    const float t = (float)(min(y - win.x + 1, win.x + win.z - y) *
-                            min(x - win.y + 1, win.y + win.w - x));
-    float* dst = ws + (bh * N + qtok) * D;
+    if (P.cover[(int64_t)b * P.N + qtok] == 1) {
+      // the only window containing this token: its output is the merge
+      T* dst = o + (bh * N + qtok) * D;
 #pragma unroll
-    for (int i = 0; i < DPT; ++i) atomicAdd(dst + part + kSimtTPQ * i, t * acc[i] * inv);
+      for (int i = 0; i < DPT; ++i) store_from_float(dst, part + kSimtTPQ * i, acc[i] * inv);
+    } else {
+      const int y = qtok / P.Wg, x = qtok % P.Wg;
+      const float t = (float)(min(y - win.x + 1, win.x + win.z - y) *
+                              min(x - win.y + 1, win.y + win.w - x));
+      float* dst = ws + (bh * N + qtok) * D;
+#pragma unroll
+      for (int i = 0; i < DPT; ++i) atomicAdd(dst + part + kSimtTPQ * i, t * acc[i] * inv);
+    }
   } else {
     T* dst = o + (bh * N + qtok) * D;
 #pragma unroll
@@ -150,10 +158,17 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
   }
 }
 
-__global__ void __launch_bounds__(256) ws_zero_kernel(float4* ws, int64_t n4) {
+// Zero the workspace rows of tokens covered by more than one window (the
+// only rows the window kernels accumulate into).
+__global__ void __launch_bounds__(256) ws_zero_kernel(float4* ws, PlanView P, int H, int D) {
+  const int64_t n4 = (int64_t)P.B * H * P.N * D / 4;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
-       i += (int64_t)gridDim.x * blockDim.x)
-    ws[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = (i * 4) / D;          // (b*H + h)*N + n
+    const int n = (int)(row % P.N);
+    const int b = (int)(row / P.N / H);
+    if (P.cover[(int64_t)b * P.N + n] > 1) ws[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 }
 
 template <typename T>
@@ -166,6 +181,7 @@ __global__ void __launch_bounds__(256) window_finalize_kernel(const float4* __re
     const int64_t row = (i * 4) / D;          // (b*H + h)*N + n
     const int n = (int)(row % P.N);
     const int b = (int)(row / P.N / H);
+    if (P.cover[(int64_t)b * P.N + n] <= 1) continue;    // written by its window
     const float inv = 1.f / P.wsum[(int64_t)b * P.N + n];
     const float4 a = ws[i];
     store_from_float(o, 4 * i + 0, a.x * inv);
@@ -212,22 +228,24 @@ cudaError_t launch_dense_attn_simt(const void* q, const void* k, const void* v, 
 }
 
 cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v,
-                                    const PlanLayout& L, const void* plan, float* ws, int H,
-                                    int D, float scale, int dtype, cudaStream_t s) {
+                                    const PlanLayout& L, const void* plan, void* o, float* ws,
+                                    int H, int D, float scale, int dtype, cudaStream_t s) {
   PlanView P = plan_view(L, const_cast<void*>(plan));
   dim3 grid((unsigned)(L.nitem_max * (kQTile / kSimtQ)), H, (unsigned)L.B);
   DenseRows dr{(int)L.N, (int)L.N};
   if (dtype == AREA_DTYPE_F32) {
-    if (D == 64) return launch_simt<float, 64, true>(grid, q, k, v, nullptr, ws, H, dr, P, scale, s);
-    return launch_simt<float, 128, true>(grid, q, k, v, nullptr, ws, H, dr, P, scale, s);
+    if (D == 64) return launch_simt<float, 64, true>(grid, q, k, v, o, ws, H, dr, P, scale, s);
+    return launch_simt<float, 128, true>(grid, q, k, v, o, ws, H, dr, P, scale, s);
   }
-  if (D == 64) return launch_simt<__nv_bfloat16, 64, true>(grid, q, k, v, nullptr, ws, H, dr, P, scale, s);
-  return launch_simt<__nv_bfloat16, 128, true>(grid, q, k, v, nullptr, ws, H, dr, P, scale, s);
+  if (D == 64) return launch_simt<__nv_bfloat16, 64, true>(grid, q, k, v, o, ws, H, dr, P, scale, s);
+  return launch_simt<__nv_bfloat16, 128, true>(grid, q, k, v, o, ws, H, dr, P, scale, s);
 }
 
-cudaError_t launch_ws_zero(float* ws, int64_t n, cudaStream_t s) {
-  const int64_t n4 = n / 4;
-  ws_zero_kernel<<<grid_cap(n4, 256), 256, 0, s>>>(reinterpret_cast<float4*>(ws), n4);
+cudaError_t launch_ws_zero(float* ws, const PlanLayout& L, const void* plan, int H, int D,
+                           cudaStream_t s) {
+  PlanView P = plan_view(L, const_cast<void*>(plan));
+  const int64_t n4 = L.B * H * L.N * D / 4;
+  ws_zero_kernel<<<grid_cap(n4, 256), 256, 0, s>>>(reinterpret_cast<float4*>(ws), P, H, D);
   return cudaGetLastError();
 }
 

@@ -705,17 +705,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
         }
       } else {
+        // A token inside one window only takes that window's output as it is;
+        // tokens in overlaps add their tent-weighted share to the workspace.
         const int tok = window_query_token(x, qpos, Wg);
+        const bool single = prm.P.cover[(int64_t)x.b * Ntok + tok] == 1;
         const int y = tok / Wg, xx = tok % Wg;
         const float t = (float)(min(y - x.win.x + 1, x.win.x + x.win.z - y) *
                                 min(xx - x.win.y + 1, x.win.y + x.win.w - xx));
-        const float sc = t * inv;
+        const float sc = single ? inv : t * inv;
         float* dst = prm.ws + ((int64_t)x.bh * Ntok + tok) * 128;
+        __nv_bfloat16* dsto = prm.o + ((int64_t)x.bh * Ntok + tok) * 128;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t orr[32];
           tmem_ld32(tO + c * 32, orr);
-          if (qvalid) {
+          if (qvalid && single) {
+            uint4* d4 = reinterpret_cast<uint4*>(dsto + c * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              uint4 w;
+              w.x = pack_bf16(__uint_as_float(orr[8 * v4 + 0]) * sc, __uint_as_float(orr[8 * v4 + 1]) * sc);
+              w.y = pack_bf16(__uint_as_float(orr[8 * v4 + 2]) * sc, __uint_as_float(orr[8 * v4 + 3]) * sc);
+              w.z = pack_bf16(__uint_as_float(orr[8 * v4 + 4]) * sc, __uint_as_float(orr[8 * v4 + 5]) * sc);
+              w.w = pack_bf16(__uint_as_float(orr[8 * v4 + 6]) * sc, __uint_as_float(orr[8 * v4 + 7]) * sc);
+              d4[v4] = w;
+            }
+          } else if (qvalid) {
 #pragma unroll
             for (int v4 = 0; v4 < 8; ++v4)
               red_add_v4(dst + c * 32 + 4 * v4, __uint_as_float(orr[4 * v4]) * sc,
@@ -828,8 +843,8 @@ cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, vo
 }
 
 cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v,
-                                  const PlanLayout& L, const void* plan, float* ws, int H,
-                                  float scale, cudaStream_t s) {
+                                  const PlanLayout& L, const void* plan, void* o, float* ws,
+                                  int H, float scale, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
   cudaError_t e;
   const int64_t rows = L.B * H * L.N;
@@ -845,6 +860,7 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v,
   prm.P = plan_view(L, const_cast<void*>(plan));
   prm.num_units = (int)(L.nitem_max * L.B * H);
   prm.ws = ws;
+  prm.o = static_cast<__nv_bfloat16*>(o);
   return launch_tc<true>(mq, mk, mv, mkp, mvp, prm, s);
 }
 

@@ -18,6 +18,10 @@ namespace area {
 
 static int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
+// Radix-sort tile: 256 threads x 16 ordered rounds of one element each.
+constexpr int kSortRounds = 16;
+constexpr int kSortTile = 256 * kSortRounds;
+
 int plan_layout(const area_plan_cfg* cfg, PlanLayout* L) {
   if (!cfg || !L) return AREA_EINVAL;
   if (cfg->B < 1 || cfg->Hg < 2 || cfg->Wg < 2 || (cfg->Hg & 1) || (cfg->Wg & 1) ||
@@ -35,13 +39,13 @@ int plan_layout(const area_plan_cfg* cfg, PlanLayout* L) {
   L->nb = L->nby * L->nbx;
   L->nw = 4 * L->nb;
   L->nitem_max = L->nb * ((L->hy * L->wx + kQTile - 1) / kQTile + 3);
-  L->ntile_sort = (N + 255) / 256;
+  L->ntile_sort = (N + kSortTile - 1) / kSortTile;
   const int64_t B = L->B;
   const int64_t sizes[AREA_PLAN_NSEC] = {
       B * L->nb * 16, B * L->nb * 4, B * L->nb, B * 4,
       B * L->nw * 16, B * L->nw * 4, B * L->nw * 16, B * L->nw * 4,
       B * L->nw * L->G * 4, B * N * 4, B * N * 4, (B + 1) * 4,
-      B * L->nitem_max * 8, 0};
+      B * L->nitem_max * 8, B * N * 4, 0};
   int64_t off = 256;  // header
   for (int s = 0; s < AREA_PLAN_NSEC; ++s) {
     L->off[s] = off;
@@ -74,6 +78,7 @@ PlanView plan_view(const PlanLayout& L, void* plan) {
   v.gcount = reinterpret_cast<int*>(p + L.off[AREA_PLAN_SEC_GCOUNT]);
   v.gidx = reinterpret_cast<int*>(p + L.off[AREA_PLAN_SEC_GIDX]);
   v.wsum = reinterpret_cast<float*>(p + L.off[AREA_PLAN_SEC_WSUM]);
+  v.cover = reinterpret_cast<int*>(p + L.off[AREA_PLAN_SEC_COVER]);
   v.order = reinterpret_cast<int*>(p + L.off[AREA_PLAN_SEC_ORDER]);
   v.nitem = reinterpret_cast<int*>(p + L.off[AREA_PLAN_SEC_NITEM]);
   v.items = reinterpret_cast<int2*>(p + L.off[AREA_PLAN_SEC_ITEMS]);
@@ -243,8 +248,12 @@ __global__ void __launch_bounds__(256) sort_hist_kernel(const uint32_t* __restri
   __shared__ uint32_t s_h[256];
   s_h[threadIdx.x] = 0;
   __syncthreads();
-  const int i = blockIdx.x * 256 + threadIdx.x;
-  if (i < n) atomicAdd(&s_h[(keys[i] >> shift) & 255u], 1u);
+  const int base = blockIdx.x * kSortTile;
+#pragma unroll 4
+  for (int r = 0; r < kSortRounds; ++r) {
+    const int i = base + r * 256 + threadIdx.x;
+    if (i < n) atomicAdd(&s_h[(keys[i] >> shift) & 255u], 1u);
+  }
   __syncthreads();
   hist[(int64_t)threadIdx.x * ntile + blockIdx.x] = s_h[threadIdx.x];
 }
@@ -264,25 +273,32 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(uint32_t* hist, int m) 
   }
 }
 
+// Stable scatter of one tile: elements are taken in index order (round r,
+// then warp, then lane); each element's rank among equal digits is its
+// rank within its warp, plus the equal digits of earlier warps of the same
+// round, plus those of earlier rounds.
 __global__ void __launch_bounds__(256) sort_scatter_kernel(const uint32_t* __restrict__ kin,
                                                           const int* __restrict__ vin,
                                                           uint32_t* kout, int* vout, int n,
                                                           int shift, const uint32_t* hist,
                                                           int ntile) {
   __shared__ int s_cnt[8][257];
+  __shared__ int s_run[256];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int j = threadIdx.x; j < 8 * 257; j += 256) (&s_cnt[0][0])[j] = 0;
-  __syncthreads();
-  const int i = blockIdx.x * 256 + threadIdx.x;
-  const bool valid = i < n;
-  const uint32_t key = valid ? kin[i] : 0u;
-  const int val = valid ? vin[i] : 0;
-  const int d = valid ? (int)((key >> shift) & 255u) : 256;
-  const unsigned peers = __match_any_sync(0xffffffffu, d);
-  const int rank = __popc(peers & ((1u << lane) - 1u));
-  if (lane == __ffs(peers) - 1) s_cnt[warp][d] = __popc(peers);
-  __syncthreads();
-  {  // exclusive prefix over warps, one digit per thread
+  s_run[threadIdx.x] = (int)hist[(int64_t)threadIdx.x * ntile + blockIdx.x];
+  for (int r = 0; r < kSortRounds; ++r) {
+    for (int j = threadIdx.x; j < 8 * 257; j += 256) (&s_cnt[0][0])[j] = 0;
+    __syncthreads();
+    const int i = blockIdx.x * kSortTile + r * 256 + threadIdx.x;
+    const bool valid = i < n;
+    const uint32_t key = valid ? kin[i] : 0u;
+    const int val = valid ? vin[i] : 0;
+    const int d = valid ? (int)((key >> shift) & 255u) : 256;
+    const unsigned peers = __match_any_sync(0xffffffffu, d);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (lane == __ffs(peers) - 1) s_cnt[warp][d] = __popc(peers);
+    __syncthreads();
+    // exclusive prefix over warps for digit dd; the round total advances s_run
     const int dd = threadIdx.x;
     int run = 0;
 #pragma unroll
@@ -291,12 +307,14 @@ __global__ void __launch_bounds__(256) sort_scatter_kernel(const uint32_t* __res
       s_cnt[w][dd] = run;
       run += c;
     }
-  }
-  __syncthreads();
-  if (valid) {
-    const int pos = (int)hist[(int64_t)d * ntile + blockIdx.x] + s_cnt[warp][d] + rank;
-    kout[pos] = key;
-    vout[pos] = val;
+    __syncthreads();
+    if (valid) {
+      const int pos = s_run[d] + s_cnt[warp][d] + rank;
+      kout[pos] = key;
+      vout[pos] = val;
+    }
+    __syncthreads();
+    s_run[dd] += run;
   }
 }
 
@@ -325,14 +343,14 @@ __global__ void __launch_bounds__(1024) plan_global_kernel(PlanView P) {
   for (int j = gw + threadIdx.x; j < P.G; j += blockDim.x) out[j] = -1;
 }
 
-// Sum of tent weights per token over the final windows that contain it.
+// Sum of tent weights, and count, of the final windows that contain each token.
 __global__ void __launch_bounds__(256) plan_wsum_kernel(PlanView P) {
   const int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (g >= (int64_t)P.B * P.N) return;
   const int b = (int)(g / P.N);
   const int t = (int)(g % P.N);
   const int y = t / P.Wg, x = t % P.Wg;
-  int total = 0;
+  int total = 0, count = 0;
   for (int iy = 0; iy < P.nby; ++iy) {
     const int y0 = tile_start(iy, P.nby, P.Hg, P.hy);
     if (y < y0 || y >= y0 + P.hy) continue;
@@ -346,9 +364,11 @@ __global__ void __launch_bounds__(256) plan_wsum_kernel(PlanView P) {
         if (x < x0 + wl) { qwx = wl; } else { qx0 = x0 + wl; qwx = P.wx - wl; }
       }
       total += min(y - qy0 + 1, qy0 + qhy - y) * min(x - qx0 + 1, qx0 + qwx - x);
+      ++count;
     }
   }
   P.wsum[g] = (float)total;
+  P.cover[g] = count;
 }
 
 }  // namespace
@@ -380,7 +400,7 @@ cudaError_t launch_window_plan(const float* energy, const area_plan_cfg* cfg,
   uint32_t* hist = reinterpret_cast<uint32_t*>(base + L.scratch_hist);
   const int n = (int)L.N, nt = (int)L.ntile_sort;
   for (int b = 0; b < L.B; ++b) {
-    sort_init_kernel<<<nt, 256, 0, s>>>(energy, b, P, ka, va);
+    sort_init_kernel<<<(n + 255) / 256, 256, 0, s>>>(energy, b, P, ka, va);
     for (int pass = 0; pass < 4; ++pass) {
       const int shift = 8 * pass;
       const uint32_t* kin = (pass & 1) ? kb : ka;

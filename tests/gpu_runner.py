@@ -135,3 +135,7 @@ def compare_plan(got: dict, want, b: int = 0):
     if want.G:
         assert np.array_equal(got["gidx"][b, :nw], want.gidx)
     assert np.array_equal(got["wsum"][b].view(np.uint32), want.wsum.view(np.uint32))
+    cover = np.zeros((want.Hg, want.Wg), dtype=np.int32)
+    for (y0, x0, hy, wx) in want.windows:
+        cover[y0:y0 + hy, x0:x0 + wx] += 1
+    assert np.array_equal(got["cover"][b], cover.reshape(-1))
