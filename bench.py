@@ -33,6 +33,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "AReA attention TFLOP/s per schedule step (bf16, 1 B200)"
+# Bumped whenever attn_tc.cu changes, so that stale DRAM counters are not reported.
+KERNEL_REVISION = "attn_tc r5 (patch loader, single-pass f32x2 softmax, direct single-cover stores)"
 DEFAULT_CONFIG = "flux6144"
 
 
@@ -287,13 +289,19 @@ def load_peaks():
             "source": "fallback"}
 
 
-def load_traffic():
-    """dram bytes per launch of the dominant kernel from a committed ncu summary."""
+def load_traffic(workload: str, kernel_tag: str):
+    """DRAM bytes (read + write) per call of a kernel, from the committed ncu
+    summary profiles/traffic.json, or None when the summary does not cover this
+    workload or was taken from an older build of the kernel."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(path):
-        with open(path) as fh:
-            return json.load(fh)
-    return {}
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        t = json.load(fh)
+    entry = t.get(workload, {}).get(kernel_tag)
+    if not entry or entry.get("kernel_revision") != KERNEL_REVISION:
+        return None
+    return entry.get("bytes_per_call")
 
 
 # ---------------------------------------------------------------------------
@@ -471,7 +479,6 @@ def run_area(args):
 
     # ---- roofline of the dominant kernel
     peaks = load_peaks()
-    traffic = load_traffic()
     n1 = st.n_phase1
     coarse_ms = med["coarse_attn"]
     t_coarse = coarse_ms * n1
@@ -485,7 +492,7 @@ def run_area(args):
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "traffic": traffic.get(dom),
+            "frac": achieved / peak, "traffic": load_traffic(cfg.name, dom),
             "kernel": dom, "per_call": dom_launches,
             "peak_kind": f"bf16 dense, {peaks['source']} sustained",
             "frac_of_burst_peak": achieved / peaks["bf16_tflops"]}

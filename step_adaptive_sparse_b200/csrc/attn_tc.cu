@@ -285,6 +285,25 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Packed fp32 pair arithmetic of sm_100 (one instruction for two lanes of work).
+__device__ __forceinline__ void fma2(float& y0, float& y1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\t"
+      "mov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %4};\n\tmov.b64 pc, {%5, %5};\n\t"
+      "fma.rn.f32x2 pd, pa, pb, pc;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(y0), "=f"(y1) : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+__device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1) {
+  asm("{\n\t.reg .b64 pa, ps;\n\t"
+      "mov.b64 pa, {%2, %3};\n\tmov.b64 ps, {%0, %1};\n\t"
+      "add.rn.f32x2 ps, ps, pa;\n\tmov.b64 {%0, %1}, ps;\n\t}"
+      : "+f"(s0), "+f"(s1) : "f"(a0), "f"(a1));
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -639,8 +658,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
         for (int t = 0; t < 4; ++t) pm[t] = __uint_as_float(sr[t]);
 #pragma unroll
-        for (int i = 4; i < 128; ++i) pm[i & 3] = fmaxf(pm[i & 3], __uint_as_float(sr[i]));
-        const float mx = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
+        for (int i = 4; i < 128; i += 2)
+          pm[(i >> 1) & 3] = max3(pm[(i >> 1) & 3], __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
+        const float mx = max3(pm[0], pm[1], fmaxf(pm[2], pm[3]));
         const float mnew = fmaxf(mx * sl2, m);
         // Rescale O only when some row of the warp gained more than 2^8; the
         // decision is warp-uniform because the TMEM accesses are .sync.aligned.
@@ -651,15 +671,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // P = exp2(S * scale * log2(e) - m) as bf16, two keys per TMEM column,
         // written over the S columns already read
         // packed pairs go in place into sr[0..63]: slot i/2 was already read
-        float ls[2] = {0.f, 0.f};
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        const float negm = -m;
 #pragma unroll
         for (int i = 0; i < 128; i += 2) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(sr[i]), sl2, -m));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(sr[i + 1]), sl2, -m));
-          ls[(i >> 1) & 1] += p0 + p1;
+          float x0, x1;
+          fma2(x0, x1, __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]), sl2, negm);
+          const float p0 = fast_exp2(x0);
+          const float p1 = fast_exp2(x1);
+          if ((i >> 1) & 1) add2(ls[2], ls[3], p0, p1); else add2(ls[0], ls[1], p0, p1);
           sr[i >> 1] = pack_bf16(p0, p1);
         }
-        l += ls[0] + ls[1];
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         tmem_st64(tS, sr);
         if (rescale) {
 #pragma unroll 1
