@@ -34,7 +34,7 @@ if ROOT not in sys.path:
 
 METRIC = "AReA attention TFLOP/s per schedule step (bf16, 1 B200)"
 # Bumped whenever attn_tc.cu changes, so that stale DRAM counters are not reported.
-KERNEL_REVISION = "attn_tc r5 (patch loader, single-pass f32x2 softmax, direct single-cover stores)"
+KERNEL_REVISION = "attn_tc r6 (patch loader, f32x2 softmax, single-cover stores, text-key tiles)"
 DEFAULT_CONFIG = "flux6144"
 
 
@@ -458,22 +458,49 @@ def run_area(args):
     full_ms = fe0.elapsed_time(fe1) / args.full_reps
     del o_full
 
-    # ---- end to end through the C-ABI from pinned host buffers
+    # ---- end to end through the C-ABI from pinned host buffers.  Each step
+    # copies its inputs host->device and its output device->host; two device
+    # buffer sets let the copies of one step overlap the kernels of the next
+    # (one stream per copy direction), as a serving loop would.
     out_h = torch.empty(q.shape, dtype=tdt).pin_memory()
     h2d = sum(p.numel() * p.element_size() for p in pin)
     d2h = out_h.numel() * out_h.element_size()
+    sets = [(q, k, v, src, st.o2),
+            tuple(torch.empty_like(t) for t in (q, k, v, src, st.o2))]
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    ev_in, ev_used, ev_out = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+    def upload(i):
+        s_in.wait_event(ev_used[i])          # the kernels of step i-2 are done with set i
+        with torch.cuda.stream(s_in):
+            for dst_t, src_t in zip(sets[i][:4], pin):
+                dst_t.copy_(src_t, non_blocking=True)
+        ev_in[i].record(s_in)
+
     barrier(dist, local)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(args.steps):
-            for dst_t, src_t in zip((q, k, v, src), pin):
-                dst_t.copy_(src_t, non_blocking=True)
+    e0.record(s_in)
+    upload(0)
+    for step in range(args.steps):
+        cur = step % 2
+        if step + 1 < args.steps:
+            upload(1 - cur)
+        stream.wait_event(ev_in[cur])
+        stream.wait_event(ev_out[cur])           # step-2's output has left this buffer
+        st.q, st.k, st.v, st.src, st.o2 = sets[cur]
+        with torch.cuda.stream(stream):
             st.run()
-            out_h.copy_(st.o2, non_blocking=True)
-    e1.record(stream)
+        ev_used[cur].record(stream)
+        s_out.wait_event(ev_used[cur])
+        with torch.cuda.stream(s_out):
+            out_h.copy_(sets[cur][4], non_blocking=True)
+        ev_out[cur].record(s_out)
+    e1.record(s_out)
     torch.cuda.synchronize()
+    st.q, st.k, st.v, st.src, st.o2 = sets[0]
+    del sets
     e2e_ms = reduce_max(dist, e0.elapsed_time(e1), device=str(dev))
     e2e_val = flops_all / (e2e_ms * 1e-3) / 1e12
 

@@ -108,6 +108,20 @@ int area_coarse_attn(const void* q, const void* kp, const void* vp, void* o,
                      int dtype, cudaStream_t stream);
 
 /*
+ * area_coarse_attn_text -- Phase I with text tokens ([ai] Phase I: text tokens
+ * are never pooled, so each of the N queries attends to T + N/f^2 keys):
+ *   O = softmax(scale * Q [Kp; Kt]^T) [Vp; Vt]   per (b, h).
+ *   kt, vt : [B, H, T, D] text keys and values (dtype), T >= 0 (0 = none).
+ * Outputs are the image queries' rows only; text queries are the caller's.
+ * Errors: as area_coarse_attn, and AREA_EINVAL for T < 0 or null kt/vt with
+ * T > 0.
+ */
+int area_coarse_attn_text(const void* q, const void* kp, const void* vp,
+                          const void* kt, const void* vt, void* o,
+                          int B, int H, int N, int Nk, int T, int D,
+                          float scale, int dtype, cudaStream_t stream);
+
+/*
  * area_full_attn -- full global attention over all N tokens, the operation
  * AReA replaces ([ai] "Main Findings": speedups are quoted against it).
  * Same kernels as area_coarse_attn with Nk = N.
@@ -248,6 +262,22 @@ int area_window_attn(const void* q, const void* k, const void* v,
                      size_t plan_bytes, void* o, void* ws, size_t ws_bytes,
                      int H, int D, float scale, int dtype,
                      cudaStream_t stream);
+
+/*
+ * area_window_attn_text -- area_window_attn with text tokens: every window's
+ * key set is ext(W), then G_W, then all T text keys [B, H, T, D] (kt, vt).
+ * The pages state that text tokens are never pooled and every query attends
+ * to them in Phase I; applying the same to Phase II windows is this
+ * library's reading.  The merge is unchanged.
+ * Errors: as area_window_attn, and AREA_EINVAL for T < 0 or null kt/vt with
+ * T > 0.
+ */
+int area_window_attn_text(const void* q, const void* k, const void* v,
+                          const void* kt, const void* vt, int T,
+                          const area_plan_cfg* cfg, const void* plan,
+                          size_t plan_bytes, void* o, void* ws, size_t ws_bytes,
+                          int H, int D, float scale, int dtype,
+                          cudaStream_t stream);
 
 /*
  * area_window_attn_noalloc -- area_window_attn for callers that cannot

@@ -87,11 +87,13 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.n
     return np.matmul(p, v)
 
 
-def coarse_attn(q, kp, vp, scale, rows: Optional[np.ndarray] = None) -> np.ndarray:
+def coarse_attn(q, kp, vp, scale, rows: Optional[np.ndarray] = None,
+                kt: Optional[np.ndarray] = None, vt: Optional[np.ndarray] = None) -> np.ndarray:
     """Phase I cross-scale coarse attention ([blog] Fase I, [ai] Phase I).
 
-    Every full-resolution query attends to all pooled keys, text tokens
-    absent (T = 0).  q: [B, H, N, D]; kp, vp: [B, H, Nk, D].  ``rows``
+    Every full-resolution query attends to all pooled keys and, when given,
+    to all T text keys, which are never pooled: T + N/f^2 keys per query.
+    q: [B, H, N, D]; kp, vp: [B, H, Nk, D]; kt, vt: [B, H, T, D].  ``rows``
     (optional) restricts the computation to those query indices.
     """
     if rows is not None:
@@ -100,7 +102,11 @@ def coarse_attn(q, kp, vp, scale, rows: Optional[np.ndarray] = None) -> np.ndarr
     out = np.empty(q.shape, dtype=np.float64)
     for b in range(B):
         for h in range(H):
-            out[b, h] = attention(q[b, h], kp[b, h], vp[b, h], scale)
+            kk, vv = kp[b, h], vp[b, h]
+            if kt is not None:
+                kk = np.concatenate([np.asarray(kk), np.asarray(kt[b, h])])
+                vv = np.concatenate([np.asarray(vv), np.asarray(vt[b, h])])
+            out[b, h] = attention(q[b, h], kk, vv, scale)
     return out
 
 
@@ -352,15 +358,19 @@ def window_kv_tokens(plan: Plan, i: int) -> np.ndarray:
 
 
 def window_attn(q, k, v, plans: Sequence[Plan], scale: float,
-                rows: Optional[np.ndarray] = None, heads: Optional[Sequence[int]] = None
+                rows: Optional[np.ndarray] = None, heads: Optional[Sequence[int]] = None,
+                kt: Optional[np.ndarray] = None, vt: Optional[np.ndarray] = None
                 ) -> np.ndarray:
     """Phase II windowed attention with centre-weighted merge ([ai] Phase II).
 
     For each final window W: O_W(q) = softmax(scale * q K_S^T) V_S over
-    S = ext(W) u G_W; then O(q) = sum_W t_W(q) O_W(q) / sum_W t_W(q), over
-    the windows that contain q.  q, k, v: [B, H, N, D]; plans: one per batch
-    element.  ``rows`` restricts the output to those token indices and
-    ``heads`` to those heads; the result is [B, len(heads), len(rows), D].
+    S = ext(W) u G_W (u the T text keys when kt, vt [B, H, T, D] are given:
+    the pages keep text keys unpooled and visible to every query in Phase I;
+    keeping them in every window is the reading taken for Phase II); then
+    O(q) = sum_W t_W(q) O_W(q) / sum_W t_W(q), over the windows that contain
+    q.  q, k, v: [B, H, N, D]; plans: one per batch element.  ``rows``
+    restricts the output to those token indices and ``heads`` to those heads;
+    the result is [B, len(heads), len(rows), D].
     """
     B, H, N, D = q.shape
     heads = list(range(H)) if heads is None else list(heads)
@@ -382,7 +392,11 @@ def window_attn(q, k, v, plans: Sequence[Plan], scale: float,
                  np.minimum(tx - x0 + 1, x0 + wx - tx)).astype(np.float64)
             kv = window_kv_tokens(plan, i)
             for hi, h in enumerate(heads):
-                o = attention(q[b, h][toks], k[b, h][kv], v[b, h][kv], scale)
+                kk, vv = k[b, h][kv], v[b, h][kv]
+                if kt is not None:
+                    kk = np.concatenate([kk, np.asarray(kt[b, h])])
+                    vv = np.concatenate([vv, np.asarray(vt[b, h])])
+                o = attention(q[b, h][toks], kk, vv, scale)
                 out[b, hi, pos[toks]] += t[:, None] * o
         ws = plan.wsum.astype(np.float64)[rows]
         out[b] /= ws[None, :, None]

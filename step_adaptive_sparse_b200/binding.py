@@ -27,7 +27,7 @@ SECTIONS = ("BASE", "SCORE", "SPLIT", "NWIN", "WIN", "PARENT", "EXT", "GCOUNT", 
             "WSUM", "ORDER", "NITEM", "ITEMS", "COVER", "SCRATCH")
 
 EXPORTED = ("area_status_string", "area_last_cuda_error", "area_version", "area_kernel_error",
-            "area_pool_kv",
+            "area_pool_kv", "area_coarse_attn_text", "area_window_attn_text",
             "area_coarse_attn", "area_full_attn", "area_dwt_detail", "area_window_plan_bytes",
             "area_window_plan", "area_window_attn_ws_bytes", "area_window_attn")
 
@@ -60,6 +60,9 @@ _SIGS = {
     "area_pool_kv": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P]),
     "area_coarse_attn": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
     "area_full_attn": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "area_coarse_attn_text": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "area_window_attn_text": (_I, [_P, _P, _P, _P, _P, _I, ctypes.POINTER(area_plan_cfg), _P, _SZ,
+                                   _P, _P, _SZ, _I, _I, _F, _I, _P]),
     "area_dwt_detail": (_I, [_P, _I, _I, _P, _I, _I, _I, _I, _P]),
     "area_window_plan_bytes": (_I, [ctypes.POINTER(area_plan_cfg), ctypes.POINTER(_SZ)]),
     "area_window_plan": (_I, [_P, ctypes.POINTER(area_plan_cfg), _P, _SZ, _P]),
@@ -140,6 +143,21 @@ def area_pool_kv(k, v, kp, vp, B, H, Hg, Wg, D, f, mode, dtype, stream=None) -> 
 def area_coarse_attn(q, kp, vp, o, B, H, N, Nk, D, scale, dtype, stream=None) -> None:
     _check(_lib().area_coarse_attn(_ptr(q), _ptr(kp), _ptr(vp), _ptr(o), B, H, N, Nk, D, scale,
                                    dtype, _stream(stream)), "area_coarse_attn")
+
+
+def area_coarse_attn_text(q, kp, vp, kt, vt, o, B, H, N, Nk, T, D, scale, dtype,
+                          stream=None) -> None:
+    _check(_lib().area_coarse_attn_text(_ptr(q), _ptr(kp), _ptr(vp), _ptr(kt), _ptr(vt), _ptr(o),
+                                        B, H, N, Nk, T, D, scale, dtype, _stream(stream)),
+           "area_coarse_attn_text")
+
+
+def area_window_attn_text(q, k, v, kt, vt, T, cfg: area_plan_cfg, plan, plan_bytes, o, ws,
+                          ws_bytes, H, D, scale, dtype, stream=None) -> None:
+    _check(_lib().area_window_attn_text(_ptr(q), _ptr(k), _ptr(v), _ptr(kt), _ptr(vt), T,
+                                        ctypes.byref(cfg), _ptr(plan), plan_bytes, _ptr(o),
+                                        _ptr(ws), ws_bytes, H, D, scale, dtype, _stream(stream)),
+           "area_window_attn_text")
 
 
 def area_full_attn(q, k, v, o, B, H, N, D, scale, dtype, stream=None) -> None:

@@ -32,14 +32,44 @@ int check_attn(const void* q, const void* k, const void* v, const void* o, int B
   return AREA_OK;
 }
 
-int dense_attn(const void* q, const void* k, const void* v, void* o, int B, int H, int N, int Nk,
-               int D, float scale, int dtype, cudaStream_t s) {
+int dense_attn(const void* q, const void* k, const void* v, const void* kt, const void* vt,
+               int T, void* o, int B, int H, int N, int Nk, int D, float scale, int dtype,
+               cudaStream_t s) {
   int st = check_attn(q, k, v, o, B, H, N, Nk, D, dtype);
   if (st != AREA_OK) return st;
   if (B > 65535 || H > 65535) return AREA_EINVAL;
+  if (T < 0 || (T > 0 && (!kt || !vt || !aligned16(kt) || !aligned16(vt)))) return AREA_EINVAL;
   if (dtype == AREA_DTYPE_BF16 && D == 128)
-    return finish(area::launch_dense_attn_tc(q, k, v, o, B, H, N, Nk, scale, s));
-  return finish(area::launch_dense_attn_simt(q, k, v, o, B, H, N, Nk, D, scale, dtype, s));
+    return finish(area::launch_dense_attn_tc(q, k, v, kt, vt, o, B, H, N, Nk, T, scale, s));
+  return finish(
+      area::launch_dense_attn_simt(q, k, v, kt, vt, o, B, H, N, Nk, T, D, scale, dtype, s));
+}
+
+int window_attn(const void* q, const void* k, const void* v, const void* kt, const void* vt,
+                int T, const area_plan_cfg* cfg, const void* plan, size_t plan_bytes, void* o,
+                void* ws, size_t ws_bytes, int H, int D, float scale, int dtype,
+                cudaStream_t stream) {
+  if (!plan || !ws) return AREA_EINVAL;
+  area::PlanLayout L;
+  int st = area::plan_layout(cfg, &L);
+  if (st != AREA_OK) return st;
+  st = check_attn(q, k, v, o, (int)L.B, H, (int)L.N, (int)L.N, D, dtype);
+  if (st != AREA_OK) return st;
+  if (T < 0 || (T > 0 && (!kt || !vt || !aligned16(kt) || !aligned16(vt)))) return AREA_EINVAL;
+  if (plan_bytes < (size_t)L.total) return AREA_ENOSPACE;
+  if (ws_bytes < (size_t)(L.B * H * L.N * D * 4)) return AREA_ENOSPACE;
+  if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(plan) & 255) != 0) return AREA_EINVAL;
+  if (H > 65535 || L.B > 65535) return AREA_EINVAL;
+  float* w = static_cast<float*>(ws);
+  cudaError_t e = area::launch_ws_zero(w, L, plan, H, D, stream);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (dtype == AREA_DTYPE_BF16 && D == 128)
+    e = area::launch_window_attn_tc(q, k, v, kt, vt, T, L, plan, o, w, H, scale, stream);
+  else
+    e = area::launch_window_attn_simt(q, k, v, kt, vt, T, L, plan, o, w, H, D, scale, dtype,
+                                      stream);
+  if (e != cudaSuccess) return fail_cuda(e);
+  return finish(area::launch_window_finalize(w, L, plan, o, H, D, dtype, stream));
 }
 
 }  // namespace
@@ -80,12 +110,18 @@ int area_pool_kv(const void* k, const void* v, void* kp, void* vp, int B, int H,
 
 int area_coarse_attn(const void* q, const void* kp, const void* vp, void* o, int B, int H, int N,
                      int Nk, int D, float scale, int dtype, cudaStream_t stream) {
-  return dense_attn(q, kp, vp, o, B, H, N, Nk, D, scale, dtype, stream);
+  return dense_attn(q, kp, vp, nullptr, nullptr, 0, o, B, H, N, Nk, D, scale, dtype, stream);
+}
+
+int area_coarse_attn_text(const void* q, const void* kp, const void* vp, const void* kt,
+                          const void* vt, void* o, int B, int H, int N, int Nk, int T, int D,
+                          float scale, int dtype, cudaStream_t stream) {
+  return dense_attn(q, kp, vp, kt, vt, T, o, B, H, N, Nk, D, scale, dtype, stream);
 }
 
 int area_full_attn(const void* q, const void* k, const void* v, void* o, int B, int H, int N,
                    int D, float scale, int dtype, cudaStream_t stream) {
-  return dense_attn(q, k, v, o, B, H, N, N, D, scale, dtype, stream);
+  return dense_attn(q, k, v, nullptr, nullptr, 0, o, B, H, N, N, D, scale, dtype, stream);
 }
 
 int area_dwt_detail(const void* src, int src_dtype, int C, float* energy, int B, int Hg, int Wg,
@@ -129,25 +165,16 @@ int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D, size_t* ws
 int area_window_attn(const void* q, const void* k, const void* v, const area_plan_cfg* cfg,
                      const void* plan, size_t plan_bytes, void* o, void* ws, size_t ws_bytes,
                      int H, int D, float scale, int dtype, cudaStream_t stream) {
-  if (!plan || !ws) return AREA_EINVAL;
-  area::PlanLayout L;
-  int st = area::plan_layout(cfg, &L);
-  if (st != AREA_OK) return st;
-  st = check_attn(q, k, v, o, (int)L.B, H, (int)L.N, (int)L.N, D, dtype);
-  if (st != AREA_OK) return st;
-  if (plan_bytes < (size_t)L.total) return AREA_ENOSPACE;
-  if (ws_bytes < (size_t)(L.B * H * L.N * D * 4)) return AREA_ENOSPACE;
-  if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(plan) & 255) != 0) return AREA_EINVAL;
-  if (H > 65535 || L.B > 65535) return AREA_EINVAL;
-  float* w = static_cast<float*>(ws);
-  cudaError_t e = area::launch_ws_zero(w, L, plan, H, D, stream);
-  if (e != cudaSuccess) return fail_cuda(e);
-  if (dtype == AREA_DTYPE_BF16 && D == 128)
-    e = area::launch_window_attn_tc(q, k, v, L, plan, o, w, H, scale, stream);
-  else
-    e = area::launch_window_attn_simt(q, k, v, L, plan, o, w, H, D, scale, dtype, stream);
-  if (e != cudaSuccess) return fail_cuda(e);
-  return finish(area::launch_window_finalize(w, L, plan, o, H, D, dtype, stream));
+  return window_attn(q, k, v, nullptr, nullptr, 0, cfg, plan, plan_bytes, o, ws, ws_bytes, H, D,
+                     scale, dtype, stream);
+}
+
+int area_window_attn_text(const void* q, const void* k, const void* v, const void* kt,
+                          const void* vt, int T, const area_plan_cfg* cfg, const void* plan,
+                          size_t plan_bytes, void* o, void* ws, size_t ws_bytes, int H, int D,
+                          float scale, int dtype, cudaStream_t stream) {
+  return window_attn(q, k, v, kt, vt, T, cfg, plan, plan_bytes, o, ws, ws_bytes, H, D, scale,
+                     dtype, stream);
 }
 
 }  // extern "C"

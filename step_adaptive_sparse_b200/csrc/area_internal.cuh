@@ -81,24 +81,27 @@ cudaError_t launch_window_plan(const float* energy, const area_plan_cfg* cfg,
                                const PlanLayout& L, void* plan, cudaStream_t s);
 
 // CUDA-core attention (fp32 any supported D; bf16 fallback for D = 64).
-cudaError_t launch_dense_attn_simt(const void* q, const void* k, const void* v, void* o, int B,
-                                   int H, int N, int Nk, int D, float scale, int dtype,
-                                   cudaStream_t s);
-cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v,
-                                    const PlanLayout& L, const void* plan, void* o, float* ws,
-                                    int H, int D, float scale, int dtype, cudaStream_t s);
+cudaError_t launch_dense_attn_simt(const void* q, const void* k, const void* v, const void* kt,
+                                   const void* vt, void* o, int B, int H, int N, int Nk, int T,
+                                   int D, float scale, int dtype, cudaStream_t s);
+cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v, const void* kt,
+                                    const void* vt, int T, const PlanLayout& L, const void* plan,
+                                    void* o, float* ws, int H, int D, float scale, int dtype,
+                                    cudaStream_t s);
 // Shared by both window-attention paths.
 cudaError_t launch_ws_zero(float* ws, const PlanLayout& L, const void* plan, int H, int D,
                            cudaStream_t s);
 cudaError_t launch_window_finalize(const float* ws, const PlanLayout& L, const void* plan,
                                    void* o, int H, int D, int dtype, cudaStream_t s);
 
-// tcgen05 tensor-core attention (bf16, D = 128).
-cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, void* o, int B,
-                                 int H, int N, int Nk, float scale, cudaStream_t s);
+// tcgen05 tensor-core attention (bf16, D = 128).  kt, vt: [B, H, T, 128] text
+// keys appended after the image keys of every query (T = 0: none).
+cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, const void* kt,
+                                 const void* vt, void* o, int B, int H, int N, int Nk, int T,
+                                 float scale, cudaStream_t s);
 cudaError_t read_and_clear_tc_error(int* code);
-cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v,
-                                  const PlanLayout& L, const void* plan, void* o, float* ws,
-                                  int H, float scale, cudaStream_t s);
+cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, const void* kt,
+                                  const void* vt, int T, const PlanLayout& L, const void* plan,
+                                  void* o, float* ws, int H, float scale, cudaStream_t s);
 
 }  // namespace area

@@ -26,12 +26,14 @@ struct DenseRows {
 template <typename T, int D, bool WINDOW>
 __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-    T* __restrict__ o, float* __restrict__ ws, int H, DenseRows dr, PlanView P, float scale) {
+    const T* __restrict__ kt, const T* __restrict__ vt, int ntext, T* __restrict__ o,
+    float* __restrict__ ws, int H, DenseRows dr, PlanView P, float scale) {
   constexpr int DPT = D / kSimtTPQ;
   extern __shared__ float smem[];
   float* Ks = smem;                       // [kSimtKV][D]
   float* Vs = smem + kSimtKV * D;         // [kSimtKV][D]
   __shared__ int s_kvtok[kSimtKV];
+  __shared__ bool s_kvtxt[kSimtKV];
 
   const int b = blockIdx.z, h = blockIdx.y;
   const int tid = threadIdx.x;
@@ -70,6 +72,10 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
   const T* qrow = q + (bh * N + qtok) * D;
   const T* kb = k + bh * Nkv_rows * D;
   const T* vb = v + bh * Nkv_rows * D;
+  const T* ktb = kt ? kt + bh * ntext * D : nullptr;   // text keys after the image keys
+  const T* vtb = vt ? vt + bh * ntext * D : nullptr;
+  const int nimg = nkv;
+  nkv += ntext;
 
   float qv[DPT], acc[DPT];
 #pragma unroll
@@ -83,9 +89,13 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     const int cn = min(kSimtKV, nkv - c0);
     if (tid < kSimtKV) {
       int tok = 0;
+      bool txt = false;
       const int j = c0 + tid;
       if (tid < cn) {
-        if (WINDOW) {
+        if (j >= nimg) {
+          tok = j - nimg;
+          txt = true;
+        } else if (WINDOW) {
           const int ne = ext.z * ext.w;
           tok = j < ne ? (ext.x + j / ext.w) * P.Wg + ext.y + j % ext.w : glist[j - ne];
         } else {
@@ -93,17 +103,20 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
         }
       }
       s_kvtok[tid] = tok;
+      s_kvtxt[tid] = txt;
     }
     __syncthreads();
     // cooperative load: thread -> (row, quarter of the row)
     for (int e = tid; e < kSimtKV * 4; e += kSimtThreads) {
       const int row = e >> 2, qd = e & 3;
       const int64_t src = (int64_t)s_kvtok[row] * D;
+      const T* ks = s_kvtxt[row] ? ktb : kb;
+      const T* vs = s_kvtxt[row] ? vtb : vb;
 #pragma unroll 4
       for (int d = qd * (D / 4); d < (qd + 1) * (D / 4); ++d) {
         const bool ok = row < cn;
-        Ks[row * D + d] = ok ? load_as_float(kb, src + d) : 0.f;
-        Vs[row * D + d] = ok ? load_as_float(vb, src + d) : 0.f;
+        Ks[row * D + d] = ok ? load_as_float(ks, src + d) : 0.f;
+        Vs[row * D + d] = ok ? load_as_float(vs, src + d) : 0.f;
       }
     }
     __syncthreads();
@@ -192,16 +205,17 @@ __global__ void __launch_bounds__(256) window_finalize_kernel(const float4* __re
 }
 
 template <typename T, int D, bool WINDOW>
-cudaError_t launch_simt(dim3 grid, const void* q, const void* k, const void* v, void* o,
-                        float* ws, int H, DenseRows dr, PlanView P, float scale,
-                        cudaStream_t s) {
+cudaError_t launch_simt(dim3 grid, const void* q, const void* k, const void* v, const void* kt,
+                        const void* vt, int ntext, void* o, float* ws, int H, DenseRows dr,
+                        PlanView P, float scale, cudaStream_t s) {
   const int smem = 2 * kSimtKV * D * (int)sizeof(float);
   auto fn = attn_simt_kernel<T, D, WINDOW>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   fn<<<grid, kSimtThreads, smem, s>>>(static_cast<const T*>(q), static_cast<const T*>(k),
-                                      static_cast<const T*>(v), static_cast<T*>(o), ws, H, dr, P,
-                                      scale);
+                                      static_cast<const T*>(v), static_cast<const T*>(kt),
+                                      static_cast<const T*>(vt), ntext, static_cast<T*>(o), ws, H,
+                                      dr, P, scale);
   return cudaGetLastError();
 }
 
@@ -213,32 +227,33 @@ int grid_cap(int64_t n, int block) {
 
 }  // namespace
 
-cudaError_t launch_dense_attn_simt(const void* q, const void* k, const void* v, void* o, int B,
-                                   int H, int N, int Nk, int D, float scale, int dtype,
-                                   cudaStream_t s) {
+cudaError_t launch_dense_attn_simt(const void* q, const void* k, const void* v, const void* kt,
+                                   const void* vt, void* o, int B, int H, int N, int Nk, int T,
+                                   int D, float scale, int dtype, cudaStream_t s) {
   dim3 grid((N + kSimtQ - 1) / kSimtQ, H, B);
   DenseRows dr{N, Nk};
   PlanView P{};
   if (dtype == AREA_DTYPE_F32) {
-    if (D == 64) return launch_simt<float, 64, false>(grid, q, k, v, o, nullptr, H, dr, P, scale, s);
-    return launch_simt<float, 128, false>(grid, q, k, v, o, nullptr, H, dr, P, scale, s);
+    if (D == 64) return launch_simt<float, 64, false>(grid, q, k, v, kt, vt, T, o, nullptr, H, dr, P, scale, s);
+    return launch_simt<float, 128, false>(grid, q, k, v, kt, vt, T, o, nullptr, H, dr, P, scale, s);
   }
-  if (D == 64) return launch_simt<__nv_bfloat16, 64, false>(grid, q, k, v, o, nullptr, H, dr, P, scale, s);
-  return launch_simt<__nv_bfloat16, 128, false>(grid, q, k, v, o, nullptr, H, dr, P, scale, s);
+  if (D == 64) return launch_simt<__nv_bfloat16, 64, false>(grid, q, k, v, kt, vt, T, o, nullptr, H, dr, P, scale, s);
+  return launch_simt<__nv_bfloat16, 128, false>(grid, q, k, v, kt, vt, T, o, nullptr, H, dr, P, scale, s);
 }
 
-cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v,
-                                    const PlanLayout& L, const void* plan, void* o, float* ws,
-                                    int H, int D, float scale, int dtype, cudaStream_t s) {
+cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v, const void* kt,
+                                    const void* vt, int T, const PlanLayout& L, const void* plan,
+                                    void* o, float* ws, int H, int D, float scale, int dtype,
+                                    cudaStream_t s) {
   PlanView P = plan_view(L, const_cast<void*>(plan));
   dim3 grid((unsigned)(L.nitem_max * (kQTile / kSimtQ)), H, (unsigned)L.B);
   DenseRows dr{(int)L.N, (int)L.N};
   if (dtype == AREA_DTYPE_F32) {
-    if (D == 64) return launch_simt<float, 64, true>(grid, q, k, v, o, ws, H, dr, P, scale, s);
-    return launch_simt<float, 128, true>(grid, q, k, v, o, ws, H, dr, P, scale, s);
+    if (D == 64) return launch_simt<float, 64, true>(grid, q, k, v, kt, vt, T, o, ws, H, dr, P, scale, s);
+    return launch_simt<float, 128, true>(grid, q, k, v, kt, vt, T, o, ws, H, dr, P, scale, s);
   }
-  if (D == 64) return launch_simt<__nv_bfloat16, 64, true>(grid, q, k, v, o, ws, H, dr, P, scale, s);
-  return launch_simt<__nv_bfloat16, 128, true>(grid, q, k, v, o, ws, H, dr, P, scale, s);
+  if (D == 64) return launch_simt<__nv_bfloat16, 64, true>(grid, q, k, v, kt, vt, T, o, ws, H, dr, P, scale, s);
+  return launch_simt<__nv_bfloat16, 128, true>(grid, q, k, v, kt, vt, T, o, ws, H, dr, P, scale, s);
 }
 
 cudaError_t launch_ws_zero(float* ws, const PlanLayout& L, const void* plan, int H, int D,

@@ -331,7 +331,8 @@ struct Unit {
   int q0;          // first query position of tile 0 (tile 1 = q0 + 128)
   int nq;          // number of valid query positions from q0 (window: area)
   int nkv;         // dense: number of keys; window: G_W (global-KV count)
-  int nt;          // key tiles of this unit
+  int nti;         // key tiles of image tokens (rectangle patches + global / dense keys)
+  int nt;          // key tiles of this unit, text tiles included
   int ncx;         // window: patches per row of the Halo rectangle
   int ntr;         // window: patch tiles of the Halo rectangle
   int4 win, ext;   // window mode
@@ -339,7 +340,8 @@ struct Unit {
 };
 
 template <bool WINDOW>
-__device__ __forceinline__ Unit get_unit(int u, const DenseArgs& da, const PlanView& P, int H) {
+__device__ __forceinline__ Unit get_unit(int u, const DenseArgs& da, const PlanView& P, int H,
+                                         int T) {
   Unit x;
   x.valid = true;
   x.glist = nullptr;
@@ -349,7 +351,8 @@ __device__ __forceinline__ Unit get_unit(int u, const DenseArgs& da, const PlanV
     x.q0 = (u % da.units_per_head) * 256;
     x.nq = da.N;
     x.nkv = da.Nk;
-    x.nt = (da.Nk + 127) / 128;
+    x.nti = (da.Nk + 127) / 128;
+    x.nt = x.nti + (T + 127) / 128;
     x.ncx = x.ntr = 0;
     x.win = x.ext = make_int4(0, 0, 0, 0);
   } else {
@@ -372,7 +375,8 @@ __device__ __forceinline__ Unit get_unit(int u, const DenseArgs& da, const PlanV
     x.nkv = P.gcount[wo];
     x.ncx = (x.ext.w + kPW - 1) / kPW;
     x.ntr = x.ncx * ((x.ext.z + kPH - 1) / kPH);
-    x.nt = x.ntr + (x.nkv + 127) / 128;
+    x.nti = x.ntr + (x.nkv + 127) / 128;
+    x.nt = x.nti + (T + 127) / 128;
     x.glist = P.gidx + wo * P.G;
   }
   return x;
@@ -391,6 +395,7 @@ __device__ __forceinline__ int window_query_token(const Unit& x, int p, int Wg) 
 struct TcParams {
   float scale_log2;
   int H;
+  int T;              // text keys per (b, h), appended after the image keys
   int num_units;
   DenseArgs da;
   PlanView P;
@@ -402,7 +407,8 @@ template <bool WINDOW>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
-               const __grid_constant__ CUtensorMap tm_vp, const TcParams prm) {
+               const __grid_constant__ CUtensorMap tm_vp, const __grid_constant__ CUtensorMap tm_kt,
+               const __grid_constant__ CUtensorMap tm_vt, const TcParams prm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -450,7 +456,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // ------------------------------------------------------------ producer
     uint32_t kv_it = 0, unit_count = 0;
     for (int u = blockIdx.x; u < prm.num_units; u += gridDim.x) {
-      const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H);
+      const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T);
       if (!x.valid) continue;
       if (!warp_wait0(bar(BAR_Q_EMPTY), (unit_count & 1u) ^ 1u, abort_flag)) break;
       if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL), 2 * kTileBytes);
@@ -486,7 +492,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           __syncwarp();
           const CUtensorMap* tm = kv ? &tm_v : &tm_k;
           const uint32_t dst = sbase + kSmemKV + s * kTileBytes;
-          if constexpr (!WINDOW) {
+          if (j >= x.nti) {
+            // text keys: rows of the [B*H*T, 128] text tensors
+            if (lane == 0) {
+              const CUtensorMap* tt = kv ? &tm_vt : &tm_kt;
+              for (int hf = 0; hf < 2; ++hf)
+                tma_load_2d(dst + hf * kHalfBytes, tt, bar(BAR_KV_FULL + s), hf * 64,
+                            x.bh * prm.T + (j - x.nti) * 128);
+            }
+          } else if constexpr (!WINDOW) {
             if (lane == 0)
               for (int hf = 0; hf < 2; ++hf)
                 tma_load_2d(dst + hf * kHalfBytes, tm, bar(BAR_KV_FULL + s), hf * 64,
@@ -545,7 +559,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                  (first && kk == 0) ? 0u : 1u);
       };
       for (int u = blockIdx.x; u < prm.num_units && ok; u += gridDim.x) {
-        const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H);
+        const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T);
         if (!x.valid) continue;
         const int nt = x.nt;
         if (!(ok = mbar_wait(bar(BAR_Q_FULL), unit_count & 1u, abort_flag))) break;
@@ -621,11 +635,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     for (int u = blockIdx.x; u < prm.num_units && ok; u += gridDim.x) {
       // key-tile geometry of this unit (the rest is looked up again for the
       // epilogue rather than kept live in registers across the key loop)
-      int nkv, nt, ntr, ncx, ew, eh;
+      int nkv, nt, nti, ntr, ncx, ew, eh;
       {
-        const Unit x0 = get_unit<WINDOW>(u, prm.da, prm.P, prm.H);
+        const Unit x0 = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T);
         if (!x0.valid) continue;
-        nkv = x0.nkv; nt = x0.nt; ntr = x0.ntr; ncx = x0.ncx;
+        nkv = x0.nkv; nt = x0.nt; nti = x0.nti; ntr = x0.ntr; ncx = x0.ncx;
         ew = x0.ext.w; eh = x0.ext.z;
       }
       float m = -INFINITY, l = 0.f;
@@ -635,11 +649,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc_fence_after();
         uint32_t sr[128];
         tmem_ld128(tS, sr);
-        // Key validity (warp-uniform): dense and global-KV tiles are a prefix
-        // of `valid` keys; a rectangle patch keeps columns dx < rem_x of rows
-        // dy < rem_y (key k = dy * kPW + dx).
+        // Key validity (warp-uniform): dense, global-KV and text tiles are a
+        // prefix of `valid` keys; a rectangle patch keeps columns dx < rem_x of
+        // rows dy < rem_y (key k = dy * kPW + dx).
         if (!WINDOW || j >= ntr) {
-          const int valid = min(128, nkv - (j - ntr) * 128);
+          const int valid = j < nti ? min(128, nkv - (j - ntr) * 128)
+                                    : min(128, prm.T - (j - nti) * 128);
           if (valid < 128) {
 #pragma unroll
             for (int i = 0; i < 128; ++i)
@@ -701,7 +716,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (!ok) break;
       // epilogue (the unit is looked up again rather than kept live in
       // registers across the key loop)
-      const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H);
+      const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T);
       if (!(ok = warp_wait_all(bO, o_cnt & 1u, abort_flag))) break;
       ++o_cnt;
       tc_fence_after();
@@ -828,13 +843,13 @@ int num_sms() {
 
 template <bool WINDOW>
 cudaError_t launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                      const CUtensorMap& mkp, const CUtensorMap& mvp, const TcParams& prm,
-                      cudaStream_t s) {
+                      const CUtensorMap& mkp, const CUtensorMap& mvp, const CUtensorMap& mkt,
+                      const CUtensorMap& mvt, const TcParams& prm, cudaStream_t s) {
   auto fn = attn_tc_kernel<WINDOW>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int grid = prm.num_units < num_sms() ? prm.num_units : num_sms();
-  fn<<<grid > 0 ? grid : 1, kThreads, kSmemBytes, s>>>(mq, mk, mv, mkp, mvp, prm);
+  fn<<<grid > 0 ? grid : 1, kThreads, kSmemBytes, s>>>(mq, mk, mv, mkp, mvp, mkt, mvt, prm);
   return cudaGetLastError();
 }
 
@@ -849,26 +864,35 @@ cudaError_t read_and_clear_tc_error(int* code) {
   return cudaMemcpyToSymbol(g_tc_error, &zero, sizeof(int));
 }
 
-cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, void* o, int B,
-                                 int H, int N, int Nk, float scale, cudaStream_t s) {
-  CUtensorMap mq, mk, mv;
+cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, const void* kt,
+                                 const void* vt, void* o, int B, int H, int N, int Nk, int T,
+                                 float scale, cudaStream_t s) {
+  CUtensorMap mq, mk, mv, mkt, mvt;
   cudaError_t e;
   if ((e = make_map(&mq, q, (int64_t)B * H * N, 128)) != cudaSuccess) return e;
   if ((e = make_map(&mk, k, (int64_t)B * H * Nk, 128)) != cudaSuccess) return e;
   if ((e = make_map(&mv, v, (int64_t)B * H * Nk, 128)) != cudaSuccess) return e;
+  if (T > 0) {
+    if ((e = make_map(&mkt, kt, (int64_t)B * H * T, 128)) != cudaSuccess) return e;
+    if ((e = make_map(&mvt, vt, (int64_t)B * H * T, 128)) != cudaSuccess) return e;
+  } else {
+    mkt = mk;   // never read without text keys
+    mvt = mv;
+  }
   TcParams prm{};
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.H = H;
+  prm.T = T;
   prm.da = DenseArgs{B, H, N, Nk, (N + 255) / 256};
   prm.num_units = B * H * prm.da.units_per_head;
   prm.o = static_cast<__nv_bfloat16*>(o);
-  return launch_tc<false>(mq, mk, mv, mk, mv, prm, s);   // no patch maps in dense mode
+  return launch_tc<false>(mq, mk, mv, mk, mv, mkt, mvt, prm, s);   // no patch maps in dense mode
 }
 
-cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v,
-                                  const PlanLayout& L, const void* plan, void* o, float* ws,
-                                  int H, float scale, cudaStream_t s) {
-  CUtensorMap mq, mk, mv;
+cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, const void* kt,
+                                  const void* vt, int T, const PlanLayout& L, const void* plan,
+                                  void* o, float* ws, int H, float scale, cudaStream_t s) {
+  CUtensorMap mq, mk, mv, mkt, mvt;
   cudaError_t e;
   const int64_t rows = L.B * H * L.N;
   if ((e = make_map(&mq, q, rows, 1)) != cudaSuccess) return e;
@@ -877,14 +901,22 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v,
   CUtensorMap mkp, mvp;
   if ((e = make_map_patch(&mkp, k, L.B * H * L.Hg, (int)L.Wg)) != cudaSuccess) return e;
   if ((e = make_map_patch(&mvp, v, L.B * H * L.Hg, (int)L.Wg)) != cudaSuccess) return e;
+  if (T > 0) {
+    if ((e = make_map(&mkt, kt, L.B * H * T, 128)) != cudaSuccess) return e;
+    if ((e = make_map(&mvt, vt, L.B * H * T, 128)) != cudaSuccess) return e;
+  } else {
+    mkt = mq;   // never read without text keys
+    mvt = mq;
+  }
   TcParams prm{};
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.H = H;
+  prm.T = T;
   prm.P = plan_view(L, const_cast<void*>(plan));
   prm.num_units = (int)(L.nitem_max * L.B * H);
   prm.ws = ws;
   prm.o = static_cast<__nv_bfloat16*>(o);
-  return launch_tc<true>(mq, mk, mv, mkp, mvp, prm, s);
+  return launch_tc<true>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
 }
 
 }  // namespace area

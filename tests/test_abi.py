@@ -65,6 +65,8 @@ def test_null_and_bad_arguments_rejected_on_host(area):
         (lambda: area.area_coarse_attn(fake, fake, fake, fake, 1, 1, 16, 4, 96, 1.0, 1), area.AREA_EUNSUPPORTED),
         (lambda: area.area_coarse_attn(fake, fake, fake, fake, 1, 1, 16, 4, 128, 1.0, 3), area.AREA_EUNSUPPORTED),
         (lambda: area.area_full_attn(None, fake, fake, fake, 1, 1, 16, 128, 1.0, 1), area.AREA_EINVAL),
+        (lambda: area.area_coarse_attn_text(fake, fake, fake, None, None, fake, 1, 1, 16, 4, 3, 128, 1.0, 1), area.AREA_EINVAL),
+        (lambda: area.area_coarse_attn_text(fake, fake, fake, fake, fake, fake, 1, 1, 16, 4, -1, 128, 1.0, 1), area.AREA_EINVAL),
         (lambda: area.area_dwt_detail(fake, 1, 16, fake, 1, 7, 8), area.AREA_EINVAL),
         (lambda: area.area_dwt_detail(fake, 1, 0, fake, 1, 8, 8), area.AREA_EINVAL),
         (lambda: area.area_dwt_detail(fake, 1, 4, fake, 1, 8, 8, 9), area.AREA_EINVAL),

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 from oracle import area_oracle as ora
-from workloads import CONFIGS
+from workloads import CONFIGS, make_text_kv
 import gpu_runner as gr
 
 pytestmark = pytest.mark.gpu
@@ -175,6 +175,73 @@ def test_window_attn(data, step):
     got = gr.to_host(o[:, heads][:, :, torch.from_numpy(rows).cuda()])
     gr.assert_close(got, want, cfg.dtype, f"window {cfg.name} step {step} w={w}")
     assert gr.area.area_kernel_error() == 0
+
+
+def test_coarse_attn_text(data):
+    # Phase I with text tokens: T + N/f^2 keys per query (T ragged: 77)
+    cfg, q, k, v = data.cfg, data.q, data.k, data.v
+    T = 5 if cfg.tiny else 77
+    kt, vt = make_text_kv(cfg, T)
+    dkt, dvt = gr.to_dev(kt, cfg.dtype), gr.to_dev(vt, cfg.dtype)
+    kp, vp = gr.gpu_pool(data.dk, data.dv, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, cfg.f, 0,
+                         cfg.dtype)
+    o = torch.empty_like(data.dq)
+    gr.area.area_coarse_attn_text(data.dq, kp, vp, dkt, dvt, o, cfg.B, cfg.H, cfg.N, cfg.Nk, T,
+                                  cfg.D, cfg.scale, gr.area_dtype(cfg.dtype))
+    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H - 1]
+    rows = np.arange(cfg.N) if cfg.tiny else gr.sample_rows(cfg.N, 256, seed=5)
+    okp = ora.pool_kv(k[:, heads], cfg.Hg, cfg.Wg, cfg.f)
+    ovp = ora.pool_kv(v[:, heads], cfg.Hg, cfg.Wg, cfg.f)
+    want = ora.coarse_attn(q[:, heads], okp, ovp, cfg.scale, rows=rows, kt=kt[:, heads],
+                           vt=vt[:, heads])
+    got = gr.to_host(o[:, heads][:, :, torch.from_numpy(rows).cuda()])
+    gr.assert_close(got, want, cfg.dtype, f"coarse+text {cfg.name}")
+
+
+@pytest.mark.parametrize("which", ["first", "last"])
+def test_window_attn_text(data, which):
+    cfg = data.cfg
+    step = 0 if which == "first" else len(cfg.schedule) - 1
+    if cfg.tiny and which == "last":
+        pytest.skip("one schedule step")
+    T = 5 if cfg.tiny else 77
+    kt, vt = make_text_kv(cfg, T)
+    dkt, dvt = gr.to_dev(kt, cfg.dtype), gr.to_dev(vt, cfg.dtype)
+    w = cfg.schedule[step]
+    energy = gr.gpu_dwt(data.dsrc, cfg.B, cfg.Hg, cfg.Wg, cfg.C, cfg.dtype)
+    pcfg, plan, nbytes = gr.gpu_plan(energy, cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G,
+                                     cfg.split_thr)
+    o = torch.empty_like(data.dq)
+    wsb = gr.area.area_window_attn_ws_bytes(pcfg, cfg.H, cfg.D)
+    ws = torch.empty(wsb // 4, dtype=torch.float32, device="cuda")
+    gr.area.area_window_attn_text(data.dq, data.dk, data.dv, dkt, dvt, T, pcfg, plan, nbytes, o,
+                                  ws, wsb, cfg.H, cfg.D, cfg.scale, gr.area_dtype(cfg.dtype))
+    E = ora.dwt_detail(data.src, cfg.Hg, cfg.Wg)
+    oplan = ora.window_plan(E[0], cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
+    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H - 1]
+    rows = np.arange(cfg.N) if cfg.tiny else gr.sample_rows(cfg.N, 192, seed=11 + step)
+    want = ora.window_attn(data.q, data.k, data.v, [oplan], cfg.scale, rows=rows, heads=heads,
+                           kt=kt, vt=vt)
+    got = gr.to_host(o[:, heads][:, :, torch.from_numpy(rows).cuda()])
+    gr.assert_close(got, want, cfg.dtype, f"window+text {cfg.name} step {step}")
+
+
+@pytest.mark.parametrize("N,Nk,T,D,dtype", [(300, 200, 1, 128, "bf16"), (257, 129, 300, 128, "bf16"),
+                                            (130, 70, 33, 64, "fp32"), (100, 64, 128, 64, "bf16")])
+def test_dense_attn_text_ragged(N, Nk, T, D, dtype):
+    rng = np.random.default_rng(N + T)
+    B, H = 2, 2
+    q = rng.standard_normal((B, H, N, D)).astype(np.float32)
+    k, v = (rng.standard_normal((B, H, Nk, D)).astype(np.float32) for _ in range(2))
+    kt, vt = (rng.standard_normal((B, H, T, D)).astype(np.float32) for _ in range(2))
+    d = [gr.to_dev(x, dtype) for x in (q, k, v, kt, vt)]
+    q, k, v, kt, vt = (gr.to_host(x) for x in d)
+    o = torch.empty_like(d[0])
+    scale = 1.0 / np.sqrt(D)
+    gr.area.area_coarse_attn_text(d[0], d[1], d[2], d[3], d[4], o, B, H, N, Nk, T, D, scale,
+                                  gr.area_dtype(dtype))
+    gr.assert_close(gr.to_host(o), ora.coarse_attn(q, k, v, scale, kt=kt, vt=vt), dtype,
+                    "dense+text")
 
 
 # ---------------------------------------------------------------------------

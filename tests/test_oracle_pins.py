@@ -429,3 +429,51 @@ def test_window_attention_rows_and_heads_subset():
     rows = np.array([0, 9, 33, 63])
     sub = ora.window_attn(q, k, v, [plan], 0.5, rows=rows, heads=[2])
     np.testing.assert_allclose(sub[0, 0], full[0, 2, rows], atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# text tokens (never pooled; every query attends to them)
+# --------------------------------------------------------------------------
+
+def test_coarse_with_text_matches_sdpa_over_concatenated_keys():
+    rng = np.random.default_rng(21)
+    Hg, Wg, f, D, T = 8, 6, 2, 4, 5
+    q, k, v = (rng.standard_normal((1, 2, Hg * Wg, D)) for _ in range(3))
+    kt, vt = (rng.standard_normal((1, 2, T, D)) for _ in range(2))
+    kp, vp = ora.pool_kv(k, Hg, Wg, f), ora.pool_kv(v, Hg, Wg, f)
+    got = ora.coarse_attn(q, kp, vp, 0.3, kt=kt, vt=vt)
+    kk = torch.cat([torch.from_numpy(kp), torch.from_numpy(kt)], dim=2)
+    vv = torch.cat([torch.from_numpy(vp), torch.from_numpy(vt)], dim=2)
+    assert kk.shape[2] == T + Hg * Wg // (f * f)          # T + N/f^2 keys per query
+    ref = torch.nn.functional.scaled_dot_product_attention(torch.from_numpy(q), kk, vv, scale=0.3)
+    np.testing.assert_allclose(got, ref.numpy(), atol=1e-12)
+    np.testing.assert_allclose(ora.coarse_attn(q, kp, vp, 0.3, kt=kt[:, :, :0], vt=vt[:, :, :0]),
+                               ora.coarse_attn(q, kp, vp, 0.3), atol=0)
+
+
+def test_window_with_text_equals_masked_attention_plus_text():
+    rng = np.random.default_rng(22)
+    Hg, Wg, T = 10, 12, 3
+    q, k, v = (rng.standard_normal((1, 2, Hg * Wg, 4)) for _ in range(3))
+    kt, vt = (rng.standard_normal((1, 2, T, 4)) for _ in range(2))
+    E = (rng.random((Hg // 2, Wg // 2)) ** 2).astype(np.float32)
+    plan = ora.window_plan(E, Hg, Wg, 5, 1, 4, 0.2)
+    got = ora.window_attn(q, k, v, [plan], 0.5, kt=kt, vt=vt)
+    # brute force: per window, keys = allowed image tokens (boolean mask) + all text keys
+    N = Hg * Wg
+    num = np.zeros((2, N, 4))
+    den = np.zeros(N)
+    for i, (y0, x0, hy, wx) in enumerate(plan.windows):
+        allowed = np.zeros(N, dtype=bool)
+        allowed[ora.window_kv_tokens(plan, i)] = True
+        for y in range(y0, y0 + hy):
+            for x in range(x0, x0 + wx):
+                t = y * Wg + x
+                w = min(y - y0 + 1, y0 + hy - y) * min(x - x0 + 1, x0 + wx - x)
+                den[t] += w
+                for h in range(2):
+                    s_img = np.where(allowed, 0.5 * k[0, h] @ q[0, h, t], -np.inf)
+                    s_all = np.concatenate([s_img, 0.5 * kt[0, h] @ q[0, h, t]])
+                    p = np.exp(s_all - s_all.max())
+                    num[h, t] += w * (p / p.sum()) @ np.concatenate([v[0, h], vt[0, h]])
+    np.testing.assert_allclose(got[0], num / den[None, :, None], atol=1e-12)

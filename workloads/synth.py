@@ -120,3 +120,18 @@ def make_detail_source(cfg: AreaConfig) -> np.ndarray:
     """Detail source, float32 [B, N, C] channels-last, storage-exact."""
     t = _field(cfg, cfg.seeds[3], cfg.B, cfg.C)                    # [B, Hg, Wg, C]
     return t.reshape(cfg.B, cfg.N, cfg.C)
+
+
+def make_text_kv(cfg: AreaConfig, T: int, seed: int = 5):
+    """Synthetic text-token keys and values, float32 [B, H, T, D] each.
+
+    Text tokens have no grid: iid N(0, 1) per element (bf16-rounded for the
+    bf16 configs).  They stand in for the prompt tokens of a joint-attention
+    transformer; no real prompt is used.
+    """
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(2):
+        t = rng.standard_normal((cfg.B, cfg.H, T, cfg.D)).astype(np.float32)
+        out.append(round_to_bf16(t) if cfg.dtype == "bf16" else t)
+    return tuple(out)
