@@ -444,6 +444,24 @@ def run_area(args):
     win_ms_steps = np.array(per["window_attn"]).reshape(args.steps, -1).mean(axis=0).tolist()
     kerr = area.area_kernel_error()
 
+    # ---- the same step captured once in a CUDA graph and replayed
+    graph_ms = None
+    if not args.no_graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            st.run()
+        g.replay()
+        torch.cuda.synchronize()
+        ge0, ge1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ge0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                g.replay()
+        ge1.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = ge0.elapsed_time(ge1) / args.steps
+        del g
+
     # ---- full attention: the speedup denominator (same inputs)
     o_full = torch.empty_like(q)
     fe0, fe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -457,6 +475,37 @@ def run_area(args):
     torch.cuda.synchronize()
     full_ms = fe0.elapsed_time(fe1) / args.full_reps
     del o_full
+
+    # ---- Phase I with the pages' pooling ramp (f0 -> 2 over the 8 steps),
+    # measured once after the timed region (the configs' step uses a fixed f)
+    from step_adaptive_sparse_b200 import schedule
+    ramp = schedule.pool_ramp(cfg.f, 2, st.n_phase1, cfg.Hg, cfg.Wg)
+    nk_max = (cfg.Hg // min(ramp)) * (cfg.Wg // min(ramp))
+    kp_r = torch.empty((cfg.B, cfg.H, nk_max, cfg.D), dtype=q.dtype, device=dev)
+    vp_r = torch.empty_like(kp_r)
+    o_r = torch.empty_like(q)
+    ramp_ms, ramp_tf = [], []
+    with torch.cuda.stream(stream):
+        for rep in range(2):                       # warm-up pass, then the timed pass
+            for f in ramp:
+                nk = (cfg.Hg // f) * (cfg.Wg // f)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                area.area_pool_kv(k, v, kp_r, vp_r, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, f,
+                                  area.AREA_POOL_MEAN, st.dt, stream)
+                area.area_coarse_attn(q, kp_r, vp_r, o_r, cfg.B, cfg.H, cfg.N, nk, cfg.D,
+                                      cfg.scale, st.dt, stream)
+                b.record(stream)
+                if rep:
+                    ramp_ms.append((a, b, 4.0 * cfg.B * cfg.H * cfg.N * nk * cfg.D))
+    torch.cuda.synchronize()
+    ramp_out = {"ramp": ramp, "ms": [], "tflops": []}
+    for a, b, fl in ramp_ms:
+        t = a.elapsed_time(b)
+        ramp_out["ms"].append(t)
+        ramp_out["tflops"].append(fl / (t * 1e-3) / 1e12)
+    ramp_out["total_ms"] = float(sum(ramp_out["ms"]))
+    del kp_r, vp_r, o_r
 
     # ---- end to end through the C-ABI from pinned host buffers.  Each step
     # copies its inputs host->device and its output device->host; two device
@@ -565,6 +614,11 @@ def run_area(args):
                              "dwt_detail": dwt_bytes(cfg) / (dwt_ms * 1e-3) / 1e9,
                              "hbm_peak_gbs": peaks["hbm_gbs"]},
             "split_fraction_by_step": splits,
+            "phase1_pooling_ramp": ramp_out,
+            "graph_replay": None if graph_ms is None else {
+                "ms_per_step": graph_ms,
+                "value": step_flops / (graph_ms * 1e-3) / 1e12,
+                "note": "the same step captured once in a CUDA graph (192 launches) and replayed"},
             "speedup_vs_full_attention": (full_ms * (n1 + len(cfg.schedule))) / ms_step,
         }
         print(json.dumps(line), flush=True)
@@ -583,6 +637,7 @@ def main(argv=None):
     ap.add_argument("--full-reps", type=int, default=2)
     ap.add_argument("--ref-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay leg")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)

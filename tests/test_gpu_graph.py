@@ -1,0 +1,73 @@
+"""A whole AReA schedule step captured in one CUDA graph and replayed.
+
+Every libarea call is asynchronous on the caller's stream and never reads the
+device from the host (the plan stays on the device), so a step of both phases
+can be captured once and replayed: the replay must reproduce the eager
+results (window outputs up to the order of fp32 additions in overlaps).
+"""
+import numpy as np
+import pytest
+import torch
+
+import step_adaptive_sparse_b200 as area
+from workloads import CONFIGS, make_detail_source, make_qkv
+
+pytestmark = pytest.mark.gpu
+
+
+def _step(bufs, cfg, dt, stream):
+    q, k, v, src, kp, vp, o1, o2, energy, plans, ws, wsb = bufs
+    area.area_pool_kv(k, v, kp, vp, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, cfg.f,
+                      area.AREA_POOL_MEAN, dt, stream)
+    area.area_coarse_attn(q, kp, vp, o1, cfg.B, cfg.H, cfg.N, cfg.Nk, cfg.D, cfg.scale, dt, stream)
+    for (pc, plan, nb), o in zip(plans, o2):
+        area.area_dwt_detail(src, dt, cfg.C, energy, cfg.B, cfg.Hg, cfg.Wg, area.AREA_DETAIL_HH,
+                             stream)
+        area.area_window_plan(energy, pc, plan, nb, stream)
+        area.area_window_attn(q, k, v, pc, plan, nb, o, ws, wsb, cfg.H, cfg.D, cfg.scale, dt,
+                              stream)
+
+
+@pytest.mark.parametrize("name", ["tiny", "flux2048"])
+def test_schedule_step_graph_replay_matches_eager(name):
+    cfg = CONFIGS[name]
+    dt = area.AREA_DTYPE_BF16 if cfg.dtype == "bf16" else area.AREA_DTYPE_F32
+    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    q, k, v = (torch.from_numpy(x).cuda().to(tdt) for x in make_qkv(cfg))
+    src = torch.from_numpy(make_detail_source(cfg)).cuda().to(tdt)
+    kp = torch.empty((cfg.B, cfg.H, cfg.Nk, cfg.D), dtype=tdt, device="cuda")
+    vp = torch.empty_like(kp)
+    energy = torch.empty((cfg.B, cfg.Hg // 2, cfg.Wg // 2), dtype=torch.float32, device="cuda")
+    plans, wsb = [], 0
+    for w in cfg.schedule:
+        pc = area.make_cfg(cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
+        nb = area.area_window_plan_bytes(pc)
+        plans.append((pc, torch.empty(nb, dtype=torch.uint8, device="cuda"), nb))
+        wsb = max(wsb, area.area_window_attn_ws_bytes(pc, cfg.H, cfg.D))
+    ws = torch.empty(wsb // 4, dtype=torch.float32, device="cuda")
+    o1 = torch.empty_like(q)
+    o2 = [torch.empty_like(q) for _ in cfg.schedule]
+    bufs = (q, k, v, src, kp, vp, o1, o2, energy, plans, ws, wsb)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        _step(bufs, cfg, dt, stream)            # eager, also the capture warm-up
+    torch.cuda.synchronize()
+    ref1 = o1.clone()
+    ref2 = [o.clone() for o in o2]
+    ref_plans = [p.clone() for _, p, _ in plans]
+    for t in [o1] + o2 + [p for _, p, _ in plans]:
+        t.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        _step(bufs, cfg, dt, stream)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(o1, ref1)
+    for (_, p, _), rp in zip(plans, ref_plans):
+        assert torch.equal(p[:256], rp[:256])
+    tol = 2e-3 if cfg.dtype == "bf16" else 1e-6
+    for o, r in zip(o2, ref2):
+        assert (o.float() - r.float()).abs().max().item() <= tol
+    assert area.area_kernel_error() == 0
+    del g

@@ -177,6 +177,24 @@ def test_window_attn(data, step):
     assert gr.area.area_kernel_error() == 0
 
 
+def test_coarse_attn_ramp_floor(data):
+    # Phase I at the floor of the pooling ramp (f = 2): 4x-16x more keys than
+    # the configs' fixed factor (16384 keys at 4096^2)
+    cfg, q, k, v = data.cfg, data.q, data.k, data.v
+    if cfg.f == 2:
+        pytest.skip("the config already pools with f = 2")
+    f = 2
+    Nk = (cfg.Hg // f) * (cfg.Wg // f)
+    kp, vp = gr.gpu_pool(data.dk, data.dv, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, f, 0, cfg.dtype)
+    o = gr.gpu_dense(data.dq, kp, vp, cfg.B, cfg.H, cfg.N, Nk, cfg.D, cfg.scale, cfg.dtype)
+    heads = [0, cfg.H - 1]
+    rows = gr.sample_rows(cfg.N, 128, seed=9)
+    want = ora.coarse_attn(q[:, heads], ora.pool_kv(k[:, heads], cfg.Hg, cfg.Wg, f),
+                           ora.pool_kv(v[:, heads], cfg.Hg, cfg.Wg, f), cfg.scale, rows=rows)
+    got = gr.to_host(o[:, heads][:, :, torch.from_numpy(rows).cuda()])
+    gr.assert_close(got, want, cfg.dtype, f"coarse f=2 {cfg.name}")
+
+
 def test_coarse_attn_text(data):
     # Phase I with text tokens: T + N/f^2 keys per query (T ragged: 77)
     cfg, q, k, v = data.cfg, data.q, data.k, data.v
