@@ -150,8 +150,17 @@ int area_full_attn(const void* q, const void* k, const void* v, void* o,
 int area_dwt_detail(const void* src, int src_dtype, int C, float* energy,
                     int B, int Hg, int Wg, int mode, cudaStream_t stream);
 
-/* Configuration of one Phase II step.  jitter_seed must be 0 (no border
- * shift).  split_thr is the mean-energy bound below which a window splits. */
+/* Configuration of one Phase II step.  split_thr is the mean-energy bound
+ * below which a window splits.  jitter_seed = 0 gives the fixed plan; any
+ * other value turns on the seeded randomness of [ai] Phase II and [blog]
+ * README notes (the seed sets border jitter and Halo widths):
+ *   - border shift s in [0, w_e) per axis (SplitMix64 output number 2^32 and
+ *     2^32 + 1 of the sequence seeded with jitter_seed, mod w_e): the base
+ *     tiling is the even tiling of the extended axis [-s, L), clipped to
+ *     [0, L);
+ *   - Halo width per final window i of batch element b: output number
+ *     2 * 2^32 + b * 2^20 + i of the same sequence, mod (halo + 1).
+ * Pass a different seed per denoising step to move the seams. */
 typedef struct area_plan_cfg {
   int B;            /* batch elements (one plan each)                        */
   int Hg, Wg;       /* token grid                                            */
@@ -159,20 +168,22 @@ typedef struct area_plan_cfg {
   int halo;         /* Halo width h >= 0                                     */
   int G;            /* global-KV tokens per window, 0 <= G <= 4096           */
   float split_thr;  /* split when score < fl32(split_thr * hy * wx)          */
-  unsigned long long jitter_seed;   /* must be 0                            */
+  unsigned long long jitter_seed;   /* 0: no jitter, fixed Halo             */
 } area_plan_cfg;
 
 /*
  * Plan buffer layout (device memory, written by area_window_plan).  The
  * first 256 bytes hold an int64 header; every section starts 256-byte
  * aligned at the byte offset stored in the header.  Windows are indexed per
- * batch element b in [0, B); "nb" = base windows per element, "nw" = 4*nb
- * (room for a full split).
+ * batch element b in [0, B); "nb" = base-window capacity per element (room
+ * for one extra window per axis under a border shift), "nw" = 4*nb.
  *   header[0]  = AREA_PLAN_MAGIC        header[1] = AREA_PLAN_VERSION
  *   header[2..8] = B, Hg, Wg, w, halo, G, nb
  *   header[9]  = nw
  *   header[10+s] = byte offset of section s (AREA_PLAN_SEC_*)
- *   header[25] = work-item capacity per element ("ni"), header[26] = N
+ *   header[25] = work-item capacity per element ("ni"), header[26] = N,
+ *   header[27] = base windows of this plan (<= nb; fewer than the capacity
+ *   when a border shift is drawn), header[28..29] = border shift (sy, sx)
  * Sections:
  *   BASE    int32 [B][nb][4]   base windows (y0, x0, hy, wx), row-major
  *   SCORE   f32   [B][nb]      sum of token energy over the base window
@@ -212,7 +223,7 @@ typedef struct area_plan_cfg {
 
 /*
  * area_window_plan_bytes -- size of the plan buffer for cfg (host only).
- * Errors: AREA_EINVAL (null, bad sizes, jitter_seed != 0, G > 4096).
+ * Errors: AREA_EINVAL (null, bad sizes, G > 4096, B > 2048).
  */
 int area_window_plan_bytes(const area_plan_cfg* cfg, size_t* plan_bytes);
 

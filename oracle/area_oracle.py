@@ -201,6 +201,70 @@ def tile_starts(L: int, w: int) -> Tuple[List[int], int]:
     return [(i * (L - we)) // (n - 1) for i in range(n)], we
 
 
+# ----------------------------------------------------------------------------
+# Seeded randomness: border jitter and Halo widths
+# ----------------------------------------------------------------------------
+
+_GAMMA = 0x9E3779B97F4A7C15
+_M64 = (1 << 64) - 1
+STREAM_JITTER, STREAM_HALO = 1, 2
+
+
+def splitmix64(state: int) -> int:
+    """One SplitMix64 step (Steele, Lea and Flood, "Fast splittable pseudorandom
+    number generators", OOPSLA 2014; finaliser constants of Vigna's reference
+    version): advance the state by the golden-ratio increment, then mix."""
+    z = (state + _GAMMA) & _M64
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _M64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _M64
+    return z ^ (z >> 31)
+
+
+def counter_random(seed: int, stream: int, index: int) -> int:
+    """Counter-based 64-bit draw: output number (stream * 2^32 + index) of the
+    SplitMix64 sequence seeded with `seed` (stream 0, index 0 is its first
+    output)."""
+    return splitmix64((seed + _GAMMA * ((stream << 32) + index)) & _M64)
+
+
+def jitter_shifts(seed: int, Hg: int, Wg: int, w: int) -> Tuple[int, int]:
+    """Border shift (sy, sx) of one plan ([ai] Phase II: window boundaries are
+    randomly shifted across steps so seams never form at fixed places).
+    Reading: s in [0, w_e) per axis, drawn from the seed; 0 when the window
+    spans the axis or the seed is 0."""
+    if seed == 0:
+        return 0, 0
+    hy, wx = min(w, Hg), min(w, Wg)
+    sy = counter_random(seed, STREAM_JITTER, 0) % hy if hy < Hg else 0
+    sx = counter_random(seed, STREAM_JITTER, 1) % wx if wx < Wg else 0
+    return sy, sx
+
+
+def tile_windows(L: int, w: int, shift: int = 0) -> List[Tuple[int, int]]:
+    """(start, size) of the base windows along one axis.
+
+    Reading of the border shift: the even tiling (tile_starts) of the extended
+    axis [-shift, L) with side w_e = min(w, L), clipped back to [0, L).
+    shift = 0 gives tile_starts exactly."""
+    we = min(w, L)
+    starts, _ = tile_starts(L + shift, we)
+    out = []
+    for s0 in starts:
+        a = s0 - shift
+        lo, hi = max(0, a), min(L, a + we)
+        out.append((lo, hi - lo))
+    return out
+
+
+def halo_width(seed: int, halo: int, b: int, i: int) -> int:
+    """Halo width of final window i of batch element b: fixed `halo` when the
+    seed is 0, else a draw in [0, halo] ([blog] README notes: the seed sets
+    the Halo widths, up to delta_max)."""
+    if seed == 0:
+        return halo
+    return counter_random(seed, STREAM_HALO, (b << 20) + i) % (halo + 1)
+
+
 def window_score(Etok: np.ndarray, y0: int, x0: int, hy: int, wx: int) -> np.float32:
     """Sum of token energies over a window, in a fixed float32 order.
 
@@ -276,15 +340,16 @@ class Plan:
 
 
 def window_plan(E: np.ndarray, Hg: int, Wg: int, w: int, halo: int, G: int,
-                thr: float) -> Plan:
+                thr: float, seed: int = 0, b: int = 0) -> Plan:
     """Phase II plan of one batch element from its detail map E [Hg/2, Wg/2].
 
     Steps in the pages' order ([ai] Phase II, [blog] Fase II):
-      1. base tiling (tile_starts per axis; windows row-major, y then x);
+      1. base tiling (tile_windows per axis, shifted by jitter_shifts(seed);
+         windows row-major, y then x);
       2. detail score per base window (window_score);
       3. windows over smooth regions (score < split_threshold) are split
          into four quadrants (one level; sides < 2 never split);
-      4. Halo rectangle per final window (halo_rect);
+      4. Halo rectangle per final window (halo_rect; width halo_width(seed));
       5. global-KV bridge: the first G_W = min(G, N - |ext|) tokens of
          global_rank that lie outside the Halo rectangle, in rank order (the
          pages select by deviation from the global mean key; the rule used
@@ -293,11 +358,12 @@ def window_plan(E: np.ndarray, Hg: int, Wg: int, w: int, halo: int, G: int,
     """
     Etok = token_energy(E)
     assert Etok.shape == (Hg, Wg)
-    ys, hy = tile_starts(Hg, w)
-    xs, wx = tile_starts(Wg, w)
+    sy, sx = jitter_shifts(seed, Hg, Wg, w)
+    ywin = tile_windows(Hg, w, sy)
+    xwin = tile_windows(Wg, w, sx)
     base, score, split, wins, parent = [], [], [], [], []
-    for y0 in ys:
-        for x0 in xs:
+    for (y0, hy) in ywin:
+        for (x0, wx) in xwin:
             bi = len(base)
             base.append((y0, x0, hy, wx))
             s = window_score(Etok, y0, x0, hy, wx)
@@ -318,7 +384,7 @@ def window_plan(E: np.ndarray, Hg: int, Wg: int, w: int, halo: int, G: int,
     gidx = np.full((len(wins), G), -1, dtype=np.int32)
     wsum = np.zeros((Hg, Wg), dtype=F32)
     for i, (y0, x0, h_, w_) in enumerate(wins):
-        e = halo_rect(y0, x0, h_, w_, halo, Hg, Wg)
+        e = halo_rect(y0, x0, h_, w_, halo_width(seed, halo, b, i), Hg, Wg)
         ext.append(e)
         ey0, ex0, ehy, ewx = e
         gw = min(G, N - ehy * ewx)

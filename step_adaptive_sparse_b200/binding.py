@@ -226,10 +226,13 @@ def parse_plan(buf: np.ndarray) -> dict:
 
     nitem = sec("NITEM", np.int32, B + 1)
     nitem_max = int(hdr[10 + len(SECTIONS)])
-    out = {"B": B, "Hg": Hg, "Wg": Wg, "w": w, "halo": halo, "G": G, "nb": nb, "nw": nw,
-           "base": sec("BASE", np.int32, B * nb * 4).reshape(B, nb, 4),
-           "score": sec("SCORE", np.float32, B * nb).reshape(B, nb),
-           "split": sec("SPLIT", np.uint8, B * nb).reshape(B, nb),
+    nb_act = int(hdr[12 + len(SECTIONS)])          # base windows of this plan
+    sy, sx = int(hdr[13 + len(SECTIONS)]), int(hdr[14 + len(SECTIONS)])
+    out = {"B": B, "Hg": Hg, "Wg": Wg, "w": w, "halo": halo, "G": G, "nb": nb_act,
+           "nb_cap": nb, "nw": nw, "shift": (sy, sx),
+           "base": sec("BASE", np.int32, B * nb * 4).reshape(B, nb, 4)[:, :nb_act],
+           "score": sec("SCORE", np.float32, B * nb).reshape(B, nb)[:, :nb_act],
+           "split": sec("SPLIT", np.uint8, B * nb).reshape(B, nb)[:, :nb_act],
            "nwin": sec("NWIN", np.int32, B),
            "win": sec("WIN", np.int32, B * nw * 4).reshape(B, nw, 4),
            "parent": sec("PARENT", np.int32, B * nw).reshape(B, nw),

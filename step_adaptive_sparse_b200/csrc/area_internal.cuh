@@ -18,8 +18,11 @@ constexpr int kMaxGrid = 1 << 15;    // largest grid side accepted (tokens)
 // ---------------------------------------------------------------------------
 struct PlanLayout {
   int64_t B, Hg, Wg, w, halo, G;
-  int64_t nby, nbx, hy, wx;     // base tiling: counts and window sides
-  int64_t nb, nw;               // base windows / final-window capacity per element
+  uint64_t seed;                // border jitter and Halo widths (0: none)
+  int64_t sy, sx;               // border shift of this plan per axis
+  int64_t nby, nbx, hy, wx;     // base tiling: counts (this plan) and window sides
+  int64_t nb_cap;               // base-window capacity per element (section strides)
+  int64_t nb, nw;               // base windows of this plan / final-window capacity
   int64_t nitem_max;            // work-item capacity per element
   int64_t N;                    // tokens per element
   int64_t ntile_sort;           // 256-element tiles of the radix sort
@@ -34,7 +37,9 @@ int plan_layout(const area_plan_cfg* cfg, PlanLayout* L);
 // Device view of a plan (pointers into the plan buffer).
 struct PlanView {
   int B, Hg, Wg, w, halo, G;
-  int nby, nbx, hy, wx, nb, nw, nitem_max, N;
+  unsigned long long seed;
+  int sy, sx;
+  int nby, nbx, hy, wx, nb, nb_cap, nw, nitem_max, N;
   int4* base;          // [B][nb]
   float* score;        // [B][nb]
   uint8_t* split;      // [B][nb]
@@ -69,6 +74,32 @@ __device__ __forceinline__ void store_from_float(__nv_bfloat16* p, int64_t i, fl
 __host__ __device__ __forceinline__ int tile_start(int i, int n, int L, int we) {
   return n > 1 ? (int)(((int64_t)i * (L - we)) / (n - 1)) : 0;
 }
+
+// Window i of an axis of length L under a border shift: the even tiling of
+// the extended axis [-shift, L) (n windows of side we), clipped to [0, L).
+__host__ __device__ __forceinline__ void axis_window(int i, int n, int L, int we, int shift,
+                                                     int* start, int* size) {
+  const int a = tile_start(i, n, L + shift, we) - shift;
+  const int lo = a > 0 ? a : 0;
+  const int hi = a + we < L ? a + we : L;
+  *start = lo;
+  *size = hi - lo;
+}
+
+// Counter-based draws: output number (stream * 2^32 + index) of the SplitMix64
+// sequence (Steele, Lea, Flood 2014) seeded with `seed`.
+__host__ __device__ __forceinline__ unsigned long long splitmix64(unsigned long long s) {
+  unsigned long long z = s + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+__host__ __device__ __forceinline__ unsigned long long counter_random(unsigned long long seed,
+                                                                     unsigned long long stream,
+                                                                     unsigned long long index) {
+  return splitmix64(seed + 0x9E3779B97F4A7C15ull * ((stream << 32) + index));
+}
+constexpr unsigned long long kStreamJitter = 1, kStreamHalo = 2;
 
 // ---------------------------------------------------------------------------
 // launchers (return cudaError_t of the launch)

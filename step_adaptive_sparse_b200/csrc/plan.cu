@@ -26,7 +26,7 @@ int plan_layout(const area_plan_cfg* cfg, PlanLayout* L) {
   if (!cfg || !L) return AREA_EINVAL;
   if (cfg->B < 1 || cfg->Hg < 2 || cfg->Wg < 2 || (cfg->Hg & 1) || (cfg->Wg & 1) ||
       cfg->Hg > kMaxGrid || cfg->Wg > kMaxGrid || cfg->w < 1 || cfg->halo < 0 || cfg->G < 0 ||
-      cfg->G > kMaxG || cfg->jitter_seed != 0)
+      cfg->G > kMaxG || cfg->B > (1 << 11))
     return AREA_EINVAL;
   const int64_t N = (int64_t)cfg->Hg * cfg->Wg;
   if (N > (int64_t(1) << 26)) return AREA_EINVAL;
@@ -34,15 +34,29 @@ int plan_layout(const area_plan_cfg* cfg, PlanLayout* L) {
   L->G = cfg->G; L->N = N;
   L->hy = cfg->w < cfg->Hg ? cfg->w : cfg->Hg;
   L->wx = cfg->w < cfg->Wg ? cfg->w : cfg->Wg;
-  L->nby = (cfg->Hg + L->hy - 1) / L->hy;
-  L->nbx = (cfg->Wg + L->wx - 1) / L->wx;
+  L->seed = cfg->jitter_seed;
+  // border shift of this plan (0 without a seed or when the window spans the axis)
+  L->sy = (L->seed && L->hy < L->Hg)
+              ? (int64_t)(counter_random(L->seed, kStreamJitter, 0) % (unsigned long long)L->hy)
+              : 0;
+  L->sx = (L->seed && L->wx < L->Wg)
+              ? (int64_t)(counter_random(L->seed, kStreamJitter, 1) % (unsigned long long)L->wx)
+              : 0;
+  L->nby = (cfg->Hg + L->sy + L->hy - 1) / L->hy;
+  L->nbx = (cfg->Wg + L->sx + L->wx - 1) / L->wx;
   L->nb = L->nby * L->nbx;
-  L->nw = 4 * L->nb;
-  L->nitem_max = L->nb * ((L->hy * L->wx + kQTile - 1) / kQTile + 3);
+  // capacity covers every shift in [0, side): one more window per axis at most
+  const int64_t cy = L->seed && L->hy < L->Hg ? (cfg->Hg + 2 * L->hy - 2) / L->hy
+                                              : (cfg->Hg + L->hy - 1) / L->hy;
+  const int64_t cx = L->seed && L->wx < L->Wg ? (cfg->Wg + 2 * L->wx - 2) / L->wx
+                                              : (cfg->Wg + L->wx - 1) / L->wx;
+  L->nb_cap = cy * cx;
+  L->nw = 4 * L->nb_cap;
+  L->nitem_max = L->nb_cap * ((L->hy * L->wx + kQTile - 1) / kQTile + 3);
   L->ntile_sort = (N + kSortTile - 1) / kSortTile;
   const int64_t B = L->B;
   const int64_t sizes[AREA_PLAN_NSEC] = {
-      B * L->nb * 16, B * L->nb * 4, B * L->nb, B * 4,
+      B * L->nb_cap * 16, B * L->nb_cap * 4, B * L->nb_cap, B * 4,
       B * L->nw * 16, B * L->nw * 4, B * L->nw * 16, B * L->nw * 4,
       B * L->nw * L->G * 4, B * N * 4, B * N * 4, (B + 1) * 4,
       B * L->nitem_max * 8, B * N * 4, 0};
@@ -67,6 +81,7 @@ PlanView plan_view(const PlanLayout& L, void* plan) {
   PlanView v;
   v.B = (int)L.B; v.Hg = (int)L.Hg; v.Wg = (int)L.Wg; v.w = (int)L.w; v.halo = (int)L.halo;
   v.G = (int)L.G; v.nby = (int)L.nby; v.nbx = (int)L.nbx; v.hy = (int)L.hy; v.wx = (int)L.wx;
+  v.seed = L.seed; v.sy = (int)L.sy; v.sx = (int)L.sx; v.nb_cap = (int)L.nb_cap;
   v.nb = (int)L.nb; v.nw = (int)L.nw; v.nitem_max = (int)L.nitem_max; v.N = (int)L.N;
   v.base = reinterpret_cast<int4*>(p + L.off[AREA_PLAN_SEC_BASE]);
   v.score = reinterpret_cast<float*>(p + L.off[AREA_PLAN_SEC_SCORE]);
@@ -133,26 +148,28 @@ __device__ int block_exclusive_scan(int x, int* total) {
 __global__ void __launch_bounds__(256) plan_base_kernel(const float* __restrict__ E, PlanView P,
                                                        float thr) {
   extern __shared__ float s_rows[];
-  const int b = blockIdx.x / P.nb, bi = blockIdx.x % P.nb;
+  const int b = blockIdx.x / P.nb_cap, bi = blockIdx.x % P.nb_cap;
+  if (bi >= P.nb) return;
   const int iy = bi / P.nbx, ix = bi % P.nbx;
-  const int y0 = tile_start(iy, P.nby, P.Hg, P.hy);
-  const int x0 = tile_start(ix, P.nbx, P.Wg, P.wx);
+  int y0, hy, x0, wx;
+  axis_window(iy, P.nby, P.Hg, P.hy, P.sy, &y0, &hy);
+  axis_window(ix, P.nbx, P.Wg, P.wx, P.sx, &x0, &wx);
   const int Wc = P.Wg / 2;
   const float* Eb = E + (int64_t)b * (P.Hg / 2) * Wc;
-  for (int y = threadIdx.x; y < P.hy; y += blockDim.x) {
+  for (int y = threadIdx.x; y < hy; y += blockDim.x) {
     const float* er = Eb + (int64_t)((y0 + y) >> 1) * Wc;
     float acc = 0.f;
-    for (int x = x0; x < x0 + P.wx; ++x) acc = __fadd_rn(acc, er[x >> 1]);
+    for (int x = x0; x < x0 + wx; ++x) acc = __fadd_rn(acc, er[x >> 1]);
     s_rows[y] = acc;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
     float S = 0.f;
-    for (int y = 0; y < P.hy; ++y) S = __fadd_rn(S, s_rows[y]);
-    const float T = __fmul_rn(thr, (float)(P.hy * P.wx));
-    const bool split = P.hy >= 2 && P.wx >= 2 && S < T;
-    const int64_t o = (int64_t)b * P.nb + bi;
-    P.base[o] = make_int4(y0, x0, P.hy, P.wx);
+    for (int y = 0; y < hy; ++y) S = __fadd_rn(S, s_rows[y]);
+    const float T = __fmul_rn(thr, (float)(hy * wx));
+    const bool split = hy >= 2 && wx >= 2 && S < T;
+    const int64_t o = (int64_t)b * P.nb_cap + bi;
+    P.base[o] = make_int4(y0, x0, hy, wx);
     P.score[o] = S;
     P.split[o] = split ? 1 : 0;
   }
@@ -167,8 +184,8 @@ __device__ __forceinline__ int4 halo_rect(int4 w, int h, int Hg, int Wg) {
 // Final windows, Halo rectangles, G_W and the work list of one batch element.
 __global__ void __launch_bounds__(1024) plan_windows_kernel(PlanView P) {
   const int b = blockIdx.x;
-  const int4* base = P.base + (int64_t)b * P.nb;
-  const uint8_t* split = P.split + (int64_t)b * P.nb;
+  const int4* base = P.base + (int64_t)b * P.nb_cap;
+  const uint8_t* split = P.split + (int64_t)b * P.nb_cap;
   int4* win = P.win + (int64_t)b * P.nw;
   int* parent = P.parent + (int64_t)b * P.nw;
   int4* ext = P.ext + (int64_t)b * P.nw;
@@ -195,7 +212,12 @@ __global__ void __launch_bounds__(1024) plan_windows_kernel(PlanView P) {
         q[0] = bw;
       }
       for (int j = 0; j < nq; ++j) {
-        const int4 e = halo_rect(q[j], P.halo, P.Hg, P.Wg);
+        // Halo width: fixed, or drawn in [0, halo] per final window with a seed
+        const int h = P.seed ? (int)(counter_random(P.seed, kStreamHalo,
+                                                    ((unsigned long long)b << 20) + at + j) %
+                                     (unsigned long long)(P.halo + 1))
+                             : P.halo;
+        const int4 e = halo_rect(q[j], h, P.Hg, P.Wg);
         const int64_t rest = (int64_t)P.N - (int64_t)e.z * e.w;
         win[at + j] = q[j];
         parent[at + j] = i;
@@ -352,16 +374,18 @@ __global__ void __launch_bounds__(256) plan_wsum_kernel(PlanView P) {
   const int y = t / P.Wg, x = t % P.Wg;
   int total = 0, count = 0;
   for (int iy = 0; iy < P.nby; ++iy) {
-    const int y0 = tile_start(iy, P.nby, P.Hg, P.hy);
-    if (y < y0 || y >= y0 + P.hy) continue;
+    int y0, hy;
+    axis_window(iy, P.nby, P.Hg, P.hy, P.sy, &y0, &hy);
+    if (y < y0 || y >= y0 + hy) continue;
     for (int ix = 0; ix < P.nbx; ++ix) {
-      const int x0 = tile_start(ix, P.nbx, P.Wg, P.wx);
-      if (x < x0 || x >= x0 + P.wx) continue;
-      int qy0 = y0, qhy = P.hy, qx0 = x0, qwx = P.wx;
-      if (P.split[(int64_t)b * P.nb + iy * P.nbx + ix]) {
-        const int ht = P.hy / 2, wl = P.wx / 2;
-        if (y < y0 + ht) { qhy = ht; } else { qy0 = y0 + ht; qhy = P.hy - ht; }
-        if (x < x0 + wl) { qwx = wl; } else { qx0 = x0 + wl; qwx = P.wx - wl; }
+      int x0, wx;
+      axis_window(ix, P.nbx, P.Wg, P.wx, P.sx, &x0, &wx);
+      if (x < x0 || x >= x0 + wx) continue;
+      int qy0 = y0, qhy = hy, qx0 = x0, qwx = wx;
+      if (P.split[(int64_t)b * P.nb_cap + iy * P.nbx + ix]) {
+        const int ht = hy / 2, wl = wx / 2;
+        if (y < y0 + ht) { qhy = ht; } else { qy0 = y0 + ht; qhy = hy - ht; }
+        if (x < x0 + wl) { qwx = wl; } else { qx0 = x0 + wl; qwx = wx - wl; }
       }
       total += min(y - qy0 + 1, qy0 + qhy - y) * min(x - qx0 + 1, qx0 + qwx - x);
       ++count;
@@ -380,10 +404,13 @@ cudaError_t launch_window_plan(const float* energy, const area_plan_cfg* cfg,
   HeaderArgs h = {};
   h.v[0] = AREA_PLAN_MAGIC; h.v[1] = AREA_PLAN_VERSION;
   h.v[2] = L.B; h.v[3] = L.Hg; h.v[4] = L.Wg; h.v[5] = L.w; h.v[6] = L.halo; h.v[7] = L.G;
-  h.v[8] = L.nb; h.v[9] = L.nw;
+  h.v[8] = L.nb_cap; h.v[9] = L.nw;
   for (int i = 0; i < AREA_PLAN_NSEC; ++i) h.v[10 + i] = L.off[i];
   h.v[10 + AREA_PLAN_NSEC] = L.nitem_max;
   h.v[11 + AREA_PLAN_NSEC] = L.N;
+  h.v[12 + AREA_PLAN_NSEC] = L.nb;
+  h.v[13 + AREA_PLAN_NSEC] = L.sy;
+  h.v[14 + AREA_PLAN_NSEC] = L.sx;
   plan_header_kernel<<<1, 32, 0, s>>>(reinterpret_cast<int64_t*>(base), h, P.nitem + L.B);
   const int smem = (int)(L.hy * sizeof(float));
   if (smem > 48 * 1024) {
@@ -391,7 +418,7 @@ cudaError_t launch_window_plan(const float* energy, const area_plan_cfg* cfg,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
   }
-  plan_base_kernel<<<(unsigned)(L.B * L.nb), 256, smem, s>>>(energy, P, cfg->split_thr);
+  plan_base_kernel<<<(unsigned)(L.B * L.nb_cap), 256, smem, s>>>(energy, P, cfg->split_thr);
   plan_windows_kernel<<<(unsigned)L.B, 1024, 0, s>>>(P);
   uint32_t* ka = reinterpret_cast<uint32_t*>(base + L.scratch_keys_a);
   uint32_t* kb = reinterpret_cast<uint32_t*>(base + L.scratch_keys_b);

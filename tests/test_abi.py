@@ -91,10 +91,17 @@ def test_plan_config_validation_and_sizes(area):
                 area.make_cfg(1, 256, 256, 0, 4, 512, 0.4),
                 area.make_cfg(1, 256, 256, 64, -1, 512, 0.4),
                 area.make_cfg(1, 256, 256, 64, 4, 5000, 0.4),
-                area.make_cfg(1, 256, 256, 64, 4, 512, 0.4, jitter_seed=7)]:
+                area.make_cfg(4096, 256, 256, 64, 4, 512, 0.4)]:
         with pytest.raises(area.AreaError) as e:
             area.area_window_plan_bytes(bad)
         assert e.value.status == area.AREA_EINVAL
+
+
+def test_plan_size_with_seed_covers_every_shift(area):
+    # a seeded plan may hold one more base window per axis
+    base = area.area_window_plan_bytes(area.make_cfg(1, 384, 384, 72, 4, 512, 0.4))
+    seeded = area.area_window_plan_bytes(area.make_cfg(1, 384, 384, 72, 4, 512, 0.4, 99))
+    assert seeded >= base
 
 
 def test_window_calls_reject_small_buffers_on_host(area):

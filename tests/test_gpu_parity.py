@@ -83,6 +83,42 @@ def test_plan_bitexact(name, step):
     _check_items(got, want)
 
 
+@pytest.mark.parametrize("name", ALL)
+@pytest.mark.parametrize("seed", [1, 12345, 2 ** 63 + 7])
+def test_plan_seeded_bitexact(name, seed):
+    # border jitter and random Halo widths drawn from the seed, at every step
+    cfg = CONFIGS[name]
+    src = gr.host_src(name)
+    E = ora.dwt_detail(src, cfg.Hg, cfg.Wg)
+    energy = torch.from_numpy(E).cuda()
+    for step, w in enumerate(cfg.schedule):
+        s = seed + step
+        want = ora.window_plan(E[0], cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr, seed=s)
+        pcfg = gr.area.make_cfg(cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr, s)
+        nbytes = gr.area.area_window_plan_bytes(pcfg)
+        plan = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        gr.area.area_window_plan(energy, pcfg, plan, nbytes)
+        got = gr.parse(plan)
+        assert got["shift"] == ora.jitter_shifts(s, cfg.Hg, cfg.Wg, w)
+        gr.compare_plan(got, want)
+        _check_items(got, want)
+
+
+def test_plan_seeded_two_batch_elements():
+    rng = np.random.default_rng(5)
+    Hg, Wg, w, h, G, seed = 40, 28, 12, 6, 9, 777
+    E = (rng.random((2, Hg // 2, Wg // 2)) ** 2).astype(np.float32)
+    pcfg = gr.area.make_cfg(2, Hg, Wg, w, h, G, 0.2, seed)
+    nbytes = gr.area.area_window_plan_bytes(pcfg)
+    plan = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    gr.area.area_window_plan(torch.from_numpy(E).cuda(), pcfg, plan, nbytes)
+    got = gr.parse(plan)
+    for b in range(2):
+        want = ora.window_plan(E[b], Hg, Wg, w, h, G, 0.2, seed=seed, b=b)
+        gr.compare_plan(got, want, b)
+        _check_items(got, want, b)
+
+
 @pytest.mark.parametrize("Hg,Wg,w,h,G,thr", [
     (16, 16, 7, 2, 5, 0.3),      # odd window side: unequal quadrants
     (12, 20, 64, 0, 3, 0.0),     # one window covers the grid, no halo
@@ -260,6 +296,29 @@ def test_dense_attn_text_ragged(N, Nk, T, D, dtype):
                                   gr.area_dtype(dtype))
     gr.assert_close(gr.to_host(o), ora.coarse_attn(q, k, v, scale, kt=kt, vt=vt), dtype,
                     "dense+text")
+
+
+def test_window_attn_seeded(data):
+    # jittered borders and random Halo widths change the plan; the attention
+    # kernels consume it unchanged
+    cfg = data.cfg
+    step = len(cfg.schedule) // 2
+    w, seed = cfg.schedule[step], 4242 + step
+    energy = gr.gpu_dwt(data.dsrc, cfg.B, cfg.Hg, cfg.Wg, cfg.C, cfg.dtype)
+    pcfg = gr.area.make_cfg(cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr, seed)
+    nbytes = gr.area.area_window_plan_bytes(pcfg)
+    plan = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    gr.area.area_window_plan(energy, pcfg, plan, nbytes)
+    o = gr.gpu_window(data.dq, data.dk, data.dv, pcfg, plan, nbytes, cfg.H, cfg.D, cfg.scale,
+                      cfg.dtype)
+    E = ora.dwt_detail(data.src, cfg.Hg, cfg.Wg)
+    oplan = ora.window_plan(E[0], cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr, seed=seed)
+    gr.compare_plan(gr.parse(plan), oplan)
+    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H - 1]
+    rows = np.arange(cfg.N) if cfg.tiny else gr.sample_rows(cfg.N, 192, seed=21)
+    want = ora.window_attn(data.q, data.k, data.v, [oplan], cfg.scale, rows=rows, heads=heads)
+    got = gr.to_host(o[:, heads][:, :, torch.from_numpy(rows).cuda()])
+    gr.assert_close(got, want, cfg.dtype, f"window seeded {cfg.name} step {step}")
 
 
 # ---------------------------------------------------------------------------

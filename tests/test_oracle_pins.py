@@ -265,8 +265,8 @@ def test_tent_weight_closed_form():
     assert ora.tent_weight(5, 7, 2, 3, 8, 8) == 4 * 4
 
 
-def _brute_plan_checks(plan, E, thr):
-    Hg, Wg, h, G = plan.Hg, plan.Wg, plan.halo, plan.G
+def _brute_plan_checks(plan, E, thr, seed=0):
+    Hg, Wg, G = plan.Hg, plan.Wg, plan.G
     N = Hg * Wg
     Etok = ora.token_energy(E)
     rank_key = lambda t: (-float(Etok[t // Wg, t % Wg]), t)
@@ -288,6 +288,8 @@ def _brute_plan_checks(plan, E, thr):
     assert cover.min() >= 1
     wsum = np.zeros(N)
     for i, (y0, x0, hy, wx) in enumerate(plan.windows):
+        h = ora.halo_width(seed, plan.halo, 0, i)
+        assert 0 <= h <= plan.halo
         ext = set()
         for t in range(N):
             y, x = divmod(t, Wg)
@@ -477,3 +479,67 @@ def test_window_with_text_equals_masked_attention_plus_text():
                     p = np.exp(s_all - s_all.max())
                     num[h, t] += w * (p / p.sum()) @ np.concatenate([v[0, h], vt[0, h]])
     np.testing.assert_allclose(got[0], num / den[None, :, None], atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# seeded border jitter and Halo widths
+# --------------------------------------------------------------------------
+
+def test_splitmix64_reference_sequence():
+    g = _golden("splitmix64.json")
+    got = [ora.counter_random(g["seed"], 0, i) for i in range(3)]
+    assert got == [int(x, 16) for x in g["outputs_hex"]]
+    # counter_random(seed, stream, i) is output number stream*2^32 + i
+    assert ora.counter_random(7, 1, 5) == ora.counter_random(7, 0, (1 << 32) + 5)
+
+
+def test_tile_windows_shift_zero_is_the_base_tiling():
+    for L in range(2, 60):
+        for w in range(1, 70):
+            starts, we = ora.tile_starts(L, w)
+            assert ora.tile_windows(L, w, 0) == [(s0, we) for s0 in starts]
+
+
+def test_tile_windows_shifted_cover_the_axis_and_move_the_seams():
+    for L in range(3, 50):
+        for w in range(2, 40):
+            we = min(w, L)
+            for shift in range(0, we):
+                wins = ora.tile_windows(L, w, shift)
+                cover = np.zeros(L, dtype=int)
+                for a, n in wins:
+                    assert n >= 1 and 0 <= a and a + n <= L and n <= we
+                    cover[a:a + n] += 1
+                assert cover.min() >= 1
+                if shift and we < L:
+                    # the first window is clipped by exactly the shift
+                    assert wins[0] == (0, we - shift)
+
+
+def test_jitter_and_halo_draws():
+    assert ora.jitter_shifts(0, 384, 384, 64) == (0, 0)
+    assert ora.jitter_shifts(99, 256, 256, 256) == (0, 0)      # window spans the grid
+    seen = set()
+    for seed in range(1, 200):
+        sy, sx = ora.jitter_shifts(seed, 384, 128, 96)
+        assert 0 <= sy < 96 and 0 <= sx < 96
+        seen.add(sy)
+        h = ora.halo_width(seed, 8, 0, seed % 7)
+        assert 0 <= h <= 8
+    assert len(seen) > 50                                       # the shift really varies
+    assert ora.halo_width(0, 4, 0, 3) == 4
+
+
+def test_plan_with_seed_brute_force_invariants():
+    rng = np.random.default_rng(31)
+    for (Hg, Wg, w, h, G, seed) in [(16, 16, 6, 2, 5, 11), (20, 12, 7, 3, 9, 12345),
+                                    (12, 18, 5, 1, 4, 2 ** 40 + 3)]:
+        E = rng.random((Hg // 2, Wg // 2)).astype(np.float32)
+        E[:, : E.shape[1] // 2] += 0.5
+        plan = ora.window_plan(E, Hg, Wg, w, h, G, 0.2, seed=seed)
+        sy, sx = ora.jitter_shifts(seed, Hg, Wg, w)
+        assert (sy, sx) != (0, 0)
+        ys = [(a, n) for a, n in ora.tile_windows(Hg, w, sy)]
+        xs = [(a, n) for a, n in ora.tile_windows(Wg, w, sx)]
+        assert [tuple(r) for r in plan.base] == [(a, c, n, m) for a, n in ys for c, m in xs]
+        _brute_plan_checks(plan, E, 0.2, seed=seed)
