@@ -291,6 +291,42 @@ int area_window_attn_text(const void* q, const void* k, const void* v,
                           cudaStream_t stream);
 
 /*
+ * area_bridge_select -- the global-KV bridge as the pages describe it ([ai]
+ * Phase II: R = (rho w)^2 tokens from the rest of the grid, selected by
+ * their deviation from the global mean key and spread spatially, rho = 0.5).
+ * Per (b, h), with K widened to fp32 and every operation round-to-nearest:
+ *   mean_d = (in-order sum over 1024-token chunks of the in-order chunk
+ *            sums of K[t, d]) * fl32(1/N);
+ *   dev(t) = (((0 + e_0) + e_1) + ...), e_d = (K[t, d] - mean_d)^2;
+ * the grid is cut into ry x rx cells (cell (cy, cx) holds rows
+ * floor(cy Hg/ry) .. floor((cy+1) Hg/ry) - 1 and likewise for columns); each
+ * cell contributes its token of largest dev, the lowest index among equals.
+ * Choose ry, rx = round(rho * window side) per axis for R = (rho w)^2.
+ *   k    : [B, H, Hg*Wg, D] (dtype)
+ *   cand : int32 [B, H, ry*rx] output, cells row-major
+ *   ws   : B*H*D*4 bytes of scratch (the mean keys)
+ * Errors: AREA_EINVAL, AREA_EUNSUPPORTED (D, or N above 232448*256/D tokens),
+ * AREA_ENOSPACE (ws too small).
+ */
+int area_bridge_select(const void* k, int dtype, int B, int H, int Hg, int Wg,
+                       int D, int ry, int rx, int* cand, void* ws,
+                       size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * area_window_attn_bridge -- area_window_attn with the pages' bridge: the
+ * global part of window W's key set, for head h, is the candidates of
+ * area_bridge_select for (b, h) that lie outside ext(W), instead of the
+ * plan's energy-ranked list (the plan's G is ignored; build it with G = 0).
+ *   cand : int32 [B, H, R] from area_bridge_select (R = ry*rx)
+ * Errors: as area_window_attn, and AREA_EINVAL for null cand or R < 1.
+ */
+int area_window_attn_bridge(const void* q, const void* k, const void* v,
+                            const int* cand, int R, const area_plan_cfg* cfg,
+                            const void* plan, size_t plan_bytes, void* o,
+                            void* ws, size_t ws_bytes, int H, int D,
+                            float scale, int dtype, cudaStream_t stream);
+
+/*
  * area_window_attn_noalloc -- area_window_attn for callers that cannot
  * allocate device memory.  The paper has no counterpart: this is a library
  * convenience, not part of the method.

@@ -29,6 +29,7 @@ function here is "parity unpinned".
 """
 from __future__ import annotations
 
+import math
 from dataclasses import dataclass, field
 from typing import Dict, List, Optional, Sequence, Tuple
 
@@ -408,6 +409,77 @@ def window_plan(E: np.ndarray, Hg: int, Wg: int, w: int, halo: int, G: int,
                 wsum=wsum.reshape(-1))
 
 
+# ----------------------------------------------------------------------------
+# The pages' global-KV bridge: distinctive keys by deviation, spread spatially
+# ----------------------------------------------------------------------------
+
+BRIDGE_CHUNK = 1024
+
+
+def bridge_lattice(w: int, Hg: int, Wg: int, rho: float = 0.5) -> Tuple[int, int]:
+    """Cells per axis of the bridge lattice: R = (rho * w)^2 tokens per window
+    ([ai] Phase II, rho = 0.5).  Reading: r = round(rho * side) per axis of
+    the (clipped) window, at least 1 and at most the grid side."""
+    hy, wx = min(w, Hg), min(w, Wg)
+    ry = min(Hg, max(1, int(math.floor(rho * hy + 0.5))))
+    rx = min(Wg, max(1, int(math.floor(rho * wx + 0.5))))
+    return ry, rx
+
+
+def key_deviation(k: np.ndarray) -> np.ndarray:
+    """Squared deviation of every key from the mean key of its head, float32.
+
+    k: [N, D] (storage values).  Mean: per dimension, tokens summed in order
+    within chunks of 1024, the chunk sums added in order, times the float32
+    reciprocal of N.  dev(t) = (((0 + e_0) + e_1) + ...) over dimensions with
+    e_d = (k[t, d] - mean_d)^2; float32, no fused multiply-add."""
+    k = np.asarray(k, dtype=F32)
+    N, D = k.shape
+    total = np.zeros(D, dtype=F32)
+    for c0 in range(0, N, BRIDGE_CHUNK):
+        part = np.zeros(D, dtype=F32)
+        for t in range(c0, min(N, c0 + BRIDGE_CHUNK)):
+            part = part + k[t]
+        total = total + part
+    mean = total * (F32(1) / F32(N))
+    dev = np.zeros(N, dtype=F32)
+    for d in range(D):
+        e = k[:, d] - mean[d]
+        dev = dev + e * e
+    return dev
+
+
+def bridge_candidates(k: np.ndarray, Hg: int, Wg: int, ry: int, rx: int) -> np.ndarray:
+    """Distinctive tokens of one head ([ai] Phase II: drawn from the rest of
+    the grid, selected by their deviation from the global mean key and spread
+    spatially).  Reading: the grid is cut into ry x rx cells (cell (cy, cx)
+    holds rows floor(cy*Hg/ry) .. floor((cy+1)*Hg/ry) - 1 and likewise for
+    columns); each cell gives its token of largest key_deviation, the lowest
+    token index among equals.  Returns int32 [ry * rx], cells row-major."""
+    dev = key_deviation(k).reshape(Hg, Wg)
+    out = np.empty(ry * rx, dtype=np.int32)
+    for cy in range(ry):
+        y0, y1 = (cy * Hg) // ry, ((cy + 1) * Hg) // ry
+        for cx in range(rx):
+            x0, x1 = (cx * Wg) // rx, ((cx + 1) * Wg) // rx
+            best, bt = None, -1
+            for y in range(y0, y1):
+                for x in range(x0, x1):
+                    v = dev[y, x]
+                    if best is None or v > best:
+                        best, bt = v, y * Wg + x
+            out[cy * rx + cx] = bt
+    return out
+
+
+def bridge_window_tokens(cand: np.ndarray, ext_rect, Wg: int) -> np.ndarray:
+    """The bridge keys of one window: the candidates outside its Halo rectangle."""
+    ey0, ex0, ehy, ewx = (int(v) for v in ext_rect)
+    cy, cx = cand // Wg, cand % Wg
+    inside = (cy >= ey0) & (cy < ey0 + ehy) & (cx >= ex0) & (cx < ex0 + ewx)
+    return cand[~inside].astype(np.int64)
+
+
 def window_tokens(rect, Wg: int) -> np.ndarray:
     """Token indices of a rectangle (y0, x0, hy, wx), row-major."""
     y0, x0, hy, wx = (int(v) for v in rect)
@@ -425,8 +497,8 @@ def window_kv_tokens(plan: Plan, i: int) -> np.ndarray:
 
 def window_attn(q, k, v, plans: Sequence[Plan], scale: float,
                 rows: Optional[np.ndarray] = None, heads: Optional[Sequence[int]] = None,
-                kt: Optional[np.ndarray] = None, vt: Optional[np.ndarray] = None
-                ) -> np.ndarray:
+                kt: Optional[np.ndarray] = None, vt: Optional[np.ndarray] = None,
+                bridge: Optional[np.ndarray] = None) -> np.ndarray:
     """Phase II windowed attention with centre-weighted merge ([ai] Phase II).
 
     For each final window W: O_W(q) = softmax(scale * q K_S^T) V_S over
@@ -458,6 +530,9 @@ def window_attn(q, k, v, plans: Sequence[Plan], scale: float,
                  np.minimum(tx - x0 + 1, x0 + wx - tx)).astype(np.float64)
             kv = window_kv_tokens(plan, i)
             for hi, h in enumerate(heads):
+                if bridge is not None:
+                    kv = np.concatenate([window_tokens(plan.ext[i], plan.Wg),
+                                         bridge_window_tokens(bridge[b, h], plan.ext[i], plan.Wg)])
                 kk, vv = k[b, h][kv], v[b, h][kv]
                 if kt is not None:
                     kk = np.concatenate([kk, np.asarray(kt[b, h])])

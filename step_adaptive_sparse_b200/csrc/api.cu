@@ -46,9 +46,9 @@ int dense_attn(const void* q, const void* k, const void* v, const void* kt, cons
 }
 
 int window_attn(const void* q, const void* k, const void* v, const void* kt, const void* vt,
-                int T, const area_plan_cfg* cfg, const void* plan, size_t plan_bytes, void* o,
-                void* ws, size_t ws_bytes, int H, int D, float scale, int dtype,
-                cudaStream_t stream) {
+                int T, const int* cand, int R, const area_plan_cfg* cfg, const void* plan,
+                size_t plan_bytes, void* o, void* ws, size_t ws_bytes, int H, int D, float scale,
+                int dtype, cudaStream_t stream) {
   if (!plan || !ws) return AREA_EINVAL;
   area::PlanLayout L;
   int st = area::plan_layout(cfg, &L);
@@ -56,6 +56,7 @@ int window_attn(const void* q, const void* k, const void* v, const void* kt, con
   st = check_attn(q, k, v, o, (int)L.B, H, (int)L.N, (int)L.N, D, dtype);
   if (st != AREA_OK) return st;
   if (T < 0 || (T > 0 && (!kt || !vt || !aligned16(kt) || !aligned16(vt)))) return AREA_EINVAL;
+  if (cand && R < 1) return AREA_EINVAL;
   if (plan_bytes < (size_t)L.total) return AREA_ENOSPACE;
   if (ws_bytes < (size_t)(L.B * H * L.N * D * 4)) return AREA_ENOSPACE;
   if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(plan) & 255) != 0) return AREA_EINVAL;
@@ -64,10 +65,10 @@ int window_attn(const void* q, const void* k, const void* v, const void* kt, con
   cudaError_t e = area::launch_ws_zero(w, L, plan, H, D, stream);
   if (e != cudaSuccess) return fail_cuda(e);
   if (dtype == AREA_DTYPE_BF16 && D == 128)
-    e = area::launch_window_attn_tc(q, k, v, kt, vt, T, L, plan, o, w, H, scale, stream);
+    e = area::launch_window_attn_tc(q, k, v, kt, vt, T, cand, R, L, plan, o, w, H, scale, stream);
   else
-    e = area::launch_window_attn_simt(q, k, v, kt, vt, T, L, plan, o, w, H, D, scale, dtype,
-                                      stream);
+    e = area::launch_window_attn_simt(q, k, v, kt, vt, T, cand, R, L, plan, o, w, H, D, scale,
+                                      dtype, stream);
   if (e != cudaSuccess) return fail_cuda(e);
   return finish(area::launch_window_finalize(w, L, plan, o, H, D, dtype, stream));
 }
@@ -165,16 +166,40 @@ int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D, size_t* ws
 int area_window_attn(const void* q, const void* k, const void* v, const area_plan_cfg* cfg,
                      const void* plan, size_t plan_bytes, void* o, void* ws, size_t ws_bytes,
                      int H, int D, float scale, int dtype, cudaStream_t stream) {
-  return window_attn(q, k, v, nullptr, nullptr, 0, cfg, plan, plan_bytes, o, ws, ws_bytes, H, D,
-                     scale, dtype, stream);
+  return window_attn(q, k, v, nullptr, nullptr, 0, nullptr, 0, cfg, plan, plan_bytes, o, ws,
+                     ws_bytes, H, D, scale, dtype, stream);
 }
 
 int area_window_attn_text(const void* q, const void* k, const void* v, const void* kt,
                           const void* vt, int T, const area_plan_cfg* cfg, const void* plan,
                           size_t plan_bytes, void* o, void* ws, size_t ws_bytes, int H, int D,
                           float scale, int dtype, cudaStream_t stream) {
-  return window_attn(q, k, v, kt, vt, T, cfg, plan, plan_bytes, o, ws, ws_bytes, H, D, scale,
-                     dtype, stream);
+  return window_attn(q, k, v, kt, vt, T, nullptr, 0, cfg, plan, plan_bytes, o, ws, ws_bytes, H,
+                     D, scale, dtype, stream);
+}
+
+int area_bridge_select(const void* k, int dtype, int B, int H, int Hg, int Wg, int D, int ry,
+                       int rx, int* cand, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!k || !cand || !ws) return AREA_EINVAL;
+  if (B < 1 || H < 1 || Hg < 1 || Wg < 1 || ry < 1 || rx < 1 || ry > Hg || rx > Wg)
+    return AREA_EINVAL;
+  if (!valid_dtype(dtype)) return AREA_EINVAL;
+  if (D != 64 && D != 128) return AREA_EUNSUPPORTED;
+  const int64_t N = (int64_t)Hg * Wg;
+  if (((N + 1023) / 1024) * D * 4 > 227 * 1024) return AREA_EUNSUPPORTED;   // chunk sums in smem
+  if (ws_bytes < (size_t)B * H * D * sizeof(float)) return AREA_ENOSPACE;
+  if (!aligned16(k) || !aligned16(ws)) return AREA_EINVAL;
+  return finish(area::launch_bridge_select(k, dtype, B, H, Hg, Wg, D, ry, rx, cand,
+                                           static_cast<float*>(ws), stream));
+}
+
+int area_window_attn_bridge(const void* q, const void* k, const void* v, const int* cand, int R,
+                            const area_plan_cfg* cfg, const void* plan, size_t plan_bytes,
+                            void* o, void* ws, size_t ws_bytes, int H, int D, float scale,
+                            int dtype, cudaStream_t stream) {
+  if (!cand) return AREA_EINVAL;
+  return window_attn(q, k, v, nullptr, nullptr, 0, cand, R, cfg, plan, plan_bytes, o, ws,
+                     ws_bytes, H, D, scale, dtype, stream);
 }
 
 }  // extern "C"

@@ -116,9 +116,9 @@ cudaError_t launch_dense_attn_simt(const void* q, const void* k, const void* v, 
                                    const void* vt, void* o, int B, int H, int N, int Nk, int T,
                                    int D, float scale, int dtype, cudaStream_t s);
 cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v, const void* kt,
-                                    const void* vt, int T, const PlanLayout& L, const void* plan,
-                                    void* o, float* ws, int H, int D, float scale, int dtype,
-                                    cudaStream_t s);
+                                    const void* vt, int T, const int* cand, int R,
+                                    const PlanLayout& L, const void* plan, void* o, float* ws,
+                                    int H, int D, float scale, int dtype, cudaStream_t s);
 // Shared by both window-attention paths.
 cudaError_t launch_ws_zero(float* ws, const PlanLayout& L, const void* plan, int H, int D,
                            cudaStream_t s);
@@ -131,8 +131,14 @@ cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, co
                                  const void* vt, void* o, int B, int H, int N, int Nk, int T,
                                  float scale, cudaStream_t s);
 cudaError_t read_and_clear_tc_error(int* code);
+// cand (may be null): per-head bridge candidates [B*H][R]; when given they
+// replace the plan's global-KV lists, candidates inside a window's Halo
+// rectangle are skipped.
 cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, const void* kt,
-                                  const void* vt, int T, const PlanLayout& L, const void* plan,
-                                  void* o, float* ws, int H, float scale, cudaStream_t s);
+                                  const void* vt, int T, const int* cand, int R,
+                                  const PlanLayout& L, const void* plan, void* o, float* ws,
+                                  int H, float scale, cudaStream_t s);
+cudaError_t launch_bridge_select(const void* k, int dtype, int B, int H, int Hg, int Wg, int D,
+                                 int ry, int rx, int* cand, float* mean, cudaStream_t s);
 
 }  // namespace area

@@ -26,14 +26,16 @@ struct DenseRows {
 template <typename T, int D, bool WINDOW>
 __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-    const T* __restrict__ kt, const T* __restrict__ vt, int ntext, T* __restrict__ o,
-    float* __restrict__ ws, int H, DenseRows dr, PlanView P, float scale) {
+    const T* __restrict__ kt, const T* __restrict__ vt, int ntext, const int* __restrict__ cand,
+    int R, T* __restrict__ o, float* __restrict__ ws, int H, DenseRows dr, PlanView P,
+    float scale) {
   constexpr int DPT = D / kSimtTPQ;
   extern __shared__ float smem[];
   float* Ks = smem;                       // [kSimtKV][D]
   float* Vs = smem + kSimtKV * D;         // [kSimtKV][D]
   __shared__ int s_kvtok[kSimtKV];
   __shared__ bool s_kvtxt[kSimtKV];
+  __shared__ bool s_kvok[kSimtKV];
 
   const int b = blockIdx.z, h = blockIdx.y;
   const int tid = threadIdx.x;
@@ -55,8 +57,8 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     const int64_t wo = (int64_t)b * P.nw + wi;
     win = P.win[wo];
     ext = P.ext[wo];
-    nkv = ext.z * ext.w + P.gcount[wo];
-    glist = P.gidx + wo * P.G;
+    nkv = ext.z * ext.w + (cand ? R : P.gcount[wo]);
+    glist = cand ? cand + ((int64_t)b * H + h) * R : P.gidx + wo * P.G;
     r = it.y * kQTile + sub * kSimtQ + ql;
     qvalid = r < win.z * win.w;
     qtok = qvalid ? (win.x + r / win.w) * P.Wg + win.y + r % win.w : 0;
@@ -89,7 +91,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     const int cn = min(kSimtKV, nkv - c0);
     if (tid < kSimtKV) {
       int tok = 0;
-      bool txt = false;
+      bool txt = false, ok = true;
       const int j = c0 + tid;
       if (tid < cn) {
         if (j >= nimg) {
@@ -98,12 +100,17 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
         } else if (WINDOW) {
           const int ne = ext.z * ext.w;
           tok = j < ne ? (ext.x + j / ext.w) * P.Wg + ext.y + j % ext.w : glist[j - ne];
+          if (cand && j >= ne) {     // bridge candidates inside the rectangle are skipped
+            const int ty = tok / P.Wg, tx = tok % P.Wg;
+            ok = !(ty >= ext.x && ty < ext.x + ext.z && tx >= ext.y && tx < ext.y + ext.w);
+          }
         } else {
           tok = j;
         }
       }
       s_kvtok[tid] = tok;
       s_kvtxt[tid] = txt;
+      s_kvok[tid] = ok;
     }
     __syncthreads();
     // cooperative load: thread -> (row, quarter of the row)
@@ -130,7 +137,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
       part_dot += __shfl_xor_sync(0xffffffffu, part_dot, 1);
       part_dot += __shfl_xor_sync(0xffffffffu, part_dot, 2);
       part_dot += __shfl_xor_sync(0xffffffffu, part_dot, 4);
-      s[j] = j < cn ? part_dot : -INFINITY;
+      s[j] = (j < cn && s_kvok[j]) ? part_dot : -INFINITY;
       mc = fmaxf(mc, s[j]);
     }
     const float mn = fmaxf(m, mc);
@@ -206,16 +213,16 @@ __global__ void __launch_bounds__(256) window_finalize_kernel(const float4* __re
 
 template <typename T, int D, bool WINDOW>
 cudaError_t launch_simt(dim3 grid, const void* q, const void* k, const void* v, const void* kt,
-                        const void* vt, int ntext, void* o, float* ws, int H, DenseRows dr,
-                        PlanView P, float scale, cudaStream_t s) {
+                        const void* vt, int ntext, const int* cand, int R, void* o, float* ws,
+                        int H, DenseRows dr, PlanView P, float scale, cudaStream_t s) {
   const int smem = 2 * kSimtKV * D * (int)sizeof(float);
   auto fn = attn_simt_kernel<T, D, WINDOW>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   fn<<<grid, kSimtThreads, smem, s>>>(static_cast<const T*>(q), static_cast<const T*>(k),
                                       static_cast<const T*>(v), static_cast<const T*>(kt),
-                                      static_cast<const T*>(vt), ntext, static_cast<T*>(o), ws, H,
-                                      dr, P, scale);
+                                      static_cast<const T*>(vt), ntext, cand, R,
+                                      static_cast<T*>(o), ws, H, dr, P, scale);
   return cudaGetLastError();
 }
 
@@ -234,26 +241,26 @@ cudaError_t launch_dense_attn_simt(const void* q, const void* k, const void* v, 
   DenseRows dr{N, Nk};
   PlanView P{};
   if (dtype == AREA_DTYPE_F32) {
-    if (D == 64) return launch_simt<float, 64, false>(grid, q, k, v, kt, vt, T, o, nullptr, H, dr, P, scale, s);
-    return launch_simt<float, 128, false>(grid, q, k, v, kt, vt, T, o, nullptr, H, dr, P, scale, s);
+    if (D == 64) return launch_simt<float, 64, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, nullptr, H, dr, P, scale, s);
+    return launch_simt<float, 128, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, nullptr, H, dr, P, scale, s);
   }
-  if (D == 64) return launch_simt<__nv_bfloat16, 64, false>(grid, q, k, v, kt, vt, T, o, nullptr, H, dr, P, scale, s);
-  return launch_simt<__nv_bfloat16, 128, false>(grid, q, k, v, kt, vt, T, o, nullptr, H, dr, P, scale, s);
+  if (D == 64) return launch_simt<__nv_bfloat16, 64, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, nullptr, H, dr, P, scale, s);
+  return launch_simt<__nv_bfloat16, 128, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, nullptr, H, dr, P, scale, s);
 }
 
 cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v, const void* kt,
-                                    const void* vt, int T, const PlanLayout& L, const void* plan,
-                                    void* o, float* ws, int H, int D, float scale, int dtype,
-                                    cudaStream_t s) {
+                                    const void* vt, int T, const int* cand, int R,
+                                    const PlanLayout& L, const void* plan, void* o, float* ws,
+                                    int H, int D, float scale, int dtype, cudaStream_t s) {
   PlanView P = plan_view(L, const_cast<void*>(plan));
   dim3 grid((unsigned)(L.nitem_max * (kQTile / kSimtQ)), H, (unsigned)L.B);
   DenseRows dr{(int)L.N, (int)L.N};
   if (dtype == AREA_DTYPE_F32) {
-    if (D == 64) return launch_simt<float, 64, true>(grid, q, k, v, kt, vt, T, o, ws, H, dr, P, scale, s);
-    return launch_simt<float, 128, true>(grid, q, k, v, kt, vt, T, o, ws, H, dr, P, scale, s);
+    if (D == 64) return launch_simt<float, 64, true>(grid, q, k, v, kt, vt, T, cand, R, o, ws, H, dr, P, scale, s);
+    return launch_simt<float, 128, true>(grid, q, k, v, kt, vt, T, cand, R, o, ws, H, dr, P, scale, s);
   }
-  if (D == 64) return launch_simt<__nv_bfloat16, 64, true>(grid, q, k, v, kt, vt, T, o, ws, H, dr, P, scale, s);
-  return launch_simt<__nv_bfloat16, 128, true>(grid, q, k, v, kt, vt, T, o, ws, H, dr, P, scale, s);
+  if (D == 64) return launch_simt<__nv_bfloat16, 64, true>(grid, q, k, v, kt, vt, T, cand, R, o, ws, H, dr, P, scale, s);
+  return launch_simt<__nv_bfloat16, 128, true>(grid, q, k, v, kt, vt, T, cand, R, o, ws, H, dr, P, scale, s);
 }
 
 cudaError_t launch_ws_zero(float* ws, const PlanLayout& L, const void* plan, int H, int D,

@@ -341,7 +341,7 @@ struct Unit {
 
 template <bool WINDOW>
 __device__ __forceinline__ Unit get_unit(int u, const DenseArgs& da, const PlanView& P, int H,
-                                         int T) {
+                                         int T, const int* cand = nullptr, int R = 0) {
   Unit x;
   x.valid = true;
   x.glist = nullptr;
@@ -372,12 +372,12 @@ __device__ __forceinline__ Unit get_unit(int u, const DenseArgs& da, const PlanV
     x.ext = P.ext[wo];
     x.q0 = it.y * 256;
     x.nq = x.win.z * x.win.w;
-    x.nkv = P.gcount[wo];
+    x.nkv = cand ? R : P.gcount[wo];
     x.ncx = (x.ext.w + kPW - 1) / kPW;
     x.ntr = x.ncx * ((x.ext.z + kPH - 1) / kPH);
     x.nti = x.ntr + (x.nkv + 127) / 128;
     x.nt = x.nti + (T + 127) / 128;
-    x.glist = P.gidx + wo * P.G;
+    x.glist = cand ? cand + (int64_t)x.bh * R : P.gidx + wo * P.G;
   }
   return x;
 }
@@ -396,6 +396,8 @@ struct TcParams {
   float scale_log2;
   int H;
   int T;              // text keys per (b, h), appended after the image keys
+  const int* cand;    // bridge mode: per-head candidate tokens [B*H][R] (else null)
+  int R;
   int num_units;
   DenseArgs da;
   PlanView P;
@@ -403,7 +405,7 @@ struct TcParams {
   float* ws;          // window workspace
 };
 
-template <bool WINDOW>
+template <bool WINDOW, bool BRIDGE>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
@@ -456,7 +458,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // ------------------------------------------------------------ producer
     uint32_t kv_it = 0, unit_count = 0;
     for (int u = blockIdx.x; u < prm.num_units; u += gridDim.x) {
-      const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T);
+      const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T, BRIDGE ? prm.cand : nullptr, prm.R);
       if (!x.valid) continue;
       if (!warp_wait0(bar(BAR_Q_EMPTY), (unit_count & 1u) ^ 1u, abort_flag)) break;
       if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL), 2 * kTileBytes);
@@ -559,7 +561,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                  (first && kk == 0) ? 0u : 1u);
       };
       for (int u = blockIdx.x; u < prm.num_units && ok; u += gridDim.x) {
-        const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T);
+        const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T, BRIDGE ? prm.cand : nullptr, prm.R);
         if (!x.valid) continue;
         const int nt = x.nt;
         if (!(ok = mbar_wait(bar(BAR_Q_FULL), unit_count & 1u, abort_flag))) break;
@@ -637,7 +639,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       // epilogue rather than kept live in registers across the key loop)
       int nkv, nt, nti, ntr, ncx, ew, eh;
       {
-        const Unit x0 = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T);
+        const Unit x0 = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T, BRIDGE ? prm.cand : nullptr, prm.R);
         if (!x0.valid) continue;
         nkv = x0.nkv; nt = x0.nt; nti = x0.nti; ntr = x0.ntr; ncx = x0.ncx;
         ew = x0.ext.w; eh = x0.ext.z;
@@ -652,7 +654,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // Key validity (warp-uniform): dense, global-KV and text tiles are a
         // prefix of `valid` keys; a rectangle patch keeps columns dx < rem_x of
         // rows dy < rem_y (key k = dy * kPW + dx).
-        if (!WINDOW || j >= ntr) {
+        if (BRIDGE && j >= ntr && j < nti) {
+          // bridge candidates: drop those past the list or inside the Halo
+          // rectangle; lane l tests keys 4l..4l+3 and ballots the result
+          const Unit xb = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T, prm.cand, prm.R);
+          uint32_t keep[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int p = (j - ntr) * 128 + lane * 4 + i;
+            bool ok = p < nkv;
+            if (ok) {
+              const int tok = xb.glist[p];
+              const int ty = tok / prm.P.Wg, tx = tok % prm.P.Wg;
+              ok = !(ty >= xb.ext.x && ty < xb.ext.x + eh && tx >= xb.ext.y && tx < xb.ext.y + ew);
+            }
+            keep[i] = __ballot_sync(0xffffffffu, ok);
+          }
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (!((keep[i & 3] >> (i >> 2)) & 1u)) sr[i] = 0xff800000u;
+        } else if (!WINDOW || j >= ntr) {
           const int valid = j < nti ? min(128, nkv - (j - ntr) * 128)
                                     : min(128, prm.T - (j - nti) * 128);
           if (valid < 128) {
@@ -716,7 +737,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (!ok) break;
       // epilogue (the unit is looked up again rather than kept live in
       // registers across the key loop)
-      const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T);
+      const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T, BRIDGE ? prm.cand : nullptr, prm.R);
       if (!(ok = warp_wait_all(bO, o_cnt & 1u, abort_flag))) break;
       ++o_cnt;
       tc_fence_after();
@@ -841,11 +862,11 @@ int num_sms() {
   return n;
 }
 
-template <bool WINDOW>
+template <bool WINDOW, bool BRIDGE>
 cudaError_t launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const CUtensorMap& mkp, const CUtensorMap& mvp, const CUtensorMap& mkt,
                       const CUtensorMap& mvt, const TcParams& prm, cudaStream_t s) {
-  auto fn = attn_tc_kernel<WINDOW>;
+  auto fn = attn_tc_kernel<WINDOW, BRIDGE>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int grid = prm.num_units < num_sms() ? prm.num_units : num_sms();
@@ -886,12 +907,13 @@ cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, co
   prm.da = DenseArgs{B, H, N, Nk, (N + 255) / 256};
   prm.num_units = B * H * prm.da.units_per_head;
   prm.o = static_cast<__nv_bfloat16*>(o);
-  return launch_tc<false>(mq, mk, mv, mk, mv, mkt, mvt, prm, s);   // no patch maps in dense mode
+  return launch_tc<false, false>(mq, mk, mv, mk, mv, mkt, mvt, prm, s);   // no patch maps in dense mode
 }
 
 cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, const void* kt,
-                                  const void* vt, int T, const PlanLayout& L, const void* plan,
-                                  void* o, float* ws, int H, float scale, cudaStream_t s) {
+                                  const void* vt, int T, const int* cand, int R,
+                                  const PlanLayout& L, const void* plan, void* o, float* ws,
+                                  int H, float scale, cudaStream_t s) {
   CUtensorMap mq, mk, mv, mkt, mvt;
   cudaError_t e;
   const int64_t rows = L.B * H * L.N;
@@ -913,10 +935,13 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, c
   prm.H = H;
   prm.T = T;
   prm.P = plan_view(L, const_cast<void*>(plan));
+  prm.cand = cand;
+  prm.R = R;
   prm.num_units = (int)(L.nitem_max * L.B * H);
   prm.ws = ws;
   prm.o = static_cast<__nv_bfloat16*>(o);
-  return launch_tc<true>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
+  if (cand) return launch_tc<true, true>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
+  return launch_tc<true, false>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
 }
 
 }  // namespace area

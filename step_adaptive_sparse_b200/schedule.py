@@ -41,3 +41,13 @@ def window_schedule(w0: int, w_min: int, steps: int = 8) -> List[int]:
         w = w0 * (w_min / w0) ** (t / (steps - 1) if steps > 1 else 0.0)
         out.append(8 * int(math.floor(w / 8 + 0.5)))
     return out
+
+
+def bridge_lattice(w: int, Hg: int, Wg: int, rho: float = 0.5):
+    """Cells per axis (ry, rx) of the global-KV bridge for window side w: the
+    pages' R = (rho * w)^2 tokens per window, rho = 0.5, as round(rho * side)
+    per axis of the window clipped to the grid (at least 1, at most the side)."""
+    hy, wx = min(w, Hg), min(w, Wg)
+    ry = min(Hg, max(1, int(math.floor(rho * hy + 0.5))))
+    rx = min(Wg, max(1, int(math.floor(rho * wx + 0.5))))
+    return ry, rx

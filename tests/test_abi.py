@@ -68,6 +68,9 @@ def test_null_and_bad_arguments_rejected_on_host(area):
         (lambda: area.area_coarse_attn_text(fake, fake, fake, None, None, fake, 1, 1, 16, 4, 3, 128, 1.0, 1), area.AREA_EINVAL),
         (lambda: area.area_coarse_attn_text(fake, fake, fake, fake, fake, fake, 1, 1, 16, 4, -1, 128, 1.0, 1), area.AREA_EINVAL),
         (lambda: area.area_dwt_detail(fake, 1, 16, fake, 1, 7, 8), area.AREA_EINVAL),
+        (lambda: area.area_bridge_select(fake, 1, 1, 2, 8, 8, 128, 9, 2, fake, fake, 1024), area.AREA_EINVAL),
+        (lambda: area.area_bridge_select(fake, 1, 1, 2, 8, 8, 128, 4, 4, fake, fake, 1023), area.AREA_ENOSPACE),
+        (lambda: area.area_bridge_select(fake, 1, 1, 2, 8, 8, 96, 4, 4, fake, fake, 4096), area.AREA_EUNSUPPORTED),
         (lambda: area.area_dwt_detail(fake, 1, 0, fake, 1, 8, 8), area.AREA_EINVAL),
         (lambda: area.area_dwt_detail(fake, 1, 4, fake, 1, 8, 8, 9), area.AREA_EINVAL),
     ]

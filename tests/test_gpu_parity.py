@@ -321,6 +321,53 @@ def test_window_attn_seeded(data):
     gr.assert_close(got, want, cfg.dtype, f"window seeded {cfg.name} step {step}")
 
 
+def _bridge(data, step):
+    cfg = data.cfg
+    from step_adaptive_sparse_b200 import schedule
+    w = cfg.schedule[step]
+    ry, rx = schedule.bridge_lattice(w, cfg.Hg, cfg.Wg)
+    assert (ry, rx) == ora.bridge_lattice(w, cfg.Hg, cfg.Wg)
+    R = ry * rx
+    cand = torch.empty((cfg.B, cfg.H, R), dtype=torch.int32, device="cuda")
+    wsb = cfg.B * cfg.H * cfg.D * 4
+    ws = torch.empty(wsb // 4, dtype=torch.float32, device="cuda")
+    gr.area.area_bridge_select(data.dk, gr.area_dtype(cfg.dtype), cfg.B, cfg.H, cfg.Hg, cfg.Wg,
+                               cfg.D, ry, rx, cand, ws, wsb)
+    return w, ry, rx, cand
+
+
+def test_bridge_select_bitexact(data):
+    # the pages' rule: per head, most-deviant key per lattice cell
+    cfg = data.cfg
+    for step in sorted({0, len(cfg.schedule) - 1}):
+        w, ry, rx, cand = _bridge(data, step)
+        got = cand.cpu().numpy()
+        for h in ([0, 1] if cfg.tiny else [0, cfg.H // 2, cfg.H - 1]):
+            want = ora.bridge_candidates(data.k[0, h], cfg.Hg, cfg.Wg, ry, rx)
+            assert np.array_equal(got[0, h], want), (cfg.name, w, h)
+
+
+def test_window_attn_bridge(data):
+    cfg = data.cfg
+    step = len(cfg.schedule) - 1
+    w, ry, rx, cand = _bridge(data, step)
+    energy = gr.gpu_dwt(data.dsrc, cfg.B, cfg.Hg, cfg.Wg, cfg.C, cfg.dtype)
+    pcfg, plan, nbytes = gr.gpu_plan(energy, cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, 0, cfg.split_thr)
+    o = torch.empty_like(data.dq)
+    wsb = gr.area.area_window_attn_ws_bytes(pcfg, cfg.H, cfg.D)
+    ws = torch.empty(wsb // 4, dtype=torch.float32, device="cuda")
+    gr.area.area_window_attn_bridge(data.dq, data.dk, data.dv, cand, ry * rx, pcfg, plan, nbytes,
+                                    o, ws, wsb, cfg.H, cfg.D, cfg.scale, gr.area_dtype(cfg.dtype))
+    E = ora.dwt_detail(data.src, cfg.Hg, cfg.Wg)
+    oplan = ora.window_plan(E[0], cfg.Hg, cfg.Wg, w, cfg.halo, 0, cfg.split_thr)
+    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H - 1]
+    rows = np.arange(cfg.N) if cfg.tiny else gr.sample_rows(cfg.N, 160, seed=31)
+    want = ora.window_attn(data.q, data.k, data.v, [oplan], cfg.scale, rows=rows, heads=heads,
+                           bridge=cand.cpu().numpy())
+    got = gr.to_host(o[:, heads][:, :, torch.from_numpy(rows).cuda()])
+    gr.assert_close(got, want, cfg.dtype, f"window bridge {cfg.name} w={w}")
+
+
 # ---------------------------------------------------------------------------
 # Ragged and degenerate shapes
 # ---------------------------------------------------------------------------

@@ -543,3 +543,78 @@ def test_plan_with_seed_brute_force_invariants():
         xs = [(a, n) for a, n in ora.tile_windows(Wg, w, sx)]
         assert [tuple(r) for r in plan.base] == [(a, c, n, m) for a, n in ys for c, m in xs]
         _brute_plan_checks(plan, E, 0.2, seed=seed)
+
+
+# --------------------------------------------------------------------------
+# the pages' global-KV bridge (deviation from the mean key, spread spatially)
+# --------------------------------------------------------------------------
+
+def test_bridge_lattice_is_rho_w_squared():
+    # [ai] Phase II: R = (rho * w)^2 with rho = 0.5
+    assert ora.bridge_lattice(64, 384, 384) == (32, 32)
+    assert ora.bridge_lattice(72, 384, 384) == (36, 36)
+    assert ora.bridge_lattice(272, 384, 128) == (136, 64)      # window clipped to 128 columns
+    ry, rx = ora.bridge_lattice(8, 32, 32)
+    assert ry * rx == 16
+
+
+def test_key_deviation_matches_float64_definition():
+    rng = np.random.default_rng(40)
+    k = rng.standard_normal((3000, 16)).astype(np.float32)
+    got = ora.key_deviation(k).astype(np.float64)
+    mu = k.astype(np.float64).mean(0)
+    want = ((k.astype(np.float64) - mu) ** 2).sum(1)
+    np.testing.assert_allclose(got, want, rtol=2e-5, atol=2e-5)
+    assert not ora.key_deviation(np.full((50, 4), 0.75, dtype=np.float32)).any()
+
+
+def test_bridge_picks_planted_outliers_and_lowest_index_on_ties():
+    Hg, Wg, D, ry, rx = 12, 16, 8, 3, 4
+    rng = np.random.default_rng(41)
+    k = np.zeros((Hg * Wg, D), dtype=np.float32)
+    planted = []
+    for cy in range(ry):
+        for cx in range(rx):
+            y = (cy * Hg) // ry + rng.integers(0, Hg // ry)
+            x = (cx * Wg) // rx + rng.integers(0, Wg // rx)
+            k[y * Wg + x] = 5.0 + cy + cx                  # far from the mean
+            planted.append(y * Wg + x)
+    assert ora.bridge_candidates(k, Hg, Wg, ry, rx).tolist() == planted
+    # constant keys: every deviation is 0, so each cell gives its first token
+    firsts = [((cy * Hg) // ry) * Wg + (cx * Wg) // rx for cy in range(ry) for cx in range(rx)]
+    const = np.ones((Hg * Wg, D), dtype=np.float32)
+    assert ora.bridge_candidates(const, Hg, Wg, ry, rx).tolist() == firsts
+
+
+def test_window_attention_with_bridge_equals_masked_attention():
+    rng = np.random.default_rng(42)
+    Hg, Wg = 12, 10
+    q, k, v = (rng.standard_normal((1, 2, Hg * Wg, 4)) for _ in range(3))
+    E = (rng.random((Hg // 2, Wg // 2)) ** 2).astype(np.float32)
+    plan = ora.window_plan(E, Hg, Wg, 6, 1, 0, 0.2)
+    ry, rx = ora.bridge_lattice(6, Hg, Wg)
+    cand = np.stack([ora.bridge_candidates(k[0, h].astype(np.float32), Hg, Wg, ry, rx)
+                     for h in range(2)])[None]
+    got = ora.window_attn(q, k, v, [plan], 0.5, bridge=cand)
+    N = Hg * Wg
+    num = np.zeros((2, N, 4))
+    den = np.zeros(N)
+    for i, (y0, x0, hy, wx) in enumerate(plan.windows):
+        ey0, ex0, ehy, ewx = plan.ext[i]
+        for h in range(2):
+            allowed = np.zeros(N, dtype=bool)
+            allowed[cand[0, h]] = True                          # all candidates ...
+            for t in range(N):
+                y, x = divmod(t, Wg)
+                if ey0 <= y < ey0 + ehy and ex0 <= x < ex0 + ewx:
+                    allowed[t] = True                           # ... and the Halo rectangle
+            for y in range(y0, y0 + hy):
+                for x in range(x0, x0 + wx):
+                    t = y * Wg + x
+                    w = min(y - y0 + 1, y0 + hy - y) * min(x - x0 + 1, x0 + wx - x)
+                    if h == 0:
+                        den[t] += w
+                    sc = np.where(allowed, 0.5 * k[0, h] @ q[0, h, t], -np.inf)
+                    p = np.exp(sc - sc.max())
+                    num[h, t] += w * (p / p.sum()) @ v[0, h]
+    np.testing.assert_allclose(got[0], num / den[None, :, None], atol=1e-12)

@@ -28,3 +28,9 @@ def test_config_schedules_follow_the_geometric_formula():
     assert list(CONFIGS["flux4096"].schedule) == schedule.window_schedule(256, 64)
     assert list(CONFIGS["flux6144"].schedule) == schedule.window_schedule(192, 64)
     assert list(CONFIGS["qwen6144x2048"].schedule) == schedule.window_schedule(272, 64)
+
+
+def test_bridge_lattice_matches_oracle():
+    for cfg in CONFIGS.values():
+        for w in list(cfg.schedule) + [2, 5, 1000]:
+            assert schedule.bridge_lattice(w, cfg.Hg, cfg.Wg) == ora.bridge_lattice(w, cfg.Hg, cfg.Wg)
