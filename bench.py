@@ -34,7 +34,7 @@ if ROOT not in sys.path:
 
 METRIC = "AReA attention TFLOP/s per schedule step (bf16, 1 B200)"
 # Bumped whenever attn_tc.cu changes, so that stale DRAM counters are not reported.
-KERNEL_REVISION = "attn_tc r6 (patch loader, f32x2 softmax, single-cover stores, text-key tiles)"
+KERNEL_REVISION = "attn_tc r7 (patch loader, f32x2 softmax, single-cover stores, text-key tiles, bridge variant)"
 DEFAULT_CONFIG = "flux6144"
 
 
@@ -87,6 +87,15 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return rank, world, local
+
+
+def head_range(rank: int, world: int, H: int):
+    """Contiguous heads [h0, h1) of a rank when the heads are sharded: the
+    attention of each head is independent and the plan depends only on the
+    detail source, so sharding needs no exchange step."""
+    base, extra = divmod(H, world)
+    h0 = rank * base + min(rank, extra)
+    return h0, h0 + base + (1 if rank < extra else 0)
 
 
 def init_dist(world: int, backend: str):
@@ -400,6 +409,14 @@ def run_area(args):
     cfg = CONFIGS[args.config]
     qh, kh, vh = make_qkv(cfg)
     srch = make_detail_source(cfg)
+    sharded = args.shard == "heads" and world > 1
+    H_all = cfg.H
+    if sharded:
+        # strong scaling: this rank computes its heads of the one problem
+        from dataclasses import replace
+        h0, h1 = head_range(rank, world, cfg.H)
+        qh, kh, vh = (np.ascontiguousarray(x[:, h0:h1]) for x in (qh, kh, vh))
+        cfg = replace(cfg, H=h1 - h0)
     tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     # pinned host copies for the end-to-end leg
     pin = [torch.from_numpy(x).to(tdt).pin_memory() for x in (qh, kh, vh, srch)]
@@ -507,6 +524,48 @@ def run_area(args):
     ramp_out["total_ms"] = float(sum(ramp_out["ms"]))
     del kp_r, vp_r, o_r
 
+    # ---- the pages' own bridge rule on the last (smallest) window size,
+    # measured once: candidate selection plus window attention
+    from step_adaptive_sparse_b200 import schedule as _sched
+    w_b = cfg.schedule[-1]
+    ry, rx = _sched.bridge_lattice(w_b, cfg.Hg, cfg.Wg)
+    cand = torch.empty((cfg.B, cfg.H, ry * rx), dtype=torch.int32, device=dev)
+    mws = torch.empty(cfg.B * cfg.H * cfg.D, dtype=torch.float32, device=dev)
+    pc0 = area.make_cfg(cfg.B, cfg.Hg, cfg.Wg, w_b, cfg.halo, 0, cfg.split_thr)
+    nb0 = area.area_window_plan_bytes(pc0)
+    plan0 = torch.empty(nb0, dtype=torch.uint8, device=dev)
+    bridge_out = {}
+    with torch.cuda.stream(stream):
+        area.area_dwt_detail(src, st.dt, cfg.C, st.energy, cfg.B, cfg.Hg, cfg.Wg,
+                             area.AREA_DETAIL_HH, stream)
+        area.area_window_plan(st.energy, pc0, plan0, nb0, stream)
+        for rep in range(2):
+            a, b2, c2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            a.record(stream)
+            area.area_bridge_select(k, st.dt, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, ry, rx, cand,
+                                    mws, mws.numel() * 4, stream)
+            b2.record(stream)
+            area.area_window_attn_bridge(q, k, v, cand, ry * rx, pc0, plan0, nb0, st.o2, st.ws,
+                                         st.ws_bytes, cfg.H, cfg.D, cfg.scale, st.dt, stream)
+            c2.record(stream)
+    torch.cuda.synchronize()
+    d0 = area.parse_plan(plan0.cpu().numpy())
+    cnd = cand.cpu().numpy().astype(np.int64)
+    pairs = 0.0
+    nwin0 = int(d0["nwin"][0])
+    for i in range(nwin0):
+        y0, x0, hy, wx = (int(t) for t in d0["win"][0, i])
+        ey0, ex0, ehy, ewx = (int(t) for t in d0["ext"][0, i])
+        cy, cx = cnd[0] // cfg.Wg, cnd[0] % cfg.Wg                # [H, R]
+        outside = ~((cy >= ey0) & (cy < ey0 + ehy) & (cx >= ex0) & (cx < ex0 + ewx))
+        pairs += hy * wx * (ehy * ewx * cfg.H + float(outside.sum()))
+    bflops = 4.0 * cfg.D * cfg.B * pairs
+    battn_ms = b2.elapsed_time(c2)
+    bridge_out = {"window": w_b, "lattice": [ry, rx], "select_ms": a.elapsed_time(b2),
+                  "window_attn_ms": battn_ms,
+                  "window_attn_tflops": bflops / (battn_ms * 1e-3) / 1e12}
+    del cand, mws, plan0
+
     # ---- end to end through the C-ABI from pinned host buffers.  Each step
     # copies its inputs host->device and its output device->host; two device
     # buffer sets let the copies of one step overlap the kernels of the next
@@ -568,7 +627,8 @@ def run_area(args):
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "traffic": load_traffic(cfg.name, dom),
+            "frac": achieved / peak,
+            "traffic": None if sharded else load_traffic(cfg.name, dom),
             "kernel": dom, "per_call": dom_launches,
             "peak_kind": f"bf16 dense, {peaks['source']} sustained",
             "frac_of_burst_peak": achieved / peaks["bf16_tflops"]}
@@ -585,15 +645,19 @@ def run_area(args):
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True,
+            "scaling": "strong" if sharded else "weak",
+            "vs_baseline": None,
             "dtype": "bf16" if cfg.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": cfg.name, "grid": [cfg.Hg, cfg.Wg], "tokens": cfg.N,
-                       "heads": cfg.H, "head_dim": cfg.D, "batch": cfg.B, "pool_f": cfg.f,
+                       "heads": H_all, "head_dim": cfg.D, "batch": cfg.B, "pool_f": cfg.f,
                        "schedule": list(cfg.schedule), "halo": cfg.halo, "G": cfg.G,
                        "split_thr": cfg.split_thr, "phase1_calls": n1,
                        "phase2_calls": len(cfg.schedule),
                        "l2": "inputs larger than L2 (0.9 GB per Q/K/V tensor)",
-                       "parallelism": f"replicas x{world}"},
+                       "parallelism": (f"heads sharded over {world} GPUs, "
+                                       f"{cfg.H} or fewer per GPU" if sharded
+                                       else f"replicas x{world}")},
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
@@ -615,6 +679,7 @@ def run_area(args):
                              "hbm_peak_gbs": peaks["hbm_gbs"]},
             "split_fraction_by_step": splits,
             "phase1_pooling_ramp": ramp_out,
+            "pages_bridge_rule": bridge_out,
             "graph_replay": None if graph_ms is None else {
                 "ms_per_step": graph_ms,
                 "value": step_flops / (graph_ms * 1e-3) / 1e12,
@@ -638,6 +703,9 @@ def main(argv=None):
     ap.add_argument("--ref-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay leg")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="N > 1: independent replicas (weak scaling) or the heads of one "
+                         "problem split across ranks (strong scaling)")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)

@@ -95,3 +95,45 @@ def test_window_flops_from_plan_dict():
 def test_plan_launch_count():
     assert bench.plan_launches(1) == 18
     assert bench.plan_launches(2) == 31
+
+
+def test_head_range_partitions_the_heads():
+    for H in (1, 2, 5, 24, 25):
+        for world in range(1, 9):
+            ranges = [bench.head_range(r, world, H) for r in range(world)]
+            assert ranges[0][0] == 0 and ranges[-1][1] == H
+            for (a0, a1), (b0, b1) in zip(ranges, ranges[1:]):
+                assert a1 == b0                                   # contiguous, no overlap
+            sizes = [b - a for a, b in ranges]
+            assert max(sizes) - min(sizes) <= 1                   # balanced
+
+
+def _shard_worker(rank, world, port, out):
+    import datetime
+
+    import torch.distributed as dist
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        h0, h1 = bench.head_range(rank, world, 24)
+        work = 1.0e12 * (h1 - h0)                      # per-rank share of one problem
+        ms = 100.0 + rank                              # slowest rank sets the time
+        out[rank] = (bench.reduce_sum(dist, work), bench.reduce_max(dist, ms))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_sharded_job_value_over_gloo():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, 3, port, out)) for r in range(3)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    for r in range(3):
+        total, ms = out[r]
+        assert total == 24.0e12 and ms == 102.0           # whole problem over the slowest rank
