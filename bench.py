@@ -530,7 +530,8 @@ def run_area(args):
     w_b = cfg.schedule[-1]
     ry, rx = _sched.bridge_lattice(w_b, cfg.Hg, cfg.Wg)
     cand = torch.empty((cfg.B, cfg.H, ry * rx), dtype=torch.int32, device=dev)
-    mws = torch.empty(cfg.B * cfg.H * cfg.D, dtype=torch.float32, device=dev)
+    mws = torch.empty(area.area_bridge_select_ws_bytes(cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D) // 4,
+                      dtype=torch.float32, device=dev)
     pc0 = area.make_cfg(cfg.B, cfg.Hg, cfg.Wg, w_b, cfg.halo, 0, cfg.split_thr)
     nb0 = area.area_window_plan_bytes(pc0)
     plan0 = torch.empty(nb0, dtype=torch.uint8, device=dev)
@@ -561,7 +562,11 @@ def run_area(args):
         pairs += hy * wx * (ehy * ewx * cfg.H + float(outside.sum()))
     bflops = 4.0 * cfg.D * cfg.B * pairs
     battn_ms = b2.elapsed_time(c2)
-    bridge_out = {"window": w_b, "lattice": [ry, rx], "select_ms": a.elapsed_time(b2),
+    sel_ms = a.elapsed_time(b2)
+    k_bytes = float(k.numel() * k.element_size())
+    bridge_out = {"window": w_b, "lattice": [ry, rx], "select_ms": sel_ms,
+                  "select_gbs": 2.0 * k_bytes / (sel_ms * 1e-3) / 1e9,
+                  "select_note": "algorithmic bytes: K read twice (chunk sums, then deviations)",
                   "window_attn_ms": battn_ms,
                   "window_attn_tflops": bflops / (battn_ms * 1e-3) / 1e12}
     del cand, mws, plan0

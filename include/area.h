@@ -302,12 +302,23 @@ int area_window_attn_text(const void* q, const void* k, const void* v,
  * floor(cy Hg/ry) .. floor((cy+1) Hg/ry) - 1 and likewise for columns); each
  * cell contributes its token of largest dev, the lowest index among equals.
  * Choose ry, rx = round(rho * window side) per axis for R = (rho w)^2.
- *   k    : [B, H, Hg*Wg, D] (dtype)
+ *   k    : [B, H, Hg*Wg, D] (dtype), 16-byte aligned
  *   cand : int32 [B, H, ry*rx] output, cells row-major
- *   ws   : B*H*D*4 bytes of scratch (the mean keys)
- * Errors: AREA_EINVAL, AREA_EUNSUPPORTED (D, or N above 232448*256/D tokens),
- * AREA_ENOSPACE (ws too small).
+ *   ws   : device scratch of ws_bytes >= area_bridge_select_ws_bytes(),
+ *          16-byte aligned, owned by the caller; it holds the mean keys and
+ *          the 1024-token chunk sums and needs no initial value
+ * K is read twice (chunk sums, then deviations); three kernels on `stream`.
+ * Errors: AREA_EINVAL, AREA_EUNSUPPORTED (D, N above 232448*256/D tokens, or
+ * rx above 16384), AREA_ENOSPACE (ws too small).
  */
+/*
+ * area_bridge_select_ws_bytes -- scratch size of area_bridge_select:
+ * B*H*D*(1 + ceil(Hg*Wg/1024))*4 bytes.  Errors: AREA_EINVAL (null output,
+ * a size below 1), AREA_EUNSUPPORTED (Hg*Wg above 2^31 - 1).
+ */
+int area_bridge_select_ws_bytes(int B, int H, int Hg, int Wg, int D,
+                                size_t* ws_bytes);
+
 int area_bridge_select(const void* k, int dtype, int B, int H, int Hg, int Wg,
                        int D, int ry, int rx, int* cand, void* ws,
                        size_t ws_bytes, cudaStream_t stream);

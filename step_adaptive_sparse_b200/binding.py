@@ -28,7 +28,7 @@ SECTIONS = ("BASE", "SCORE", "SPLIT", "NWIN", "WIN", "PARENT", "EXT", "GCOUNT", 
 
 EXPORTED = ("area_status_string", "area_last_cuda_error", "area_version", "area_kernel_error",
             "area_pool_kv", "area_coarse_attn_text", "area_window_attn_text",
-            "area_bridge_select", "area_window_attn_bridge",
+            "area_bridge_select_ws_bytes", "area_bridge_select", "area_window_attn_bridge",
             "area_coarse_attn", "area_full_attn", "area_dwt_detail", "area_window_plan_bytes",
             "area_window_plan", "area_window_attn_ws_bytes", "area_window_attn")
 
@@ -72,6 +72,7 @@ _SIGS = {
                               _I, _I, _F, _I, _P]),
     "area_window_attn_noalloc": (_I, [_P, _P, _P, ctypes.POINTER(area_plan_cfg), _P, _SZ, _P,
                                       _I, _I, _F, _I, _P]),
+    "area_bridge_select_ws_bytes": (_I, [_I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]),
     "area_bridge_select": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "area_window_attn_bridge": (_I, [_P, _P, _P, _P, _I, ctypes.POINTER(area_plan_cfg), _P, _SZ,
                                      _P, _P, _SZ, _I, _I, _F, _I, _P]),
@@ -208,6 +209,13 @@ def area_window_attn_noalloc(q, k, v, cfg: area_plan_cfg, plan, plan_bytes, o, H
     _check(_lib().area_window_attn_noalloc(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(cfg),
                                            _ptr(plan), plan_bytes, _ptr(o), H, D, scale, dtype,
                                            _stream(stream)), "area_window_attn_noalloc")
+
+
+def area_bridge_select_ws_bytes(B: int, H: int, Hg: int, Wg: int, D: int) -> int:
+    out = _SZ(0)
+    _check(_lib().area_bridge_select_ws_bytes(B, H, Hg, Wg, D, ctypes.byref(out)),
+           "area_bridge_select_ws_bytes")
+    return out.value
 
 
 def area_bridge_select(k, dtype, B, H, Hg, Wg, D, ry, rx, cand, ws, ws_bytes, stream=None) -> None:

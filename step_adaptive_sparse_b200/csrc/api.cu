@@ -178,6 +178,13 @@ int area_window_attn_text(const void* q, const void* k, const void* v, const voi
                      D, scale, dtype, stream);
 }
 
+int area_bridge_select_ws_bytes(int B, int H, int Hg, int Wg, int D, size_t* ws_bytes) {
+  if (!ws_bytes || B < 1 || H < 1 || Hg < 1 || Wg < 1 || D < 1) return AREA_EINVAL;
+  if ((int64_t)Hg * Wg > INT32_MAX) return AREA_EUNSUPPORTED;
+  *ws_bytes = area::bridge_ws_bytes(B, H, Hg, Wg, D);
+  return AREA_OK;
+}
+
 int area_bridge_select(const void* k, int dtype, int B, int H, int Hg, int Wg, int D, int ry,
                        int rx, int* cand, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (!k || !cand || !ws) return AREA_EINVAL;
@@ -186,8 +193,10 @@ int area_bridge_select(const void* k, int dtype, int B, int H, int Hg, int Wg, i
   if (!valid_dtype(dtype)) return AREA_EINVAL;
   if (D != 64 && D != 128) return AREA_EUNSUPPORTED;
   const int64_t N = (int64_t)Hg * Wg;
+  if (N > INT32_MAX) return AREA_EUNSUPPORTED;
   if (((N + 1023) / 1024) * D * 4 > 227 * 1024) return AREA_EUNSUPPORTED;   // chunk sums in smem
-  if (ws_bytes < (size_t)B * H * D * sizeof(float)) return AREA_ENOSPACE;
+  if (rx > 16384) return AREA_EUNSUPPORTED;                                  // cell keys in smem
+  if (ws_bytes < area::bridge_ws_bytes(B, H, Hg, Wg, D)) return AREA_ENOSPACE;
   if (!aligned16(k) || !aligned16(ws)) return AREA_EINVAL;
   return finish(area::launch_bridge_select(k, dtype, B, H, Hg, Wg, D, ry, rx, cand,
                                            static_cast<float*>(ws), stream));

@@ -138,6 +138,9 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, c
                                   const void* vt, int T, const int* cand, int R,
                                   const PlanLayout& L, const void* plan, void* o, float* ws,
                                   int H, float scale, cudaStream_t s);
+// Scratch of area_bridge_select: the mean keys [B*H][D] then the chunk sums
+// [B*H][ceil(N/1024)][D], fp32.
+size_t bridge_ws_bytes(int B, int H, int Hg, int Wg, int D);
 cudaError_t launch_bridge_select(const void* k, int dtype, int B, int H, int Hg, int Wg, int D,
                                  int ry, int rx, int* cand, float* mean, cudaStream_t s);
 

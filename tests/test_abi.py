@@ -69,7 +69,8 @@ def test_null_and_bad_arguments_rejected_on_host(area):
         (lambda: area.area_coarse_attn_text(fake, fake, fake, fake, fake, fake, 1, 1, 16, 4, -1, 128, 1.0, 1), area.AREA_EINVAL),
         (lambda: area.area_dwt_detail(fake, 1, 16, fake, 1, 7, 8), area.AREA_EINVAL),
         (lambda: area.area_bridge_select(fake, 1, 1, 2, 8, 8, 128, 9, 2, fake, fake, 1024), area.AREA_EINVAL),
-        (lambda: area.area_bridge_select(fake, 1, 1, 2, 8, 8, 128, 4, 4, fake, fake, 1023), area.AREA_ENOSPACE),
+        (lambda: area.area_bridge_select(fake, 1, 1, 2, 8, 8, 128, 4, 4, fake, fake, 2047), area.AREA_ENOSPACE),
+        (lambda: area.area_bridge_select_ws_bytes(1, 0, 8, 8, 128), area.AREA_EINVAL),
         (lambda: area.area_bridge_select(fake, 1, 1, 2, 8, 8, 96, 4, 4, fake, fake, 4096), area.AREA_EUNSUPPORTED),
         (lambda: area.area_dwt_detail(fake, 1, 0, fake, 1, 8, 8), area.AREA_EINVAL),
         (lambda: area.area_dwt_detail(fake, 1, 4, fake, 1, 8, 8, 9), area.AREA_EINVAL),
@@ -78,6 +79,14 @@ def test_null_and_bad_arguments_rejected_on_host(area):
         with pytest.raises(area.AreaError) as e:
             fn()
         assert e.value.status == status
+
+
+def test_bridge_ws_bytes(area):
+    # mean keys [B*H][D] plus one row of D chunk sums per 1024 tokens, fp32
+    assert area.area_bridge_select_ws_bytes(1, 2, 8, 8, 128) == 2 * 128 * 2 * 4
+    assert area.area_bridge_select_ws_bytes(1, 24, 384, 384, 128) == 24 * 128 * (1 + 144) * 4
+    assert area.area_bridge_select_ws_bytes(2, 1, 33, 31, 64) == 2 * 64 * (1 + 1) * 4
+    assert area.area_bridge_select_ws_bytes(1, 1, 32, 33, 64) == 64 * (1 + 2) * 4
 
 
 def test_plan_config_validation_and_sizes(area):

@@ -329,7 +329,7 @@ def _bridge(data, step):
     assert (ry, rx) == ora.bridge_lattice(w, cfg.Hg, cfg.Wg)
     R = ry * rx
     cand = torch.empty((cfg.B, cfg.H, R), dtype=torch.int32, device="cuda")
-    wsb = cfg.B * cfg.H * cfg.D * 4
+    wsb = gr.area.area_bridge_select_ws_bytes(cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D)
     ws = torch.empty(wsb // 4, dtype=torch.float32, device="cuda")
     gr.area.area_bridge_select(data.dk, gr.area_dtype(cfg.dtype), cfg.B, cfg.H, cfg.Hg, cfg.Wg,
                                cfg.D, ry, rx, cand, ws, wsb)
@@ -422,3 +422,50 @@ def test_window_attn_edge_cases(Hg, Wg, w, h, G, D, dtype, H):
     for b in range(B):
         want = ora.window_attn(q[b:b + 1], k[b:b + 1], v[b:b + 1], [plans[b]], scale)
         gr.assert_close(gr.to_host(o[b:b + 1]), want, dtype, "window edge")
+
+
+# ---------------------------------------------------------------------------
+# the pages' bridge: edge cases of the candidate selection (bit-exact)
+# ---------------------------------------------------------------------------
+
+def _gpu_bridge(dk, B, H, Hg, Wg, D, ry, rx, dtype):
+    cand = torch.full((B, H, ry * rx), -1, dtype=torch.int32, device="cuda")
+    wsb = gr.area.area_bridge_select_ws_bytes(B, H, Hg, Wg, D)
+    ws = torch.empty(wsb // 4, dtype=torch.float32, device="cuda")
+    gr.area.area_bridge_select(dk, gr.area_dtype(dtype), B, H, Hg, Wg, D, ry, rx, cand, ws, wsb)
+    return cand.cpu().numpy()
+
+
+@pytest.mark.parametrize("B,H,Hg,Wg,ry,rx,D,dtype", [
+    (1, 3, 37, 53, 5, 7, 64, "bf16"),      # ragged bands, cells and last chunk
+    (2, 1, 33, 64, 33, 64, 128, "bf16"),   # one token per cell
+    (1, 2, 40, 41, 3, 2, 128, "fp32"),     # fp32 keys
+    (1, 2, 64, 64, 1, 1, 128, "bf16"),     # one cell: the argmax of the whole grid
+    (1, 1, 48, 80, 24, 40, 64, "fp32"),    # 2 x 2 cells, fp32 head_dim 64
+    (1, 2, 72, 72, 36, 36, 128, "bf16"),   # 2 x 2 cells, band of several tiles
+])
+def test_bridge_select_edge_cases(B, H, Hg, Wg, ry, rx, D, dtype):
+    rng = np.random.default_rng(Hg * 131 + Wg * 7 + D)
+    N = Hg * Wg
+    k = (rng.standard_normal((B, H, N, D)) * rng.random((B, H, N, 1)) * 3).astype(np.float32)
+    dk = gr.to_dev(k, dtype)
+    k = gr.to_host(dk)
+    got = _gpu_bridge(dk, B, H, Hg, Wg, D, ry, rx, dtype)
+    for b in range(B):
+        for h in range(H):
+            want = ora.bridge_candidates(k[b, h], Hg, Wg, ry, rx)
+            assert np.array_equal(got[b, h], want), (b, h)
+    if (ry, rx) == (Hg, Wg):
+        assert np.array_equal(got[0, 0], np.arange(N))
+
+
+def test_bridge_select_ties_take_the_first_token():
+    # every key equal: all deviations tie, so each cell gives its top-left token
+    B, H, Hg, Wg, D, ry, rx = 1, 2, 30, 50, 128, 4, 6
+    k = np.full((B, H, Hg * Wg, D), 0.375, dtype=np.float32)
+    got = _gpu_bridge(gr.to_dev(k, "bf16"), B, H, Hg, Wg, D, ry, rx, "bf16")
+    want = np.array([((cy * Hg) // ry) * Wg + (cx * Wg) // rx
+                     for cy in range(ry) for cx in range(rx)], dtype=np.int32)
+    for h in range(H):
+        assert np.array_equal(got[0, h], want)
+        assert np.array_equal(ora.bridge_candidates(k[0, h], Hg, Wg, ry, rx), want)
