@@ -59,6 +59,9 @@ extern "C" {
 #define AREA_DETAIL_HH     0   /* e = HH^2                                     */
 #define AREA_DETAIL_ALL3   1   /* e = (LH^2 + HL^2) + HH^2                     */
 
+#define AREA_PHASE_COARSE  1   /* Phase I step: pool K/V by f, coarse attention */
+#define AREA_PHASE_WINDOW  2   /* Phase II step: DWT, plan, window attention    */
+
 /* Returns a static, human-readable string for a status code. */
 const char* area_status_string(int status);
 /* CUDA error code of the most recent AREA_ECUDA return on this thread. */
@@ -367,6 +370,64 @@ int area_window_attn_noalloc(const void* q, const void* k, const void* v,
                              const area_plan_cfg* cfg, const void* plan,
                              size_t plan_bytes, void* o, int H, int D,
                              float scale, int dtype, cudaStream_t stream);
+
+/* ---- schedule (host functions: no device memory, no stream) ------------ */
+
+/*
+ * area_pool_ramp -- Phase I pooling factor per step ([ai] Phase I: the factor
+ * starts at f0 and ramps down linearly to the floor f_min, each value snapped
+ * to a valid grid divisor; [blog] Fase I prints [4,4,4,4,2,2,2,2] for f0 = 4
+ * over 8 steps at a 256 x 256 grid).  Step t's linear value
+ * f0 + (f_min - f0) * t / (steps - 1) (double precision) goes to the nearest
+ * factor that divides both Hg and Wg, the larger one on a tie.
+ *   ramp : host int[steps] output.   Errors: AREA_EINVAL.
+ */
+int area_pool_ramp(int f0, int f_min, int steps, int Hg, int Wg, int* ramp);
+
+/*
+ * area_window_sides -- Phase II window side per step ([ai] Phase II: windows
+ * shrink geometrically from w_start to w_min): w_t = w0 * (w_min / w0)^(t /
+ * (steps - 1)) in double precision, rounded to the nearest multiple of 8
+ * (halves up), at least 8.
+ *   sides : host int[steps] output.   Errors: AREA_EINVAL.
+ */
+int area_window_sides(int w0, int w_min, int steps, int* sides);
+
+/*
+ * area_bridge_lattice -- cells per axis of the global-KV bridge for window
+ * side w ([ai] Phase II: R = (rho w)^2 tokens, rho = 0.5): round(0.5 * side)
+ * per axis of the window clipped to the grid, at least 1, at most the grid
+ * side.  Outputs are host ints.   Errors: AREA_EINVAL.
+ */
+int area_bridge_lattice(int w, int Hg, int Wg, int* ry, int* rx);
+
+/*
+ * area_phase_switch -- number of Phase I steps for a sampler's noise levels
+ * ([ai] "Scheduling the switch": Phase I ends at a noise level sigma*, not at
+ * a step count; [wiki] usage notes: sigma* between 0.86 and 0.96 for the
+ * tuned models).  Phase I is the leading run of steps with
+ * sigmas[t] >= sigma_star (fp32 comparison); every later step is Phase II.
+ *   sigmas : host float[steps], the sampler's noise level at each step.
+ * Errors: AREA_EINVAL.
+ */
+int area_phase_switch(const float* sigmas, int steps, float sigma_star,
+                      int* n_phase1);
+
+/*
+ * area_schedule -- the whole AReA schedule of a sampling run: the phase
+ * switch above, the pooling ramp f0 -> f_min over the Phase I steps and the
+ * window sides w0 -> w_min over the Phase II steps.
+ *   kind  : host int[steps] output, AREA_PHASE_COARSE or AREA_PHASE_WINDOW;
+ *   param : host int[steps] output, the pooling factor f (Phase I) or the
+ *           window side w (Phase II) of each step.
+ * The step calls are then area_pool_kv + area_coarse_attn (Phase I) and
+ * area_dwt_detail + area_window_plan + area_window_attn (Phase II), all
+ * asynchronous on one stream, so a whole schedule can be captured in one
+ * CUDA graph.   Errors: AREA_EINVAL.
+ */
+int area_schedule(const float* sigmas, int steps, float sigma_star, int f0,
+                  int f_min, int w0, int w_min, int Hg, int Wg, int* kind,
+                  int* param);
 
 #ifdef __cplusplus
 }  /* extern "C" */

@@ -133,6 +133,46 @@ def pool_ramp(f0: int, f_min: int, steps: int, Hg: int, Wg: int) -> List[int]:
     return out
 
 
+def window_sides(w0: int, w_min: int, steps: int) -> List[int]:
+    """Phase II window side per step ([ai] Phase II: windows shrink
+    geometrically from w_start to w_min).  Reading: the geometric sequence
+    w0 * (w_min / w0)^(t / (steps - 1)), each value rounded to the nearest
+    multiple of 8 (halves up), at least 8."""
+    out = []
+    for t in range(steps):
+        e = t / (steps - 1) if steps > 1 else 0.0
+        w = w0 * (w_min / w0) ** e
+        out.append(max(8, 8 * int(math.floor(w / 8 + 0.5))))
+    return out
+
+
+def phase_switch(sigmas: Sequence[float], sigma_star: float) -> int:
+    """Number of Phase I steps ([ai] "Scheduling the switch": the transition
+    is a noise level sigma*, not a step count).  Reading: Phase I is the
+    leading run of steps whose noise level is at least sigma* (compared in
+    float32); every later step is Phase II."""
+    star = np.float32(sigma_star)
+    n = 0
+    for sg in sigmas:
+        if np.float32(sg) >= star:
+            n += 1
+        else:
+            break
+    return n
+
+
+def phase_schedule(sigmas: Sequence[float], sigma_star: float, f0: int, f_min: int,
+                   w0: int, w_min: int, Hg: int, Wg: int) -> List[Tuple[str, int]]:
+    """The schedule of a sampling run: ("coarse", f) for each Phase I step
+    (the pooling ramp over those steps), then ("window", w) for each Phase II
+    step (the shrinking window sides over those steps)."""
+    n1 = phase_switch(sigmas, sigma_star)
+    n2 = len(sigmas) - n1
+    out = [("coarse", f) for f in (pool_ramp(f0, f_min, n1, Hg, Wg) if n1 else [])]
+    out += [("window", w) for w in (window_sides(w0, w_min, n2) if n2 else [])]
+    return out
+
+
 # ----------------------------------------------------------------------------
 # Phase II: Haar DWT detail map
 # ----------------------------------------------------------------------------

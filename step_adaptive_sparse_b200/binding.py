@@ -22,6 +22,7 @@ AREA_OK, AREA_EINVAL, AREA_EUNSUPPORTED, AREA_ENOSPACE, AREA_ECUDA = 0, 1, 2, 3,
 AREA_DTYPE_F32, AREA_DTYPE_BF16 = 0, 1
 AREA_POOL_MEAN, AREA_POOL_CENTER = 0, 1
 AREA_DETAIL_HH, AREA_DETAIL_ALL3 = 0, 1
+AREA_PHASE_COARSE, AREA_PHASE_WINDOW = 1, 2
 AREA_PLAN_MAGIC = 0x4145524150414C4E
 SECTIONS = ("BASE", "SCORE", "SPLIT", "NWIN", "WIN", "PARENT", "EXT", "GCOUNT", "GIDX",
             "WSUM", "ORDER", "NITEM", "ITEMS", "COVER", "SCRATCH")
@@ -29,6 +30,8 @@ SECTIONS = ("BASE", "SCORE", "SPLIT", "NWIN", "WIN", "PARENT", "EXT", "GCOUNT", 
 EXPORTED = ("area_status_string", "area_last_cuda_error", "area_version", "area_kernel_error",
             "area_pool_kv", "area_coarse_attn_text", "area_window_attn_text",
             "area_bridge_select_ws_bytes", "area_bridge_select", "area_window_attn_bridge",
+            "area_pool_ramp", "area_window_sides", "area_bridge_lattice", "area_phase_switch",
+            "area_schedule",
             "area_coarse_attn", "area_full_attn", "area_dwt_detail", "area_window_plan_bytes",
             "area_window_plan", "area_window_attn_ws_bytes", "area_window_attn")
 
@@ -72,6 +75,11 @@ _SIGS = {
                               _I, _I, _F, _I, _P]),
     "area_window_attn_noalloc": (_I, [_P, _P, _P, ctypes.POINTER(area_plan_cfg), _P, _SZ, _P,
                                       _I, _I, _F, _I, _P]),
+    "area_pool_ramp": (_I, [_I, _I, _I, _I, _I, _P]),
+    "area_window_sides": (_I, [_I, _I, _I, _P]),
+    "area_bridge_lattice": (_I, [_I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
+    "area_phase_switch": (_I, [_P, _I, _F, ctypes.POINTER(_I)]),
+    "area_schedule": (_I, [_P, _I, _F, _I, _I, _I, _I, _I, _I, _P, _P]),
     "area_bridge_select_ws_bytes": (_I, [_I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]),
     "area_bridge_select": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "area_window_attn_bridge": (_I, [_P, _P, _P, _P, _I, ctypes.POINTER(area_plan_cfg), _P, _SZ,
@@ -209,6 +217,53 @@ def area_window_attn_noalloc(q, k, v, cfg: area_plan_cfg, plan, plan_bytes, o, H
     _check(_lib().area_window_attn_noalloc(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(cfg),
                                            _ptr(plan), plan_bytes, _ptr(o), H, D, scale, dtype,
                                            _stream(stream)), "area_window_attn_noalloc")
+
+
+def _ints(n: int):
+    return (ctypes.c_int * n)()
+
+
+def _floats(values):
+    arr = (ctypes.c_float * len(values))(*[float(x) for x in values])
+    return arr
+
+
+def area_pool_ramp(f0: int, f_min: int, steps: int, Hg: int, Wg: int) -> list:
+    out = _ints(max(steps, 1))
+    _check(_lib().area_pool_ramp(f0, f_min, steps, Hg, Wg, out), "area_pool_ramp")
+    return list(out)[:steps]
+
+
+def area_window_sides(w0: int, w_min: int, steps: int) -> list:
+    out = _ints(max(steps, 1))
+    _check(_lib().area_window_sides(w0, w_min, steps, out), "area_window_sides")
+    return list(out)[:steps]
+
+
+def area_bridge_lattice(w: int, Hg: int, Wg: int):
+    ry, rx = _I(0), _I(0)
+    _check(_lib().area_bridge_lattice(w, Hg, Wg, ctypes.byref(ry), ctypes.byref(rx)),
+           "area_bridge_lattice")
+    return ry.value, rx.value
+
+
+def area_phase_switch(sigmas, sigma_star: float) -> int:
+    arr = _floats(sigmas)
+    n = _I(0)
+    _check(_lib().area_phase_switch(arr, len(arr), sigma_star, ctypes.byref(n)),
+           "area_phase_switch")
+    return n.value
+
+
+def area_schedule(sigmas, sigma_star: float, f0: int, f_min: int, w0: int, w_min: int,
+                  Hg: int, Wg: int):
+    """Per step (kind, param): (AREA_PHASE_COARSE, f) or (AREA_PHASE_WINDOW, w)."""
+    arr = _floats(sigmas)
+    n = len(arr)
+    kind, param = _ints(max(n, 1)), _ints(max(n, 1))
+    _check(_lib().area_schedule(arr, n, sigma_star, f0, f_min, w0, w_min, Hg, Wg, kind, param),
+           "area_schedule")
+    return [(kind[t], param[t]) for t in range(n)]
 
 
 def area_bridge_select_ws_bytes(B: int, H: int, Hg: int, Wg: int, D: int) -> int:

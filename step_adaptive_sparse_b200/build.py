@@ -15,7 +15,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libarea.so")
 SOURCES = ["api.cu", "pool_dwt.cu", "plan.cu", "attn_simt.cu", "attn_tc.cu", "noalloc.cu",
-           "bridge.cu"]
+           "bridge.cu", "schedule.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -71,6 +71,10 @@ def test_null_and_bad_arguments_rejected_on_host(area):
         (lambda: area.area_bridge_select(fake, 1, 1, 2, 8, 8, 128, 9, 2, fake, fake, 1024), area.AREA_EINVAL),
         (lambda: area.area_bridge_select(fake, 1, 1, 2, 8, 8, 128, 4, 4, fake, fake, 2047), area.AREA_ENOSPACE),
         (lambda: area.area_bridge_select_ws_bytes(1, 0, 8, 8, 128), area.AREA_EINVAL),
+        (lambda: area.area_pool_ramp(4, 2, 0, 8, 8), area.AREA_EINVAL),
+        (lambda: area.area_window_sides(0, 64, 8), area.AREA_EINVAL),
+        (lambda: area.area_bridge_lattice(0, 8, 8), area.AREA_EINVAL),
+        (lambda: area.area_schedule([], 0.9, 4, 2, 64, 32, 8, 8), area.AREA_EINVAL),
         (lambda: area.area_bridge_select(fake, 1, 1, 2, 8, 8, 96, 4, 4, fake, fake, 4096), area.AREA_EUNSUPPORTED),
         (lambda: area.area_dwt_detail(fake, 1, 0, fake, 1, 8, 8), area.AREA_EINVAL),
         (lambda: area.area_dwt_detail(fake, 1, 4, fake, 1, 8, 8, 9), area.AREA_EINVAL),

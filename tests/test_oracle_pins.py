@@ -15,7 +15,7 @@ import pytest
 import torch
 
 from oracle import area_oracle as ora
-from workloads import CONFIGS, make_detail_source, texture_mask
+from workloads import CONFIGS, flow_sigmas, make_detail_source, texture_mask
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -145,6 +145,62 @@ def test_pool_ramp_reproduces_printed_example():
     g = _golden("ramp_flux4096.json")
     assert ora.pool_ramp(g["f0"], g["f_min"], g["steps"], g["Hg"], g["Wg"]) == g["ramp"]
     assert [g["Hg"] // g["f0"], g["Wg"] // g["f0"]] == g["pooled_grid_at_f0"]
+
+
+def test_phase_switch_reproduces_the_flux_split():
+    # a sampler whose noise level crosses the pages' sigma* range between
+    # steps 8 and 9 gives the 8 Phase I steps the pages state for FLUX.1
+    g = _golden("phase_switch_flux.json")
+    sig = flow_sigmas(g["steps"], 3.0)
+    lo, hi = g["sigma_star_range"]
+    n = g["phase1_steps"]
+    assert lo <= sig[n] < sig[n - 1] <= hi
+    for star in (float(sig[n]) + 1e-4, 0.5 * float(sig[n] + sig[n - 1]), float(sig[n - 1])):
+        assert ora.phase_switch(sig, star) == n
+    assert ora.phase_switch(sig, 1.5) == 0 and ora.phase_switch(sig, 0.0) == g["steps"]
+
+
+def test_phase_switch_is_the_leading_run():
+    # invariant on arbitrary (also non-monotone) lists: every step before the
+    # switch is at or above sigma*, the step at the switch is below it
+    rng = np.random.default_rng(7)
+    for _ in range(200):
+        sig = rng.random(rng.integers(1, 12)).astype(np.float32)
+        star = float(rng.random())
+        n = ora.phase_switch(sig, star)
+        assert all(sig[:n] >= np.float32(star))
+        assert n == len(sig) or sig[n] < np.float32(star)
+    # a later step above sigma* does not re-enter Phase I
+    assert ora.phase_switch([0.99, 0.5, 0.99], 0.9) == 1
+
+
+def test_window_sides_reproduce_the_config_tables():
+    # the configs' 8-step tables (integers) follow the geometric shrink
+    assert ora.window_sides(64, 32, 8) == list(CONFIGS["flux2048"].schedule)
+    assert ora.window_sides(256, 64, 8) == list(CONFIGS["flux4096"].schedule)
+    assert ora.window_sides(192, 64, 8) == list(CONFIGS["flux6144"].schedule)
+    assert ora.window_sides(272, 64, 8) == list(CONFIGS["qwen6144x2048"].schedule)
+
+
+def test_window_sides_are_geometric_up_to_rounding():
+    for w0, wm, n in [(192, 64, 20), (256, 64, 20), (272, 64, 40), (96, 96, 5), (64, 32, 1)]:
+        ws = ora.window_sides(w0, wm, n)
+        assert len(ws) == n and ws[0] == w0 and (n == 1 or ws[-1] == wm)
+        assert all(a >= b for a, b in zip(ws, ws[1:]))
+        assert all(w % 8 == 0 for w in ws)
+        for t, w in enumerate(ws):
+            exact = w0 * (wm / w0) ** (t / (n - 1) if n > 1 else 0.0)
+            assert abs(w - exact) <= 4.0
+
+
+def test_phase_schedule_concatenates_ramp_and_windows():
+    g = _golden("ramp_flux4096.json")
+    sig = flow_sigmas(28, 3.0)
+    sched = ora.phase_schedule(sig, 0.89, g["f0"], g["f_min"], 256, 64, g["Hg"], g["Wg"])
+    assert [p for k, p in sched if k == "coarse"] == g["ramp"]           # printed ramp
+    wins = [p for k, p in sched if k == "window"]
+    assert len(wins) == 20 and wins[0] == 256 and wins[-1] == 64
+    assert [k for k, _ in sched] == ["coarse"] * 8 + ["window"] * 20
 
 
 # --------------------------------------------------------------------------

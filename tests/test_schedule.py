@@ -1,10 +1,12 @@
 """Host schedules of the package against the oracle and the printed example."""
 import json
+
+import numpy as np
 import os
 
 from oracle import area_oracle as ora
 from step_adaptive_sparse_b200 import schedule
-from workloads import CONFIGS
+from workloads import CONFIGS, flow_sigmas
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -34,3 +36,30 @@ def test_bridge_lattice_matches_oracle():
     for cfg in CONFIGS.values():
         for w in list(cfg.schedule) + [2, 5, 1000]:
             assert schedule.bridge_lattice(w, cfg.Hg, cfg.Wg) == ora.bridge_lattice(w, cfg.Hg, cfg.Wg)
+
+
+def test_window_sides_match_oracle():
+    for w0 in (64, 96, 192, 256, 272):
+        for wm in (32, 64, 96):
+            for n in (1, 2, 8, 20, 33):
+                assert schedule.window_schedule(w0, wm, n) == ora.window_sides(w0, wm, n)
+
+
+def test_phase_switch_matches_oracle():
+    rng = np.random.default_rng(3)
+    lists = [flow_sigmas(28, 3.0), flow_sigmas(50, 4.0), np.array([0.99, 0.5, 0.99], np.float32)]
+    lists += [rng.random(rng.integers(1, 30)).astype(np.float32) for _ in range(50)]
+    for sig in lists:
+        for star in (0.0, 0.3, 0.86, 0.89, 0.9, 0.96, 1.0, float(sig[0])):
+            assert schedule.phase_switch(sig, star) == ora.phase_switch(sig, star)
+
+
+def test_schedule_matches_oracle():
+    names = {schedule.PHASE_COARSE: "coarse", schedule.PHASE_WINDOW: "window"}
+    for cfg in CONFIGS.values():
+        for steps, shift, star in [(28, 3.0, 0.89), (28, 3.0, 0.96), (50, 3.0, 0.9), (8, 1.0, 0.5)]:
+            sig = flow_sigmas(steps, shift)
+            w0, wm = cfg.schedule[0], cfg.schedule[-1]
+            got = schedule.schedule(sig, star, cfg.f, 2, w0, wm, cfg.Hg, cfg.Wg)
+            want = ora.phase_schedule(sig, star, cfg.f, 2, w0, wm, cfg.Hg, cfg.Wg)
+            assert [(names[k], p) for k, p in got] == want

@@ -5,4 +5,5 @@ generators.  It contains none of the method's arithmetic: neither the oracle
 nor the CUDA path is imported here, and neither imports this package.
 """
 from .configs import CONFIGS, AreaConfig, get_config  # noqa: F401
-from .synth import make_qkv, make_detail_source, make_text_kv, texture_mask  # noqa: F401
+from .synth import (flow_sigmas, make_detail_source, make_qkv, make_text_kv,  # noqa: F401
+                    texture_mask)

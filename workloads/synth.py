@@ -135,3 +135,16 @@ def make_text_kv(cfg: AreaConfig, T: int, seed: int = 5):
         t = rng.standard_normal((cfg.B, cfg.H, T, cfg.D)).astype(np.float32)
         out.append(round_to_bf16(t) if cfg.dtype == "bf16" else t)
     return tuple(out)
+
+
+def flow_sigmas(steps: int = 28, shift: float = 3.0) -> np.ndarray:
+    """Noise levels of a synthetic flow-matching sampler, float32 [steps].
+
+    Stand-in for the sampler that drives the phase switch (the pages name a
+    noise level sigma* and 28 steps for FLUX.1, but print no noise schedule):
+    times t_i = 1 - i / steps, shifted as sigma = s t / (1 + (s - 1) t).  With
+    28 steps and s = 3 the levels cross the pages' sigma* range 0.86..0.96
+    near step 8.
+    """
+    t = 1.0 - np.arange(steps, dtype=np.float64) / steps
+    return (shift * t / (1.0 + (shift - 1.0) * t)).astype(np.float32)
