@@ -395,6 +395,79 @@ def run_reference(args):
     return 0
 
 
+def schedule_graph_leg(cfg, st, stream, full_ms, steps=28, shift=3.0, sigma_star=0.89):
+    """A whole sampling run of attention calls: the noise-level phase switch
+    over a synthetic flow-matching sampler, the pooling ramp over the Phase I
+    steps and the shrinking windows over the Phase II steps, captured once in
+    one CUDA graph and replayed.  Returns the summary for the JSON line."""
+    import torch
+
+    import step_adaptive_sparse_b200 as area
+    from step_adaptive_sparse_b200 import schedule
+    from workloads import flow_sigmas
+    dev = st.q.device
+    sig = flow_sigmas(steps, shift)
+    sched = schedule.schedule(sig, sigma_star, cfg.f, 2, cfg.schedule[0], cfg.schedule[-1],
+                              cfg.Hg, cfg.Wg)
+    fs = [p for kd, p in sched if kd == schedule.PHASE_COARSE]
+    ws_sides = [p for kd, p in sched if kd == schedule.PHASE_WINDOW]
+    nk_max = max([(cfg.Hg // f) * (cfg.Wg // f) for f in fs], default=1)
+    kp = torch.empty((cfg.B, cfg.H, nk_max, cfg.D), dtype=st.q.dtype, device=dev)
+    vp = torch.empty_like(kp)
+    plans = {}
+    for w in sorted(set(ws_sides)):
+        pc = area.make_cfg(cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
+        nb = area.area_window_plan_bytes(pc)
+        assert area.area_window_attn_ws_bytes(pc, cfg.H, cfg.D) <= st.ws_bytes
+        plans[w] = (pc, torch.empty(nb, dtype=torch.uint8, device=dev), nb)
+
+    def run():
+        for kd, p in sched:
+            if kd == schedule.PHASE_COARSE:
+                nk = (cfg.Hg // p) * (cfg.Wg // p)
+                area.area_pool_kv(st.k, st.v, kp, vp, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, p,
+                                  area.AREA_POOL_MEAN, st.dt, stream)
+                area.area_coarse_attn(st.q, kp, vp, st.o1, cfg.B, cfg.H, cfg.N, nk, cfg.D,
+                                      cfg.scale, st.dt, stream)
+            else:
+                pc, plan, nb = plans[p]
+                area.area_dwt_detail(st.src, st.dt, cfg.C, st.energy, cfg.B, cfg.Hg, cfg.Wg,
+                                     area.AREA_DETAIL_HH, stream)
+                area.area_window_plan(st.energy, pc, plan, nb, stream)
+                area.area_window_attn(st.q, st.k, st.v, pc, plan, nb, st.o2, st.ws, st.ws_bytes,
+                                      cfg.H, cfg.D, cfg.scale, st.dt, stream)
+
+    with torch.cuda.stream(stream):
+        run()                                       # eager pass: capture warm-up, plans
+    torch.cuda.synchronize()
+    flops = sum(4.0 * cfg.B * cfg.H * cfg.N * (cfg.Hg // f) * (cfg.Wg // f) * cfg.D for f in fs)
+    wfl = {w: window_flops(area.parse_plan(pl.cpu().numpy()), cfg.H, cfg.D)
+           for w, (_, pl, _) in plans.items()}
+    flops += sum(wfl[w] for w in ws_sides)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        run()
+    g.replay()
+    torch.cuda.synchronize()
+    reps = 2
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    del g
+    launches = 2 * len(fs) + len(ws_sides) * (1 + plan_launches(cfg.B) + 3)
+    return {"steps": steps, "sampler": f"flow matching, shift {shift}", "sigma_star": sigma_star,
+            "phase1_steps": len(fs), "ramp": fs, "window_sides": ws_sides,
+            "graph_launches": launches, "ms": ms,
+            "tflops": flops / (ms * 1e-3) / 1e12,
+            "speedup_vs_full_attention": steps * full_ms / ms,
+            "note": "all attention calls of the run captured in one CUDA graph; "
+                    "speedup against the same number of full-attention calls"}
+
+
 def run_area(args):
     import torch
 
@@ -571,6 +644,35 @@ def run_area(args):
                   "window_attn_tflops": bflops / (battn_ms * 1e-3) / 1e12}
     del cand, mws, plan0
 
+    # ---- detail map + planner: one cooperative launch against the separate
+    # calls, at the last schedule step (eager, 10 calls each)
+    fused = {}
+    with torch.cuda.stream(stream):
+        i_last = len(cfg.schedule) - 1
+        pc_l, pl_l, nb_l = st.pcfg[i_last], st.plan[i_last], st.plan_bytes[i_last]
+        for tag in ("separate", "fused"):
+            def call():
+                if tag == "fused":
+                    area.area_dwt_window_plan(st.src, st.dt, cfg.C, area.AREA_DETAIL_HH, st.energy,
+                                              pc_l, pl_l, nb_l, stream)
+                else:
+                    area.area_dwt_detail(st.src, st.dt, cfg.C, st.energy, cfg.B, cfg.Hg, cfg.Wg,
+                                         area.AREA_DETAIL_HH, stream)
+                    area.area_window_plan(st.energy, pc_l, pl_l, nb_l, stream)
+            for _ in range(3):
+                call()
+            fa, fb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            fa.record(stream)
+            for _ in range(10):
+                call()
+            fb.record(stream)
+            torch.cuda.synchronize()
+            fused[tag + "_us"] = fa.elapsed_time(fb) / 10 * 1e3
+    fused["launches"] = {"separate": 1 + plan_launches(cfg.B), "fused": 1}
+
+    # ---- a whole 28-step sampling run in one CUDA graph
+    sched_out = None if args.no_graph else schedule_graph_leg(cfg, st, stream, full_ms)
+
     # ---- end to end through the C-ABI from pinned host buffers.  Each step
     # copies its inputs host->device and its output device->host; two device
     # buffer sets let the copies of one step overlap the kernels of the next
@@ -685,6 +787,8 @@ def run_area(args):
             "split_fraction_by_step": splits,
             "phase1_pooling_ramp": ramp_out,
             "pages_bridge_rule": bridge_out,
+            "schedule_28_steps_graph": sched_out,
+            "dwt_plan_one_launch": fused,
             "graph_replay": None if graph_ms is None else {
                 "ms_per_step": graph_ms,
                 "value": step_flops / (graph_ms * 1e-3) / 1e12,

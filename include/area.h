@@ -68,12 +68,14 @@ const char* area_status_string(int status);
 int area_last_cuda_error(void);
 /* Library version, e.g. "libarea 0.1.0 sm_100a". */
 const char* area_version(void);
+#define AREA_KERR_TC_WAIT        1  /* a tensor-core kernel's mbarrier wait expired */
+#define AREA_KERR_PLAN_BARRIER    2  /* a grid barrier of area_dwt_window_plan expired */
 /*
  * area_kernel_error -- synchronises the current device, then reports in
- * *code whether a tensor-core kernel gave up a bounded wait since the last
- * call (0 = none, 1 = a wait expired; that launch's output is invalid), and
- * clears the flag.  Meant for tests and health checks, not the hot path.
- * Errors: AREA_EINVAL (null), AREA_ECUDA.
+ * *code whether a kernel gave up a bounded wait since the last call (0 =
+ * none; else an OR of AREA_KERR_* bits; the output of that launch is
+ * invalid), and clears the flags.  Meant for tests and health checks, not
+ * the hot path.   Errors: AREA_EINVAL (null), AREA_ECUDA.
  */
 int area_kernel_error(int* code);
 
@@ -252,6 +254,26 @@ int area_window_plan_bytes(const area_plan_cfg* cfg, size_t* plan_bytes);
  */
 int area_window_plan(const float* energy, const area_plan_cfg* cfg,
                      void* plan, size_t plan_bytes, cudaStream_t stream);
+
+/*
+ * area_dwt_window_plan -- area_dwt_detail followed by area_window_plan in ONE
+ * cooperative kernel launch (plus a 8-byte memset of the plan's barrier
+ * words): every block runs every stage -- detail map, split scores, windows,
+ * the four radix-sort passes, global-KV lists, merge-weight sums -- over its
+ * share of the work, with a grid barrier between stages.  Results are
+ * bit-identical to the two separate calls.  The grid is at most two blocks of
+ * 256 threads per SM, all resident at once (cooperative launch); each barrier
+ * wait is bounded (2 s), after which the kernel stops and area_kernel_error
+ * reports AREA_KERR_PLAN_BARRIER.
+ *   src, src_dtype, C, mode : as area_dwt_detail (B, Hg, Wg from cfg);
+ *   energy : fp32 [B, Hg/2, Wg/2] output, as area_dwt_detail;
+ *   cfg, plan, plan_bytes   : as area_window_plan.
+ * Errors: as area_dwt_detail and area_window_plan; AREA_ECUDA when the
+ * device cannot co-schedule the grid.
+ */
+int area_dwt_window_plan(const void* src, int src_dtype, int C, int mode,
+                         float* energy, const area_plan_cfg* cfg, void* plan,
+                         size_t plan_bytes, cudaStream_t stream);
 
 /*
  * area_window_attn_ws_bytes -- fp32 merge workspace for area_window_attn:

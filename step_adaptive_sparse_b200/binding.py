@@ -23,6 +23,7 @@ AREA_DTYPE_F32, AREA_DTYPE_BF16 = 0, 1
 AREA_POOL_MEAN, AREA_POOL_CENTER = 0, 1
 AREA_DETAIL_HH, AREA_DETAIL_ALL3 = 0, 1
 AREA_PHASE_COARSE, AREA_PHASE_WINDOW = 1, 2
+AREA_KERR_TC_WAIT, AREA_KERR_PLAN_BARRIER = 1, 2
 AREA_PLAN_MAGIC = 0x4145524150414C4E
 SECTIONS = ("BASE", "SCORE", "SPLIT", "NWIN", "WIN", "PARENT", "EXT", "GCOUNT", "GIDX",
             "WSUM", "ORDER", "NITEM", "ITEMS", "COVER", "SCRATCH")
@@ -30,7 +31,7 @@ SECTIONS = ("BASE", "SCORE", "SPLIT", "NWIN", "WIN", "PARENT", "EXT", "GCOUNT", 
 EXPORTED = ("area_status_string", "area_last_cuda_error", "area_version", "area_kernel_error",
             "area_pool_kv", "area_coarse_attn_text", "area_window_attn_text",
             "area_bridge_select_ws_bytes", "area_bridge_select", "area_window_attn_bridge",
-            "area_pool_ramp", "area_window_sides", "area_bridge_lattice", "area_phase_switch",
+            "area_dwt_window_plan", "area_pool_ramp", "area_window_sides", "area_bridge_lattice", "area_phase_switch",
             "area_schedule",
             "area_coarse_attn", "area_full_attn", "area_dwt_detail", "area_window_plan_bytes",
             "area_window_plan", "area_window_attn_ws_bytes", "area_window_attn")
@@ -75,6 +76,8 @@ _SIGS = {
                               _I, _I, _F, _I, _P]),
     "area_window_attn_noalloc": (_I, [_P, _P, _P, ctypes.POINTER(area_plan_cfg), _P, _SZ, _P,
                                       _I, _I, _F, _I, _P]),
+    "area_dwt_window_plan": (_I, [_P, _I, _I, _I, _P, ctypes.POINTER(area_plan_cfg), _P, _SZ,
+                                  _P]),
     "area_pool_ramp": (_I, [_I, _I, _I, _I, _I, _P]),
     "area_window_sides": (_I, [_I, _I, _I, _P]),
     "area_bridge_lattice": (_I, [_I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
@@ -193,6 +196,13 @@ def area_window_plan_bytes(cfg: area_plan_cfg) -> int:
 def area_window_plan(energy, cfg: area_plan_cfg, plan, plan_bytes: int, stream=None) -> None:
     _check(_lib().area_window_plan(_ptr(energy), ctypes.byref(cfg), _ptr(plan), plan_bytes,
                                    _stream(stream)), "area_window_plan")
+
+
+def area_dwt_window_plan(src, src_dtype, C, mode, energy, cfg: area_plan_cfg, plan, plan_bytes,
+                         stream=None) -> None:
+    _check(_lib().area_dwt_window_plan(_ptr(src), src_dtype, C, mode, _ptr(energy),
+                                       ctypes.byref(cfg), _ptr(plan), plan_bytes,
+                                       _stream(stream)), "area_dwt_window_plan")
 
 
 def area_window_attn_ws_bytes(cfg: area_plan_cfg, H: int, D: int) -> int:

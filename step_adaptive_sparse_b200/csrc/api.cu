@@ -94,7 +94,13 @@ const char* area_version(void) { return "libarea 0.1.0 sm_100a"; }
 
 int area_kernel_error(int* code) {
   if (!code) return AREA_EINVAL;
-  return finish(area::read_and_clear_tc_error(code));
+  int tc = 0, pl = 0;
+  int st = finish(area::read_and_clear_tc_error(&tc));
+  if (st != AREA_OK) return st;
+  st = finish(area::read_and_clear_plan_error(&pl));
+  if (st != AREA_OK) return st;
+  *code = tc | (pl ? AREA_KERR_PLAN_BARRIER : 0);
+  return AREA_OK;
 }
 
 int area_pool_kv(const void* k, const void* v, void* kp, void* vp, int B, int H, int Hg, int Wg,
@@ -152,6 +158,21 @@ int area_window_plan(const float* energy, const area_plan_cfg* cfg, void* plan,
   if (plan_bytes < (size_t)L.total) return AREA_ENOSPACE;
   if ((reinterpret_cast<uintptr_t>(plan) & 255) != 0) return AREA_EINVAL;
   return finish(area::launch_window_plan(energy, cfg, L, plan, stream));
+}
+
+int area_dwt_window_plan(const void* src, int src_dtype, int C, int mode, float* energy,
+                         const area_plan_cfg* cfg, void* plan, size_t plan_bytes,
+                         cudaStream_t stream) {
+  if (!src || !energy || !plan) return AREA_EINVAL;
+  if (C < 1 || (mode != AREA_DETAIL_HH && mode != AREA_DETAIL_ALL3)) return AREA_EINVAL;
+  if (!valid_dtype(src_dtype)) return AREA_EINVAL;
+  area::PlanLayout L;
+  const int st = area::plan_layout(cfg, &L);
+  if (st != AREA_OK) return st;
+  if (plan_bytes < (size_t)L.total) return AREA_ENOSPACE;
+  if ((reinterpret_cast<uintptr_t>(plan) & 255) != 0) return AREA_EINVAL;
+  return finish(area::launch_dwt_window_plan(src, src_dtype, C, mode, energy, cfg, L, plan,
+                                             stream));
 }
 
 int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D, size_t* ws_bytes) {

@@ -28,7 +28,8 @@ struct PlanLayout {
   int64_t ntile_sort;           // 256-element tiles of the radix sort
   int64_t off[AREA_PLAN_NSEC];  // byte offsets of the sections
   int64_t scratch_keys_a, scratch_keys_b, scratch_vals_a, scratch_vals_b,
-          scratch_hist;         // byte offsets inside the buffer
+          scratch_hist,         // byte offsets inside the buffer
+          scratch_bar;          // grid-barrier words of the fused planner
   int64_t total;                // bytes
 };
 
@@ -138,6 +139,13 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, c
                                   const void* vt, int T, const int* cand, int R,
                                   const PlanLayout& L, const void* plan, void* o, float* ws,
                                   int H, float scale, cudaStream_t s);
+// Detail map and planner in one cooperative launch (one memset of the
+// barrier words first); a barrier timeout raises the planner error flag.
+cudaError_t launch_dwt_window_plan(const void* src, int src_dtype, int C, int mode, float* energy,
+                                   const area_plan_cfg* cfg, const PlanLayout& L, void* plan,
+                                   cudaStream_t s);
+cudaError_t read_and_clear_plan_error(int* code);
+
 // Scratch of area_bridge_select: the mean keys [B*H][D] then the chunk sums
 // [B*H][ceil(N/1024)][D], fp32.
 size_t bridge_ws_bytes(int B, int H, int Hg, int Wg, int D);

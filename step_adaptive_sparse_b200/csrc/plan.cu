@@ -13,8 +13,11 @@
 // round-to-nearest operations.  The global-KV ranking is a stable LSD radix
 // sort of the energy bits (descending), which keeps token order among ties.
 #include "area_internal.cuh"
+#include "detail_cell.cuh"
 
 namespace area {
+
+__device__ int g_plan_error = 0;   // set when a fused-planner grid barrier times out
 
 static int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
 
@@ -72,6 +75,7 @@ int plan_layout(const area_plan_cfg* cfg, PlanLayout* L) {
   L->scratch_vals_a = off; off = align256(off + N * 4);
   L->scratch_vals_b = off; off = align256(off + N * 4);
   L->scratch_hist = off;   off = align256(off + 256 * L->ntile_sort * 4);
+  L->scratch_bar = off;    off = align256(off + 8);   // grid barrier of the fused planner
   L->total = off;
   return AREA_OK;
 }
@@ -106,11 +110,17 @@ struct HeaderArgs {
   int64_t v[32];
 };
 
-__global__ void plan_header_kernel(int64_t* hdr, HeaderArgs a, int* nitem_total) {
-  const int i = threadIdx.x;
-  hdr[i] = a.v[i];
-  if (i == 0) *nitem_total = 0;
-}
+// ---------------------------------------------------------------------------
+// Planner stages.  Each stage is a device function over one work item (a
+// base window, a batch element, a block of tokens, a sort tile, a final
+// window) run by a whole thread block; the separate kernels below launch one
+// block per item, the fused kernel loops its blocks over the items and
+// separates the stages with grid barriers.  Thread counts are any multiple of
+// 32 up to 1024, except the sort histogram and scatter (256 threads).
+// No stage pointer is __restrict__: in the fused kernel a stage reads what
+// other blocks wrote before the last grid barrier, which must not go through
+// the non-coherent read-only load path.
+// ---------------------------------------------------------------------------
 
 // Exclusive block-wide scan of one int per thread (blockDim.x multiple of 32,
 // at most 1024).  Returns the exclusive prefix; *total receives the sum.
@@ -144,11 +154,15 @@ __device__ int block_exclusive_scan(int x, int* total) {
   return res;
 }
 
-// Split score of one base window per block.
-__global__ void __launch_bounds__(256) plan_base_kernel(const float* __restrict__ E, PlanView P,
-                                                       float thr) {
-  extern __shared__ float s_rows[];
-  const int b = blockIdx.x / P.nb_cap, bi = blockIdx.x % P.nb_cap;
+__device__ void stage_header(int64_t* hdr, const HeaderArgs& a, int* nitem_total) {
+  if (threadIdx.x < 32) hdr[threadIdx.x] = a.v[threadIdx.x];
+  if (threadIdx.x == 0) *nitem_total = 0;
+}
+
+// Split score of base window `item` = b * nb_cap + bi.
+__device__ void stage_base(const float* E, const PlanView& P, float thr, int item,
+                           float* s_rows) {
+  const int b = item / P.nb_cap, bi = item % P.nb_cap;
   if (bi >= P.nb) return;
   const int iy = bi / P.nbx, ix = bi % P.nbx;
   int y0, hy, x0, wx;
@@ -173,6 +187,7 @@ __global__ void __launch_bounds__(256) plan_base_kernel(const float* __restrict_
     P.score[o] = S;
     P.split[o] = split ? 1 : 0;
   }
+  __syncthreads();                             // s_rows is reused by the next item
 }
 
 __device__ __forceinline__ int4 halo_rect(int4 w, int h, int Hg, int Wg) {
@@ -181,9 +196,8 @@ __device__ __forceinline__ int4 halo_rect(int4 w, int h, int Hg, int Wg) {
   return make_int4(ey0, ex0, ey1 - ey0, ex1 - ex0);
 }
 
-// Final windows, Halo rectangles, G_W and the work list of one batch element.
-__global__ void __launch_bounds__(1024) plan_windows_kernel(PlanView P) {
-  const int b = blockIdx.x;
+// Final windows, Halo rectangles, G_W and the work list of batch element b.
+__device__ void stage_windows(const PlanView& P, int b) {
   const int4* base = P.base + (int64_t)b * P.nb_cap;
   const uint8_t* split = P.split + (int64_t)b * P.nb_cap;
   int4* win = P.win + (int64_t)b * P.nw;
@@ -254,9 +268,10 @@ __global__ void __launch_bounds__(1024) plan_windows_kernel(PlanView P) {
 }
 
 // ---- stable LSD radix sort of (~energy bits, token) ------------------------
-__global__ void __launch_bounds__(256) sort_init_kernel(const float* __restrict__ E, int b,
-                                                       PlanView P, uint32_t* keys, int* vals) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+// Keys and values of the tokens t in [t0, t0 + blockDim.x).
+__device__ void stage_sort_init(const float* E, int b, const PlanView& P,
+                                uint32_t* keys, int* vals, int t0) {
+  const int t = t0 + threadIdx.x;
   if (t >= P.N) return;
   const int y = t / P.Wg, x = t % P.Wg;
   const int Wc = P.Wg / 2;
@@ -265,23 +280,25 @@ __global__ void __launch_bounds__(256) sort_init_kernel(const float* __restrict_
   vals[t] = t;
 }
 
-__global__ void __launch_bounds__(256) sort_hist_kernel(const uint32_t* __restrict__ keys, int n,
-                                                       int shift, uint32_t* hist, int ntile) {
+// Digit histogram of sort tile `tile` (256 threads).
+__device__ void stage_sort_hist(const uint32_t* keys, int n, int shift,
+                                uint32_t* hist, int ntile, int tile) {
   __shared__ uint32_t s_h[256];
   s_h[threadIdx.x] = 0;
   __syncthreads();
-  const int base = blockIdx.x * kSortTile;
+  const int base = tile * kSortTile;
 #pragma unroll 4
   for (int r = 0; r < kSortRounds; ++r) {
     const int i = base + r * 256 + threadIdx.x;
     if (i < n) atomicAdd(&s_h[(keys[i] >> shift) & 255u], 1u);
   }
   __syncthreads();
-  hist[(int64_t)threadIdx.x * ntile + blockIdx.x] = s_h[threadIdx.x];
+  hist[(int64_t)threadIdx.x * ntile + tile] = s_h[threadIdx.x];
+  __syncthreads();
 }
 
 // Exclusive scan, in place, of the digit-major histogram (one block).
-__global__ void __launch_bounds__(1024) sort_scan_kernel(uint32_t* hist, int m) {
+__device__ void stage_sort_scan(uint32_t* hist, int m) {
   const int per = (m + blockDim.x - 1) / blockDim.x;
   const int lo = threadIdx.x * per, hi = min(m, lo + per);
   int sum = 0;
@@ -295,23 +312,26 @@ __global__ void __launch_bounds__(1024) sort_scan_kernel(uint32_t* hist, int m) 
   }
 }
 
-// Stable scatter of one tile: elements are taken in index order (round r,
-// then warp, then lane); each element's rank among equal digits is its
-// rank within its warp, plus the equal digits of earlier warps of the same
-// round, plus those of earlier rounds.
-__global__ void __launch_bounds__(256) sort_scatter_kernel(const uint32_t* __restrict__ kin,
-                                                          const int* __restrict__ vin,
-                                                          uint32_t* kout, int* vout, int n,
-                                                          int shift, const uint32_t* hist,
-                                                          int ntile) {
+// Stable scatter of sort tile `tile` (256 threads): elements are taken in
+// index order (round r, then warp, then lane); each element's rank among
+// equal digits is its rank within its warp, plus the equal digits of earlier
+// warps of the same round, plus those of earlier rounds.
+__device__ void tile_offsets_from_hist(const uint32_t* hist, int ntile, int tile, int* s_run);
+
+// With raw = true the histogram is the unscanned one and the tile's offsets
+// are derived from it in the block.
+__device__ void stage_sort_scatter(const uint32_t* kin, const int* vin,
+                                   uint32_t* kout, int* vout, int n, int shift,
+                                   const uint32_t* hist, int ntile, int tile, bool raw = false) {
   __shared__ int s_cnt[8][257];
   __shared__ int s_run[256];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  s_run[threadIdx.x] = (int)hist[(int64_t)threadIdx.x * ntile + blockIdx.x];
+  if (raw) tile_offsets_from_hist(hist, ntile, tile, s_run);
+  else s_run[threadIdx.x] = (int)hist[(int64_t)threadIdx.x * ntile + tile];
   for (int r = 0; r < kSortRounds; ++r) {
     for (int j = threadIdx.x; j < 8 * 257; j += 256) (&s_cnt[0][0])[j] = 0;
     __syncthreads();
-    const int i = blockIdx.x * kSortTile + r * 256 + threadIdx.x;
+    const int i = tile * kSortTile + r * 256 + threadIdx.x;
     const bool valid = i < n;
     const uint32_t key = valid ? kin[i] : 0u;
     const int val = valid ? vin[i] : 0;
@@ -338,11 +358,32 @@ __global__ void __launch_bounds__(256) sort_scatter_kernel(const uint32_t* __res
     __syncthreads();
     s_run[dd] += run;
   }
+  __syncthreads();
 }
 
-// Global-KV bridge: first G_W tokens of the ranked order outside ext(W).
-__global__ void __launch_bounds__(1024) plan_global_kernel(PlanView P) {
-  const int b = blockIdx.x / P.nw, wi = blockIdx.x % P.nw;
+// Digit offsets of sort tile `tile` straight from the raw (unscanned)
+// digit-major histogram: s_run[d] = (keys of all tiles with a smaller digit)
+// + (keys of earlier tiles with digit d).  The same integers the scan stage
+// produces, so the fused kernel can skip that stage and its barriers.
+__device__ void tile_offsets_from_hist(const uint32_t* hist, int ntile, int tile, int* s_run) {
+  const int d = threadIdx.x;                   // 256 threads, one digit each
+  const uint32_t* row = hist + (int64_t)d * ntile;
+  int before = 0, all = 0;
+  for (int t = 0; t < ntile; ++t) {
+    const int h = (int)row[t];
+    before += t < tile ? h : 0;
+    all += h;
+  }
+  int total;
+  const int smaller = block_exclusive_scan(all, &total);
+  s_run[d] = smaller + before;
+  __syncthreads();
+}
+
+// Global-KV bridge of final window `item` = b * nw + wi: the first G_W
+// tokens of the ranked order outside ext(W).
+__device__ void stage_global(const PlanView& P, int item) {
+  const int b = item / P.nw, wi = item % P.nw;
   if (wi >= P.nwin[b] || P.G == 0) return;
   const int64_t o = (int64_t)b * P.nw + wi;
   const int4 e = P.ext[o];
@@ -365,9 +406,10 @@ __global__ void __launch_bounds__(1024) plan_global_kernel(PlanView P) {
   for (int j = gw + threadIdx.x; j < P.G; j += blockDim.x) out[j] = -1;
 }
 
-// Sum of tent weights, and count, of the final windows that contain each token.
-__global__ void __launch_bounds__(256) plan_wsum_kernel(PlanView P) {
-  const int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+// Sum of tent weights, and count, of the final windows that contain each of
+// the tokens g in [g0, g0 + blockDim.x) (g = b * N + t).
+__device__ void stage_wsum(const PlanView& P, int64_t g0) {
+  const int64_t g = g0 + threadIdx.x;
   if (g >= (int64_t)P.B * P.N) return;
   const int b = (int)(g / P.N);
   const int t = (int)(g % P.N);
@@ -395,12 +437,177 @@ __global__ void __launch_bounds__(256) plan_wsum_kernel(PlanView P) {
   P.cover[g] = count;
 }
 
+// ---------------------------------------------------------------------------
+// One launch per stage
+// ---------------------------------------------------------------------------
+__global__ void plan_header_kernel(int64_t* hdr, HeaderArgs a, int* nitem_total) {
+  stage_header(hdr, a, nitem_total);
+}
+
+__global__ void __launch_bounds__(256) plan_base_kernel(const float* __restrict__ E, PlanView P,
+                                                       float thr) {
+  extern __shared__ float s_rows[];
+  stage_base(E, P, thr, blockIdx.x, s_rows);
+}
+
+__global__ void __launch_bounds__(1024) plan_windows_kernel(PlanView P) {
+  stage_windows(P, blockIdx.x);
+}
+
+__global__ void __launch_bounds__(256) sort_init_kernel(const float* __restrict__ E, int b,
+                                                       PlanView P, uint32_t* keys, int* vals) {
+  stage_sort_init(E, b, P, keys, vals, blockIdx.x * blockDim.x);
+}
+
+__global__ void __launch_bounds__(256) sort_hist_kernel(const uint32_t* __restrict__ keys, int n,
+                                                       int shift, uint32_t* hist, int ntile) {
+  stage_sort_hist(keys, n, shift, hist, ntile, blockIdx.x);
+}
+
+__global__ void __launch_bounds__(1024) sort_scan_kernel(uint32_t* hist, int m) {
+  stage_sort_scan(hist, m);
+}
+
+__global__ void __launch_bounds__(256) sort_scatter_kernel(const uint32_t* __restrict__ kin,
+                                                          const int* __restrict__ vin,
+                                                          uint32_t* kout, int* vout, int n,
+                                                          int shift, const uint32_t* hist,
+                                                          int ntile) {
+  stage_sort_scatter(kin, vin, kout, vout, n, shift, hist, ntile, blockIdx.x);
+}
+
+__global__ void __launch_bounds__(1024) plan_global_kernel(PlanView P) {
+  stage_global(P, blockIdx.x);
+}
+
+__global__ void __launch_bounds__(256) plan_wsum_kernel(PlanView P) {
+  stage_wsum(P, blockIdx.x * (int64_t)blockDim.x);
+}
+
+// ---------------------------------------------------------------------------
+// Detail map + planner in one cooperative launch.  Every block runs every
+// stage over its share of the items; a grid barrier separates the stages.
+// The barrier is a monotone arrival counter in the plan's scratch (zeroed by
+// the launcher); each wait is bounded by kPlanWaitNs of %globaltimer, after
+// which the block raises the abort word, records g_plan_error and returns,
+// and every other block leaves at its next barrier.
+// ---------------------------------------------------------------------------
+constexpr int kFusedThreads = 256;
+constexpr uint64_t kPlanWaitNs = 2000000000ull;
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ bool grid_sync(unsigned* bar, unsigned target, int* s_ok) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();                           // this block's writes, then its arrival
+    atomicAdd(bar, 1u);
+    const uint64_t t0 = global_ns();
+    int ok = 1;
+    for (;;) {
+      unsigned v, ab;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+      if (v >= target) break;
+      asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(ab) : "l"(bar + 1) : "memory");
+      if (ab != 0u || global_ns() - t0 > kPlanWaitNs) {
+        ok = 0;
+        atomicExch(bar + 1, 1u);
+        atomicExch(&g_plan_error, 1);
+        break;
+      }
+      __nanosleep(32);
+    }
+    __threadfence();
+    *s_ok = ok;
+  }
+  __syncthreads();
+  return *s_ok != 0;
+}
+
+struct FusedArgs {
+  const void* src;       // detail source [B, N, C] (DWT stage), else null
+  int C;
+  float inv_c;           // fl32(1 / C)
+  float* energy;         // [B, Hg/2, Wg/2]
+  float thr;
+  int64_t* hdr;
+  uint32_t *ka, *kb, *hist;
+  int *va, *vb;
+  int nt;                // sort tiles
+  unsigned* bar;         // [arrivals, abort]
+};
+
+template <typename T, int MODE, bool VEC>
+__global__ void __launch_bounds__(kFusedThreads, 2) plan_fused_kernel(PlanView P, FusedArgs A,
+                                                                  HeaderArgs h) {
+  extern __shared__ float s_rows[];
+  __shared__ int s_ok;
+  unsigned nbar = 0;
+  auto sync = [&]() { return grid_sync(A.bar, ++nbar * gridDim.x, &s_ok); };
+  const int G = gridDim.x;
+  const int n = P.N;
+  // detail map
+  if (A.src) {
+    const int64_t ncell = (int64_t)P.B * (P.Hg / 2) * (P.Wg / 2);
+    for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < ncell;
+         g += (int64_t)G * blockDim.x)
+      A.energy[g] = detail_cell<T, MODE, VEC>(static_cast<const T*>(A.src), A.C, g, P.Hg, P.Wg,
+                                              A.inv_c);
+    if (!sync()) return;
+  }
+  // header, split scores, sort keys of element 0
+  {
+    const int nbase = P.B * P.nb_cap, ninit = (n + blockDim.x - 1) / blockDim.x;
+    if (blockIdx.x == 0) stage_header(A.hdr, h, P.nitem + P.B);
+    for (int it = blockIdx.x; it < nbase + ninit; it += G) {
+      if (it < nbase) stage_base(A.energy, P, A.thr, it, s_rows);
+      else stage_sort_init(A.energy, 0, P, A.ka, A.va, (it - nbase) * blockDim.x);
+    }
+    if (!sync()) return;
+  }
+  for (int b = 0; b < P.B; ++b) {
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 8 * pass;
+      const uint32_t* kin = (pass & 1) ? A.kb : A.ka;
+      const int* vin = (pass & 1) ? A.vb : A.va;
+      uint32_t* kout = (pass & 1) ? A.ka : A.kb;
+      int* vout = (pass == 3) ? P.order + (int64_t)b * n : ((pass & 1) ? A.va : A.vb);
+      // histogram (the first pass of element 0 also builds the windows)
+      const int nwin_items = (b == 0 && pass == 0) ? P.B : 0;
+      for (int it = blockIdx.x; it < nwin_items + A.nt; it += G) {
+        if (it < nwin_items) stage_windows(P, it);
+        else stage_sort_hist(kin, n, shift, A.hist, A.nt, it - nwin_items);
+      }
+      if (!sync()) return;
+      for (int it = blockIdx.x; it < A.nt; it += G)
+        stage_sort_scatter(kin, vin, kout, vout, n, shift, A.hist, A.nt, it, /*raw=*/true);
+      if (!sync()) return;
+    }
+    if (b + 1 < P.B) {                         // keys of the next element
+      for (int it = blockIdx.x; it < (n + (int)blockDim.x - 1) / (int)blockDim.x; it += G)
+        stage_sort_init(A.energy, b + 1, P, A.ka, A.va, it * blockDim.x);
+      if (!sync()) return;
+    }
+  }
+  // global-KV lists and merge-weight sums
+  {
+    const int nglob = P.B * P.nw;
+    const int nws = (int)(((int64_t)P.B * n + blockDim.x - 1) / blockDim.x);
+    for (int it = blockIdx.x; it < nglob + nws; it += G) {
+      if (it < nglob) stage_global(P, it);
+      else stage_wsum(P, (int64_t)(it - nglob) * blockDim.x);
+    }
+  }
+}
+
 }  // namespace
 
-cudaError_t launch_window_plan(const float* energy, const area_plan_cfg* cfg,
-                               const PlanLayout& L, void* plan, cudaStream_t s) {
-  PlanView P = plan_view(L, plan);
-  char* base = static_cast<char*>(plan);
+namespace {
+HeaderArgs header_args(const PlanLayout& L) {
   HeaderArgs h = {};
   h.v[0] = AREA_PLAN_MAGIC; h.v[1] = AREA_PLAN_VERSION;
   h.v[2] = L.B; h.v[3] = L.Hg; h.v[4] = L.Wg; h.v[5] = L.w; h.v[6] = L.halo; h.v[7] = L.G;
@@ -411,6 +618,15 @@ cudaError_t launch_window_plan(const float* energy, const area_plan_cfg* cfg,
   h.v[12 + AREA_PLAN_NSEC] = L.nb;
   h.v[13 + AREA_PLAN_NSEC] = L.sy;
   h.v[14 + AREA_PLAN_NSEC] = L.sx;
+  return h;
+}
+}  // namespace
+
+cudaError_t launch_window_plan(const float* energy, const area_plan_cfg* cfg,
+                               const PlanLayout& L, void* plan, cudaStream_t s) {
+  PlanView P = plan_view(L, plan);
+  char* base = static_cast<char*>(plan);
+  const HeaderArgs h = header_args(L);
   plan_header_kernel<<<1, 32, 0, s>>>(reinterpret_cast<int64_t*>(base), h, P.nitem + L.B);
   const int smem = (int)(L.hy * sizeof(float));
   if (smem > 48 * 1024) {
@@ -443,6 +659,81 @@ cudaError_t launch_window_plan(const float* energy, const area_plan_cfg* cfg,
   const int64_t ntok = L.B * L.N;
   plan_wsum_kernel<<<(unsigned)((ntok + 255) / 256), 256, 0, s>>>(P);
   return cudaGetLastError();
+}
+
+template <typename T, int MODE, bool VEC>
+static cudaError_t launch_fused_typed(const PlanLayout& L, const PlanView& P, const FusedArgs& A,
+                                     const HeaderArgs& h, cudaStream_t s) {
+  auto fn = plan_fused_kernel<T, MODE, VEC>;
+  const int smem = (int)(L.hy * sizeof(float)) > 16 ? (int)(L.hy * sizeof(float)) : 16;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kFusedThreads, smem)) !=
+      cudaSuccess)
+    return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const int grid = sms * (per_sm < 2 ? per_sm : 2);  // every block resident at once
+  if ((e = cudaMemsetAsync(A.bar, 0, 2 * sizeof(unsigned), s)) != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kFusedThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fn, P, A, h);
+}
+
+cudaError_t launch_dwt_window_plan(const void* src, int src_dtype, int C, int mode, float* energy,
+                                   const area_plan_cfg* cfg, const PlanLayout& L, void* plan,
+                                   cudaStream_t s) {
+  PlanView P = plan_view(L, plan);
+  char* base = static_cast<char*>(plan);
+  FusedArgs A = {};
+  A.src = src;
+  A.C = C;
+  A.inv_c = 1.0f / (float)C;                   // host IEEE division: fl32(1 / C)
+  A.energy = energy;
+  A.thr = cfg->split_thr;
+  A.hdr = reinterpret_cast<int64_t*>(base);
+  A.ka = reinterpret_cast<uint32_t*>(base + L.scratch_keys_a);
+  A.kb = reinterpret_cast<uint32_t*>(base + L.scratch_keys_b);
+  A.va = reinterpret_cast<int*>(base + L.scratch_vals_a);
+  A.vb = reinterpret_cast<int*>(base + L.scratch_vals_b);
+  A.hist = reinterpret_cast<uint32_t*>(base + L.scratch_hist);
+  A.nt = (int)L.ntile_sort;
+  A.bar = reinterpret_cast<unsigned*>(base + L.scratch_bar);
+  const HeaderArgs h = header_args(L);
+  const bool vec = C % (src_dtype == AREA_DTYPE_BF16 ? 8 : 4) == 0 &&
+                   (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+#define AREA_FUSED(T, M, V) launch_fused_typed<T, M, V>(L, P, A, h, s)
+  if (src_dtype == AREA_DTYPE_BF16) {
+    if (mode == AREA_DETAIL_HH)
+      return vec ? AREA_FUSED(__nv_bfloat16, AREA_DETAIL_HH, true)
+                 : AREA_FUSED(__nv_bfloat16, AREA_DETAIL_HH, false);
+    return vec ? AREA_FUSED(__nv_bfloat16, AREA_DETAIL_ALL3, true)
+               : AREA_FUSED(__nv_bfloat16, AREA_DETAIL_ALL3, false);
+  }
+  if (mode == AREA_DETAIL_HH)
+    return vec ? AREA_FUSED(float, AREA_DETAIL_HH, true) : AREA_FUSED(float, AREA_DETAIL_HH, false);
+  return vec ? AREA_FUSED(float, AREA_DETAIL_ALL3, true) : AREA_FUSED(float, AREA_DETAIL_ALL3, false);
+#undef AREA_FUSED
+}
+
+cudaError_t read_and_clear_plan_error(int* code) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyFromSymbol(code, g_plan_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_plan_error, &zero, sizeof(int));
 }
 
 }  // namespace area

@@ -8,6 +8,7 @@
 // token cell per channel, energy averaged over channels, in exact-order fp32
 // so that split decisions downstream are reproducible bit for bit.
 #include "area_internal.cuh"
+#include "detail_cell.cuh"
 
 namespace area {
 namespace {
@@ -92,58 +93,16 @@ __global__ void __launch_bounds__(256) pool_kv_kernel(const T* __restrict__ k,
   }
 }
 
-// ---------------------------------------------------------------------------
-// Haar detail energy.  Exact fp32 order: no contraction (explicit _rn ops).
-// ---------------------------------------------------------------------------
-template <int MODE>
-__device__ __forceinline__ float cell_energy(float a, float b, float c, float d) {
-  const float amb = __fsub_rn(a, b), cmd = __fsub_rn(c, d);
-  const float hh = __fmul_rn(__fsub_rn(amb, cmd), 0.5f);
-  if (MODE == AREA_DETAIL_HH) return __fmul_rn(hh, hh);
-  const float lh = __fmul_rn(__fsub_rn(__fadd_rn(a, b), __fadd_rn(c, d)), 0.5f);
-  const float hl = __fmul_rn(__fadd_rn(amb, cmd), 0.5f);
-  return __fadd_rn(__fadd_rn(__fmul_rn(lh, lh), __fmul_rn(hl, hl)), __fmul_rn(hh, hh));
-}
-
-// One thread per 2x2 cell; the C channels of each of the four tokens are
-// read as 16-byte vectors when C fills whole vectors (VEC), else one by one.
+// One thread per 2x2 cell (the cell arithmetic is in detail_cell.cuh).
 template <typename T, int MODE, bool VEC>
 __global__ void __launch_bounds__(256) dwt_detail_kernel(const T* __restrict__ src, int C,
                                                          float* __restrict__ energy, int B,
                                                          int Hg, int Wg) {
-  const int Hc = Hg / 2, Wc = Wg / 2;
-  const int64_t ncell = (int64_t)B * Hc * Wc;
+  const int64_t ncell = (int64_t)B * (Hg / 2) * (Wg / 2);
   const float inv = __frcp_rn((float)C);
   for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < ncell;
-       g += (int64_t)gridDim.x * blockDim.x) {
-    const int cx = (int)(g % Wc);
-    const int64_t r = g / Wc;
-    const int cy = (int)(r % Hc);
-    const int64_t b = r / Hc;
-    const int64_t t00 = (b * Hg + 2 * cy) * (int64_t)Wg + 2 * cx;
-    const T* pa = src + t00 * C;
-    const T* pb = pa + C;
-    const T* pc = pa + (int64_t)Wg * C;
-    const T* pd = pc + C;
-    float acc = 0.f;
-    if (VEC) {
-      constexpr int NV = Vec<T>::n;
-      for (int c0 = 0; c0 < C; c0 += NV) {
-        float a[NV], bb[NV], c[NV], d[NV];
-        Vec<T>::load(pa + c0, a);
-        Vec<T>::load(pb + c0, bb);
-        Vec<T>::load(pc + c0, c);
-        Vec<T>::load(pd + c0, d);
-#pragma unroll
-        for (int i = 0; i < NV; ++i) acc = __fadd_rn(acc, cell_energy<MODE>(a[i], bb[i], c[i], d[i]));
-      }
-    } else {
-      for (int c = 0; c < C; ++c)
-        acc = __fadd_rn(acc, cell_energy<MODE>(load_as_float(pa, c), load_as_float(pb, c),
-                                               load_as_float(pc, c), load_as_float(pd, c)));
-    }
-    energy[g] = __fmul_rn(acc, inv);
-  }
+       g += (int64_t)gridDim.x * blockDim.x)
+    energy[g] = detail_cell<T, MODE, VEC>(src, C, g, Hg, Wg, inv);
 }
 
 int grid_for(int64_t work, int block) {

@@ -72,6 +72,10 @@ def test_null_and_bad_arguments_rejected_on_host(area):
         (lambda: area.area_bridge_select(fake, 1, 1, 2, 8, 8, 128, 4, 4, fake, fake, 2047), area.AREA_ENOSPACE),
         (lambda: area.area_bridge_select_ws_bytes(1, 0, 8, 8, 128), area.AREA_EINVAL),
         (lambda: area.area_pool_ramp(4, 2, 0, 8, 8), area.AREA_EINVAL),
+        (lambda: area.area_dwt_window_plan(None, 1, 16, 0, fake, area.make_cfg(1, 16, 16, 8, 1, 4, 0.1), fake, 1 << 20), area.AREA_EINVAL),
+        (lambda: area.area_dwt_window_plan(fake, 1, 16, 7, fake, area.make_cfg(1, 16, 16, 8, 1, 4, 0.1), fake, 1 << 20), area.AREA_EINVAL),
+        (lambda: area.area_dwt_window_plan(fake, 1, 16, 0, fake, area.make_cfg(1, 16, 16, 8, 1, 4, 0.1), fake, 256), area.AREA_ENOSPACE),
+        (lambda: area.area_dwt_window_plan(fake, 1, 16, 0, fake, area.make_cfg(1, 15, 16, 8, 1, 4, 0.1), fake, 1 << 20), area.AREA_EINVAL),
         (lambda: area.area_window_sides(0, 64, 8), area.AREA_EINVAL),
         (lambda: area.area_bridge_lattice(0, 8, 8), area.AREA_EINVAL),
         (lambda: area.area_schedule([], 0.9, 4, 2, 64, 32, 8, 8), area.AREA_EINVAL),

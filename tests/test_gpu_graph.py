@@ -71,3 +71,69 @@ def test_schedule_step_graph_replay_matches_eager(name):
         assert (o.float() - r.float()).abs().max().item() <= tol
     assert area.area_kernel_error() == 0
     del g
+
+
+def test_whole_sampling_run_in_one_graph():
+    # 28 steps of a synthetic flow-matching sampler: the noise-level switch,
+    # the pooling ramp over Phase I and the shrinking windows over Phase II,
+    # every call of the run captured in one graph
+    from step_adaptive_sparse_b200 import schedule
+    from workloads import flow_sigmas
+    cfg = CONFIGS["flux2048"]
+    dt = area.AREA_DTYPE_BF16
+    q, k, v = (torch.from_numpy(x).cuda().to(torch.bfloat16) for x in make_qkv(cfg))
+    src = torch.from_numpy(make_detail_source(cfg)).cuda().to(torch.bfloat16)
+    sched = schedule.schedule(flow_sigmas(28, 3.0), 0.89, 4, 2, 64, 32, cfg.Hg, cfg.Wg)
+    kinds = [kd for kd, _ in sched]
+    assert kinds == [schedule.PHASE_COARSE] * 8 + [schedule.PHASE_WINDOW] * 20
+    fs = [p for kd, p in sched if kd == schedule.PHASE_COARSE]
+    assert fs == [4, 4, 4, 4, 2, 2, 2, 2]
+    kp = torch.empty((cfg.B, cfg.H, cfg.N // 4, cfg.D), dtype=torch.bfloat16, device="cuda")
+    vp = torch.empty_like(kp)
+    energy = torch.empty((cfg.B, cfg.Hg // 2, cfg.Wg // 2), dtype=torch.float32, device="cuda")
+    plans, wsb = {}, 0
+    for w in {p for kd, p in sched if kd == schedule.PHASE_WINDOW}:
+        pc = area.make_cfg(cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
+        nb = area.area_window_plan_bytes(pc)
+        plans[w] = (pc, torch.empty(nb, dtype=torch.uint8, device="cuda"), nb)
+        wsb = max(wsb, area.area_window_attn_ws_bytes(pc, cfg.H, cfg.D))
+    ws = torch.empty(wsb // 4, dtype=torch.float32, device="cuda")
+    o1, o2 = torch.empty_like(q), torch.empty_like(q)
+    outs1, outs2 = [], []
+
+    def run(keep):
+        for kd, p in sched:
+            if kd == schedule.PHASE_COARSE:
+                nk = (cfg.Hg // p) * (cfg.Wg // p)
+                area.area_pool_kv(k, v, kp, vp, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, p,
+                                  area.AREA_POOL_MEAN, dt, stream)
+                area.area_coarse_attn(q, kp, vp, o1, cfg.B, cfg.H, cfg.N, nk, cfg.D, cfg.scale,
+                                      dt, stream)
+                if keep:
+                    outs1.append(o1.clone())
+            else:
+                pc, plan, nb = plans[p]
+                area.area_dwt_detail(src, dt, cfg.C, energy, cfg.B, cfg.Hg, cfg.Wg,
+                                     area.AREA_DETAIL_HH, stream)
+                area.area_window_plan(energy, pc, plan, nb, stream)
+                area.area_window_attn(q, k, v, pc, plan, nb, o2, ws, wsb, cfg.H, cfg.D,
+                                      cfg.scale, dt, stream)
+                if keep:
+                    outs2.append(o2.clone())
+
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        run(True)                                   # eager, per-step outputs kept
+    torch.cuda.synchronize()
+    o1.zero_()
+    o2.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        run(False)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(o1, outs1[-1])               # last Phase I step (f = 2)
+    assert (o2.float() - outs2[-1].float()).abs().max().item() <= 2e-3
+    assert not torch.equal(outs1[0], outs1[-1])     # the ramp changed the pooled grid
+    assert area.area_kernel_error() == 0
+    del g

@@ -140,6 +140,66 @@ def test_plan_edge_cases(Hg, Wg, w, h, G, thr):
 
 
 # ---------------------------------------------------------------------------
+# Detail map + planner in one cooperative launch: bit-identical to the two
+# separate calls (whose output the tests above pin to the oracle)
+# ---------------------------------------------------------------------------
+
+def _plan_pair(dsrc, C, dtype, B, Hg, Wg, w, h, G, thr, seed=0, mode=gr.area.AREA_DETAIL_HH):
+    pcfg = gr.area.make_cfg(B, Hg, Wg, w, h, G, thr, seed)
+    nb = gr.area.area_window_plan_bytes(pcfg)
+    p_sep = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    p_fus = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    e_sep = torch.zeros((B, Hg // 2, Wg // 2), dtype=torch.float32, device="cuda")
+    e_fus = torch.zeros_like(e_sep)
+    gr.area.area_dwt_detail(dsrc, gr.area_dtype(dtype), C, e_sep, B, Hg, Wg, mode)
+    gr.area.area_window_plan(e_sep, pcfg, p_sep, nb)
+    gr.area.area_dwt_window_plan(dsrc, gr.area_dtype(dtype), C, mode, e_fus, pcfg, p_fus, nb)
+    torch.cuda.synchronize()
+    assert gr.area.area_kernel_error() == 0
+    assert torch.equal(e_fus.view(torch.int32), e_sep.view(torch.int32))
+    # header and every section up to the sort scratch, byte for byte
+    hdr = p_sep[:256].cpu().numpy().view(np.int64)
+    end = int(hdr[10 + gr.area.SECTIONS.index("SCRATCH")])
+    assert torch.equal(p_fus[:end], p_sep[:end])
+    return e_fus, p_fus
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_fused_dwt_plan_matches_separate_calls(name):
+    cfg = CONFIGS[name]
+    dsrc = gr.to_dev(gr.host_src(name), cfg.dtype)
+    for step in sorted({0, len(cfg.schedule) // 2, len(cfg.schedule) - 1}):
+        _plan_pair(dsrc, cfg.C, cfg.dtype, cfg.B, cfg.Hg, cfg.Wg, cfg.schedule[step], cfg.halo,
+                   cfg.G, cfg.split_thr)
+    # seeded border jitter and Halo widths
+    _plan_pair(dsrc, cfg.C, cfg.dtype, cfg.B, cfg.Hg, cfg.Wg, cfg.schedule[-1], cfg.halo, cfg.G,
+               cfg.split_thr, seed=99)
+
+
+@pytest.mark.parametrize("B,C,Hg,Wg,w,h,G,thr,dtype,mode", [
+    (2, 16, 40, 28, 12, 6, 9, 0.2, "bf16", 0),     # two batch elements
+    (3, 5, 34, 18, 9, 1, 7, 0.25, "fp32", 0),      # odd channel count: scalar loads
+    (1, 16, 64, 48, 24, 4, 130, 0.3, "bf16", 1),   # all three detail bands
+    (1, 8, 6, 6, 2, 3, 40, 9.0, "fp32", 0),        # halo larger than the window
+])
+def test_fused_dwt_plan_edge_cases(B, C, Hg, Wg, w, h, G, thr, dtype, mode):
+    rng = np.random.default_rng(B * 1000 + Hg)
+    src = rng.standard_normal((B, Hg * Wg, C)).astype(np.float32)
+    src[:, : Hg * Wg // 3] *= 0.05                 # smooth part: some windows split
+    dsrc = gr.to_dev(src, dtype)
+    e, plan = _plan_pair(dsrc, C, dtype, B, Hg, Wg, w, h, G, thr, seed=0, mode=mode)
+    # and against the oracle directly
+    hsrc = gr.to_host(dsrc).astype(np.float32)
+    E = ora.dwt_detail(hsrc, Hg, Wg, "hh" if mode == 0 else "all3")
+    assert np.array_equal(e.cpu().numpy().view(np.uint32), E.view(np.uint32))
+    got = gr.parse(plan)
+    for b in range(B):
+        want = ora.window_plan(E[b], Hg, Wg, w, h, G, thr)
+        gr.compare_plan(got, want, b)
+        _check_items(got, want, b)
+
+
+# ---------------------------------------------------------------------------
 # Per-configuration tests (grouped by config: inputs are generated once)
 # ---------------------------------------------------------------------------
 
