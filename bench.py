@@ -452,8 +452,9 @@ def schedule_graph_leg(cfg, st, stream, full_ms, steps=28, shift=3.0, sigma_star
     reps = 2
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(reps):
-        g.replay()
+    with torch.cuda.stream(stream):                 # replay() launches on the current stream
+        for _ in range(reps):
+            g.replay()
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
@@ -792,7 +793,8 @@ def run_area(args):
             "graph_replay": None if graph_ms is None else {
                 "ms_per_step": graph_ms,
                 "value": step_flops / (graph_ms * 1e-3) / 1e12,
-                "note": "the same step captured once in a CUDA graph (192 launches) and replayed"},
+                "note": f"the same step captured once in a CUDA graph ({st.launches} launches) "
+                        "and replayed"},
             "speedup_vs_full_attention": (full_ms * (n1 + len(cfg.schedule))) / ms_step,
         }
         print(json.dumps(line), flush=True)
