@@ -21,7 +21,9 @@
 //               thread owns one query row (TMEM lane 32*(warp mod 4) + lane).
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.  P (bf16)
 // overwrites the first 64 columns of its S tile and feeds the PV MMA straight
-// from TMEM.  Online softmax rescales O in TMEM only when some row of a warp
+// from TMEM.  P is handed over in two parts of 64 keys, each with its own
+// barrier, so the PV product of the first part runs while the softmax
+// computes the second.  Online softmax rescales O in TMEM only when some row of a warp
 // sees its running maximum grow by more than 2^8 (the final normalisation uses
 // the same stale maximum in numerator and denominator, so the result is exact).
 // Every branch around a .sync.aligned tcgen05 instruction is warp-uniform.
@@ -44,6 +46,8 @@ constexpr int kTileBytes = 128 * 128 * 2;
 constexpr int kHalfBytes = 128 * 128;   // 128 rows x 64 bf16
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr int kMaxChains = 8;                // independent partial maxima of a score row
+constexpr int kPParts = 2;                   // P handed to the PV product in this many parts
 // Window keys: the Halo rectangle is covered by patches of kPW x kPH tokens,
 // one 128-key tile each, loaded by a 3-D tiled TMA box (tokens of one grid
 // row are contiguous).  Only the global-KV list is gathered row by row.
@@ -62,7 +66,9 @@ enum {
   BAR_S_FULL0, BAR_S_FULL1,
   BAR_P_FULL0, BAR_P_FULL1,
   BAR_O_FULL0, BAR_O_FULL1,
-  BAR_KV_FULL,                       // kStages of them
+  BAR_P_PART0,                       // kPParts - 1 per query tile: leading parts of P stored
+  BAR_P_PART1 = BAR_P_PART0 + kPParts - 1,
+  BAR_KV_FULL = BAR_P_PART1 + kPParts - 1,  // kStages of them
   BAR_KV_EMPTY = BAR_KV_FULL + kStages,
   BAR_DRAIN = BAR_KV_EMPTY + kStages,  // MMA completion before TMEM release
   BAR_COUNT
@@ -430,6 +436,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     mbar_init(bar(BAR_S_FULL1), 1);
     mbar_init(bar(BAR_P_FULL0), 128);
     mbar_init(bar(BAR_P_FULL1), 128);
+    for (int h = 0; h < kPParts - 1; ++h) {
+      mbar_init(bar(BAR_P_PART0 + h), 128);
+      mbar_init(bar(BAR_P_PART1 + h), 128);
+    }
     mbar_init(bar(BAR_O_FULL0), 1);
     mbar_init(bar(BAR_O_FULL1), 1);
     for (int s = 0; s < kStages; ++s) {
@@ -560,6 +570,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           mma_ts(d, p_tmem + kk * 8, sdesc(vs + kk * 2048, kHalfBytes, 1024), kIdescPV,
                  (first && kk == 0) ? 0u : 1u);
       };
+      // PV over part h of the tile's keys (128 / kPParts keys, 16 per instruction)
+      auto pv_part = [&](uint32_t d, uint32_t p_tmem, uint32_t vs, bool first, int h) {
+        constexpr int kPer = 8 / kPParts;
+#pragma unroll
+        for (int kk = kPer * h; kk < kPer * h + kPer; ++kk)
+          mma_ts(d, p_tmem + kk * 8, sdesc(vs + kk * 2048, kHalfBytes, 1024), kIdescPV,
+                 (first && kk == 0) ? 0u : 1u);
+      };
+      // PV of one query tile, part by part as the softmax hands P over
+      auto pv_parts = [&](uint32_t d, uint32_t p_tmem, uint32_t vs, bool first, int bpart,
+                          int bfull, uint32_t cnt) {
+#pragma unroll
+        for (int h = 0; h < kPParts; ++h) {
+          const uint32_t b = h + 1 < kPParts ? bar(bpart + h) : bar(bfull);
+          if (!mbar_wait(b, cnt & 1u, abort_flag)) return false;
+          tc_fence_after();
+          pv_part(d, p_tmem, vs, first, h);
+        }
+        return true;
+      };
+      (void)pv;
       for (int u = blockIdx.x; u < prm.num_units && ok; u += gridDim.x) {
         const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T, BRIDGE ? prm.cand : nullptr, prm.R);
         if (!x.valid) continue;
@@ -581,10 +612,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const uint32_t kn = kv_it + 2 * j + 2;
           if (!(ok = mbar_wait(bar(BAR_KV_FULL + vi % kStages), (vi / kStages) & 1u, abort_flag)))
             break;
-          if (!(ok = mbar_wait(bar(BAR_P_FULL0), p_cnt0 & 1u, abort_flag))) break;
+          if (!(ok = pv_parts(tO0, tS0, kv_addr(vi), j == 0, BAR_P_PART0, BAR_P_FULL0, p_cnt0)))
+            break;
           ++p_cnt0;
-          tc_fence_after();
-          pv(tO0, tS0, kv_addr(vi), j == 0);
           if (j == nt - 1) mma_commit(bar(BAR_O_FULL0));
           if (j + 1 < nt) {
             if (!(ok = mbar_wait(bar(BAR_KV_FULL + kn % kStages), (kn / kStages) & 1u,
@@ -594,10 +624,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             qk(tS0, q0s, kv_addr(kn));
             mma_commit(bar(BAR_S_FULL0));
           }
-          if (!(ok = mbar_wait(bar(BAR_P_FULL1), p_cnt1 & 1u, abort_flag))) break;
+          if (!(ok = pv_parts(tO1, tS1, kv_addr(vi), j == 0, BAR_P_PART1, BAR_P_FULL1, p_cnt1)))
+            break;
           ++p_cnt1;
-          tc_fence_after();
-          pv(tO1, tS1, kv_addr(vi), j == 0);
           if (j == nt - 1) mma_commit(bar(BAR_O_FULL1));
           mma_commit(bar(BAR_KV_EMPTY + vi % kStages));
           if (j + 1 < nt) {
@@ -630,6 +659,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t tO = tmem + lane_off + (qt ? 384u : 256u);
     const uint32_t bS = bar(qt ? BAR_S_FULL1 : BAR_S_FULL0);
     const uint32_t bP = bar(qt ? BAR_P_FULL1 : BAR_P_FULL0);
+    const int bPpart = qt ? BAR_P_PART1 : BAR_P_PART0;
     const uint32_t bO = bar(qt ? BAR_O_FULL1 : BAR_O_FULL0);
     uint32_t s_cnt = 0, o_cnt = 0;
     const float sl2 = prm.scale_log2;
@@ -645,6 +675,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ew = x0.ext.w; eh = x0.ext.z;
       }
       float m = -INFINITY, l = 0.f;
+      int pcx = 0, pcy = 0;                          // patch of tile j in the Halo rectangle
       for (int j = 0; j < nt; ++j) {
         if (!(ok = warp_wait_all(bS, s_cnt & 1u, abort_flag))) break;
         ++s_cnt;
@@ -682,21 +713,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               if (i >= valid) sr[i] = 0xff800000u;        // -inf: no weight
           }
         } else {
-          const int rem_x = ew - (j % ncx) * kPW, rem_y = eh - (j / ncx) * kPH;
+          const int rem_x = ew - pcx * kPW, rem_y = eh - pcy * kPH;
           if (rem_x < kPW || rem_y < kPH) {
 #pragma unroll
             for (int i = 0; i < 128; ++i)
               if ((i % kPW) >= rem_x || (i / kPW) >= rem_y) sr[i] = 0xff800000u;
           }
         }
-        // row maximum: four independent partial maxima, then combine
-        float pm[4];
+        // row maximum: kMaxChains independent partial maxima, then a tree
+        float pm[kMaxChains];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) pm[t] = __uint_as_float(sr[t]);
+        for (int t = 0; t < kMaxChains; ++t) pm[t] = __uint_as_float(sr[t]);
 #pragma unroll
-        for (int i = 4; i < 128; i += 2)
-          pm[(i >> 1) & 3] = max3(pm[(i >> 1) & 3], __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
-        const float mx = max3(pm[0], pm[1], fmaxf(pm[2], pm[3]));
+        for (int i = kMaxChains; i < 128; i += 2)
+          pm[(i >> 1) % kMaxChains] = max3(pm[(i >> 1) % kMaxChains],
+                                                __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
+#pragma unroll
+        for (int t = kMaxChains / 2; t > 0; t >>= 1)
+#pragma unroll
+          for (int q = 0; q < t; ++q) pm[q] = fmaxf(pm[q], pm[q + t]);
+        const float mx = pm[0];
         const float mnew = fmaxf(mx * sl2, m);
         // Rescale O only when some row of the warp gained more than 2^8; the
         // decision is warp-uniform because the TMEM accesses are .sync.aligned.
@@ -705,34 +741,45 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (j == 0 || rescale) m = mnew;
         l *= alpha;
         // P = exp2(S * scale * log2(e) - m) as bf16, two keys per TMEM column,
-        // written over the S columns already read
-        // packed pairs go in place into sr[0..63]: slot i/2 was already read
+        // packed in place into sr[0..63] (slot i/2 was already read).  The
+        // first 64 keys go out first, so the PV product can start on them
+        // while the second 64 are computed; O is rescaled before that first
+        // hand-over, so the PV products of this tile accumulate onto it.
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
         const float negm = -m;
 #pragma unroll
-        for (int i = 0; i < 128; i += 2) {
-          float x0, x1;
-          fma2(x0, x1, __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]), sl2, negm);
-          const float p0 = fast_exp2(x0);
-          const float p1 = fast_exp2(x1);
-          if ((i >> 1) & 1) add2(ls[2], ls[3], p0, p1); else add2(ls[0], ls[1], p0, p1);
-          sr[i >> 1] = pack_bf16(p0, p1);
+        for (int h = 0; h < kPParts; ++h) {
+          constexpr int kKeys = 128 / kPParts;
+#pragma unroll
+          for (int i = kKeys * h; i < kKeys * h + kKeys; i += 2) {
+            float x0, x1;
+            fma2(x0, x1, __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]), sl2, negm);
+            const float p0 = fast_exp2(x0);
+            const float p1 = fast_exp2(x1);
+            if ((i >> 1) & 1) add2(ls[2], ls[3], p0, p1); else add2(ls[0], ls[1], p0, p1);
+            sr[i >> 1] = pack_bf16(p0, p1);
+          }
+          if (h == 0 && rescale) {
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t orr[32];
+              tmem_ld32(tO + c * 32, orr);
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+              tmem_st32(tO + c * 32, orr);
+            }
+          }
+          tmem_st32(tS + 32 * h, *reinterpret_cast<const uint32_t(*)[32]>(&sr[32 * h]));
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(h + 1 < kPParts ? bar(bPpart + h) : bP);
         }
         l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-        tmem_st64(tS, sr);
-        if (rescale) {
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t orr[32];
-            tmem_ld32(tO + c * 32, orr);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
-            tmem_st32(tO + c * 32, orr);
-          }
+        if (WINDOW && ++pcx == ncx) {
+          pcx = 0;
+          ++pcy;
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bP);
       }
       if (!ok) break;
       // epilogue (the unit is looked up again rather than kept live in
