@@ -34,7 +34,7 @@ if ROOT not in sys.path:
 
 METRIC = "AReA attention TFLOP/s per schedule step (bf16, 1 B200)"
 # Bumped whenever attn_tc.cu changes, so that stale DRAM counters are not reported.
-KERNEL_REVISION = "attn_tc r8 (patch loader, f32x2 softmax, single-cover stores, text-key tiles, bridge variant, 8-chain max, P in two parts)"
+KERNEL_REVISION = "attn_tc r9 (patch loader, f32x2 softmax, single-cover stores, text-key tiles, bridge variant, 8-chain max, P in two parts, cover read ahead of the O wait)"
 DEFAULT_CONFIG = "flux6144"
 
 

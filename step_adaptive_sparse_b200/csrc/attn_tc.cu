@@ -785,6 +785,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       // epilogue (the unit is looked up again rather than kept live in
       // registers across the key loop)
       const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T, BRIDGE ? prm.cand : nullptr, prm.R);
+      int cover1 = 1;              // window: this row's token lies in one window only
+      if constexpr (WINDOW) {      // (read before the wait, so its latency overlaps it)
+        const int qp = x.q0 + qt * 128 + row;
+        cover1 = prm.P.cover[(int64_t)x.b * Ntok + window_query_token(x, qp, Wg)];
+      }
       if (!(ok = warp_wait_all(bO, o_cnt & 1u, abort_flag))) break;
       ++o_cnt;
       tc_fence_after();
@@ -814,7 +819,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // A token inside one window only takes that window's output as it is;
         // tokens in overlaps add their tent-weighted share to the workspace.
         const int tok = window_query_token(x, qpos, Wg);
-        const bool single = prm.P.cover[(int64_t)x.b * Ntok + tok] == 1;
+        const bool single = cover1 == 1;
         const int y = tok / Wg, xx = tok % Wg;
         const float t = (float)(min(y - x.win.x + 1, x.win.x + x.win.z - y) *
                                 min(xx - x.win.y + 1, x.win.y + x.win.w - xx));
