@@ -677,19 +677,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       float m = -INFINITY, l = 0.f;
       int pcx = 0, pcy = 0;                          // patch of tile j in the Halo rectangle
       for (int j = 0; j < nt; ++j) {
-        if (!(ok = warp_wait_all(bS, s_cnt & 1u, abort_flag))) break;
-        ++s_cnt;
-        tc_fence_after();
-        uint32_t sr[128];
-        tmem_ld128(tS, sr);
-        // Key validity (warp-uniform): dense, global-KV and text tiles are a
-        // prefix of `valid` keys; a rectangle patch keeps columns dx < rem_x of
-        // rows dy < rem_y (key k = dy * kPW + dx).
-        if (BRIDGE && j >= ntr && j < nti) {
-          // bridge candidates: drop those past the list or inside the Halo
-          // rectangle; lane l tests keys 4l..4l+3 and ballots the result
+        // Bridge candidates: drop those past the list or inside the Halo
+        // rectangle; lane l tests keys 4l..4l+3 and ballots the result.  This
+        // does not depend on S, so it is done before waiting for S (the loads
+        // overlap the wait) and before S occupies 128 registers.
+        const bool bridge_tile = BRIDGE && j >= ntr && j < nti;
+        uint32_t keep[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+        if (bridge_tile) {
           const Unit xb = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T, prm.cand, prm.R);
-          uint32_t keep[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int p = (j - ntr) * 128 + lane * 4 + i;
@@ -701,6 +696,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             keep[i] = __ballot_sync(0xffffffffu, ok);
           }
+        }
+        if (!(ok = warp_wait_all(bS, s_cnt & 1u, abort_flag))) break;
+        ++s_cnt;
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld128(tS, sr);
+        // Key validity (warp-uniform): dense, global-KV and text tiles are a
+        // prefix of `valid` keys; a rectangle patch keeps columns dx < rem_x of
+        // rows dy < rem_y (key k = dy * kPW + dx).
+        if (bridge_tile) {
 #pragma unroll
           for (int i = 0; i < 128; ++i)
             if (!((keep[i & 3] >> (i >> 2)) & 1u)) sr[i] = 0xff800000u;
