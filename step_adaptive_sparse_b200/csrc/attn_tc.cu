@@ -533,7 +533,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t kv_it = 0, unit_count = 0, s_cnt0 = 0, s_cnt1 = 0;
+      uint32_t kv_it = 0, unit_count = 0;
       uint32_t p_cnt0 = 0, p_cnt1 = 0;
       const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
       const uint32_t q0s = sbase + kSmemQ, q1s = sbase + kSmemQ + kTileBytes;
@@ -545,12 +545,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
           mma_ss(d, sdesc(qs + off, 16, 1024), sdesc(ks + off, 16, 1024), kIdescQK, kk > 0);
         }
-      };
-      auto pv = [&](uint32_t d, uint32_t p_tmem, uint32_t vs, bool first) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(d, p_tmem + kk * 8, sdesc(vs + kk * 2048, kHalfBytes, 1024), kIdescPV,
-                 (first && kk == 0) ? 0u : 1u);
       };
       // PV over part h of the tile's keys (128 / kPParts keys, 16 per instruction)
       auto pv_part = [&](uint32_t d, uint32_t p_tmem, uint32_t vs, bool first, int h) {
@@ -572,7 +566,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         return true;
       };
-      (void)pv;
       for (int u = blockIdx.x; u < prm.num_units && ok; u += gridDim.x) {
         const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T, BRIDGE ? prm.cand : nullptr, prm.R);
         if (!x.valid) continue;
@@ -621,8 +614,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         kv_it += 2 * nt;
         ++unit_count;
       }
-      (void)s_cnt0;
-      (void)s_cnt1;
       // Drain: every MMA issued by this thread has completed (bounded wait).
       int drain_abort = 0;
       mma_commit(bar(BAR_DRAIN));
