@@ -363,6 +363,24 @@ def oracle_sample(cfg, q, k, v, src, budget_s: float = 15.0, rows_per_call: int 
 # arms
 # ---------------------------------------------------------------------------
 
+def l2_note(cfg) -> str:
+    tensor = cfg.B * cfg.H * cfg.N * cfg.D * (2 if cfg.dtype == "bf16" else 4)
+    rel = "larger" if tensor > 126e6 else "smaller"
+    return f"inputs {rel} than L2 ({tensor / 1e9:.2f} GB per Q/K/V tensor, L2 126 MB)"
+
+
+def workload_config(cfg, heads: int, world: int, sharded: bool) -> dict:
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": cfg.name, "grid": [cfg.Hg, cfg.Wg], "tokens": cfg.N,
+            "heads": heads, "head_dim": cfg.D, "batch": cfg.B, "pool_f": cfg.f,
+            "schedule": list(cfg.schedule), "halo": cfg.halo, "G": cfg.G,
+            "split_thr": cfg.split_thr, "phase1_calls": len(cfg.schedule),
+            "phase2_calls": len(cfg.schedule),
+            "l2": l2_note(cfg),
+            "parallelism": (f"heads sharded over {world} GPUs, {-(-heads // world)} or fewer "
+                            "per GPU" if sharded else f"replicas x{world}")}
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -385,8 +403,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * float(np.median(secs)), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": cfg.name, "grid": [cfg.Hg, cfg.Wg], "heads": cfg.H,
-                       "head_dim": cfg.D, "batch": cfg.B, "parallelism": "replicas"},
+            "config": workload_config(cfg, cfg.H, args.gpus, False),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -757,15 +774,7 @@ def run_area(args):
             "scaling": "strong" if sharded else "weak",
             "vs_baseline": None,
             "dtype": "bf16" if cfg.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": {"workload": cfg.name, "grid": [cfg.Hg, cfg.Wg], "tokens": cfg.N,
-                       "heads": H_all, "head_dim": cfg.D, "batch": cfg.B, "pool_f": cfg.f,
-                       "schedule": list(cfg.schedule), "halo": cfg.halo, "G": cfg.G,
-                       "split_thr": cfg.split_thr, "phase1_calls": n1,
-                       "phase2_calls": len(cfg.schedule),
-                       "l2": "inputs larger than L2 (0.9 GB per Q/K/V tensor)",
-                       "parallelism": (f"heads sharded over {world} GPUs, "
-                                       f"{cfg.H} or fewer per GPU" if sharded
-                                       else f"replicas x{world}")},
+            "config": workload_config(cfg, H_all, world, sharded),
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,

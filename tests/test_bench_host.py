@@ -137,3 +137,20 @@ def test_head_sharded_job_value_over_gloo():
     for r in range(3):
         total, ms = out[r]
         assert total == 24.0e12 and ms == 102.0           # whole problem over the slowest rank
+
+
+def test_reference_arm_line(capsys, monkeypatch):
+    # the reference arm (the oracle on the host cores) prints the contract's
+    # keys with the same config object as the device arm
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    import json
+    assert bench.main(["--impl", "reference", "--config", "tiny", "--steps", "1", "--warmup", "0",
+                       "--ref-budget", "0.5"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "TFLOP/s" and line["higher_is_better"] is True and line["value"] > 0
+    assert line["config"] == bench.workload_config(CONFIGS["tiny"], CONFIGS["tiny"].H, 1, False)
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
