@@ -153,3 +153,23 @@ def test_binding_has_no_oracle_dependency():
                 text = open(os.path.join(dirpath, fn)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle", text, flags=re.M), fn
                 assert "area_oracle" not in text, fn
+
+
+def test_plain_c_consumer(tmp_path):
+    # the header and the shared library are usable from C alone: compile a C
+    # program against include/area.h, link libarea.so and run its host checks
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    cuda_inc = next((p for p in ("/usr/local/cuda/include",) if os.path.isdir(p)), None)
+    if gcc is None or cuda_inc is None:
+        pytest.skip("gcc or the CUDA headers are not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.join(root, "step_adaptive_sparse_b200", "lib")
+    exe = str(tmp_path / "c_abi_check")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(root, "include"),
+                    "-I", cuda_inc, os.path.join(root, "tests", "c_abi_check.c"),
+                    "-L", libdir, "-larea", f"-Wl,-rpath,{libdir}", "-o", exe], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert "C-ABI host checks passed" in r.stdout
