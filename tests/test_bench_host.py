@@ -154,3 +154,40 @@ def test_reference_arm_line(capsys, monkeypatch):
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_clock_summary_reads_the_sampled_csv(tmp_path):
+    # nvidia-smi rows: index, sm, max sm, power, active, hw, hw_thermal, sw_thermal, sw_power_cap
+    path = tmp_path / "clocks.csv"
+    path.write_text("\n".join([
+        "0, 1965, 1965, 300.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "0, 1800, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1750, 1965, 998.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 300, 1965, 80.0, 0x0, Not Active, Not Active, Not Active, Not Active",   # idle sample
+        "garbage line",
+    ]) + "\n")
+    cs = bench.ClockSampler(0)
+    cs.path = str(path)
+    cs.proc = object()                               # as if nvidia-smi had run
+    s = cs.summary()
+    assert s["sm_max_mhz"] == 1965.0 and s["samples"] == 4
+    assert s["sm_mhz"] == 1800.0                     # median of the samples under load
+    assert s["reasons"] == ["sw_power_cap"]
+    path.write_text("0, 1500, 1965, 700.0, 0x8, Not Active, Active, Not Active, Not Active\n")
+    assert bench.ClockSampler.summary(cs)["reasons"] == ["hw_thermal_slowdown"]
+
+
+def test_clock_summary_without_nvidia_smi():
+    cs = bench.ClockSampler(0)
+    assert cs.summary() == {"sm_mhz": None, "sm_max_mhz": None,
+                            "reasons": ["nvidia-smi unavailable"]}
+
+
+def test_traffic_is_null_for_another_kernel_revision(monkeypatch):
+    # roofline.traffic comes from the committed DRAM capture only while it was
+    # taken from the same build of the kernel
+    got = bench.load_traffic("flux6144", "window_attn")
+    assert got is not None and got > 0
+    monkeypatch.setattr(bench, "KERNEL_REVISION", "some later build")
+    assert bench.load_traffic("flux6144", "window_attn") is None
+    assert bench.load_traffic("no-such-workload", "window_attn") is None
