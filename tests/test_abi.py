@@ -173,3 +173,14 @@ def test_plain_c_consumer(tmp_path):
     r = subprocess.run([exe], capture_output=True, text=True)
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
     assert "C-ABI host checks passed" in r.stdout
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    # no fallback: without the built library every call raises
+    from step_adaptive_sparse_b200 import binding
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "libarea.so"))
+    monkeypatch.setattr(binding, "_LIB", None)
+    with pytest.raises(ImportError):
+        binding.area_version()
+    with pytest.raises(ImportError):
+        binding.area_pool_ramp(4, 2, 8, 256, 256)
