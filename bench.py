@@ -24,6 +24,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -145,10 +146,11 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, path: str = ""):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{gpu_index}.csv")
+        self.path = path or os.path.join(tempfile.gettempdir(),
+                                         f"area_bench_clocks_{gpu_index}.csv")
 
     def __enter__(self):
         try:
@@ -531,7 +533,7 @@ def run_area(args):
     barrier(dist, local)
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clocks:
+    with ClockSampler(local, args.clocks_csv) as clocks:
         time.sleep(0.3)
         ev0.record(stream)
         with torch.cuda.stream(stream):
@@ -823,6 +825,9 @@ def main(argv=None):
     ap.add_argument("--ref-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay leg")
+    ap.add_argument("--clocks-csv", default="",
+                    help="where to keep the nvidia-smi clock samples of the timed region "
+                         "(default: the system temporary directory)")
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="N > 1: independent replicas (weak scaling) or the heads of one "
                          "problem split across ranks (strong scaling)")
