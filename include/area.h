@@ -26,9 +26,12 @@
  *     accumulation, D = 128 or 64) or AREA_DTYPE_F32 (storage fp32, fp32
  *     CUDA-core arithmetic, D = 64 or 128).
  *   - Every kernel call is asynchronous on the given stream (0 = legacy
- *     default stream), never synchronises the host and never waits on
- *     another CTA.  The return value reports argument validation and launch
- *     errors only; AREA_ECUDA carries the CUDA error, see area_status_string.
+ *     default stream) and never synchronises the host.  No CTA waits on
+ *     another, except in area_dwt_window_plan: a cooperative launch (every
+ *     CTA resident) whose grid barriers are bounded waits.  The return value
+ *     reports argument validation and launch errors only; AREA_ECUDA carries
+ *     the CUDA error, see area_status_string.  The schedule functions at the
+ *     end are host arithmetic (no device memory, no stream).
  *   - Device pointers passed to the attention calls must be 16-byte aligned.
  */
 #ifndef AREA_H_
