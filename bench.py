@@ -521,9 +521,13 @@ def run_area(args):
         for _ in range(args.warmup):
             st.run()
     torch.cuda.synchronize()
-    kerr = area.area_kernel_error()
+    # every rank learns of a bounded-wait expiry on any rank, and all stop
+    # together instead of leaving the others in the next collective
+    kerr = reduce_max(dist, float(area.area_kernel_error()), device=str(dev))
     if kerr:
-        raise SystemExit("bench.py: a tensor-core kernel gave up a bounded wait in warm-up")
+        if dist is not None:
+            dist.destroy_process_group()
+        raise SystemExit("bench.py: a kernel gave up a bounded wait in warm-up")
     win_flops, win_per_step = st.window_flops_per_step()
     splits = st.split_fractions()
     step_flops = phase1_flops(cfg) * st.n_phase1 + win_flops

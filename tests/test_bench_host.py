@@ -191,3 +191,32 @@ def test_traffic_is_null_for_another_kernel_revision(monkeypatch):
     monkeypatch.setattr(bench, "KERNEL_REVISION", "some later build")
     assert bench.load_traffic("flux6144", "window_attn") is None
     assert bench.load_traffic("no-such-workload", "window_attn") is None
+
+
+def _error_worker(rank, world, port, out):
+    # a failure seen by one rank reaches every rank through the same
+    # collective, so all of them take the same exit
+    import datetime
+
+    import torch.distributed as dist
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        local_error = 1.0 if rank == 1 else 0.0
+        out[rank] = bench.reduce_max(dist, local_error)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_one_ranks_error_reaches_all_ranks():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_error_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    assert out[0] == 1.0 and out[1] == 1.0
