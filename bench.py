@@ -422,14 +422,13 @@ def schedule_graph_leg(cfg, st, stream, full_ms, steps=28, shift=3.0, sigma_star
     import torch
 
     import step_adaptive_sparse_b200 as area
-    from step_adaptive_sparse_b200 import schedule
     from workloads import flow_sigmas
     dev = st.q.device
     sig = flow_sigmas(steps, shift)
-    sched = schedule.schedule(sig, sigma_star, cfg.f, 2, cfg.schedule[0], cfg.schedule[-1],
-                              cfg.Hg, cfg.Wg)
-    fs = [p for kd, p in sched if kd == schedule.PHASE_COARSE]
-    ws_sides = [p for kd, p in sched if kd == schedule.PHASE_WINDOW]
+    sched = area.area_schedule(sig, sigma_star, cfg.f, 2, cfg.schedule[0], cfg.schedule[-1],
+                               cfg.Hg, cfg.Wg)
+    fs = [p for kd, p in sched if kd == area.AREA_PHASE_COARSE]
+    ws_sides = [p for kd, p in sched if kd == area.AREA_PHASE_WINDOW]
     nk_max = max([(cfg.Hg // f) * (cfg.Wg // f) for f in fs], default=1)
     kp = torch.empty((cfg.B, cfg.H, nk_max, cfg.D), dtype=st.q.dtype, device=dev)
     vp = torch.empty_like(kp)
@@ -442,7 +441,7 @@ def schedule_graph_leg(cfg, st, stream, full_ms, steps=28, shift=3.0, sigma_star
 
     def run():
         for kd, p in sched:
-            if kd == schedule.PHASE_COARSE:
+            if kd == area.AREA_PHASE_COARSE:
                 nk = (cfg.Hg // p) * (cfg.Wg // p)
                 area.area_pool_kv(st.k, st.v, kp, vp, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, p,
                                   area.AREA_POOL_MEAN, st.dt, stream)
@@ -592,8 +591,7 @@ def run_area(args):
 
     # ---- Phase I with the pages' pooling ramp (f0 -> 2 over the 8 steps),
     # measured once after the timed region (the configs' step uses a fixed f)
-    from step_adaptive_sparse_b200 import schedule
-    ramp = schedule.pool_ramp(cfg.f, 2, st.n_phase1, cfg.Hg, cfg.Wg)
+    ramp = area.area_pool_ramp(cfg.f, 2, st.n_phase1, cfg.Hg, cfg.Wg)
     nk_max = (cfg.Hg // min(ramp)) * (cfg.Wg // min(ramp))
     kp_r = torch.empty((cfg.B, cfg.H, nk_max, cfg.D), dtype=q.dtype, device=dev)
     vp_r = torch.empty_like(kp_r)
@@ -623,9 +621,8 @@ def run_area(args):
 
     # ---- the pages' own bridge rule on the last (smallest) window size,
     # measured once: candidate selection plus window attention
-    from step_adaptive_sparse_b200 import schedule as _sched
     w_b = cfg.schedule[-1]
-    ry, rx = _sched.bridge_lattice(w_b, cfg.Hg, cfg.Wg)
+    ry, rx = area.area_bridge_lattice(w_b, cfg.Hg, cfg.Wg)
     cand = torch.empty((cfg.B, cfg.H, ry * rx), dtype=torch.int32, device=dev)
     mws = torch.empty(area.area_bridge_select_ws_bytes(cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D) // 4,
                       dtype=torch.float32, device=dev)

@@ -379,12 +379,14 @@ int area_window_attn_bridge(const void* q, const void* k, const void* v,
  * which every GPU that loads libarea holds until the process exits.
  *
  *   Arguments: as area_window_attn, without ws / ws_bytes.
- *   Limit: B * H * Hg * Wg * D * 4 bytes must not exceed 32 MiB
- *          (e.g. 2 heads of a 128x128 grid at D = 128); larger sizes return
- *          AREA_ENOSPACE before anything is launched.
- *   Set-up: the first call on a device looks up the array's device address
- *          (cudaGetSymbolAddress, with that device current); make that first
- *          call outside any stream capture.  It allocates nothing.
+ *   Limit: the workspace area_window_attn would need,
+ *          area_window_attn_ws_bytes(cfg, H, D), must not exceed 32 MiB;
+ *          larger sizes return AREA_ENOSPACE before anything is launched.
+ *   Set-up: the first call in a CUDA context (per device; again after
+ *          cudaDeviceReset or under another context) looks up the array's
+ *          device address with cudaGetSymbolAddress, with that device
+ *          current; make that first call outside any stream capture.  It
+ *          allocates nothing and calls no cudaMalloc / cudaFree.
  *   Sharing: all calls on a device use the same array.  It keeps the last
  *          call's contents; each call clears it before use.  Calls that
  *          overlap on the GPU (other streams, other threads) race on it and

@@ -34,7 +34,8 @@ EXPORTED = ("area_status_string", "area_last_cuda_error", "area_version", "area_
             "area_dwt_window_plan", "area_pool_ramp", "area_window_sides", "area_bridge_lattice", "area_phase_switch",
             "area_schedule",
             "area_coarse_attn", "area_full_attn", "area_dwt_detail", "area_window_plan_bytes",
-            "area_window_plan", "area_window_attn_ws_bytes", "area_window_attn")
+            "area_window_plan", "area_window_attn_ws_bytes", "area_window_attn",
+            "area_window_attn_noalloc")
 
 
 class AreaError(RuntimeError):

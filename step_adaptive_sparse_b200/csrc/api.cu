@@ -6,13 +6,18 @@
 #include "area_internal.cuh"
 
 namespace {
-
 thread_local int g_last_cuda_error = 0;
+}  // namespace
 
+namespace area {
 int fail_cuda(cudaError_t e) {
   g_last_cuda_error = (int)e;
   return AREA_ECUDA;
 }
+}  // namespace area
+
+namespace {
+using area::fail_cuda;
 
 int finish(cudaError_t e) { return e == cudaSuccess ? AREA_OK : fail_cuda(e); }
 

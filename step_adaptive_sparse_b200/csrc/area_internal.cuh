@@ -102,6 +102,10 @@ __host__ __device__ __forceinline__ unsigned long long counter_random(unsigned l
 }
 constexpr unsigned long long kStreamJitter = 1, kStreamHalo = 2;
 
+// Records a CUDA error for area_last_cuda_error (per host thread) and
+// returns AREA_ECUDA.
+int fail_cuda(cudaError_t e);
+
 // ---------------------------------------------------------------------------
 // launchers (return cudaError_t of the launch)
 // ---------------------------------------------------------------------------

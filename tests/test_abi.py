@@ -184,3 +184,37 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
         binding.area_version()
     with pytest.raises(ImportError):
         binding.area_pool_ramp(4, 2, 8, 256, 256)
+
+
+def test_noalloc_rejects_bad_input_with_the_status_of_area_window_attn(area):
+    # Both calls validate on the host before any CUDA call; for the same bad
+    # input they must give the same status.
+    fake = 1 << 20
+    cfg = area.make_cfg(1, 16, 16, 8, 1, 4, 0.1)
+    nb = area.area_window_plan_bytes(cfg)
+    ws_big = 1 << 40
+    cases = [
+        dict(q=None),                           # null input
+        dict(plan=None),                        # null plan
+        dict(H=0),                              # no heads
+        dict(D=96),                             # unsupported head_dim
+        dict(dtype=5),                          # unknown dtype
+        dict(cfg=area.make_cfg(1, 15, 16, 8, 1, 4, 0.1)),   # odd grid side
+        dict(cfg=area.make_cfg(1, 16, 16, 0, 1, 4, 0.1)),   # zero window side
+    ]
+    for c in cases:
+        a = dict(q=fake, k=fake, v=fake, cfg=cfg, plan=fake, o=fake, H=2, D=128, dtype=1)
+        a.update(c)
+        with pytest.raises(area.AreaError) as e1:
+            area.area_window_attn(a["q"], a["k"], a["v"], a["cfg"], a["plan"], nb, a["o"], fake,
+                                  ws_big, a["H"], a["D"], 1.0, a["dtype"])
+        with pytest.raises(area.AreaError) as e2:
+            area.area_window_attn_noalloc(a["q"], a["k"], a["v"], a["cfg"], a["plan"], nb,
+                                          a["o"], a["H"], a["D"], 1.0, a["dtype"])
+        assert e1.value.status == e2.value.status, c
+    # beyond the static workspace: refused before any launch
+    big = area.make_cfg(1, 256, 256, 64, 4, 16, 0.1)
+    with pytest.raises(area.AreaError) as e:
+        area.area_window_attn_noalloc(fake, fake, fake, big, fake, area.area_window_plan_bytes(big),
+                                      fake, 24, 128, 1.0, 1)
+    assert e.value.status == area.AREA_ENOSPACE

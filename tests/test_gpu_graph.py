@@ -86,22 +86,21 @@ def test_whole_sampling_run_in_one_graph():
     # 28 steps of a synthetic flow-matching sampler: the noise-level switch,
     # the pooling ramp over Phase I and the shrinking windows over Phase II,
     # every call of the run captured in one graph
-    from step_adaptive_sparse_b200 import schedule
     from workloads import flow_sigmas
     cfg = CONFIGS["flux2048"]
     dt = area.AREA_DTYPE_BF16
     q, k, v = (torch.from_numpy(x).cuda().to(torch.bfloat16) for x in make_qkv(cfg))
     src = torch.from_numpy(make_detail_source(cfg)).cuda().to(torch.bfloat16)
-    sched = schedule.schedule(flow_sigmas(28, 3.0), 0.89, 4, 2, 64, 32, cfg.Hg, cfg.Wg)
+    sched = area.area_schedule(flow_sigmas(28, 3.0), 0.89, 4, 2, 64, 32, cfg.Hg, cfg.Wg)
     kinds = [kd for kd, _ in sched]
-    assert kinds == [schedule.PHASE_COARSE] * 8 + [schedule.PHASE_WINDOW] * 20
-    fs = [p for kd, p in sched if kd == schedule.PHASE_COARSE]
+    assert kinds == [area.AREA_PHASE_COARSE] * 8 + [area.AREA_PHASE_WINDOW] * 20
+    fs = [p for kd, p in sched if kd == area.AREA_PHASE_COARSE]
     assert fs == [4, 4, 4, 4, 2, 2, 2, 2]
     kp = torch.empty((cfg.B, cfg.H, cfg.N // 4, cfg.D), dtype=torch.bfloat16, device="cuda")
     vp = torch.empty_like(kp)
     energy = torch.empty((cfg.B, cfg.Hg // 2, cfg.Wg // 2), dtype=torch.float32, device="cuda")
     plans, wsb = {}, 0
-    for w in {p for kd, p in sched if kd == schedule.PHASE_WINDOW}:
+    for w in {p for kd, p in sched if kd == area.AREA_PHASE_WINDOW}:
         pc = area.make_cfg(cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
         nb = area.area_window_plan_bytes(pc)
         plans[w] = (pc, torch.empty(nb, dtype=torch.uint8, device="cuda"), nb)
@@ -112,7 +111,7 @@ def test_whole_sampling_run_in_one_graph():
 
     def run(keep):
         for kd, p in sched:
-            if kd == schedule.PHASE_COARSE:
+            if kd == area.AREA_PHASE_COARSE:
                 nk = (cfg.Hg // p) * (cfg.Wg // p)
                 area.area_pool_kv(k, v, kp, vp, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, p,
                                   area.AREA_POOL_MEAN, dt, stream)

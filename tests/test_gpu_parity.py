@@ -383,9 +383,8 @@ def test_window_attn_seeded(data):
 
 def _bridge(data, step):
     cfg = data.cfg
-    from step_adaptive_sparse_b200 import schedule
     w = cfg.schedule[step]
-    ry, rx = schedule.bridge_lattice(w, cfg.Hg, cfg.Wg)
+    ry, rx = gr.area.area_bridge_lattice(w, cfg.Hg, cfg.Wg)
     assert (ry, rx) == ora.bridge_lattice(w, cfg.Hg, cfg.Wg)
     R = ry * rx
     cand = torch.empty((cfg.B, cfg.H, R), dtype=torch.int32, device="cuda")
