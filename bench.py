@@ -4,8 +4,9 @@
 One step = one AReA attention schedule on one synthetic FLUX.1-shaped
 6144x6144 image (384x384 tokens, 24 heads, head_dim 128, bf16):
   8 Phase I calls   (area_pool_kv + area_coarse_attn, f = 6 -> 64x64 keys), and
-  8 Phase II calls  (area_dwt_detail + area_window_plan + area_window_attn, one
-                     per window side of the schedule 192 -> 64).
+  8 Phase II calls  (area_dwt_window_plan: detail map + plan in one launch, then
+                     area_window_attn; one per window side of the schedule
+                     192 -> 64).
 The metric is algorithmic attention TFLOP/s: 4*D*H*(query, key) pairs the
 method defines (N*Nk per Phase I call; sum over windows of |W|*(|ext|+G_W)
 per Phase II call) divided by the step time.  Full attention over the same
@@ -74,9 +75,14 @@ def dwt_bytes(cfg) -> float:
 
 
 def plan_launches(B: int) -> int:
-    # header, base scores, windows, (sort init + 4 x (hist, scan, scatter)) per
-    # batch element, global-KV selection, weight sums
+    # the separate planner calls: header, base scores, windows, (sort init +
+    # 4 x (hist, scan, scatter)) per batch element, global-KV selection,
+    # weight sums
     return 5 + 13 * B
+
+
+# kernels of one area_window_attn call (workspace zero, attention, finalize)
+WINDOW_LAUNCHES = 3
 
 
 # ---------------------------------------------------------------------------
@@ -230,10 +236,10 @@ class AreaStep:
         self.ws = torch.empty(wsb // 4, dtype=torch.float32, device=dev)
         self.ws_bytes = wsb
         self.n_phase1 = len(cfg.schedule)
-        self.launches = (self.n_phase1 * 2 +
-                         len(cfg.schedule) * (1 + plan_launches(cfg.B) + 3))
-        self.calls = {"pool_kv": [], "coarse_attn": [], "dwt_detail": [], "window_plan": [],
-                      "window_attn": []}
+        # libarea kernels per step: pool + coarse per Phase I call; the one
+        # planner launch and the window call's launches per Phase II call
+        self.launches = self.n_phase1 * 2 + len(cfg.schedule) * (1 + WINDOW_LAUNCHES)
+        self.calls = {"pool_kv": [], "coarse_attn": [], "dwt_window_plan": [], "window_attn": []}
         self.record = False
 
     def _ev(self):
@@ -259,11 +265,9 @@ class AreaStep:
                 self.q, self.kp, self.vp, self.o1, cfg.B, cfg.H, cfg.N, cfg.Nk, cfg.D, cfg.scale,
                 self.dt, s))
         for i in range(len(cfg.schedule)):
-            self._timed("dwt_detail", lambda: area.area_dwt_detail(
-                self.src, self.dt, cfg.C, self.energy, cfg.B, cfg.Hg, cfg.Wg,
-                area.AREA_DETAIL_HH, s))
-            self._timed("window_plan", lambda: area.area_window_plan(
-                self.energy, self.pcfg[i], self.plan[i], self.plan_bytes[i], s))
+            self._timed("dwt_window_plan", lambda: area.area_dwt_window_plan(
+                self.src, self.dt, cfg.C, area.AREA_DETAIL_HH, self.energy, self.pcfg[i],
+                self.plan[i], self.plan_bytes[i], s))
             self._timed("window_attn", lambda: area.area_window_attn(
                 self.q, self.k, self.v, self.pcfg[i], self.plan[i], self.plan_bytes[i],
                 self.o2, self.ws, self.ws_bytes, cfg.H, cfg.D, cfg.scale, self.dt, s))
@@ -449,9 +453,8 @@ def schedule_graph_leg(cfg, st, stream, full_ms, steps=28, shift=3.0, sigma_star
                                       cfg.scale, st.dt, stream)
             else:
                 pc, plan, nb = plans[p]
-                area.area_dwt_detail(st.src, st.dt, cfg.C, st.energy, cfg.B, cfg.Hg, cfg.Wg,
-                                     area.AREA_DETAIL_HH, stream)
-                area.area_window_plan(st.energy, pc, plan, nb, stream)
+                area.area_dwt_window_plan(st.src, st.dt, cfg.C, area.AREA_DETAIL_HH, st.energy,
+                                          pc, plan, nb, stream)
                 area.area_window_attn(st.q, st.k, st.v, pc, plan, nb, st.o2, st.ws, st.ws_bytes,
                                       cfg.H, cfg.D, cfg.scale, st.dt, stream)
 
@@ -477,7 +480,7 @@ def schedule_graph_leg(cfg, st, stream, full_ms, steps=28, shift=3.0, sigma_star
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
     del g
-    launches = 2 * len(fs) + len(ws_sides) * (1 + plan_launches(cfg.B) + 3)
+    launches = 2 * len(fs) + len(ws_sides) * (1 + WINDOW_LAUNCHES)
     return {"steps": steps, "sampler": f"flow matching, shift {shift}", "sigma_star": sigma_star,
             "phase1_steps": len(fs), "ramp": fs, "window_sides": ws_sides,
             "graph_launches": launches, "ms": ms,
@@ -485,6 +488,106 @@ def schedule_graph_leg(cfg, st, stream, full_ms, steps=28, shift=3.0, sigma_star
             "speedup_vs_full_attention": steps * full_ms / ms,
             "note": "all attention calls of the run captured in one CUDA graph; "
                     "speedup against the same number of full-attention calls"}
+
+
+def config_leg(name: str, dev, stream, steps: int = 3, warmup: int = 3) -> dict:
+    """The metric's other configuration, timed like the main step (the same
+    call sequence, CUDA events on the launching stream, inputs larger than L2)
+    and reported per call: Phase I and Phase II ms and TFLOP/s, and the window
+    calls' fraction of the measured sustained bf16 peak."""
+    import torch
+
+    from workloads import CONFIGS, make_detail_source, make_qkv
+    cfg = CONFIGS[name]
+    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    q, k, v = (torch.from_numpy(x).to(dev).to(tdt) for x in make_qkv(cfg))
+    src = torch.from_numpy(make_detail_source(cfg)).to(dev).to(tdt)
+    st = AreaStep(cfg, q, k, v, src, stream)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            st.run()
+    torch.cuda.synchronize()
+    wfl, wper = st.window_flops_per_step()
+    st.record = True
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(steps):
+            st.run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    st.record = False
+    ms = e0.elapsed_time(e1) / steps
+    per = {n: call_ms(p) for n, p in st.calls.items()}
+    coarse_ms = float(np.median(per["coarse_attn"]))
+    win_ms = np.array(per["window_attn"]).reshape(steps, -1).mean(axis=0)
+    step_flops = phase1_flops(cfg) * st.n_phase1 + wfl
+    peak = load_peaks()["bf16_tflops_sustained"]
+    win_tf = wfl / (float(win_ms.sum()) * 1e-3) / 1e12
+    out = {"workload": name, "steps": steps, "warmup": warmup, "ms_per_step": ms,
+           "value": step_flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "coarse_attn_ms": coarse_ms,
+           "coarse_attn_tflops": phase1_flops(cfg) / (coarse_ms * 1e-3) / 1e12,
+           "window_attn_ms_by_step": win_ms.tolist(),
+           "window_attn_tflops_by_step": [f / (t * 1e-3) / 1e12 for f, t in zip(wper, win_ms)],
+           "window_attn_tflops": win_tf,
+           "window_frac_of_sustained_peak": win_tf / peak,
+           "coarse_frac_of_sustained_peak": phase1_flops(cfg) / (coarse_ms * 1e-3) / 1e12 / peak,
+           "dwt_window_plan_ms": float(np.median(per["dwt_window_plan"])),
+           "pool_kv_gbs": pool_bytes(cfg) / (float(np.median(per["pool_kv"])) * 1e-3) / 1e9,
+           "split_fraction_by_step": st.split_fractions()}
+    del st, q, k, v, src
+    torch.cuda.empty_cache()
+    return out
+
+
+def profile_pass(args) -> int:
+    """Every kernel of the path, twice, on one configuration: the input of the
+    per-kernel ncu captures (a capture selects the second launch of a kernel
+    with -s/-c).  Sequence per pass: pool_kv, coarse attention, the detail
+    map, the separate planner, the one-launch planner, window attention at
+    schedule step --profile-step, bridge selection and bridged window
+    attention.  Nothing is timed."""
+    import torch
+
+    import step_adaptive_sparse_b200 as area
+    from workloads import CONFIGS, make_detail_source, make_qkv
+    cfg = CONFIGS[args.config]
+    dev = torch.device("cuda", 0)
+    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    q, k, v = (torch.from_numpy(x).to(dev).to(tdt) for x in make_qkv(cfg))
+    src = torch.from_numpy(make_detail_source(cfg)).to(dev).to(tdt)
+    stream = torch.cuda.Stream(device=dev)
+    st = AreaStep(cfg, q, k, v, src, stream)
+    i = args.profile_step % len(cfg.schedule)
+    w = cfg.schedule[i]
+    ry, rx = area.area_bridge_lattice(w, cfg.Hg, cfg.Wg)
+    cand = torch.empty((cfg.B, cfg.H, ry * rx), dtype=torch.int32, device=dev)
+    mws = torch.empty(area.area_bridge_select_ws_bytes(cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D) // 4,
+                      dtype=torch.float32, device=dev)
+    s = stream
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            area.area_pool_kv(k, v, st.kp, st.vp, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, cfg.f,
+                              area.AREA_POOL_MEAN, st.dt, s)
+            area.area_coarse_attn(q, st.kp, st.vp, st.o1, cfg.B, cfg.H, cfg.N, cfg.Nk, cfg.D,
+                                  cfg.scale, st.dt, s)
+            area.area_dwt_detail(src, st.dt, cfg.C, st.energy, cfg.B, cfg.Hg, cfg.Wg,
+                                 area.AREA_DETAIL_HH, s)
+            area.area_window_plan(st.energy, st.pcfg[i], st.plan[i], st.plan_bytes[i], s)
+            area.area_dwt_window_plan(src, st.dt, cfg.C, area.AREA_DETAIL_HH, st.energy,
+                                      st.pcfg[i], st.plan[i], st.plan_bytes[i], s)
+            area.area_window_attn(q, k, v, st.pcfg[i], st.plan[i], st.plan_bytes[i], st.o2, st.ws,
+                                  st.ws_bytes, cfg.H, cfg.D, cfg.scale, st.dt, s)
+            area.area_bridge_select(k, st.dt, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, ry, rx, cand,
+                                    mws, mws.numel() * 4, s)
+            area.area_window_attn_bridge(q, k, v, cand, ry * rx, st.pcfg[i], st.plan[i],
+                                         st.plan_bytes[i], st.o2, st.ws, st.ws_bytes, cfg.H,
+                                         cfg.D, cfg.scale, st.dt, s)
+    torch.cuda.synchronize()
+    err = area.area_kernel_error()
+    print(json.dumps({"profile_pass": cfg.name, "window_side": w, "kernel_error": err}))
+    return 0 if err == 0 else 1
 
 
 def run_area(args):
@@ -691,6 +794,24 @@ def run_area(args):
             fused[tag + "_us"] = fa.elapsed_time(fb) / 10 * 1e3
     fused["launches"] = {"separate": 1 + plan_launches(cfg.B), "fused": 1}
 
+    # ---- the detail map alone, for its HBM figure: L2 is flushed (a 256 MB
+    # write, twice the L2) before each call so the source comes from HBM
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    dwt_pairs = []
+    with torch.cuda.stream(stream):
+        for rep in range(13):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            area.area_dwt_detail(st.src, st.dt, cfg.C, st.energy, cfg.B, cfg.Hg, cfg.Wg,
+                                 area.AREA_DETAIL_HH, stream)
+            b.record(stream)
+            if rep >= 3:
+                dwt_pairs.append((a, b))
+    torch.cuda.synchronize()
+    dwt_ms = float(np.median(call_ms(dwt_pairs)))
+    del flush
+
     # ---- a whole 28-step sampling run in one CUDA graph
     sched_out = None if args.no_graph else schedule_graph_leg(cfg, st, stream, full_ms)
 
@@ -740,6 +861,11 @@ def run_area(args):
     e2e_ms = reduce_max(dist, e0.elapsed_time(e1), device=str(dev))
     e2e_val = flops_all / (e2e_ms * 1e-3) / 1e12
 
+    # ---- the metric's other configuration (4096^2), reported per call
+    other = None
+    if world == 1 and args.config == DEFAULT_CONFIG and args.other_config:
+        other = config_leg(args.other_config, dev, stream)
+
     # ---- roofline of the dominant kernel
     peaks = load_peaks()
     n1 = st.n_phase1
@@ -769,7 +895,7 @@ def run_area(args):
 
     clk = clocks.summary()
     if rank == 0:
-        pool_ms, dwt_ms = med["pool_kv"], med["dwt_detail"]
+        pool_ms = med["pool_kv"]
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -786,8 +912,8 @@ def run_area(args):
             "clocks": clk,
             "kernel_error": kerr,
             "per_call_ms": {
-                "pool_kv": pool_ms, "coarse_attn": coarse_ms, "dwt_detail": dwt_ms,
-                "window_plan": med["window_plan"], "window_attn_by_step": win_ms_steps,
+                "pool_kv": pool_ms, "coarse_attn": coarse_ms, "dwt_detail_alone": dwt_ms,
+                "dwt_window_plan": med["dwt_window_plan"], "window_attn_by_step": win_ms_steps,
                 "full_attn": full_ms},
             "per_call_tflops": {
                 "coarse_attn": phase1_flops(cfg) / (coarse_ms * 1e-3) / 1e12,
@@ -795,13 +921,14 @@ def run_area(args):
                                         zip(win_per_step, win_ms_steps)],
                 "full_attn": full_flops(cfg) / (full_ms * 1e-3) / 1e12},
             "per_call_gbs": {"pool_kv": pool_bytes(cfg) / (pool_ms * 1e-3) / 1e9,
-                             "dwt_detail": dwt_bytes(cfg) / (dwt_ms * 1e-3) / 1e9,
+                             "dwt_detail_alone": dwt_bytes(cfg) / (dwt_ms * 1e-3) / 1e9,
                              "hbm_peak_gbs": peaks["hbm_gbs"]},
             "split_fraction_by_step": splits,
             "phase1_pooling_ramp": ramp_out,
             "pages_bridge_rule": bridge_out,
             "schedule_28_steps_graph": sched_out,
             "dwt_plan_one_launch": fused,
+            "other_config": other,
             "graph_replay": None if graph_ms is None else {
                 "ms_per_step": graph_ms,
                 "value": step_flops / (graph_ms * 1e-3) / 1e12,
@@ -825,6 +952,9 @@ def main(argv=None):
     ap.add_argument("--full-reps", type=int, default=2)
     ap.add_argument("--ref-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--other-config", default="flux4096",
+                    help="the metric's second configuration, timed after the main one at "
+                         "N = 1 (empty string: skip)")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay leg")
     ap.add_argument("--clocks-csv", default="",
                     help="where to keep the nvidia-smi clock samples of the timed region "
@@ -832,7 +962,14 @@ def main(argv=None):
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="N > 1: independent replicas (weak scaling) or the heads of one "
                          "problem split across ranks (strong scaling)")
+    ap.add_argument("--profile-pass", action="store_true",
+                    help="run every kernel of the path twice on --config, untimed (the "
+                         "input of the per-kernel ncu captures)")
+    ap.add_argument("--profile-step", type=int, default=-1,
+                    help="schedule step of the window calls in --profile-pass")
     args = ap.parse_args(argv)
+    if args.profile_pass:
+        return profile_pass(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_area(args)

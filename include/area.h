@@ -398,6 +398,25 @@ int area_window_attn_noalloc(const void* q, const void* k, const void* v,
                              size_t plan_bytes, void* o, int H, int D,
                              float scale, int dtype, cudaStream_t stream);
 
+/*
+ * area_test_plan_barrier_expiry -- TEST HOOK, not part of the method (the
+ * pages have no counterpart).  Runs the one-launch detail map + planner of
+ * area_dwt_window_plan (AREA_DETAIL_HH) with every grid-barrier target set
+ * one above the number of blocks and each barrier wait bounded by 1 ms, so
+ * the first barrier cannot complete.  Every block gives up after about 1 ms
+ * and returns; the launch ends and the context stays usable.  A following
+ * area_kernel_error reports AREA_KERR_PLAN_BARRIER (and clears it).  The
+ * energy and plan buffers are left partly written: their contents are
+ * unspecified.  Exists so that tests can drive the bounded-wait path of the
+ * cooperative planner to expiry without a fault or a hang.
+ *   Arguments: as area_dwt_window_plan, without the detail mode.
+ * Errors: AREA_EINVAL, AREA_ENOSPACE, AREA_ECUDA.
+ */
+int area_test_plan_barrier_expiry(const void* src, int src_dtype, int C,
+                                  float* energy, const area_plan_cfg* cfg,
+                                  void* plan, size_t plan_bytes,
+                                  cudaStream_t stream);
+
 /* ---- schedule (host functions: no device memory, no stream) ------------ */
 
 /*

@@ -35,7 +35,7 @@ EXPORTED = ("area_status_string", "area_last_cuda_error", "area_version", "area_
             "area_schedule",
             "area_coarse_attn", "area_full_attn", "area_dwt_detail", "area_window_plan_bytes",
             "area_window_plan", "area_window_attn_ws_bytes", "area_window_attn",
-            "area_window_attn_noalloc")
+            "area_window_attn_noalloc", "area_test_plan_barrier_expiry")
 
 
 class AreaError(RuntimeError):
@@ -79,6 +79,8 @@ _SIGS = {
                                       _I, _I, _F, _I, _P]),
     "area_dwt_window_plan": (_I, [_P, _I, _I, _I, _P, ctypes.POINTER(area_plan_cfg), _P, _SZ,
                                   _P]),
+    "area_test_plan_barrier_expiry": (_I, [_P, _I, _I, _P, ctypes.POINTER(area_plan_cfg), _P,
+                                           _SZ, _P]),
     "area_pool_ramp": (_I, [_I, _I, _I, _I, _I, _P]),
     "area_window_sides": (_I, [_I, _I, _I, _P]),
     "area_bridge_lattice": (_I, [_I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
@@ -204,6 +206,16 @@ def area_dwt_window_plan(src, src_dtype, C, mode, energy, cfg: area_plan_cfg, pl
     _check(_lib().area_dwt_window_plan(_ptr(src), src_dtype, C, mode, _ptr(energy),
                                        ctypes.byref(cfg), _ptr(plan), plan_bytes,
                                        _stream(stream)), "area_dwt_window_plan")
+
+
+def area_test_plan_barrier_expiry(src, src_dtype, C, energy, cfg: area_plan_cfg, plan,
+                                  plan_bytes, stream=None) -> None:
+    """Test hook: the one-launch planner with barriers that cannot complete
+    and 1 ms wait bounds (see include/area.h)."""
+    _check(_lib().area_test_plan_barrier_expiry(_ptr(src), src_dtype, C, _ptr(energy),
+                                                ctypes.byref(cfg), _ptr(plan), plan_bytes,
+                                                _stream(stream)),
+           "area_test_plan_barrier_expiry")
 
 
 def area_window_attn_ws_bytes(cfg: area_plan_cfg, H: int, D: int) -> int:

@@ -180,6 +180,21 @@ int area_dwt_window_plan(const void* src, int src_dtype, int C, int mode, float*
                                              stream));
 }
 
+int area_test_plan_barrier_expiry(const void* src, int src_dtype, int C, float* energy,
+                                  const area_plan_cfg* cfg, void* plan, size_t plan_bytes,
+                                  cudaStream_t stream) {
+  if (!src || !energy || !plan || C < 1 || !valid_dtype(src_dtype)) return AREA_EINVAL;
+  area::PlanLayout L;
+  const int st = area::plan_layout(cfg, &L);
+  if (st != AREA_OK) return st;
+  if (plan_bytes < (size_t)L.total) return AREA_ENOSPACE;
+  if ((reinterpret_cast<uintptr_t>(plan) & 255) != 0) return AREA_EINVAL;
+  // every grid-barrier target one above the grid: no barrier can complete,
+  // and each wait gives up after 1 ms
+  return finish(area::launch_dwt_window_plan(src, src_dtype, C, AREA_DETAIL_HH, energy, cfg, L,
+                                             plan, stream, 1u, 1000000ull));
+}
+
 int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D, size_t* ws_bytes) {
   if (!ws_bytes || H < 1 || D < 1) return AREA_EINVAL;
   area::PlanLayout L;

@@ -145,9 +145,13 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, c
                                   int H, float scale, cudaStream_t s);
 // Detail map and planner in one cooperative launch (one memset of the
 // barrier words first); a barrier timeout raises the planner error flag.
+// target_extra (0 in every product call) raises each grid-barrier target so
+// that the first barrier cannot complete; wait_ns bounds each barrier wait
+// (0: the default of 2 s).  Both exist for the expiry test hook.
 cudaError_t launch_dwt_window_plan(const void* src, int src_dtype, int C, int mode, float* energy,
                                    const area_plan_cfg* cfg, const PlanLayout& L, void* plan,
-                                   cudaStream_t s);
+                                   cudaStream_t s, unsigned target_extra = 0,
+                                   uint64_t wait_ns = 0);
 cudaError_t read_and_clear_plan_error(int* code);
 
 // Scratch of area_bridge_select: the mean keys [B*H][D] then the chunk sums

@@ -501,7 +501,7 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
-__device__ bool grid_sync(unsigned* bar, unsigned target, int* s_ok) {
+__device__ bool grid_sync(unsigned* bar, unsigned target, uint64_t wait_ns, int* s_ok) {
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();                           // this block's writes, then its arrival
@@ -513,7 +513,7 @@ __device__ bool grid_sync(unsigned* bar, unsigned target, int* s_ok) {
       asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
       if (v >= target) break;
       asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(ab) : "l"(bar + 1) : "memory");
-      if (ab != 0u || global_ns() - t0 > kPlanWaitNs) {
+      if (ab != 0u || global_ns() - t0 > wait_ns) {
         ok = 0;
         atomicExch(bar + 1, 1u);
         atomicExch(&g_plan_error, 1);
@@ -539,6 +539,8 @@ struct FusedArgs {
   int *va, *vb;
   int nt;                // sort tiles
   unsigned* bar;         // [arrivals, abort]
+  unsigned target_extra; // added to every barrier target (0; 1 only in the expiry test hook)
+  uint64_t wait_ns;      // bound of each barrier wait
 };
 
 template <typename T, int MODE, bool VEC>
@@ -547,7 +549,9 @@ __global__ void __launch_bounds__(kFusedThreads, 2) plan_fused_kernel(PlanView P
   extern __shared__ float s_rows[];
   __shared__ int s_ok;
   unsigned nbar = 0;
-  auto sync = [&]() { return grid_sync(A.bar, ++nbar * gridDim.x, &s_ok); };
+  auto sync = [&]() {
+    return grid_sync(A.bar, ++nbar * gridDim.x + A.target_extra, A.wait_ns, &s_ok);
+  };
   const int G = gridDim.x;
   const int n = P.N;
   // detail map
@@ -693,7 +697,7 @@ static cudaError_t launch_fused_typed(const PlanLayout& L, const PlanView& P, co
 
 cudaError_t launch_dwt_window_plan(const void* src, int src_dtype, int C, int mode, float* energy,
                                    const area_plan_cfg* cfg, const PlanLayout& L, void* plan,
-                                   cudaStream_t s) {
+                                   cudaStream_t s, unsigned target_extra, uint64_t wait_ns) {
   PlanView P = plan_view(L, plan);
   char* base = static_cast<char*>(plan);
   FusedArgs A = {};
@@ -710,6 +714,8 @@ cudaError_t launch_dwt_window_plan(const void* src, int src_dtype, int C, int mo
   A.hist = reinterpret_cast<uint32_t*>(base + L.scratch_hist);
   A.nt = (int)L.ntile_sort;
   A.bar = reinterpret_cast<unsigned*>(base + L.scratch_bar);
+  A.target_extra = target_extra;
+  A.wait_ns = wait_ns ? wait_ns : kPlanWaitNs;
   const HeaderArgs h = header_args(L);
   const bool vec = C % (src_dtype == AREA_DTYPE_BF16 ? 8 : 4) == 0 &&
                    (reinterpret_cast<uintptr_t>(src) & 15) == 0;

@@ -82,6 +82,52 @@ def test_schedule_step_graph_replay_matches_eager(name):
     del g
 
 
+@pytest.mark.parametrize("name", ["tiny", "flux2048", "flux6144"])
+def test_one_launch_planner_in_a_graph(name):
+    # the cooperative detail map + planner launch (and the reset of its
+    # barrier words) captured in a graph: replay == eager, byte for byte
+    cfg = CONFIGS[name]
+    dt = area.AREA_DTYPE_BF16 if cfg.dtype == "bf16" else area.AREA_DTYPE_F32
+    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    src = torch.from_numpy(make_detail_source(cfg)).cuda().to(tdt)
+    energy = torch.empty((cfg.B, cfg.Hg // 2, cfg.Wg // 2), dtype=torch.float32, device="cuda")
+    plans = []
+    for w in cfg.schedule:
+        pc = area.make_cfg(cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
+        nb = area.area_window_plan_bytes(pc)
+        plans.append((pc, torch.empty(nb, dtype=torch.uint8, device="cuda"), nb))
+    stream = torch.cuda.Stream()
+
+    def run():
+        for pc, plan, nb in plans:
+            area.area_dwt_window_plan(src, dt, cfg.C, area.AREA_DETAIL_HH, energy, pc, plan, nb,
+                                      stream)
+
+    with torch.cuda.stream(stream):
+        run()
+    torch.cuda.synchronize()
+    ends = []
+    for _, p, _ in plans:
+        hdr = p[:256].cpu().numpy().view(np.int64)
+        ends.append(int(hdr[10 + area.SECTIONS.index("SCRATCH")]))
+    ref = [p[:e].clone() for (_, p, _), e in zip(plans, ends)]
+    ref_e = energy.clone()
+    for _, p, _ in plans:
+        p.zero_()
+    energy.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        run()
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert area.area_kernel_error() == 0
+    assert torch.equal(energy.view(torch.int32), ref_e.view(torch.int32))
+    for (_, p, _), e, r in zip(plans, ends, ref):
+        assert torch.equal(p[:e], r)
+    del g
+
+
 def test_whole_sampling_run_in_one_graph():
     # 28 steps of a synthetic flow-matching sampler: the noise-level switch,
     # the pooling ramp over Phase I and the shrinking windows over Phase II,

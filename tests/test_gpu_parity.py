@@ -212,7 +212,7 @@ def data(request):
 
 def test_pool_kv(data):
     cfg, k, v = data.cfg, data.k, data.v
-    heads = [0, cfg.H - 1]
+    heads = [0, cfg.H // 2, cfg.H - 1]
     for mode, mname in [(0, "mean"), (1, "center")]:
         kp, vp = gr.gpu_pool(data.dk, data.dv, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, cfg.f, mode,
                              cfg.dtype)
@@ -244,7 +244,7 @@ def test_full_attn(data):
     o = torch.empty_like(data.dq)
     gr.area.area_full_attn(data.dq, data.dk, data.dv, o, cfg.B, cfg.H, cfg.N, cfg.D, cfg.scale,
                            gr.area_dtype(cfg.dtype))
-    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H - 1]
+    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H // 2, cfg.H - 1]
     rows = np.arange(cfg.N) if cfg.tiny else gr.sample_rows(cfg.N, 96, seed=2)
     want = ora.full_attn(q[:, heads], k[:, heads], v[:, heads], cfg.scale, rows=rows)
     got = gr.to_host(o[:, heads][:, :, torch.from_numpy(rows).cuda()])
@@ -265,7 +265,7 @@ def test_window_attn(data, step):
     E = ora.dwt_detail(data.src, cfg.Hg, cfg.Wg)
     oplan = ora.window_plan(E[0], cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
     gr.compare_plan(gr.parse(plan), oplan)
-    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H - 1]
+    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H // 2, cfg.H - 1]
     rows = np.arange(cfg.N) if cfg.tiny else gr.sample_rows(cfg.N, 256, seed=3 + step)
     want = ora.window_attn(data.q, data.k, data.v, [oplan], cfg.scale, rows=rows, heads=heads)
     got = gr.to_host(o[:, heads][:, :, torch.from_numpy(rows).cuda()])
@@ -302,7 +302,7 @@ def test_coarse_attn_text(data):
     o = torch.empty_like(data.dq)
     gr.area.area_coarse_attn_text(data.dq, kp, vp, dkt, dvt, o, cfg.B, cfg.H, cfg.N, cfg.Nk, T,
                                   cfg.D, cfg.scale, gr.area_dtype(cfg.dtype))
-    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H - 1]
+    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H // 2, cfg.H - 1]
     rows = np.arange(cfg.N) if cfg.tiny else gr.sample_rows(cfg.N, 256, seed=5)
     okp = ora.pool_kv(k[:, heads], cfg.Hg, cfg.Wg, cfg.f)
     ovp = ora.pool_kv(v[:, heads], cfg.Hg, cfg.Wg, cfg.f)
@@ -332,7 +332,7 @@ def test_window_attn_text(data, which):
                                   ws, wsb, cfg.H, cfg.D, cfg.scale, gr.area_dtype(cfg.dtype))
     E = ora.dwt_detail(data.src, cfg.Hg, cfg.Wg)
     oplan = ora.window_plan(E[0], cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
-    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H - 1]
+    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H // 2, cfg.H - 1]
     rows = np.arange(cfg.N) if cfg.tiny else gr.sample_rows(cfg.N, 192, seed=11 + step)
     want = ora.window_attn(data.q, data.k, data.v, [oplan], cfg.scale, rows=rows, heads=heads,
                            kt=kt, vt=vt)
@@ -374,7 +374,7 @@ def test_window_attn_seeded(data):
     E = ora.dwt_detail(data.src, cfg.Hg, cfg.Wg)
     oplan = ora.window_plan(E[0], cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr, seed=seed)
     gr.compare_plan(gr.parse(plan), oplan)
-    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H - 1]
+    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H // 2, cfg.H - 1]
     rows = np.arange(cfg.N) if cfg.tiny else gr.sample_rows(cfg.N, 192, seed=21)
     want = ora.window_attn(data.q, data.k, data.v, [oplan], cfg.scale, rows=rows, heads=heads)
     got = gr.to_host(o[:, heads][:, :, torch.from_numpy(rows).cuda()])
@@ -419,10 +419,15 @@ def test_window_attn_bridge(data):
                                     o, ws, wsb, cfg.H, cfg.D, cfg.scale, gr.area_dtype(cfg.dtype))
     E = ora.dwt_detail(data.src, cfg.Hg, cfg.Wg)
     oplan = ora.window_plan(E[0], cfg.Hg, cfg.Wg, w, cfg.halo, 0, cfg.split_thr)
-    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H - 1]
+    heads = list(range(cfg.H)) if cfg.tiny else [0, cfg.H // 2, cfg.H - 1]
     rows = np.arange(cfg.N) if cfg.tiny else gr.sample_rows(cfg.N, 160, seed=31)
+    # the oracle's own candidates, from the host keys of the heads under test
+    # (the GPU's selection is pinned separately, bit for bit)
+    ocand = np.full((cfg.B, cfg.H, ry * rx), -1, dtype=np.int64)
+    for h in heads:
+        ocand[0, h] = ora.bridge_candidates(data.k[0, h], cfg.Hg, cfg.Wg, ry, rx)
     want = ora.window_attn(data.q, data.k, data.v, [oplan], cfg.scale, rows=rows, heads=heads,
-                           bridge=cand.cpu().numpy())
+                           bridge=ocand)
     got = gr.to_host(o[:, heads][:, :, torch.from_numpy(rows).cuda()])
     gr.assert_close(got, want, cfg.dtype, f"window bridge {cfg.name} w={w}")
 

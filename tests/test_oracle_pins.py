@@ -572,6 +572,34 @@ def test_tile_windows_shifted_cover_the_axis_and_move_the_seams():
                     assert wins[0] == (0, we - shift)
 
 
+def test_tile_windows_shifted_hand_worked():
+    g = _golden("tilings.json")
+    for c in g["shifted_cases"]:
+        assert ora.tile_windows(c["L"], c["w"], c["shift"]) == [tuple(x) for x in c["windows"]], c
+
+
+def test_seeded_draws_hand_worked_from_published_outputs():
+    # seeds chosen so each stream's draws are the published SplitMix64
+    # outputs of state 0; the shifts and widths are those outputs reduced by
+    # hand (tests/golden/make_seeded_draws.py states the derivation)
+    g = _golden("seeded_draws.json")
+    for c in g["jitter"]:
+        assert ora.jitter_shifts(int(c["seed_hex"], 16), c["Hg"], c["Wg"], c["w"]) == \
+            (c["sy"], c["sx"]), c
+    for c in g["halo"]:
+        seed = int(c["seed_hex"], 16)
+        got = [ora.halo_width(seed, c["halo"], c["b"], i) for i in c["windows"]]
+        assert got == c["widths"], c
+    # the jitter seed lands on the published outputs only through stream 1
+    # and the Halo seeds only through stream 2 at index b * 2^20 + i
+    pub = [int(h, 16) for h in _golden("splitmix64.json")["outputs_hex"]]
+    sj = int(g["jitter"][0]["seed_hex"], 16)
+    assert [ora.counter_random(sj, 1, i) for i in range(2)] == pub[:2]
+    for c in g["halo"]:
+        seed = int(c["seed_hex"], 16)
+        assert [ora.counter_random(seed, 2, (c["b"] << 20) + i) for i in range(3)] == pub
+
+
 def test_jitter_and_halo_draws():
     assert ora.jitter_shifts(0, 384, 384, 64) == (0, 0)
     assert ora.jitter_shifts(99, 256, 256, 256) == (0, 0)      # window spans the grid
