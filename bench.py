@@ -36,7 +36,7 @@ if ROOT not in sys.path:
 
 METRIC = "AReA attention TFLOP/s per schedule step (bf16, 1 B200)"
 # Bumped whenever attn_tc.cu changes, so that stale DRAM counters are not reported.
-KERNEL_REVISION = "attn_tc r9 (patch loader, f32x2 softmax, single-cover stores, text-key tiles, bridge variant, 8-chain max, P in two parts, cover read ahead of the O wait)"
+KERNEL_REVISION = "attn_tc r10 (unit records in a shared-memory ring, dynamic window units in parity-class order, global-KV tiles first, merge in class order without atomics)"
 DEFAULT_CONFIG = "flux6144"
 
 
@@ -81,8 +81,10 @@ def plan_launches(B: int) -> int:
     return 5 + 13 * B
 
 
-# kernels of one area_window_attn call (workspace zero, attention, finalize)
-WINDOW_LAUNCHES = 3
+# kernels of one area_window_attn call on the tensor-core path (the merge runs
+# inside the attention kernel; a 256-byte memset of the workspace counters
+# precedes it)
+WINDOW_LAUNCHES = 1
 
 
 # ---------------------------------------------------------------------------
@@ -874,7 +876,8 @@ def run_area(args):
     t_window = float(np.sum(win_ms_steps))
     if t_window >= t_coarse:
         dom, dom_flops, dom_ms, dom_launches = ("window_attn", win_flops / len(cfg.schedule),
-                                                t_window / len(cfg.schedule), "3 launches")
+                                                t_window / len(cfg.schedule),
+                                                "1 launch after a 256-byte memset")
     else:
         dom, dom_flops, dom_ms, dom_launches = ("coarse_attn", phase1_flops(cfg), coarse_ms,
                                                 "1 launch")

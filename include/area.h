@@ -189,9 +189,9 @@ typedef struct area_plan_cfg {
  *   header[2..8] = B, Hg, Wg, w, halo, G, nb
  *   header[9]  = nw
  *   header[10+s] = byte offset of section s (AREA_PLAN_SEC_*)
- *   header[25] = work-item capacity per element ("ni"), header[26] = N,
- *   header[27] = base windows of this plan (<= nb; fewer than the capacity
- *   when a border shift is drawn), header[28..29] = border shift (sy, sx)
+ *   header[26] = work-item capacity per element ("ni"), header[27] = N,
+ *   header[28] = base windows of this plan (<= nb; fewer than the capacity
+ *   when a border shift is drawn), header[29..30] = border shift (sy, sx)
  * Sections:
  *   BASE    int32 [B][nb][4]   base windows (y0, x0, hy, wx), row-major
  *   SCORE   f32   [B][nb]      sum of token energy over the base window
@@ -207,11 +207,18 @@ typedef struct area_plan_cfg {
  *   ORDER   int32 [B][N]       tokens by (energy desc, index asc)
  *   NITEM   int32 [B+1]        work items (window, query tile) per element,
  *                              last entry = total
- *   ITEMS   int32 [B][ni][2]   (window, block of 256 queries) in cost order
+ *   ITEMS   int32 [B][ni][2]   (window, block of 256 queries), grouped by
+ *                              the parity class of the window's base window,
+ *                              class = 2 * (row index & 1) + (column index & 1)
+ *                              in the base tiling (windows of one class never
+ *                              overlap); within a class, windows of unsplit
+ *                              base windows first, then quadrants, each in
+ *                              window order
+ *   NCLASS  int32 [B+1][4]     work items per class; row B = totals
  *   SCRATCH                    sort and scan scratch (contents unspecified)
  */
 #define AREA_PLAN_MAGIC    0x4145524150414c4eLL  /* "AREAPLAN" */
-#define AREA_PLAN_VERSION  2
+#define AREA_PLAN_VERSION  3
 #define AREA_PLAN_SEC_BASE     0
 #define AREA_PLAN_SEC_SCORE    1
 #define AREA_PLAN_SEC_SPLIT    2
@@ -226,8 +233,9 @@ typedef struct area_plan_cfg {
 #define AREA_PLAN_SEC_NITEM    11
 #define AREA_PLAN_SEC_ITEMS    12
 #define AREA_PLAN_SEC_COVER    13
-#define AREA_PLAN_SEC_SCRATCH  14
-#define AREA_PLAN_NSEC         15
+#define AREA_PLAN_SEC_NCLASS   14
+#define AREA_PLAN_SEC_SCRATCH  15
+#define AREA_PLAN_NSEC         16
 
 /*
  * area_window_plan_bytes -- size of the plan buffer for cfg (host only).
@@ -250,7 +258,8 @@ int area_window_plan_bytes(const area_plan_cfg* cfg, size_t* plan_bytes);
  *   6. per-token sum of tent weights
  *      t = min(y-y0+1, y0+hy-y) * min(x-x0+1, x0+wx-x) over final windows,
  *      and the number of final windows containing the token;
- *   7. the list of (window, 256-query block) work items, costliest first.
+ *   7. the list of (window, 256-query block) work items by parity class,
+ *      costliest first within a class (see ITEMS).
  *   energy : [B, Hg/2, Wg/2] fp32 from area_dwt_detail
  *   plan   : device buffer of plan_bytes >= area_window_plan_bytes(cfg)
  * The plan never leaves the device.  Errors: AREA_EINVAL, AREA_ENOSPACE.

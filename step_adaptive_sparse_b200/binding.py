@@ -26,7 +26,7 @@ AREA_PHASE_COARSE, AREA_PHASE_WINDOW = 1, 2
 AREA_KERR_TC_WAIT, AREA_KERR_PLAN_BARRIER = 1, 2
 AREA_PLAN_MAGIC = 0x4145524150414C4E
 SECTIONS = ("BASE", "SCORE", "SPLIT", "NWIN", "WIN", "PARENT", "EXT", "GCOUNT", "GIDX",
-            "WSUM", "ORDER", "NITEM", "ITEMS", "COVER", "SCRATCH")
+            "WSUM", "ORDER", "NITEM", "ITEMS", "COVER", "NCLASS", "SCRATCH")
 
 EXPORTED = ("area_status_string", "area_last_cuda_error", "area_version", "area_kernel_error",
             "area_pool_kv", "area_coarse_attn_text", "area_window_attn_text",
@@ -346,5 +346,6 @@ def parse_plan(buf: np.ndarray) -> dict:
            "cover": sec("COVER", np.int32, B * N).reshape(B, N),
            "order": sec("ORDER", np.int32, B * N).reshape(B, N),
            "nitem": nitem,
-           "items": sec("ITEMS", np.int32, B * nitem_max * 2).reshape(B, nitem_max, 2)}
+           "items": sec("ITEMS", np.int32, B * nitem_max * 2).reshape(B, nitem_max, 2),
+           "nclass": sec("NCLASS", np.int32, (B + 1) * 4).reshape(B + 1, 4)}
     return out

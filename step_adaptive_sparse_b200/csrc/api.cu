@@ -63,19 +63,14 @@ int window_attn(const void* q, const void* k, const void* v, const void* kt, con
   if (T < 0 || (T > 0 && (!kt || !vt || !aligned16(kt) || !aligned16(vt)))) return AREA_EINVAL;
   if (cand && R < 1) return AREA_EINVAL;
   if (plan_bytes < (size_t)L.total) return AREA_ENOSPACE;
-  if (ws_bytes < (size_t)(L.B * H * L.N * D * 4)) return AREA_ENOSPACE;
+  if (ws_bytes < (size_t)area::window_ws_bytes(L, H, D)) return AREA_ENOSPACE;
   if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(plan) & 255) != 0) return AREA_EINVAL;
   if (H > 65535 || L.B > 65535) return AREA_EINVAL;
-  float* w = static_cast<float*>(ws);
-  cudaError_t e = area::launch_ws_zero(w, L, plan, H, D, stream);
-  if (e != cudaSuccess) return fail_cuda(e);
   if (dtype == AREA_DTYPE_BF16 && D == 128)
-    e = area::launch_window_attn_tc(q, k, v, kt, vt, T, cand, R, L, plan, o, w, H, scale, stream);
-  else
-    e = area::launch_window_attn_simt(q, k, v, kt, vt, T, cand, R, L, plan, o, w, H, D, scale,
-                                      dtype, stream);
-  if (e != cudaSuccess) return fail_cuda(e);
-  return finish(area::launch_window_finalize(w, L, plan, o, H, D, dtype, stream));
+    return finish(area::launch_window_attn_tc(q, k, v, kt, vt, T, cand, R, L, plan, o, ws, H,
+                                              scale, stream));
+  return finish(area::launch_window_attn_simt(q, k, v, kt, vt, T, cand, R, L, plan, o, ws, H, D,
+                                              scale, dtype, stream));
 }
 
 }  // namespace
@@ -200,7 +195,7 @@ int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D, size_t* ws
   area::PlanLayout L;
   const int st = area::plan_layout(cfg, &L);
   if (st != AREA_OK) return st;
-  *ws_bytes = (size_t)(L.B * H * L.N * D * 4);
+  *ws_bytes = (size_t)area::window_ws_bytes(L, H, D);
   return AREA_OK;
 }
 

@@ -26,6 +26,8 @@ struct PlanLayout {
   int64_t nitem_max;            // work-item capacity per element
   int64_t N;                    // tokens per element
   int64_t ntile_sort;           // 256-element tiles of the radix sort
+  int64_t ny2, nx2;             // positions covered by two base windows, per axis
+  int64_t n_ov;                 // tokens covered by more than one window (per element)
   int64_t off[AREA_PLAN_NSEC];  // byte offsets of the sections
   int64_t scratch_keys_a, scratch_keys_b, scratch_vals_a, scratch_vals_b,
           scratch_hist,         // byte offsets inside the buffer
@@ -55,6 +57,7 @@ struct PlanView {
   int* order;          // [B][N]
   int* nitem;          // [B+1]
   int2* items;         // [B][nitem_max]
+  int* nclass;         // [B+1][4] work items per parity class (row B: totals)
 };
 
 PlanView plan_view(const PlanLayout& L, void* plan);
@@ -86,6 +89,90 @@ __host__ __device__ __forceinline__ void axis_window(int i, int n, int L, int we
   *start = lo;
   *size = hi - lo;
 }
+
+// Merge geometry of base window i along one axis (n windows, shift as in
+// axis_window).  Consecutive windows may overlap; windows two apart never do
+// (their spacing exceeds half a window), so a position is covered by one or
+// two windows of an axis.  Returns
+//   x = start of window i, y = end of the overlap with window i-1 (x when
+//   none), z = start of the overlap with window i+1 (end of window i when
+//   none), w = number of twice-covered positions before the start of i.
+__host__ __device__ inline int4 axis_merge(int i, int n, int L, int we, int shift) {
+  int a, s;
+  axis_window(i, n, L, we, shift, &a, &s);
+  int lo_end = a, hi_start = a + s;
+  if (i > 0) {
+    int ap, sp;
+    axis_window(i - 1, n, L, we, shift, &ap, &sp);
+    lo_end = ap + sp > a ? ap + sp : a;
+  }
+  if (i + 1 < n) {
+    int an, sn;
+    axis_window(i + 1, n, L, we, shift, &an, &sn);
+    hi_start = an < a + s ? an : a + s;
+  }
+  int cnt = 0, ak, sk;
+  axis_window(0, n, L, we, shift, &ak, &sk);
+  for (int k = 0; k + 1 <= i - 1; ++k) {       // overlaps of windows (k, k+1) before a
+    int an, sn;
+    axis_window(k + 1, n, L, we, shift, &an, &sn);
+    cnt += ak + sk > an ? ak + sk - an : 0;
+    ak = an;
+    sk = sn;
+  }
+  return make_int4(a, lo_end, hi_start, cnt);
+}
+
+// Number of positions of an axis covered by two windows.
+__host__ __device__ inline int axis_twice_total(int n, int L, int we, int shift) {
+  int cnt = 0, ak, sk;
+  axis_window(0, n, L, we, shift, &ak, &sk);
+  for (int k = 0; k + 1 < n; ++k) {
+    int an, sn;
+    axis_window(k + 1, n, L, we, shift, &an, &sn);
+    cnt += ak + sk > an ? ak + sk - an : 0;
+    ak = an;
+    sk = sn;
+  }
+  return cnt;
+}
+
+// Parity class of a base window: windows of one class never overlap.
+__host__ __device__ inline int window_class(int parent, int nbx) {
+  return (((parent / nbx) & 1) << 1) | ((parent % nbx) & 1);
+}
+
+// Role of one output row in the centre-weighted merge.  A token inside one
+// window stores its output directly.  A token covered by several windows
+// (one per parity class at most) has one fp32 accumulator row: the window of
+// its lowest class stores, the middle ones add, the highest class adds and
+// normalises.  my/mx: axis_merge of the base window along y and x.
+struct MergeRole {
+  bool ov, first, last;
+  int64_t rank;        // accumulator row among the overlapped tokens of the element
+};
+__host__ __device__ inline MergeRole merge_role(int y, int x, int cls, int4 my, int4 mx,
+                                                int Wg, int nx2) {
+  MergeRole r;
+  const bool ty = y < my.y || y >= my.z;
+  const bool tx = x < mx.y || x >= mx.z;
+  r.ov = ty || tx;
+  const int py = cls >> 1, px = cls & 1;
+  const int minc = ((ty ? 0 : py) << 1) | (tx ? 0 : px);
+  const int maxc = ((ty ? 1 : py) << 1) | (tx ? 1 : px);
+  r.first = cls == minc;
+  r.last = cls == maxc;
+  const int by = my.w + ((y < my.y ? y : my.y) - my.x) + (y >= my.z ? y - my.z : 0);
+  const int bx = mx.w + ((x < mx.y ? x : mx.y) - mx.x) + (x >= mx.z ? x - mx.z : 0);
+  r.rank = (int64_t)by * Wg + (int64_t)(y - by) * nx2 + (ty ? x : bx);
+  return r;
+}
+
+// Window-attention workspace: a 256-byte header of counters (the dynamic
+// unit counter, then one completion counter per parity class), then one fp32
+// accumulator row per (element, head, overlapped token).
+constexpr int kWsHeaderBytes = 256;
+constexpr int kWsUnitCounter = 0, kWsClassDone = 1;
 
 // Counter-based draws: output number (stream * 2^32 + index) of the SplitMix64
 // sequence (Steele, Lea, Flood 2014) seeded with `seed`.
@@ -120,15 +207,13 @@ cudaError_t launch_window_plan(const float* energy, const area_plan_cfg* cfg,
 cudaError_t launch_dense_attn_simt(const void* q, const void* k, const void* v, const void* kt,
                                    const void* vt, void* o, int B, int H, int N, int Nk, int T,
                                    int D, float scale, int dtype, cudaStream_t s);
+// Window attention on CUDA cores: one launch per parity class, so that the
+// merge of overlapped tokens runs in class order.  ws: the window workspace
+// (header + accumulator rows).
 cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v, const void* kt,
                                     const void* vt, int T, const int* cand, int R,
-                                    const PlanLayout& L, const void* plan, void* o, float* ws,
+                                    const PlanLayout& L, const void* plan, void* o, void* ws,
                                     int H, int D, float scale, int dtype, cudaStream_t s);
-// Shared by both window-attention paths.
-cudaError_t launch_ws_zero(float* ws, const PlanLayout& L, const void* plan, int H, int D,
-                           cudaStream_t s);
-cudaError_t launch_window_finalize(const float* ws, const PlanLayout& L, const void* plan,
-                                   void* o, int H, int D, int dtype, cudaStream_t s);
 
 // tcgen05 tensor-core attention (bf16, D = 128).  kt, vt: [B, H, T, 128] text
 // keys appended after the image keys of every query (T = 0: none).
@@ -141,8 +226,10 @@ cudaError_t read_and_clear_tc_error(int* code);
 // rectangle are skipped.
 cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, const void* kt,
                                   const void* vt, int T, const int* cand, int R,
-                                  const PlanLayout& L, const void* plan, void* o, float* ws,
+                                  const PlanLayout& L, const void* plan, void* o, void* ws,
                                   int H, float scale, cudaStream_t s);
+// Bytes of the window workspace for H heads of head_dim D.
+int64_t window_ws_bytes(const PlanLayout& L, int H, int D);
 // Detail map and planner in one cooperative launch (one memset of the
 // barrier words first); a barrier timeout raises the planner error flag.
 // target_extra (0 in every product call) raises each grid-barrier target so

@@ -5,9 +5,11 @@
 //   window : per plan work item (window W, 256-query block), keys S = Halo
 //            rectangle of W followed by its global-KV tokens.  A token inside
 //            one window only takes that window's output; a token in an overlap
-//            adds its tent-weighted share to an fp32 workspace, normalised
-//            afterwards by the per-token weight sum (AReA Phase II,
-//            centre-weighted blending of overlaps).
+//            has one fp32 accumulator row, written by its lowest parity class
+//            of windows, added to by the higher ones and normalised by the
+//            per-token weight sum by the highest (AReA Phase II,
+//            centre-weighted blending of overlaps).  One launch per parity
+//            class keeps that order; windows of one class never overlap.
 // Pages: ai.info "Methodology in Plain English" (Phase I, Phase II).
 #include "area_internal.cuh"
 
@@ -27,8 +29,8 @@ template <typename T, int D, bool WINDOW>
 __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
     const T* __restrict__ kt, const T* __restrict__ vt, int ntext, const int* __restrict__ cand,
-    int R, T* __restrict__ o, float* __restrict__ ws, int H, DenseRows dr, PlanView P,
-    float scale) {
+    int R, T* __restrict__ o, float* acc, int H, DenseRows dr, PlanView P, float scale, int cls,
+    int nx2, long long n_ov) {
   constexpr int DPT = D / kSimtTPQ;
   extern __shared__ float smem[];
   float* Ks = smem;                       // [kSimtKV][D]
@@ -49,9 +51,11 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
   int qtok;
   if (WINDOW) {
     N = P.N;
-    const int item = blockIdx.x / (kQTile / kSimtQ);
+    const int ic = blockIdx.x / (kQTile / kSimtQ);       // item within the class
     const int sub = blockIdx.x % (kQTile / kSimtQ);
-    if (item >= P.nitem[b]) return;
+    if (ic >= P.nclass[b * 4 + cls]) return;
+    int item = ic;
+    for (int c = 0; c < cls; ++c) item += P.nclass[b * 4 + c];
     const int2 it = P.items[(int64_t)b * P.nitem_max + item];
     wi = it.x;
     const int64_t wo = (int64_t)b * P.nw + wi;
@@ -79,11 +83,11 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
   const int nimg = nkv;
   nkv += ntext;
 
-  float qv[DPT], acc[DPT];
+  float qv[DPT], acc_v[DPT];
 #pragma unroll
   for (int i = 0; i < DPT; ++i) {
     qv[i] = load_as_float(qrow, part + kSimtTPQ * i) * scale;
-    acc[i] = 0.f;
+    acc_v[i] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
 
@@ -144,92 +148,73 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     const float corr = expf(m - mn);
     l *= corr;
 #pragma unroll
-    for (int i = 0; i < DPT; ++i) acc[i] *= corr;
+    for (int i = 0; i < DPT; ++i) acc_v[i] *= corr;
 #pragma unroll
     for (int j = 0; j < kSimtKV; ++j) {
       const float p = expf(s[j] - mn);
       l += p;
 #pragma unroll
-      for (int i = 0; i < DPT; ++i) acc[i] += p * Vs[j * D + part + kSimtTPQ * i];
+      for (int i = 0; i < DPT; ++i) acc_v[i] += p * Vs[j * D + part + kSimtTPQ * i];
     }
     m = mn;
     __syncthreads();
   }
   if (!qvalid) return;
   const float inv = 1.f / l;
+  T* dst = o + (bh * N + qtok) * D;
   if (WINDOW) {
-    if (P.cover[(int64_t)b * P.N + qtok] == 1) {
-      // the only window containing this token: its output is the merge
-      T* dst = o + (bh * N + qtok) * D;
-#pragma unroll
-      for (int i = 0; i < DPT; ++i) store_from_float(dst, part + kSimtTPQ * i, acc[i] * inv);
-    } else {
-      const int y = qtok / P.Wg, x = qtok % P.Wg;
+    const int parent = P.parent[(int64_t)b * P.nw + wi];
+    const int4 my = axis_merge(parent / P.nbx, P.nby, P.Hg, P.hy, P.sy);
+    const int4 mx = axis_merge(parent % P.nbx, P.nbx, P.Wg, P.wx, P.sx);
+    const int y = qtok / P.Wg, x = qtok % P.Wg;
+    const MergeRole mr = merge_role(y, x, cls, my, mx, P.Wg, nx2);
+    if (mr.ov) {
+      // overlap: this class's share goes to the token's accumulator row
       const float t = (float)(min(y - win.x + 1, win.x + win.z - y) *
                               min(x - win.y + 1, win.y + win.w - x));
-      float* dst = ws + (bh * N + qtok) * D;
+      float* arow = acc + (bh * n_ov + mr.rank) * D;
+      const float winv = 1.f / P.wsum[(int64_t)b * P.N + qtok];
 #pragma unroll
-      for (int i = 0; i < DPT; ++i) atomicAdd(dst + part + kSimtTPQ * i, t * acc[i] * inv);
+      for (int i = 0; i < DPT; ++i) {
+        const int d = part + kSimtTPQ * i;
+        float a = acc_v[i] * (t * inv);
+        if (!mr.first) a += arow[d];
+        if (mr.last) store_from_float(dst, d, a * winv);
+        else arow[d] = a;
+      }
+      return;
     }
-  } else {
-    T* dst = o + (bh * N + qtok) * D;
+  }
+  // the only window containing this token (or dense attention): the output
 #pragma unroll
-    for (int i = 0; i < DPT; ++i) store_from_float(dst, part + kSimtTPQ * i, acc[i] * inv);
-  }
+  for (int i = 0; i < DPT; ++i) store_from_float(dst, part + kSimtTPQ * i, acc_v[i] * inv);
 }
 
-// Zero the workspace rows of tokens covered by more than one window (the
-// only rows the window kernels accumulate into).
-__global__ void __launch_bounds__(256) ws_zero_kernel(float4* ws, PlanView P, int H, int D) {
-  const int64_t n4 = (int64_t)P.B * H * P.N * D / 4;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = (i * 4) / D;          // (b*H + h)*N + n
-    const int n = (int)(row % P.N);
-    const int b = (int)(row / P.N / H);
-    if (P.cover[(int64_t)b * P.N + n] > 1) ws[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-}
-
-template <typename T>
-__global__ void __launch_bounds__(256) window_finalize_kernel(const float4* __restrict__ ws,
-                                                              PlanView P, T* __restrict__ o,
-                                                              int H, int D) {
-  const int64_t n4 = (int64_t)P.B * H * P.N * D / 4;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = (i * 4) / D;          // (b*H + h)*N + n
-    const int n = (int)(row % P.N);
-    const int b = (int)(row / P.N / H);
-    if (P.cover[(int64_t)b * P.N + n] <= 1) continue;    // written by its window
-    const float inv = 1.f / P.wsum[(int64_t)b * P.N + n];
-    const float4 a = ws[i];
-    store_from_float(o, 4 * i + 0, a.x * inv);
-    store_from_float(o, 4 * i + 1, a.y * inv);
-    store_from_float(o, 4 * i + 2, a.z * inv);
-    store_from_float(o, 4 * i + 3, a.w * inv);
-  }
-}
+struct MergeArgs {
+  float* acc;       // accumulator rows [B*H][n_ov][D]
+  int nx2;
+  long long n_ov;
+};
 
 template <typename T, int D, bool WINDOW>
 cudaError_t launch_simt(dim3 grid, const void* q, const void* k, const void* v, const void* kt,
-                        const void* vt, int ntext, const int* cand, int R, void* o, float* ws,
-                        int H, DenseRows dr, PlanView P, float scale, cudaStream_t s) {
+                        const void* vt, int ntext, const int* cand, int R, void* o,
+                        const MergeArgs& ma, int H, DenseRows dr, PlanView P, float scale,
+                        cudaStream_t s) {
   const int smem = 2 * kSimtKV * D * (int)sizeof(float);
   auto fn = attn_simt_kernel<T, D, WINDOW>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  fn<<<grid, kSimtThreads, smem, s>>>(static_cast<const T*>(q), static_cast<const T*>(k),
-                                      static_cast<const T*>(v), static_cast<const T*>(kt),
-                                      static_cast<const T*>(vt), ntext, cand, R,
-                                      static_cast<T*>(o), ws, H, dr, P, scale);
-  return cudaGetLastError();
-}
-
-int grid_cap(int64_t n, int block) {
-  int64_t g = (n + block - 1) / block;
-  const int64_t cap = 148LL * 32;
-  return (int)(g < 1 ? 1 : (g > cap ? cap : g));
+  // window mode: one launch per parity class, in class order
+  for (int cls = 0; cls < (WINDOW ? 4 : 1); ++cls) {
+    fn<<<grid, kSimtThreads, smem, s>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                        static_cast<const T*>(v), static_cast<const T*>(kt),
+                                        static_cast<const T*>(vt), ntext, cand, R,
+                                        static_cast<T*>(o), ma.acc, H, dr, P, scale, cls, ma.nx2,
+                                        ma.n_ov);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -241,47 +226,28 @@ cudaError_t launch_dense_attn_simt(const void* q, const void* k, const void* v, 
   DenseRows dr{N, Nk};
   PlanView P{};
   if (dtype == AREA_DTYPE_F32) {
-    if (D == 64) return launch_simt<float, 64, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, nullptr, H, dr, P, scale, s);
-    return launch_simt<float, 128, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, nullptr, H, dr, P, scale, s);
+    if (D == 64) return launch_simt<float, 64, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, MergeArgs{}, H, dr, P, scale, s);
+    return launch_simt<float, 128, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, MergeArgs{}, H, dr, P, scale, s);
   }
-  if (D == 64) return launch_simt<__nv_bfloat16, 64, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, nullptr, H, dr, P, scale, s);
-  return launch_simt<__nv_bfloat16, 128, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, nullptr, H, dr, P, scale, s);
+  if (D == 64) return launch_simt<__nv_bfloat16, 64, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, MergeArgs{}, H, dr, P, scale, s);
+  return launch_simt<__nv_bfloat16, 128, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, MergeArgs{}, H, dr, P, scale, s);
 }
 
 cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v, const void* kt,
                                     const void* vt, int T, const int* cand, int R,
-                                    const PlanLayout& L, const void* plan, void* o, float* ws,
+                                    const PlanLayout& L, const void* plan, void* o, void* ws,
                                     int H, int D, float scale, int dtype, cudaStream_t s) {
   PlanView P = plan_view(L, const_cast<void*>(plan));
+  const MergeArgs ma{reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeaderBytes),
+                     (int)L.nx2, (long long)L.n_ov};
   dim3 grid((unsigned)(L.nitem_max * (kQTile / kSimtQ)), H, (unsigned)L.B);
   DenseRows dr{(int)L.N, (int)L.N};
   if (dtype == AREA_DTYPE_F32) {
-    if (D == 64) return launch_simt<float, 64, true>(grid, q, k, v, kt, vt, T, cand, R, o, ws, H, dr, P, scale, s);
-    return launch_simt<float, 128, true>(grid, q, k, v, kt, vt, T, cand, R, o, ws, H, dr, P, scale, s);
+    if (D == 64) return launch_simt<float, 64, true>(grid, q, k, v, kt, vt, T, cand, R, o, ma, H, dr, P, scale, s);
+    return launch_simt<float, 128, true>(grid, q, k, v, kt, vt, T, cand, R, o, ma, H, dr, P, scale, s);
   }
-  if (D == 64) return launch_simt<__nv_bfloat16, 64, true>(grid, q, k, v, kt, vt, T, cand, R, o, ws, H, dr, P, scale, s);
-  return launch_simt<__nv_bfloat16, 128, true>(grid, q, k, v, kt, vt, T, cand, R, o, ws, H, dr, P, scale, s);
-}
-
-cudaError_t launch_ws_zero(float* ws, const PlanLayout& L, const void* plan, int H, int D,
-                           cudaStream_t s) {
-  PlanView P = plan_view(L, const_cast<void*>(plan));
-  const int64_t n4 = L.B * H * L.N * D / 4;
-  ws_zero_kernel<<<grid_cap(n4, 256), 256, 0, s>>>(reinterpret_cast<float4*>(ws), P, H, D);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_window_finalize(const float* ws, const PlanLayout& L, const void* plan,
-                                   void* o, int H, int D, int dtype, cudaStream_t s) {
-  PlanView P = plan_view(L, const_cast<void*>(plan));
-  const int64_t n4 = L.B * H * L.N * D / 4;
-  const int grid = grid_cap(n4, 256);
-  auto* w4 = reinterpret_cast<const float4*>(ws);
-  if (dtype == AREA_DTYPE_F32)
-    window_finalize_kernel<float><<<grid, 256, 0, s>>>(w4, P, static_cast<float*>(o), H, D);
-  else
-    window_finalize_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(w4, P, static_cast<__nv_bfloat16*>(o), H, D);
-  return cudaGetLastError();
+  if (D == 64) return launch_simt<__nv_bfloat16, 64, true>(grid, q, k, v, kt, vt, T, cand, R, o, ma, H, dr, P, scale, s);
+  return launch_simt<__nv_bfloat16, 128, true>(grid, q, k, v, kt, vt, T, cand, R, o, ma, H, dr, P, scale, s);
 }
 
 }  // namespace area

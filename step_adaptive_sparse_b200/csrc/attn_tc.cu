@@ -9,13 +9,17 @@
 // gpt-diffusion.com "Las dos fases de AReA".
 //
 // Design (one persistent CTA per SM, 320 threads):
-//   warp 0      TMA producer: Q tiles once per work unit, then a ring of K and
-//               V tiles (128 keys x 128 dims, 128B-swizzled, 32 KB each).
-//               Dense rows use tiled 2-D loads.  Window keys are the Halo
-//               rectangle, covered by 16x8-token patches (one 3-D tiled box
-//               each, masked at the rectangle's right and bottom edges), then
-//               the global-KV list (gather4, 4 rows per lane); window queries
-//               (the rectangle enumerated row-major) use gather4.
+//   warp 0      producer: claims work units (window mode: from a counter in
+//               the workspace, in the plan's parity-class order; dense mode:
+//               statically), publishes one record per unit in a shared-memory
+//               ring read by the other roles, and issues the TMA loads: Q
+//               tiles once per unit, then a ring of K and V tiles (128 keys x
+//               128 dims, 128B-swizzled, 32 KB each).  Dense rows use tiled
+//               2-D loads.  Window keys are the global-KV list first (gather4,
+//               4 rows per lane), then the Halo rectangle covered by 16x8-token
+//               patches (one 3-D tiled box each, masked at the rectangle's
+//               right and bottom edges); window queries (the rectangle
+//               enumerated row-major) use gather4.
 //   warp 1      TMEM allocator and the single MMA-issuing thread.
 //   warps 2-5   softmax of query tile 0, warps 6-9 of query tile 1: each
 //               thread owns one query row (TMEM lane 32*(warp mod 4) + lane).
@@ -26,6 +30,9 @@
 // computes the second.  Online softmax rescales O in TMEM only when some row of a warp
 // sees its running maximum grow by more than 2^8 (the final normalisation uses
 // the same stale maximum in numerator and denominator, so the result is exact).
+// Window outputs are merged without atomics: the units of one parity class
+// of windows never overlap, and the classes add into the fp32 accumulator
+// rows of overlapped tokens one after another (see the epilogue).
 // Every branch around a .sync.aligned tcgen05 instruction is warp-uniform.
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the kernel
 // records an error code, stops issuing work and still releases its TMEM.
@@ -40,7 +47,31 @@ __device__ int g_tc_error = 0;   // set on a bounded-wait expiry; read by tests
 
 namespace {
 
-constexpr int kThreads = 320;
+// Warp roles.  By default warp 0 is the producer, warp 1 the MMA issuer and
+// warps 2-9 the softmax (320 threads, every thread capped at 168 registers).
+// With AREA_TC_WG_SPLIT the CTA has three warpgroups (384 threads launched at
+// 168 registers each): warpgroup 0 (producer, MMA issuer, two idle warps)
+// gives registers back with setmaxnreg and the two softmax warpgroups take
+// them, 56 + 2 x 224 = 3 x 168 per lane of a warpgroup, the block's whole
+// launch allocation.
+#ifndef AREA_TC_WG_SPLIT
+#define AREA_TC_WG_SPLIT 0
+#endif
+// Exponentials of every 8 key pairs computed on the FMA pipe instead of the
+// MUFU unit (0..8); see exp2_poly2.
+#ifndef AREA_EXP2_POLY_PER8
+#define AREA_EXP2_POLY_PER8 0
+#endif
+constexpr bool kWgSplit = AREA_TC_WG_SPLIT != 0;
+constexpr int kSoftWarp0 = kWgSplit ? 4 : 2;          // first softmax warp
+constexpr int kThreads = kSoftWarp0 * 32 + 256;
+// The split is sized for the registers the kernel is compiled to start with
+// (ptxas, no launch bound: the setmaxnreg regions may not exceed a bound).
+// The host refuses the launch unless warpgroup 0's release covers the softmax
+// warpgroups' increase: kRegsLow * 128 + kRegsHigh * 256 <= entry * 384.
+constexpr int kRegsLow = 56, kRegsHigh = 208;
+constexpr int kPolyPer8 = AREA_EXP2_POLY_PER8;
+static_assert(kPolyPer8 >= 0 && kPolyPer8 <= 8, "polynomial share");
 constexpr int kStages = 4;              // K/V ring stages of 32 KB
 constexpr int kTileBytes = 128 * 128 * 2;
 constexpr int kHalfBytes = 128 * 128;   // 128 rows x 64 bf16
@@ -52,6 +83,7 @@ constexpr int kPParts = 2;                   // P handed to the PV product in th
 // one 128-key tile each, loaded by a 3-D tiled TMA box (tokens of one grid
 // row are contiguous).  Only the global-KV list is gathered row by row.
 constexpr int kPW = 16, kPH = 8;
+constexpr int kRecSlots = 3;                 // unit records in flight (shared-memory ring)
 
 // Shared-memory plan (offsets from a 1024-aligned base).
 constexpr int kSmemQ = 0;                              // 2 tiles x 32 KB
@@ -70,9 +102,12 @@ enum {
   BAR_P_PART1 = BAR_P_PART0 + kPParts - 1,
   BAR_KV_FULL = BAR_P_PART1 + kPParts - 1,  // kStages of them
   BAR_KV_EMPTY = BAR_KV_FULL + kStages,
-  BAR_DRAIN = BAR_KV_EMPTY + kStages,  // MMA completion before TMEM release
+  BAR_REC_FULL = BAR_KV_EMPTY + kStages,     // kRecSlots unit-record slots
+  BAR_REC_EMPTY = BAR_REC_FULL + kRecSlots,
+  BAR_DRAIN = BAR_REC_EMPTY + kRecSlots,     // MMA completion before TMEM release
   BAR_COUNT
 };
+static_assert(BAR_COUNT * 8 <= 256, "barrier area");
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -273,6 +308,43 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// 2^x for two arguments on the FMA pipe (packed f32x2 arithmetic), for
+// x <= 0 as in the softmax.  Method: Cody-Waite range reduction
+// x = n + f with n = round(x) (the 1.5 * 2^23 rounding constant), f in
+// [-0.5, 0.5]; 2^f by a cubic fitted in this project by the Remez exchange on
+// relative error over [-0.5, 0.5] (maximum relative error 7.5e-5 in fp32,
+// below the 2^-9 rounding of the bf16 probabilities it feeds); 2^n applied by
+// adding n to the exponent field.  Arguments below -126 are raised to -126,
+// so a masked key (x = -inf) gets 2^-126 instead of 0.
+constexpr float kExp2C0 = 0.9999280571937561f, kExp2C1 = 0.6932609677314758f,
+                kExp2C2 = 0.2426111251115799f, kExp2C3 = 0.0551716685295105f;
+__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  float t0, t1, p0, p1;
+  asm("{\n\t.reg .b64 px, pm, pt, pn, pf, pp, c;\n\t"
+      "mov.b64 px, {%4, %5};\n\t"
+      "mov.b64 pm, {%6, %6};\n\t"
+      "add.rn.f32x2 pt, px, pm;\n\t"          // t = x + 1.5 * 2^23: round to integer
+      "sub.rn.f32x2 pn, pt, pm;\n\t"          // n = round(x)
+      "sub.rn.f32x2 pf, px, pn;\n\t"          // f = x - n
+      "mov.b64 c, {%10, %10};\n\t"
+      "mov.b64 pp, {%9, %9};\n\t"
+      "fma.rn.f32x2 pp, c, pf, pp;\n\t"       // c3 f + c2
+      "mov.b64 c, {%8, %8};\n\t"
+      "fma.rn.f32x2 pp, pp, pf, c;\n\t"       // (..) f + c1
+      "mov.b64 c, {%7, %7};\n\t"
+      "fma.rn.f32x2 pp, pp, pf, c;\n\t"       // (..) f + c0
+      "mov.b64 {%0, %1}, pt;\n\t"
+      "mov.b64 {%2, %3}, pp;\n\t}"
+      : "=f"(t0), "=f"(t1), "=f"(p0), "=f"(p1)
+      : "f"(x0), "f"(x1), "f"(12582912.0f), "f"(kExp2C0), "f"(kExp2C1), "f"(kExp2C2),
+        "f"(kExp2C3));
+  // the low mantissa bits of t hold n: shifted into the exponent field
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 // Packed fp32 pair arithmetic of sm_100 (one instruction for two lanes of work).
 __device__ __forceinline__ void fma2(float& y0, float& y1, float a0, float a1, float b, float c) {
   asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\t"
@@ -297,88 +369,35 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
-
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
-}
-
 // ---------------------------------------------------------------------------
-// Work units
+// Work units.  The producer warp turns each unit into a record in a
+// kRecSlots-slot shared-memory ring (FULL: the producer wrote it; EMPTY: the
+// MMA thread and the eight softmax warps are done with it).  Nobody else
+// decodes the plan, so no role waits on a chain of dependent global loads at
+// a unit boundary.
 // ---------------------------------------------------------------------------
 struct DenseArgs {
   int B, H, N, Nk;
   int units_per_head;   // ceil(N / 256)
 };
 
-struct Unit {
-  bool valid;
-  int bh;          // b*H + h
-  int b;
-  int q0;          // first query position of tile 0 (tile 1 = q0 + 128)
-  int nq;          // number of valid query positions from q0 (window: area)
-  int nkv;         // dense: number of keys; window: G_W (global-KV count)
-  int nti;         // key tiles of image tokens (rectangle patches + global / dense keys)
-  int nt;          // key tiles of this unit, text tiles included
-  int ncx;         // window: patches per row of the Halo rectangle
-  int ntr;         // window: patch tiles of the Halo rectangle
-  int4 win, ext;   // window mode
-  const int* glist;
+struct UnitRec {
+  int valid;          // 0: no more work for this CTA
+  int bh, b;
+  int q0;             // first query position of tile 0 (tile 1 = q0 + 128)
+  int nq;             // valid query positions (dense: N; window: its area)
+  int nkv;            // keys of the leading list tiles (dense keys, or global-KV count)
+  int ngt;            // leading list tiles (dense key tiles, or global-KV tiles)
+  int ntr;            // window: Halo-rectangle patch tiles, after the list tiles
+  int ncx;            // window: patches per row of the Halo rectangle
+  int nt;             // all key tiles of the unit, text tiles included
+  int cls;            // window: parity class of the base window
+  int pad;
+  int4 win, ext;      // window: the window and its Halo rectangle (y0, x0, hy, wx)
+  int4 my, mx;        // window: merge geometry of the base window per axis (axis_merge)
+  long long glist;    // window: element offset of the global list in the plan or cand
 };
-
-template <bool WINDOW>
-__device__ __forceinline__ Unit get_unit(int u, const DenseArgs& da, const PlanView& P, int H,
-                                         int T, const int* cand = nullptr, int R = 0) {
-  Unit x;
-  x.valid = true;
-  x.glist = nullptr;
-  if (!WINDOW) {
-    x.bh = u / da.units_per_head;
-    x.b = x.bh / da.H;
-    x.q0 = (u % da.units_per_head) * 256;
-    x.nq = da.N;
-    x.nkv = da.Nk;
-    x.nti = (da.Nk + 127) / 128;
-    x.nt = x.nti + (T + 127) / 128;
-    x.ncx = x.ntr = 0;
-    x.win = x.ext = make_int4(0, 0, 0, 0);
-  } else {
-    // Head-major order: consecutive units are the query blocks of one
-    // (batch, head), windows costliest first, so the CTAs in flight share a
-    // few windows' keys and values in L2.
-    const int item = u % P.nitem_max;
-    x.bh = u / P.nitem_max;
-    x.b = x.bh / H;
-    if (item >= P.nitem[x.b]) {
-      x.valid = false;
-      return x;
-    }
-    const int2 it = P.items[(int64_t)x.b * P.nitem_max + item];
-    const int64_t wo = (int64_t)x.b * P.nw + it.x;
-    x.win = P.win[wo];
-    x.ext = P.ext[wo];
-    x.q0 = it.y * 256;
-    x.nq = x.win.z * x.win.w;
-    x.nkv = cand ? R : P.gcount[wo];
-    x.ncx = (x.ext.w + kPW - 1) / kPW;
-    x.ntr = x.ncx * ((x.ext.z + kPH - 1) / kPH);
-    x.nti = x.ntr + (x.nkv + 127) / 128;
-    x.nt = x.nti + (T + 127) / 128;
-    x.glist = cand ? cand + (int64_t)x.bh * R : P.gidx + wo * P.G;
-  }
-  return x;
-}
-
-// Token of the p-th global-KV key of a window unit (clamped into the list).
-__device__ __forceinline__ int window_global_token(const Unit& x, int p) {
-  return x.glist[p < x.nkv ? p : (x.nkv > 0 ? x.nkv - 1 : 0)];
-}
-
-__device__ __forceinline__ int window_query_token(const Unit& x, int p, int Wg) {
-  if (p >= x.nq) p = 0;
-  return (x.win.x + p / x.win.w) * Wg + x.win.y + p % x.win.w;
-}
+static_assert(sizeof(UnitRec) <= 128, "unit record");
 
 struct TcParams {
   float scale_log2;
@@ -386,15 +405,89 @@ struct TcParams {
   int T;              // text keys per (b, h), appended after the image keys
   const int* cand;    // bridge mode: per-head candidate tokens [B*H][R] (else null)
   int R;
-  int num_units;
+  int num_units;      // dense: all units; window: capacity (the plan holds the count)
   DenseArgs da;
   PlanView P;
-  __nv_bfloat16* o;   // dense output
-  float* ws;          // window workspace
+  __nv_bfloat16* o;   // output
+  unsigned* counters; // window: workspace header (unit counter, per-class completions)
+  float* acc;         // window: fp32 accumulator rows [B*H][n_ov][128]
+  int nx2;            // window: columns covered by two base windows
+  long long n_ov;     // window: overlapped tokens per element
 };
 
+// Query token of position p of a window enumerated row-major (clamped).
+__device__ __forceinline__ int window_query_token(const int4& win, int nq, int p, int Wg) {
+  if (p >= nq) p = 0;
+  return (win.x + p / win.w) * Wg + win.y + p % win.w;
+}
+
+// Decode unit u into a record (producer lane 0).  Dense: (b*H + h, 256-query
+// block), head-major.  Window: by parity class, then batch element, then
+// head, then the class's work items in plan order.
+template <bool WINDOW>
+__device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
+  r.valid = 1;
+  r.pad = 0;
+  r.cls = 0;
+  r.glist = 0;
+  r.ntr = r.ncx = 0;
+  r.win = r.ext = r.my = r.mx = make_int4(0, 0, 0, 0);
+  if (!WINDOW) {
+    if (u >= prm.num_units) return false;
+    r.bh = u / prm.da.units_per_head;
+    r.b = r.bh / prm.da.H;
+    r.q0 = (u % prm.da.units_per_head) * 256;
+    r.nq = prm.da.N;
+    r.nkv = prm.da.Nk;
+    r.ngt = (prm.da.Nk + 127) / 128;
+    r.nt = r.ngt + (prm.T + 127) / 128;
+    return true;
+  }
+  const PlanView& P = prm.P;
+  int rem = u;
+  for (int c = 0; c < 4; ++c) {
+    for (int b = 0; b < P.B; ++b) {
+      const int n = P.nclass[b * 4 + c];
+      const int cnt = n * prm.H;
+      if (rem >= cnt) {
+        rem -= cnt;
+        continue;
+      }
+      int coff = 0;
+      for (int c2 = 0; c2 < c; ++c2) coff += P.nclass[b * 4 + c2];
+      const int h = rem / n;
+      const int2 it = P.items[(int64_t)b * P.nitem_max + coff + rem % n];
+      const int64_t wo = (int64_t)b * P.nw + it.x;
+      r.b = b;
+      r.bh = b * prm.H + h;
+      r.win = P.win[wo];
+      r.ext = P.ext[wo];
+      const int parent = P.parent[wo];
+      r.cls = window_class(parent, P.nbx);
+      r.my = axis_merge(parent / P.nbx, P.nby, P.Hg, P.hy, P.sy);
+      r.mx = axis_merge(parent % P.nbx, P.nbx, P.Wg, P.wx, P.sx);
+      r.q0 = it.y * 256;
+      r.nq = r.win.z * r.win.w;
+      r.nkv = prm.cand ? prm.R : P.gcount[wo];
+      r.ngt = (r.nkv + 127) / 128;
+      r.ncx = (r.ext.w + kPW - 1) / kPW;
+      r.ntr = r.ncx * ((r.ext.z + kPH - 1) / kPH);
+      r.nt = r.ngt + r.ntr + (prm.T + 127) / 128;
+      r.glist = prm.cand ? (long long)r.bh * prm.R : (long long)wo * P.G;
+      return true;
+    }
+  }
+  return false;
+}
+
+#if AREA_TC_WG_SPLIT
+#define AREA_TC_BOUNDS
+#else
+#define AREA_TC_BOUNDS __launch_bounds__(kThreads, 1)
+#endif
+
 template <bool WINDOW, bool BRIDGE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void AREA_TC_BOUNDS
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
                const __grid_constant__ CUtensorMap tm_vp, const __grid_constant__ CUtensorMap tm_kt,
@@ -406,9 +499,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const uint32_t bar0 = sbase + kSmemBar;
   __shared__ uint32_t s_tmem_base;
   __shared__ int s_abort;
+  __shared__ __align__(16) UnitRec s_rec[kRecSlots];
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if constexpr (kWgSplit) {
+    // first thing: warpgroup 0 gives registers back, the softmax warpgroups
+    // take them (so almost no code runs at the entry allocation)
+    if (warp < kSoftWarp0) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+    else asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+  }
 
   if (threadIdx.x == 0) {
     s_abort = 0;
@@ -427,6 +527,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(BAR_KV_FULL + s), 1);
       mbar_init(bar(BAR_KV_EMPTY + s), 1);
+    }
+    for (int s = 0; s < kRecSlots; ++s) {
+      mbar_init(bar(BAR_REC_FULL + s), 1);
+      mbar_init(bar(BAR_REC_EMPTY + s), 9);   // the MMA thread and the 8 softmax warps
     }
     mbar_init(bar(BAR_DRAIN), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -448,10 +552,39 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    uint32_t kv_it = 0, unit_count = 0;
-    for (int u = blockIdx.x; u < prm.num_units; u += gridDim.x) {
-      const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T, BRIDGE ? prm.cand : nullptr, prm.R);
-      if (!x.valid) continue;
+    // Units are claimed from a counter in the workspace (window mode) or
+    // statically (dense mode).  The record of the next unit is written while
+    // the current unit's first key tiles are in flight.
+    uint32_t kv_it = 0, unit_count = 0, claims = 0;
+    bool ok = true;
+    auto claim = [&]() -> int {
+      int u = 0;
+      if (lane == 0) {
+        if (WINDOW) u = (int)atomicAdd(prm.counters + kWsUnitCounter, 1u);
+        else u = blockIdx.x + (int)claims * gridDim.x;
+      }
+      ++claims;
+      return __shfl_sync(0xffffffffu, u, 0);
+    };
+    // Claim, decode and publish the record of this CTA's k-th unit.
+    auto publish = [&](uint32_t k) -> bool {
+      const int u = claim();
+      const uint32_t slot = k % kRecSlots;
+      if (!warp_wait0(bar(BAR_REC_EMPTY + slot), ((k / kRecSlots) & 1u) ^ 1u, abort_flag))
+        return false;
+      if (lane == 0) {
+        UnitRec r;
+        if (!decode_unit<WINDOW>(u, prm, r)) r.valid = 0;
+        s_rec[slot] = r;
+        mbar_arrive(bar(BAR_REC_FULL + slot));
+      }
+      __syncwarp();
+      return true;
+    };
+    ok = publish(0);
+    while (ok) {
+      const UnitRec& R = s_rec[unit_count % kRecSlots];
+      if (!R.valid) break;
       if (!warp_wait0(bar(BAR_Q_EMPTY), (unit_count & 1u) ^ 1u, abort_flag)) break;
       if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL), 2 * kTileBytes);
       __syncwarp();
@@ -460,22 +593,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           for (int t = 0; t < 2; ++t)
             for (int hf = 0; hf < 2; ++hf)
               tma_load_2d(sbase + kSmemQ + t * kTileBytes + hf * kHalfBytes, &tm_q,
-                          bar(BAR_Q_FULL), hf * 64, x.bh * Ntok + x.q0 + t * 128);
+                          bar(BAR_Q_FULL), hf * 64, R.bh * Ntok + R.q0 + t * 128);
         }
       } else {
         for (int t = 0; t < 2; ++t) {
           int r[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            r[i] = x.bh * Ntok + window_query_token(x, x.q0 + t * 128 + lane * 4 + i, Wg);
+            r[i] = R.bh * Ntok + window_query_token(R.win, R.nq, R.q0 + t * 128 + lane * 4 + i, Wg);
           for (int hf = 0; hf < 2; ++hf)
             tma_gather4(sbase + kSmemQ + t * kTileBytes + hf * kHalfBytes + lane * 512, &tm_q,
                         bar(BAR_Q_FULL), hf * 64, r[0], r[1], r[2], r[3]);
         }
       }
-      const int nt = x.nt;
-      bool ok = true;
+      const int nt = R.nt, ngt = R.ngt, ntr = R.ntr, ncx = R.ncx, nkv = R.nkv;
+      const int nti = ngt + ntr;
+      const int bh = R.bh;
+      const int4 ext = R.ext;
+      const int* glist = (BRIDGE ? prm.cand : prm.P.gidx) + R.glist;
+      const int jn = nt < 2 ? nt : 2;         // the next record is published before tile jn
+      bool published = false;
       for (int j = 0; j < nt && ok; ++j) {
+        if (j == jn) {
+          published = true;
+          if (!(ok = publish(unit_count + 1))) break;
+        }
         for (int kv = 0; kv < 2; ++kv) {       // K then V
           const int s = (int)(kv_it % kStages);
           if (!warp_wait0(bar(BAR_KV_EMPTY + s), ((kv_it / kStages) & 1u) ^ 1u, abort_flag)) {
@@ -486,42 +628,48 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           __syncwarp();
           const CUtensorMap* tm = kv ? &tm_v : &tm_k;
           const uint32_t dst = sbase + kSmemKV + s * kTileBytes;
-          if (j >= x.nti) {
+          if (j >= nti) {
             // text keys: rows of the [B*H*T, 128] text tensors
             if (lane == 0) {
               const CUtensorMap* tt = kv ? &tm_vt : &tm_kt;
               for (int hf = 0; hf < 2; ++hf)
                 tma_load_2d(dst + hf * kHalfBytes, tt, bar(BAR_KV_FULL + s), hf * 64,
-                            x.bh * prm.T + (j - x.nti) * 128);
+                            bh * prm.T + (j - nti) * 128);
             }
-          } else if constexpr (!WINDOW) {
+          } else if (!WINDOW) {
             if (lane == 0)
               for (int hf = 0; hf < 2; ++hf)
                 tma_load_2d(dst + hf * kHalfBytes, tm, bar(BAR_KV_FULL + s), hf * 64,
-                            x.bh * Nkrows + j * 128);
-          } else if (j < x.ntr) {
-            // patch (px, py) of the Halo rectangle: kPH grid rows of kPW tokens
-            if (lane == 0) {
-              const CUtensorMap* tp = kv ? &tm_vp : &tm_kp;
-              const int px = j % x.ncx, py = j / x.ncx;
-              const int cx = x.ext.y + px * kPW;
-              const int cy = x.bh * prm.P.Hg + x.ext.x + py * kPH;
-              for (int hf = 0; hf < 2; ++hf)
-                tma_load_3d(dst + hf * kHalfBytes, tp, bar(BAR_KV_FULL + s), hf * 64, cx, cy);
-            }
-          } else {
-            const int g0 = (j - x.ntr) * 128 + lane * 4;
+                            bh * Nkrows + j * 128);
+          } else if (j < ngt) {
+            // global-KV list (or bridge candidates), gathered 4 rows per lane
+            const int g0 = j * 128 + lane * 4;
             int r[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) r[i] = x.bh * Nkrows + window_global_token(x, g0 + i);
+            for (int i = 0; i < 4; ++i) {
+              const int p = g0 + i < nkv ? g0 + i : nkv - 1;
+              r[i] = bh * Nkrows + glist[p];
+            }
             for (int hf = 0; hf < 2; ++hf)
               tma_gather4(dst + hf * kHalfBytes + lane * 512, tm, bar(BAR_KV_FULL + s), hf * 64,
                           r[0], r[1], r[2], r[3]);
+          } else {
+            // patch (px, py) of the Halo rectangle: kPH grid rows of kPW tokens
+            if (lane == 0) {
+              const CUtensorMap* tp = kv ? &tm_vp : &tm_kp;
+              const int jj = j - ngt;
+              const int px = jj % ncx, py = jj / ncx;
+              const int cx = ext.y + px * kPW;
+              const int cy = bh * prm.P.Hg + ext.x + py * kPH;
+              for (int hf = 0; hf < 2; ++hf)
+                tma_load_3d(dst + hf * kHalfBytes, tp, bar(BAR_KV_FULL + s), hf * 64, cx, cy);
+            }
           }
           ++kv_it;
         }
       }
       if (!ok) break;
+      if (!published && !(ok = publish(unit_count + 1))) break;
       ++unit_count;
     }
     // Drain: the most recent load of every stage has landed (bounded wait).
@@ -566,10 +714,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         return true;
       };
-      for (int u = blockIdx.x; u < prm.num_units && ok; u += gridDim.x) {
-        const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T, BRIDGE ? prm.cand : nullptr, prm.R);
-        if (!x.valid) continue;
-        const int nt = x.nt;
+      while (ok) {
+        const uint32_t slot = unit_count % kRecSlots;
+        if (!(ok = mbar_wait(bar(BAR_REC_FULL + slot), (unit_count / kRecSlots) & 1u, abort_flag)))
+          break;
+        const int valid = s_rec[slot].valid, nt = s_rec[slot].nt;
+        mbar_arrive(bar(BAR_REC_EMPTY + slot));
+        if (!valid) break;
         if (!(ok = mbar_wait(bar(BAR_Q_FULL), unit_count & 1u, abort_flag))) break;
         // prologue: S(0)
         const uint32_t k0 = kv_it;
@@ -620,12 +771,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_wait(bar(BAR_DRAIN), 0, &drain_abort);
     }
     __syncwarp();
-  } else {
+  } else if (warp >= kSoftWarp0) {
     // ------------------------------------------------------------ softmax / epilogue
-    // Warps 2-5 own query tile 0 and warps 6-9 query tile 1.  A warp may only
-    // touch the TMEM lane quarter (warp id mod 4), and each group of four
-    // consecutive warps covers all four quarters.
-    const int qt = (warp - 2) >> 2;                  // query tile of this warpgroup
+    // The first four softmax warps own query tile 0, the next four query
+    // tile 1.  A warp may only touch the TMEM lane quarter (warp id mod 4),
+    // and each group of four consecutive warps covers all four quarters.
+    const int qt = (warp - kSoftWarp0) >> 2;         // query tile of this warpgroup
     const int row = ((warp & 3) << 5) + lane;        // TMEM lane = query row in the tile
     const uint32_t lane_off = (uint32_t)((warp & 3) << 5) << 16;
     const uint32_t tS = tmem + lane_off + (qt ? 128u : 0u);
@@ -634,19 +785,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t bP = bar(qt ? BAR_P_FULL1 : BAR_P_FULL0);
     const int bPpart = qt ? BAR_P_PART1 : BAR_P_PART0;
     const uint32_t bO = bar(qt ? BAR_O_FULL1 : BAR_O_FULL0);
-    uint32_t s_cnt = 0, o_cnt = 0;
+    uint32_t s_cnt = 0, o_cnt = 0, unit_count = 0;
     const float sl2 = prm.scale_log2;
     bool ok = true;
-    for (int u = blockIdx.x; u < prm.num_units && ok; u += gridDim.x) {
-      // key-tile geometry of this unit (the rest is looked up again for the
-      // epilogue rather than kept live in registers across the key loop)
-      int nkv, nt, nti, ntr, ncx, ew, eh;
-      {
-        const Unit x0 = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T, BRIDGE ? prm.cand : nullptr, prm.R);
-        if (!x0.valid) continue;
-        nkv = x0.nkv; nt = x0.nt; nti = x0.nti; ntr = x0.ntr; ncx = x0.ncx;
-        ew = x0.ext.w; eh = x0.ext.z;
-      }
+    while (ok) {
+      const uint32_t slot = unit_count % kRecSlots;
+      if (!(ok = warp_wait_all(bar(BAR_REC_FULL + slot), (unit_count / kRecSlots) & 1u,
+                               abort_flag)))
+        break;
+      const UnitRec& R = s_rec[slot];
+      if (!R.valid) break;
+      const int nkv = R.nkv, nt = R.nt, ngt = R.ngt, ntr = R.ntr, ncx = R.ncx;
+      const int nti = ngt + ntr;
+      const int ew = R.ext.w, eh = R.ext.z;
       float m = -INFINITY, l = 0.f;
       int pcx = 0, pcy = 0;                          // patch of tile j in the Halo rectangle
       for (int j = 0; j < nt; ++j) {
@@ -654,20 +805,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // rectangle; lane l tests keys 4l..4l+3 and ballots the result.  This
         // does not depend on S, so it is done before waiting for S (the loads
         // overlap the wait) and before S occupies 128 registers.
-        const bool bridge_tile = BRIDGE && j >= ntr && j < nti;
+        const bool bridge_tile = BRIDGE && j < ngt;
         uint32_t keep[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
         if (bridge_tile) {
-          const Unit xb = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T, prm.cand, prm.R);
+          const int* cl = prm.cand + R.glist;
+          const int4 ex = R.ext;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const int p = (j - ntr) * 128 + lane * 4 + i;
-            bool ok = p < nkv;
-            if (ok) {
-              const int tok = xb.glist[p];
+            const int p = j * 128 + lane * 4 + i;
+            bool in = p < nkv;
+            if (in) {
+              const int tok = cl[p];
               const int ty = tok / prm.P.Wg, tx = tok % prm.P.Wg;
-              ok = !(ty >= xb.ext.x && ty < xb.ext.x + eh && tx >= xb.ext.y && tx < xb.ext.y + ew);
+              in = !(ty >= ex.x && ty < ex.x + eh && tx >= ex.y && tx < ex.y + ew);
             }
-            keep[i] = __ballot_sync(0xffffffffu, ok);
+            keep[i] = __ballot_sync(0xffffffffu, in);
           }
         }
         if (!(ok = warp_wait_all(bS, s_cnt & 1u, abort_flag))) break;
@@ -675,16 +827,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc_fence_after();
         uint32_t sr[128];
         tmem_ld128(tS, sr);
-        // Key validity (warp-uniform): dense, global-KV and text tiles are a
-        // prefix of `valid` keys; a rectangle patch keeps columns dx < rem_x of
-        // rows dy < rem_y (key k = dy * kPW + dx).
+        // Key validity (warp-uniform): list and text tiles are a prefix of
+        // `valid` keys; a rectangle patch keeps columns dx < rem_x of rows
+        // dy < rem_y (key k = dy * kPW + dx).
         if (bridge_tile) {
 #pragma unroll
           for (int i = 0; i < 128; ++i)
             if (!((keep[i & 3] >> (i >> 2)) & 1u)) sr[i] = 0xff800000u;
-        } else if (!WINDOW || j >= ntr) {
-          const int valid = j < nti ? min(128, nkv - (j - ntr) * 128)
-                                    : min(128, prm.T - (j - nti) * 128);
+        } else if (!WINDOW || j < ngt || j >= nti) {
+          const int valid = j < ngt ? min(128, nkv - j * 128) : min(128, prm.T - (j - nti) * 128);
           if (valid < 128) {
 #pragma unroll
             for (int i = 0; i < 128; ++i)
@@ -714,8 +865,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const float mnew = fmaxf(mx * sl2, m);
         // Rescale O only when some row of the warp gained more than 2^8; the
         // decision is warp-uniform because the TMEM accesses are .sync.aligned.
+        // A row whose earlier keys were all masked has m = -inf (its l and O
+        // are zero): it takes alpha = 0.
         const bool rescale = j > 0 && __any_sync(0xffffffffu, mnew > m + kRescaleThreshold);
-        const float alpha = rescale ? fast_exp2(m - mnew) : 1.f;
+        const float alpha = rescale ? (m == -INFINITY ? 0.f : fast_exp2(m - mnew)) : 1.f;
         if (j == 0 || rescale) m = mnew;
         l *= alpha;
         // P = exp2(S * scale * log2(e) - m) as bf16, two keys per TMEM column,
@@ -723,8 +876,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // first 64 keys go out first, so the PV product can start on them
         // while the second 64 are computed; O is rescaled before that first
         // hand-over, so the PV products of this tile accumulate onto it.
+        // While every key so far is masked (m = -inf) the reference is 0.
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
-        const float negm = -m;
+        const float negm = m == -INFINITY ? 0.f : -m;
 #pragma unroll
         for (int h = 0; h < kPParts; ++h) {
           constexpr int kKeys = 128 / kPParts;
@@ -732,8 +886,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           for (int i = kKeys * h; i < kKeys * h + kKeys; i += 2) {
             float x0, x1;
             fma2(x0, x1, __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]), sl2, negm);
-            const float p0 = fast_exp2(x0);
-            const float p1 = fast_exp2(x1);
+            float p0, p1;
+            if (kPolyPer8 > 0 && ((i >> 1) & 7) < kPolyPer8) {
+              exp2_poly2(p0, p1, x0, x1);
+            } else {
+              p0 = fast_exp2(x0);
+              p1 = fast_exp2(x1);
+            }
             if ((i >> 1) & 1) add2(ls[2], ls[3], p0, p1); else add2(ls[0], ls[1], p0, p1);
             sr[i >> 1] = pack_bf16(p0, p1);
           }
@@ -754,28 +913,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           mbar_arrive(h + 1 < kPParts ? bar(bPpart + h) : bP);
         }
         l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-        if (WINDOW && ++pcx == ncx) {
+        if (WINDOW && j >= ngt && j < nti && ++pcx == ncx) {
           pcx = 0;
           ++pcy;
         }
       }
       if (!ok) break;
-      // epilogue (the unit is looked up again rather than kept live in
-      // registers across the key loop)
-      const Unit x = get_unit<WINDOW>(u, prm.da, prm.P, prm.H, prm.T, BRIDGE ? prm.cand : nullptr, prm.R);
-      int cover1 = 1;              // window: this row's token lies in one window only
-      if constexpr (WINDOW) {      // (read before the wait, so its latency overlaps it)
-        const int qp = x.q0 + qt * 128 + row;
-        cover1 = prm.P.cover[(int64_t)x.b * Ntok + window_query_token(x, qp, Wg)];
-      }
-      if (!(ok = warp_wait_all(bO, o_cnt & 1u, abort_flag))) break;
-      ++o_cnt;
-      tc_fence_after();
-      const int qpos = x.q0 + qt * 128 + row;
-      const bool qvalid = qpos < x.nq;
-      const float inv = 1.f / l;
+      // ---- epilogue
+      const int qpos = R.q0 + qt * 128 + row;
+      const bool qvalid = qpos < R.nq;
+      const int bh = R.bh;
       if constexpr (!WINDOW) {
-        __nv_bfloat16* dst = prm.o + ((int64_t)x.bh * Ntok + qpos) * 128;
+        if (!(ok = warp_wait_all(bO, o_cnt & 1u, abort_flag))) break;
+        ++o_cnt;
+        tc_fence_after();
+        const float inv = 1.f / l;
+        __nv_bfloat16* dst = prm.o + ((int64_t)bh * Ntok + qpos) * 128;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t orr[32];
@@ -794,42 +947,109 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
         }
       } else {
-        // A token inside one window only takes that window's output as it is;
-        // tokens in overlaps add their tent-weighted share to the workspace.
-        const int tok = window_query_token(x, qpos, Wg);
-        const bool single = cover1 == 1;
-        const int y = tok / Wg, xx = tok % Wg;
-        const float t = (float)(min(y - x.win.x + 1, x.win.x + x.win.z - y) *
-                                min(xx - x.win.y + 1, x.win.y + x.win.w - xx));
-        const float sc = single ? inv : t * inv;
-        float* dst = prm.ws + ((int64_t)x.bh * Ntok + tok) * 128;
-        __nv_bfloat16* dsto = prm.o + ((int64_t)x.bh * Ntok + tok) * 128;
+        // Centre-weighted merge.  A token inside one window stores its output
+        // directly.  A token in an overlap has one fp32 accumulator row: the
+        // window of its lowest parity class stores t * O, the middle classes
+        // add, the highest class adds and divides by the weight sum.  Windows
+        // of one class never overlap, and a class adds only after every unit
+        // of the lower classes has completed (a bounded wait on their
+        // completion counters), so the sum runs in a fixed order.
+        const int tok = window_query_token(R.win, R.nq, qpos, Wg);
+        const int y = tok / Wg, x = tok % Wg;
+        const MergeRole mr = merge_role(y, x, R.cls, R.my, R.mx, Wg, prm.nx2);
+        const bool rmw = qvalid && mr.ov;
+        // read before the O wait, so its latency overlaps it
+        const float wsum = rmw && mr.last ? prm.P.wsum[(int64_t)R.b * Ntok + tok] : 1.f;
+        const float tent = (float)(min(y - R.win.x + 1, R.win.x + R.win.z - y) *
+                                   min(x - R.win.y + 1, R.win.y + R.win.w - x));
+        const int cls = R.cls;
+        if (!(ok = warp_wait_all(bO, o_cnt & 1u, abort_flag))) break;
+        ++o_cnt;
+        tc_fence_after();
+        const float inv = 1.f / l;
+        if (__any_sync(0xffffffffu, rmw && !mr.first)) {
+          int wok = 1;
+          if (lane == 0) {
+            const uint64_t t0 = global_ns();
+            for (int c = 0; c < cls && wok; ++c) {
+              // completions class c needs: 8 warps per unit, H units per item
+              const unsigned target = 8u * (unsigned)prm.H * (unsigned)prm.P.nclass[prm.P.B * 4 + c];
+              uint32_t it = 0;
+              for (;;) {
+                unsigned v;
+                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];"
+                             : "=r"(v) : "l"(prm.counters + kWsClassDone + c) : "memory");
+                if (v >= target) break;
+                if ((++it & 63u) == 0) {
+                  if (*(volatile int*)abort_flag) { wok = 0; break; }
+                  if (global_ns() - t0 > kWaitNs) {
+                    *(volatile int*)abort_flag = 1;
+                    atomicExch(&g_tc_error, 1);
+                    wok = 0;
+                    break;
+                  }
+                }
+                __nanosleep(64);
+              }
+            }
+          }
+          wok = __shfl_sync(0xffffffffu, wok, 0);
+          __threadfence();
+          if (!(ok = wok != 0)) break;
+        }
+        const float sc = mr.ov ? tent * inv : inv;
+        const float winv = 1.f / wsum;
+        __nv_bfloat16* dsto = prm.o + ((int64_t)bh * Ntok + tok) * 128;
+        float* acc = prm.acc + ((int64_t)bh * prm.n_ov + mr.rank) * 128;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t orr[32];
           tmem_ld32(tO + c * 32, orr);
-          if (qvalid && single) {
-            uint4* d4 = reinterpret_cast<uint4*>(dsto + c * 32);
+          if (!qvalid) continue;
+          float vals[32];
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) {
-              uint4 w;
-              w.x = pack_bf16(__uint_as_float(orr[8 * v4 + 0]) * sc, __uint_as_float(orr[8 * v4 + 1]) * sc);
-              w.y = pack_bf16(__uint_as_float(orr[8 * v4 + 2]) * sc, __uint_as_float(orr[8 * v4 + 3]) * sc);
-              w.z = pack_bf16(__uint_as_float(orr[8 * v4 + 4]) * sc, __uint_as_float(orr[8 * v4 + 5]) * sc);
-              w.w = pack_bf16(__uint_as_float(orr[8 * v4 + 6]) * sc, __uint_as_float(orr[8 * v4 + 7]) * sc);
-              d4[v4] = w;
+          for (int i = 0; i < 32; ++i) vals[i] = __uint_as_float(orr[i]) * sc;
+          if (rmw) {
+            float4* a4 = reinterpret_cast<float4*>(acc + c * 32);
+            if (!mr.first) {
+#pragma unroll
+              for (int v4 = 0; v4 < 8; ++v4) {
+                const float4 a = a4[v4];
+                vals[4 * v4 + 0] += a.x;
+                vals[4 * v4 + 1] += a.y;
+                vals[4 * v4 + 2] += a.z;
+                vals[4 * v4 + 3] += a.w;
+              }
             }
-          } else if (qvalid) {
+            if (!mr.last) {
 #pragma unroll
-            for (int v4 = 0; v4 < 8; ++v4)
-              red_add_v4(dst + c * 32 + 4 * v4, __uint_as_float(orr[4 * v4]) * sc,
-                         __uint_as_float(orr[4 * v4 + 1]) * sc,
-                         __uint_as_float(orr[4 * v4 + 2]) * sc,
-                         __uint_as_float(orr[4 * v4 + 3]) * sc);
+              for (int v4 = 0; v4 < 8; ++v4)
+                a4[v4] = make_float4(vals[4 * v4], vals[4 * v4 + 1], vals[4 * v4 + 2],
+                                     vals[4 * v4 + 3]);
+              continue;
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) vals[i] *= winv;
+          }
+          uint4* d4 = reinterpret_cast<uint4*>(dsto + c * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w;
+            w.x = pack_bf16(vals[8 * v4 + 0], vals[8 * v4 + 1]);
+            w.y = pack_bf16(vals[8 * v4 + 2], vals[8 * v4 + 3]);
+            w.z = pack_bf16(vals[8 * v4 + 4], vals[8 * v4 + 5]);
+            w.w = pack_bf16(vals[8 * v4 + 6], vals[8 * v4 + 7]);
+            d4[v4] = w;
           }
         }
+        // this warp's rows of the unit are complete
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(prm.counters + kWsClassDone + cls, 1u);
       }
       tc_fence_before();
+      if (lane == 0) mbar_arrive(bar(BAR_REC_EMPTY + slot));
+      ++unit_count;
     }
   }
   tc_fence_before();
@@ -899,6 +1119,17 @@ cudaError_t launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
   auto fn = attn_tc_kernel<WINDOW, BRIDGE>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
+  if constexpr (kWgSplit) {
+    // setmaxnreg.inc waits until registers are free: launch only when the
+    // registers warpgroup 0 gives back cover what the softmax warpgroups take
+    // (entry count rounded up to the allocation unit of 8 per thread)
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, fn)) != cudaSuccess) return e;
+    const int entry = (fa.numRegs + 7) & ~7;
+    if (entry < kRegsLow || entry > kRegsHigh ||
+        (entry - kRegsLow) * 128 < (kRegsHigh - entry) * 256)
+      return cudaErrorInvalidConfiguration;
+  }
   const int grid = prm.num_units < num_sms() ? prm.num_units : num_sms();
   fn<<<grid > 0 ? grid : 1, kThreads, kSmemBytes, s>>>(mq, mk, mv, mkp, mvp, mkt, mvt, prm);
   return cudaGetLastError();
@@ -940,9 +1171,13 @@ cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, co
   return launch_tc<false, false>(mq, mk, mv, mk, mv, mkt, mvt, prm, s);   // no patch maps in dense mode
 }
 
+int64_t window_ws_bytes(const PlanLayout& L, int H, int D) {
+  return kWsHeaderBytes + L.B * H * L.n_ov * D * 4;
+}
+
 cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, const void* kt,
                                   const void* vt, int T, const int* cand, int R,
-                                  const PlanLayout& L, const void* plan, void* o, float* ws,
+                                  const PlanLayout& L, const void* plan, void* o, void* ws,
                                   int H, float scale, cudaStream_t s) {
   CUtensorMap mq, mk, mv, mkt, mvt;
   cudaError_t e;
@@ -968,8 +1203,13 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, c
   prm.cand = cand;
   prm.R = R;
   prm.num_units = (int)(L.nitem_max * L.B * H);
-  prm.ws = ws;
   prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.counters = static_cast<unsigned*>(ws);
+  prm.acc = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeaderBytes);
+  prm.nx2 = (int)L.nx2;
+  prm.n_ov = L.n_ov;
+  // unit counter and class completion counters start at zero
+  if ((e = cudaMemsetAsync(ws, 0, kWsHeaderBytes, s)) != cudaSuccess) return e;
   if (cand) return launch_tc<true, true>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
   return launch_tc<true, false>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
 }

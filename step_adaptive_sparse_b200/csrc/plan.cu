@@ -57,12 +57,15 @@ int plan_layout(const area_plan_cfg* cfg, PlanLayout* L) {
   L->nw = 4 * L->nb_cap;
   L->nitem_max = L->nb_cap * ((L->hy * L->wx + kQTile - 1) / kQTile + 3);
   L->ntile_sort = (N + kSortTile - 1) / kSortTile;
+  L->ny2 = axis_twice_total((int)L->nby, (int)L->Hg, (int)L->hy, (int)L->sy);
+  L->nx2 = axis_twice_total((int)L->nbx, (int)L->Wg, (int)L->wx, (int)L->sx);
+  L->n_ov = L->ny2 * L->Wg + (L->Hg - L->ny2) * L->nx2;
   const int64_t B = L->B;
   const int64_t sizes[AREA_PLAN_NSEC] = {
       B * L->nb_cap * 16, B * L->nb_cap * 4, B * L->nb_cap, B * 4,
       B * L->nw * 16, B * L->nw * 4, B * L->nw * 16, B * L->nw * 4,
       B * L->nw * L->G * 4, B * N * 4, B * N * 4, (B + 1) * 4,
-      B * L->nitem_max * 8, B * N * 4, 0};
+      B * L->nitem_max * 8, B * N * 4, (B + 1) * 16, 0};
   int64_t off = 256;  // header
   for (int s = 0; s < AREA_PLAN_NSEC; ++s) {
     L->off[s] = off;
@@ -101,6 +104,7 @@ PlanView plan_view(const PlanLayout& L, void* plan) {
   v.order = reinterpret_cast<int*>(p + L.off[AREA_PLAN_SEC_ORDER]);
   v.nitem = reinterpret_cast<int*>(p + L.off[AREA_PLAN_SEC_NITEM]);
   v.items = reinterpret_cast<int2*>(p + L.off[AREA_PLAN_SEC_ITEMS]);
+  v.nclass = reinterpret_cast<int*>(p + L.off[AREA_PLAN_SEC_NCLASS]);
   return v;
 }
 
@@ -154,9 +158,13 @@ __device__ int block_exclusive_scan(int x, int* total) {
   return res;
 }
 
-__device__ void stage_header(int64_t* hdr, const HeaderArgs& a, int* nitem_total) {
+// Header; zeroes the totals that stage_windows accumulates (the work-item
+// total and the per-class totals, row B of NCLASS).
+__device__ void stage_header(int64_t* hdr, const HeaderArgs& a, int* nitem_total,
+                             int* nclass_total) {
   if (threadIdx.x < 32) hdr[threadIdx.x] = a.v[threadIdx.x];
   if (threadIdx.x == 0) *nitem_total = 0;
+  if (threadIdx.x < 4) nclass_total[threadIdx.x] = 0;
 }
 
 // Split score of base window `item` = b * nb_cap + bi.
@@ -244,21 +252,30 @@ __device__ void stage_windows(const PlanView& P, int b) {
   const int nwin = running;
   if (threadIdx.x == 0) P.nwin[b] = nwin;
   __syncthreads();
-  // Work items: windows whose parent kept its size first (largest KV sets),
-  // then the quadrants; within each class in window order.
+  // Work items, grouped by the parity class of the base window (windows of
+  // one class never overlap, so the merge can run class after class); within
+  // a class, windows whose parent kept its size first (largest KV sets), then
+  // the quadrants, each in window order.
   int2* items = P.items + (int64_t)b * P.nitem_max;
   running = 0;
-  for (int cls = 0; cls < 2; ++cls) {
-    for (int c0 = 0; c0 < nwin; c0 += blockDim.x) {
-      const int wi = c0 + threadIdx.x;
-      int nq = 0;
-      if (wi < nwin && (int)split[parent[wi]] == cls) {
-        const int4 w = win[wi];
-        nq = (w.z * w.w + kQTile - 1) / kQTile;
+  for (int pc = 0; pc < 4; ++pc) {
+    const int start = running;
+    for (int sc = 0; sc < 2; ++sc) {
+      for (int c0 = 0; c0 < nwin; c0 += blockDim.x) {
+        const int wi = c0 + threadIdx.x;
+        int nq = 0;
+        if (wi < nwin && (int)split[parent[wi]] == sc && window_class(parent[wi], P.nbx) == pc) {
+          const int4 w = win[wi];
+          nq = (w.z * w.w + kQTile - 1) / kQTile;
+        }
+        const int at = running + block_exclusive_scan(nq, &total);
+        for (int t = 0; t < nq; ++t) items[at + t] = make_int2(wi, t);
+        running += total;
       }
-      const int at = running + block_exclusive_scan(nq, &total);
-      for (int t = 0; t < nq; ++t) items[at + t] = make_int2(wi, t);
-      running += total;
+    }
+    if (threadIdx.x == 0) {
+      P.nclass[b * 4 + pc] = running - start;
+      atomicAdd(P.nclass + P.B * 4 + pc, running - start);
     }
   }
   if (threadIdx.x == 0) {
@@ -440,8 +457,9 @@ __device__ void stage_wsum(const PlanView& P, int64_t g0) {
 // ---------------------------------------------------------------------------
 // One launch per stage
 // ---------------------------------------------------------------------------
-__global__ void plan_header_kernel(int64_t* hdr, HeaderArgs a, int* nitem_total) {
-  stage_header(hdr, a, nitem_total);
+__global__ void plan_header_kernel(int64_t* hdr, HeaderArgs a, int* nitem_total,
+                                   int* nclass_total) {
+  stage_header(hdr, a, nitem_total, nclass_total);
 }
 
 __global__ void __launch_bounds__(256) plan_base_kernel(const float* __restrict__ E, PlanView P,
@@ -566,7 +584,7 @@ __global__ void __launch_bounds__(kFusedThreads, 2) plan_fused_kernel(PlanView P
   // header, split scores, sort keys of element 0
   {
     const int nbase = P.B * P.nb_cap, ninit = (n + blockDim.x - 1) / blockDim.x;
-    if (blockIdx.x == 0) stage_header(A.hdr, h, P.nitem + P.B);
+    if (blockIdx.x == 0) stage_header(A.hdr, h, P.nitem + P.B, P.nclass + P.B * 4);
     for (int it = blockIdx.x; it < nbase + ninit; it += G) {
       if (it < nbase) stage_base(A.energy, P, A.thr, it, s_rows);
       else stage_sort_init(A.energy, 0, P, A.ka, A.va, (it - nbase) * blockDim.x);
@@ -631,7 +649,8 @@ cudaError_t launch_window_plan(const float* energy, const area_plan_cfg* cfg,
   PlanView P = plan_view(L, plan);
   char* base = static_cast<char*>(plan);
   const HeaderArgs h = header_args(L);
-  plan_header_kernel<<<1, 32, 0, s>>>(reinterpret_cast<int64_t*>(base), h, P.nitem + L.B);
+  plan_header_kernel<<<1, 32, 0, s>>>(reinterpret_cast<int64_t*>(base), h, P.nitem + L.B,
+                                      P.nclass + L.B * 4);
   const int smem = (int)(L.hy * sizeof(float));
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(plan_base_kernel,

@@ -105,7 +105,8 @@ def test_plan_config_validation_and_sizes(area):
     assert area.area_window_plan_bytes(area.make_cfg(1, 256, 256, 64, 4, 1024, 0.4)) > n
     assert area.area_window_plan_bytes(area.make_cfg(1, 256, 256, 32, 4, 512, 0.4)) > n
     assert area.area_window_plan_bytes(area.make_cfg(2, 256, 256, 64, 4, 512, 0.4)) > n
-    assert area.area_window_attn_ws_bytes(good, 24, 128) == 24 * 65536 * 128 * 4
+    # 64-token windows tile 256 exactly: no overlap, only the counter header
+    assert area.area_window_attn_ws_bytes(good, 24, 128) == 256
     for bad in [area.make_cfg(0, 256, 256, 64, 4, 512, 0.4),
                 area.make_cfg(1, 255, 256, 64, 4, 512, 0.4),
                 area.make_cfg(1, 256, 256, 0, 4, 512, 0.4),
@@ -213,8 +214,32 @@ def test_noalloc_rejects_bad_input_with_the_status_of_area_window_attn(area):
                                           a["o"], a["H"], a["D"], 1.0, a["dtype"])
         assert e1.value.status == e2.value.status, c
     # beyond the static workspace: refused before any launch
-    big = area.make_cfg(1, 256, 256, 64, 4, 16, 0.1)
+    big = area.make_cfg(1, 256, 256, 80, 4, 16, 0.1)
     with pytest.raises(area.AreaError) as e:
         area.area_window_attn_noalloc(fake, fake, fake, big, fake, area.area_window_plan_bytes(big),
                                       fake, 24, 128, 1.0, 1)
     assert e.value.status == area.AREA_ENOSPACE
+
+
+def test_window_ws_bytes_count_the_overlapped_tokens(area):
+    # Workspace = 256-byte counter header + one fp32 row of D per (element,
+    # head, token covered by more than one base window).  The overlapped
+    # tokens are counted here by brute force over the oracle's base tiling
+    # (with the border shift the seed draws).
+    from oracle import area_oracle as ora
+    import numpy as np
+    for (B, Hg, Wg, w, seed) in [(1, 256, 256, 80, 0), (2, 384, 128, 96, 0), (1, 32, 32, 10, 0),
+                                 (1, 384, 384, 168, 0), (1, 384, 384, 192, 0), (1, 40, 28, 12, 777),
+                                 (3, 64, 48, 24, 5), (1, 20, 12, 6, 2 ** 40 + 3)]:
+        sy, sx = ora.jitter_shifts(seed, Hg, Wg, w)
+        cy = np.zeros(Hg, dtype=int)
+        cx = np.zeros(Wg, dtype=int)
+        for a, n in ora.tile_windows(Hg, w, sy):
+            cy[a:a + n] += 1
+        for a, n in ora.tile_windows(Wg, w, sx):
+            cx[a:a + n] += 1
+        assert cy.max() <= 2 and cx.max() <= 2       # only neighbours overlap
+        n_ov = int(((cy[:, None] * cx[None, :]) > 1).sum())
+        for H, D in [(1, 64), (24, 128)]:
+            cfg = area.make_cfg(B, Hg, Wg, w, 4, 16, 0.1, seed)
+            assert area.area_window_attn_ws_bytes(cfg, H, D) == 256 + B * H * n_ov * D * 4

@@ -63,8 +63,23 @@ def _check_items(got, want, b=0):
         for t in range(-(-(hy * wx) // 256)):
             expect.add((i, t))
     assert len(items) == len(expect) and set(map(tuple, items.tolist())) == expect
-    kept = want.split[want.parent[items[:, 0]]] == 0
-    assert not np.any(np.diff(kept.astype(int)) > 0), "unsplit windows must come first"
+    # grouped by the parity class of the base window (row and column index of
+    # the base tiling); within a class unsplit windows first
+    nbx = int(np.sum(want.base[:, 0] == want.base[0, 0]))
+    parent = want.parent[items[:, 0]]
+    cls = ((parent // nbx) % 2) * 2 + (parent % nbx) % 2
+    split = want.split[parent].astype(int)
+    key = cls * 2 + split
+    assert not np.any(np.diff(key) < 0), "items must run class by class, unsplit first"
+    for c in range(4):
+        assert int(got["nclass"][b, c]) == int(np.sum(cls == c))
+    # windows of one class never overlap
+    for c in range(4):
+        cover = np.zeros((want.Hg, want.Wg), dtype=np.int32)
+        for i in sorted(set(items[cls == c, 0].tolist())):
+            y0, x0, hy, wx = want.windows[i]
+            cover[y0:y0 + hy, x0:x0 + wx] += 1
+        assert cover.max() <= 1
 
 
 @pytest.mark.parametrize("name,step", [(n, s) for n in ALL for s in _steps(n)])

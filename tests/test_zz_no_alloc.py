@@ -51,8 +51,8 @@ def _close(a, b, dtype):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("Hg,Wg,H,D,w,h,G,dtype", [
-    (32, 32, 2, 64, 8, 1, 16, area.AREA_DTYPE_F32),      # CUDA-core path
-    (64, 64, 4, 128, 24, 4, 70, area.AREA_DTYPE_BF16),   # tensor-core path
+    (32, 32, 2, 64, 10, 1, 16, area.AREA_DTYPE_F32),     # CUDA-core path, overlapping windows
+    (64, 64, 4, 128, 24, 4, 70, area.AREA_DTYPE_BF16),   # tensor-core path, overlapping windows
 ])
 def test_noalloc_matches_window_attn_on_two_calls(Hg, Wg, H, D, w, h, G, dtype):
     scale = 1.0 / np.sqrt(D)
@@ -67,9 +67,12 @@ def test_noalloc_matches_window_attn_on_two_calls(Hg, Wg, H, D, w, h, G, dtype):
 
 
 def test_noalloc_refuses_sizes_beyond_the_static_workspace():
-    # 24 heads of a 128x128 grid at D = 128 need 192 MiB > 32 MiB: refused on
-    # the host, before any device work (the pointers are never touched).
-    cfg = area.make_cfg(1, 128, 128, 64, 4, 256, 0.4)
+    # 48-token windows on a 128x128 grid overlap on 3840 tokens; 24 heads at
+    # D = 128 need 3840 * 24 * 128 * 4 bytes = 45 MiB of accumulator rows,
+    # more than the 32 MiB array: refused on the host, before any device work
+    # (the pointers are never touched).
+    cfg = area.make_cfg(1, 128, 128, 48, 4, 256, 0.4)
+    assert area.area_window_attn_ws_bytes(cfg, 24, 128) > 32 << 20
     nbytes = area.area_window_plan_bytes(cfg)
     fake = 1 << 20
     with pytest.raises(area.AreaError) as e:
