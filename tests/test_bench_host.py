@@ -183,11 +183,16 @@ def test_clock_summary_without_nvidia_smi():
                             "reasons": ["nvidia-smi unavailable"]}
 
 
-def test_traffic_is_null_for_another_kernel_revision(monkeypatch):
+def test_traffic_is_null_for_another_kernel_revision(monkeypatch, tmp_path):
     # roofline.traffic comes from the committed DRAM capture only while it was
     # taken from the same build of the kernel
-    got = bench.load_traffic("flux6144", "window_attn")
-    assert got is not None and got > 0
+    import json
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"flux6144": {"window_attn": {"kernel_revision": bench.KERNEL_REVISION,
+                                      "bytes_per_call": 123.0}}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.load_traffic("flux6144", "window_attn") == 123.0
     monkeypatch.setattr(bench, "KERNEL_REVISION", "some later build")
     assert bench.load_traffic("flux6144", "window_attn") is None
     assert bench.load_traffic("no-such-workload", "window_attn") is None
