@@ -288,8 +288,15 @@ int area_dwt_window_plan(const void* src, int src_dtype, int C, int mode,
                          size_t plan_bytes, cudaStream_t stream);
 
 /*
- * area_window_attn_ws_bytes -- fp32 merge workspace for area_window_attn:
- * B*H*Hg*Wg*D*4 bytes (host only).
+ * area_window_attn_ws_bytes -- workspace for area_window_attn (host only):
+ * 256 bytes of counters, then one fp32 row of D values per (batch element,
+ * head, token covered by more than one base window):
+ *   256 + B * H * n_ov * D * 4 bytes,
+ * n_ov = ny2 * Wg + (Hg - ny2) * nx2, where ny2 (nx2) counts the rows
+ * (columns) of the grid that two base windows share along that axis under
+ * the plan's border shift.  Windows that tile an axis exactly share nothing
+ * (e.g. 64-token windows on a 384-token axis), and then the workspace is the
+ * 256-byte header alone.
  */
 int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D,
                               size_t* ws_bytes);
@@ -301,8 +308,13 @@ int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D,
  * then O(q) = sum_W t_W(q) O_W(q) / sum_W t_W(q).
  *   q, k, v, o : [B, H, Hg*Wg, D] (dtype)
  *   cfg, plan  : the configuration and buffer given to area_window_plan
- *   ws         : fp32 workspace of ws_bytes >= area_window_attn_ws_bytes();
- *                contents on entry are ignored, on exit unspecified.
+ *   ws         : workspace of ws_bytes >= area_window_attn_ws_bytes(),
+ *                16-byte aligned; contents on entry are ignored, on exit
+ *                unspecified.  The call resets its 256-byte header (a memset
+ *                on the stream) before the kernel.
+ * Merge order: a token covered by several windows is summed over them in a
+ * fixed order (by the parity class of the base window, see the plan's ITEMS),
+ * so the output is bit-identical from run to run and in CUDA-graph replays.
  * Errors: AREA_EINVAL, AREA_EUNSUPPORTED (D, dtype), AREA_ENOSPACE.
  */
 int area_window_attn(const void* q, const void* k, const void* v,
@@ -397,7 +409,8 @@ int area_window_attn_bridge(const void* q, const void* k, const void* v,
  *          current; make that first call outside any stream capture.  It
  *          allocates nothing and calls no cudaMalloc / cudaFree.
  *   Sharing: all calls on a device use the same array.  It keeps the last
- *          call's contents; each call clears it before use.  Calls that
+ *          call's contents; each call resets the counters at its start, and
+ *          every accumulator row is written before it is read.  Calls that
  *          overlap on the GPU (other streams, other threads) race on it and
  *          must be serialised by the caller.
  * Errors: AREA_EINVAL, AREA_EUNSUPPORTED, AREA_ENOSPACE, AREA_ECUDA.

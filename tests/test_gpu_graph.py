@@ -87,7 +87,8 @@ def test_one_launch_planner_in_a_graph(name):
     for w in cfg.schedule:
         pc = area.make_cfg(cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
         nb = area.area_window_plan_bytes(pc)
-        plans.append((pc, torch.empty(nb, dtype=torch.uint8, device="cuda"), nb))
+        # zero-filled: the 256-byte padding after each section is never written
+        plans.append((pc, torch.zeros(nb, dtype=torch.uint8, device="cuda"), nb))
     stream = torch.cuda.Stream()
 
     def run():
