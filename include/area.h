@@ -27,8 +27,13 @@
  *     CUDA-core arithmetic, D = 64 or 128).
  *   - Every kernel call is asynchronous on the given stream (0 = legacy
  *     default stream) and never synchronises the host.  No CTA waits on
- *     another, except in area_dwt_window_plan: a cooperative launch (every
- *     CTA resident) whose grid barriers are bounded waits.  The return value
+ *     another, except in two calls, always with bounded waits:
+ *     area_dwt_window_plan, a cooperative launch (every CTA resident) with
+ *     grid barriers; and the window-attention calls on the tensor cores,
+ *     where a CTA about to add a later parity class of windows into an
+ *     overlapped token's accumulator row waits until every unit of the
+ *     earlier classes has completed (units are claimed in class order by
+ *     running CTAs, so every unit waited on is held by a running CTA).  The return value
  *     reports argument validation and launch errors only; AREA_ECUDA carries
  *     the CUDA error, see area_status_string.  The schedule functions at the
  *     end are host arithmetic (no device memory, no stream).
@@ -106,8 +111,8 @@ int area_pool_kv(const void* k, const void* v, void* kp, void* vp,
  * area_coarse_attn -- Phase I cross-scale coarse attention ([ai] Phase I):
  *   O = softmax(scale * Q Kp^T) Vp   per (b, h), text tokens absent.
  *   q  : [B, H, N, D]; kp, vp : [B, H, Nk, D]; o : [B, H, N, D] (dtype).
- * bf16 with D = 128 runs on the tcgen05 tensor-core kernel; every other
- * supported combination on the CUDA-core kernel.
+ * bf16 (D = 64 or 128) runs on the tcgen05 tensor-core kernel, fp32 on the
+ * CUDA-core kernel.
  * Errors: AREA_EINVAL (null, N < 1, Nk < 1), AREA_EUNSUPPORTED (D not 64/128,
  * unknown dtype).
  */
@@ -438,6 +443,17 @@ int area_test_plan_barrier_expiry(const void* src, int src_dtype, int C,
                                   float* energy, const area_plan_cfg* cfg,
                                   void* plan, size_t plan_bytes,
                                   cudaStream_t stream);
+
+/*
+ * area_test_exp2_poly -- TEST HOOK, not part of the method (the pages have no
+ * counterpart).  y[i] = 2^x[i] by the polynomial exponent the attention
+ * softmax uses for part of its keys: Cody-Waite range reduction to
+ * f in [-0.5, 0.5] and a cubic fitted in this project by the Remez exchange
+ * (relative error below 7.5e-5 for -126 <= x <= 0; arguments below -126
+ * give 2^-126).  x, y: device fp32 arrays of n elements.
+ * Errors: AREA_EINVAL, AREA_ECUDA.
+ */
+int area_test_exp2_poly(const float* x, float* y, long long n, cudaStream_t stream);
 
 /* ---- schedule (host functions: no device memory, no stream) ------------ */
 

@@ -44,8 +44,8 @@ int dense_attn(const void* q, const void* k, const void* v, const void* kt, cons
   if (st != AREA_OK) return st;
   if (B > 65535 || H > 65535) return AREA_EINVAL;
   if (T < 0 || (T > 0 && (!kt || !vt || !aligned16(kt) || !aligned16(vt)))) return AREA_EINVAL;
-  if (dtype == AREA_DTYPE_BF16 && D == 128)
-    return finish(area::launch_dense_attn_tc(q, k, v, kt, vt, o, B, H, N, Nk, T, scale, s));
+  if (dtype == AREA_DTYPE_BF16)       // tensor cores, head_dim 64 or 128
+    return finish(area::launch_dense_attn_tc(q, k, v, kt, vt, o, B, H, N, Nk, T, D, scale, s));
   return finish(
       area::launch_dense_attn_simt(q, k, v, kt, vt, o, B, H, N, Nk, T, D, scale, dtype, s));
 }
@@ -66,8 +66,8 @@ int window_attn(const void* q, const void* k, const void* v, const void* kt, con
   if (ws_bytes < (size_t)area::window_ws_bytes(L, H, D)) return AREA_ENOSPACE;
   if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(plan) & 255) != 0) return AREA_EINVAL;
   if (H > 65535 || L.B > 65535) return AREA_EINVAL;
-  if (dtype == AREA_DTYPE_BF16 && D == 128)
-    return finish(area::launch_window_attn_tc(q, k, v, kt, vt, T, cand, R, L, plan, o, ws, H,
+  if (dtype == AREA_DTYPE_BF16)       // tensor cores, head_dim 64 or 128
+    return finish(area::launch_window_attn_tc(q, k, v, kt, vt, T, cand, R, L, plan, o, ws, H, D,
                                               scale, stream));
   return finish(area::launch_window_attn_simt(q, k, v, kt, vt, T, cand, R, L, plan, o, ws, H, D,
                                               scale, dtype, stream));
@@ -188,6 +188,12 @@ int area_test_plan_barrier_expiry(const void* src, int src_dtype, int C, float* 
   // and each wait gives up after 1 ms
   return finish(area::launch_dwt_window_plan(src, src_dtype, C, AREA_DETAIL_HH, energy, cfg, L,
                                              plan, stream, 1u, 1000000ull));
+}
+
+int area_test_exp2_poly(const float* x, float* y, long long n, cudaStream_t stream) {
+  if (!x || !y || n < 0 || n > (1ll << 40)) return AREA_EINVAL;
+  if (n == 0) return AREA_OK;
+  return finish(area::launch_exp2_poly(x, y, (int64_t)n, stream));
 }
 
 int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D, size_t* ws_bytes) {

@@ -203,7 +203,7 @@ cudaError_t launch_dwt_detail(const void* src, int src_dtype, int C, float* ener
 cudaError_t launch_window_plan(const float* energy, const area_plan_cfg* cfg,
                                const PlanLayout& L, void* plan, cudaStream_t s);
 
-// CUDA-core attention (fp32 any supported D; bf16 fallback for D = 64).
+// CUDA-core attention (fp32, D = 64 or 128).
 cudaError_t launch_dense_attn_simt(const void* q, const void* k, const void* v, const void* kt,
                                    const void* vt, void* o, int B, int H, int N, int Nk, int T,
                                    int D, float scale, int dtype, cudaStream_t s);
@@ -215,19 +215,21 @@ cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v,
                                     const PlanLayout& L, const void* plan, void* o, void* ws,
                                     int H, int D, float scale, int dtype, cudaStream_t s);
 
-// tcgen05 tensor-core attention (bf16, D = 128).  kt, vt: [B, H, T, 128] text
-// keys appended after the image keys of every query (T = 0: none).
+// tcgen05 tensor-core attention (bf16, D = 64 or 128).  kt, vt: [B, H, T, D]
+// text keys appended after the image keys of every query (T = 0: none).
 cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, const void* kt,
                                  const void* vt, void* o, int B, int H, int N, int Nk, int T,
-                                 float scale, cudaStream_t s);
+                                 int D, float scale, cudaStream_t s);
 cudaError_t read_and_clear_tc_error(int* code);
+// The softmax's polynomial 2^x (exp2_poly2) over an array, for its accuracy test.
+cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s);
 // cand (may be null): per-head bridge candidates [B*H][R]; when given they
 // replace the plan's global-KV lists, candidates inside a window's Halo
 // rectangle are skipped.
 cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, const void* kt,
                                   const void* vt, int T, const int* cand, int R,
                                   const PlanLayout& L, const void* plan, void* o, void* ws,
-                                  int H, float scale, cudaStream_t s);
+                                  int H, int D, float scale, cudaStream_t s);
 // Bytes of the window workspace for H heads of head_dim D.
 int64_t window_ws_bytes(const PlanLayout& L, int H, int D);
 // Detail map and planner in one cooperative launch (one memset of the

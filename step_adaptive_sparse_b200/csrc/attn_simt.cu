@@ -1,5 +1,6 @@
-// CUDA-core attention: the fp32 path (tiny configuration, tolerance 1e-4) and
-// the bf16 path for head_dim 64.  Same semantics as the tensor-core kernels:
+// CUDA-core attention: the fp32 path (the tiny configuration, tolerance 1e-4;
+// bf16 runs on the tensor-core kernel).  Same semantics as the tensor-core
+// kernels:
 //   dense  : O = softmax(scale * Q K^T) V over all Nk keys (coarse and full
 //            attention, AReA Phase I / the speedup denominator);
 //   window : per plan work item (window W, 256-query block), keys S = Halo
@@ -229,8 +230,7 @@ cudaError_t launch_dense_attn_simt(const void* q, const void* k, const void* v, 
     if (D == 64) return launch_simt<float, 64, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, MergeArgs{}, H, dr, P, scale, s);
     return launch_simt<float, 128, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, MergeArgs{}, H, dr, P, scale, s);
   }
-  if (D == 64) return launch_simt<__nv_bfloat16, 64, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, MergeArgs{}, H, dr, P, scale, s);
-  return launch_simt<__nv_bfloat16, 128, false>(grid, q, k, v, kt, vt, T, nullptr, 0, o, MergeArgs{}, H, dr, P, scale, s);
+  return cudaErrorNotSupported;           // bf16 runs on the tensor-core kernel
 }
 
 cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v, const void* kt,
@@ -246,8 +246,7 @@ cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v,
     if (D == 64) return launch_simt<float, 64, true>(grid, q, k, v, kt, vt, T, cand, R, o, ma, H, dr, P, scale, s);
     return launch_simt<float, 128, true>(grid, q, k, v, kt, vt, T, cand, R, o, ma, H, dr, P, scale, s);
   }
-  if (D == 64) return launch_simt<__nv_bfloat16, 64, true>(grid, q, k, v, kt, vt, T, cand, R, o, ma, H, dr, P, scale, s);
-  return launch_simt<__nv_bfloat16, 128, true>(grid, q, k, v, kt, vt, T, cand, R, o, ma, H, dr, P, scale, s);
+  return cudaErrorNotSupported;           // bf16 runs on the tensor-core kernel
 }
 
 }  // namespace area

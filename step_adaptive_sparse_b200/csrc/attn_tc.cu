@@ -73,8 +73,7 @@ constexpr int kRegsLow = 56, kRegsHigh = 208;
 constexpr int kPolyPer8 = AREA_EXP2_POLY_PER8;
 static_assert(kPolyPer8 >= 0 && kPolyPer8 <= 8, "polynomial share");
 constexpr int kStages = 4;              // K/V ring stages of 32 KB
-constexpr int kTileBytes = 128 * 128 * 2;
-constexpr int kHalfBytes = 128 * 128;   // 128 rows x 64 bf16
+constexpr int kHalfBytes = 128 * 128;   // 128 rows x 64 bf16: one 128B-swizzled half tile
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr int kMaxChains = 8;                // independent partial maxima of a score row
@@ -85,11 +84,20 @@ constexpr int kPParts = 2;                   // P handed to the PV product in th
 constexpr int kPW = 16, kPH = 8;
 constexpr int kRecSlots = 3;                 // unit records in flight (shared-memory ring)
 
-// Shared-memory plan (offsets from a 1024-aligned base).
-constexpr int kSmemQ = 0;                              // 2 tiles x 32 KB
-constexpr int kSmemKV = 2 * kTileBytes;                // kStages x 32 KB
-constexpr int kSmemBar = kSmemKV + kStages * kTileBytes;
-constexpr int kSmemBytes = kSmemBar + 256 + 1024;      // barriers + alignment slack
+// Tile geometry for head_dim D (64 or 128): a tile is 128 rows of D bf16,
+// stored as D / 64 halves of 64 columns, each the canonical K-major SW128
+// layout of UMMA.  Shared-memory plan (offsets from a 1024-aligned base): the
+// two Q tiles, the K/V ring, then the barriers.
+template <int D>
+struct Geo {
+  static_assert(D == 64 || D == 128, "head_dim");
+  static constexpr int kHalves = D / 64;
+  static constexpr int kTileBytes = kHalves * kHalfBytes;
+  static constexpr int kSmemQ = 0;
+  static constexpr int kSmemKV = 2 * kTileBytes;
+  static constexpr int kSmemBar = kSmemKV + kStages * kTileBytes;
+  static constexpr int kSmemBytes = kSmemBar + 256 + 1024;   // barriers + alignment slack
+};
 
 // barrier indices
 enum {
@@ -218,10 +226,13 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
   return d;
 }
 
-// Instruction descriptor: fp32 accumulate, bf16 A and B, M = N = 128.
-constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) |
-                              ((128u >> 4) << 24);
-constexpr uint32_t kIdescPV = kIdescQK | (1u << 16);   // B (V) is MN-major
+// Instruction descriptors: fp32 accumulate, bf16 A and B, M = 128.  QK^T has
+// N = 128 keys; PV has N = D with B (V) MN-major.
+__host__ __device__ constexpr uint32_t idesc(uint32_t n, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major ? (1u << 16) : 0u) | ((n >> 3) << 17) |
+         ((128u >> 4) << 24);
+}
+constexpr uint32_t kIdescQK = idesc(128, false);
 
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                        uint32_t accum) {
@@ -486,17 +497,19 @@ __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
 #define AREA_TC_BOUNDS __launch_bounds__(kThreads, 1)
 #endif
 
-template <bool WINDOW, bool BRIDGE>
+template <bool WINDOW, bool BRIDGE, int D>
 __global__ void AREA_TC_BOUNDS
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
                const __grid_constant__ CUtensorMap tm_vp, const __grid_constant__ CUtensorMap tm_kt,
                const __grid_constant__ CUtensorMap tm_vt, const TcParams prm) {
+  using G = Geo<D>;
+  constexpr uint32_t kIdescPV = idesc(D, true);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar0 = sbase + kSmemBar;
+  const uint32_t bar0 = sbase + G::kSmemBar;
   __shared__ uint32_t s_tmem_base;
   __shared__ int s_abort;
   __shared__ __align__(16) UnitRec s_rec[kRecSlots];
@@ -586,13 +599,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const UnitRec& R = s_rec[unit_count % kRecSlots];
       if (!R.valid) break;
       if (!warp_wait0(bar(BAR_Q_EMPTY), (unit_count & 1u) ^ 1u, abort_flag)) break;
-      if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL), 2 * kTileBytes);
+      if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL), 2 * G::kTileBytes);
       __syncwarp();
       if constexpr (!WINDOW) {
         if (lane == 0) {
           for (int t = 0; t < 2; ++t)
-            for (int hf = 0; hf < 2; ++hf)
-              tma_load_2d(sbase + kSmemQ + t * kTileBytes + hf * kHalfBytes, &tm_q,
+            for (int hf = 0; hf < G::kHalves; ++hf)
+              tma_load_2d(sbase + G::kSmemQ + t * G::kTileBytes + hf * kHalfBytes, &tm_q,
                           bar(BAR_Q_FULL), hf * 64, R.bh * Ntok + R.q0 + t * 128);
         }
       } else {
@@ -601,8 +614,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             r[i] = R.bh * Ntok + window_query_token(R.win, R.nq, R.q0 + t * 128 + lane * 4 + i, Wg);
-          for (int hf = 0; hf < 2; ++hf)
-            tma_gather4(sbase + kSmemQ + t * kTileBytes + hf * kHalfBytes + lane * 512, &tm_q,
+          for (int hf = 0; hf < G::kHalves; ++hf)
+            tma_gather4(sbase + G::kSmemQ + t * G::kTileBytes + hf * kHalfBytes + lane * 512, &tm_q,
                         bar(BAR_Q_FULL), hf * 64, r[0], r[1], r[2], r[3]);
         }
       }
@@ -624,21 +637,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ok = false;
             break;
           }
-          if (lane == 0) mbar_arrive_tx(bar(BAR_KV_FULL + s), kTileBytes);
+          if (lane == 0) mbar_arrive_tx(bar(BAR_KV_FULL + s), G::kTileBytes);
           __syncwarp();
           const CUtensorMap* tm = kv ? &tm_v : &tm_k;
-          const uint32_t dst = sbase + kSmemKV + s * kTileBytes;
+          const uint32_t dst = sbase + G::kSmemKV + s * G::kTileBytes;
           if (j >= nti) {
             // text keys: rows of the [B*H*T, 128] text tensors
             if (lane == 0) {
               const CUtensorMap* tt = kv ? &tm_vt : &tm_kt;
-              for (int hf = 0; hf < 2; ++hf)
+              for (int hf = 0; hf < G::kHalves; ++hf)
                 tma_load_2d(dst + hf * kHalfBytes, tt, bar(BAR_KV_FULL + s), hf * 64,
                             bh * prm.T + (j - nti) * 128);
             }
           } else if (!WINDOW) {
             if (lane == 0)
-              for (int hf = 0; hf < 2; ++hf)
+              for (int hf = 0; hf < G::kHalves; ++hf)
                 tma_load_2d(dst + hf * kHalfBytes, tm, bar(BAR_KV_FULL + s), hf * 64,
                             bh * Nkrows + j * 128);
           } else if (j < ngt) {
@@ -650,7 +663,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               const int p = g0 + i < nkv ? g0 + i : nkv - 1;
               r[i] = bh * Nkrows + glist[p];
             }
-            for (int hf = 0; hf < 2; ++hf)
+            for (int hf = 0; hf < G::kHalves; ++hf)
               tma_gather4(dst + hf * kHalfBytes + lane * 512, tm, bar(BAR_KV_FULL + s), hf * 64,
                           r[0], r[1], r[2], r[3]);
           } else {
@@ -661,7 +674,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               const int px = jj % ncx, py = jj / ncx;
               const int cx = ext.y + px * kPW;
               const int cy = bh * prm.P.Hg + ext.x + py * kPH;
-              for (int hf = 0; hf < 2; ++hf)
+              for (int hf = 0; hf < G::kHalves; ++hf)
                 tma_load_3d(dst + hf * kHalfBytes, tp, bar(BAR_KV_FULL + s), hf * 64, cx, cy);
             }
           }
@@ -684,12 +697,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       uint32_t kv_it = 0, unit_count = 0;
       uint32_t p_cnt0 = 0, p_cnt1 = 0;
       const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
-      const uint32_t q0s = sbase + kSmemQ, q1s = sbase + kSmemQ + kTileBytes;
+      const uint32_t q0s = sbase + G::kSmemQ, q1s = sbase + G::kSmemQ + G::kTileBytes;
       bool ok = true;
-      auto kv_addr = [&](uint32_t it) { return sbase + kSmemKV + (it % kStages) * kTileBytes; };
+      auto kv_addr = [&](uint32_t it) { return sbase + G::kSmemKV + (it % kStages) * G::kTileBytes; };
       auto qk = [&](uint32_t d, uint32_t qs, uint32_t ks) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
           mma_ss(d, sdesc(qs + off, 16, 1024), sdesc(ks + off, 16, 1024), kIdescQK, kk > 0);
         }
@@ -898,7 +911,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
           if (h == 0 && rescale) {
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
               uint32_t orr[32];
               tmem_ld32(tO + c * 32, orr);
 #pragma unroll
@@ -928,9 +941,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ++o_cnt;
         tc_fence_after();
         const float inv = 1.f / l;
-        __nv_bfloat16* dst = prm.o + ((int64_t)bh * Ntok + qpos) * 128;
+        __nv_bfloat16* dst = prm.o + ((int64_t)bh * Ntok + qpos) * D;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           uint32_t orr[32];
           tmem_ld32(tO + c * 32, orr);
           if (qvalid) {
@@ -999,10 +1012,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         const float sc = mr.ov ? tent * inv : inv;
         const float winv = 1.f / wsum;
-        __nv_bfloat16* dsto = prm.o + ((int64_t)bh * Ntok + tok) * 128;
-        float* acc = prm.acc + ((int64_t)bh * prm.n_ov + mr.rank) * 128;
+        __nv_bfloat16* dsto = prm.o + ((int64_t)bh * Ntok + tok) * D;
+        float* acc = prm.acc + ((int64_t)bh * prm.n_ov + mr.rank) * D;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           uint32_t orr[32];
           tmem_ld32(tO + c * 32, orr);
           if (!qvalid) continue;
@@ -1076,12 +1089,12 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// 2-D bf16 map over [rows, 128] with a box of 64 columns x box_rows rows.
-cudaError_t make_map(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
+// 2-D bf16 map over [rows, D] with a box of 64 columns x box_rows rows.
+cudaError_t make_map(CUtensorMap* m, const void* base, int64_t rows, int box_rows, int D) {
   auto enc = get_encode();
   if (!enc) return cudaErrorNotSupported;
-  cuuint64_t dims[2] = {128, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {128 * 2};
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
   cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
@@ -1090,13 +1103,13 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int64_t rows, int box_row
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// 3-D bf16 map over [rows_y, Wg, 128] (token-grid rows of all (b, h), grid
+// 3-D bf16 map over [rows_y, Wg, D] (token-grid rows of all (b, h), grid
 // columns, head dims) with a box of 64 dims x kPW tokens x kPH grid rows.
-cudaError_t make_map_patch(CUtensorMap* m, const void* base, int64_t rows_y, int Wg) {
+cudaError_t make_map_patch(CUtensorMap* m, const void* base, int64_t rows_y, int Wg, int D) {
   auto enc = get_encode();
   if (!enc) return cudaErrorNotSupported;
-  cuuint64_t dims[3] = {128, (cuuint64_t)Wg, (cuuint64_t)rows_y};
-  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)Wg * 128 * 2};
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Wg, (cuuint64_t)rows_y};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Wg * D * 2};
   cuuint32_t box[3] = {64, (cuuint32_t)kPW, (cuuint32_t)kPH};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
@@ -1112,11 +1125,12 @@ int num_sms() {
   return n;
 }
 
-template <bool WINDOW, bool BRIDGE>
+template <bool WINDOW, bool BRIDGE, int D>
 cudaError_t launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const CUtensorMap& mkp, const CUtensorMap& mvp, const CUtensorMap& mkt,
                       const CUtensorMap& mvt, const TcParams& prm, cudaStream_t s) {
-  auto fn = attn_tc_kernel<WINDOW, BRIDGE>;
+  constexpr int kSmemBytes = Geo<D>::kSmemBytes;
+  auto fn = attn_tc_kernel<WINDOW, BRIDGE, D>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   if constexpr (kWgSplit) {
@@ -1137,6 +1151,27 @@ cudaError_t launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
 
 }  // namespace
 
+namespace {
+// exp2_poly2 over an array (the accuracy test of the polynomial exponent)
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+  const int64_t i = 2 * (blockIdx.x * (int64_t)blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    exp2_poly2(y[i], y[i + 1], x[i], x[i + 1]);
+  } else if (i < n) {
+    float a, b;
+    exp2_poly2(a, b, x[i], 0.f);
+    y[i] = a;
+  }
+}
+}  // namespace
+
+cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s) {
+  const int64_t pairs = (n + 1) / 2;
+  const int64_t blocks = (pairs + 255) / 256;
+  exp2_poly_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, s>>>(x, y, n);
+  return cudaGetLastError();
+}
+
 cudaError_t read_and_clear_tc_error(int* code) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return e;
@@ -1148,15 +1183,15 @@ cudaError_t read_and_clear_tc_error(int* code) {
 
 cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, const void* kt,
                                  const void* vt, void* o, int B, int H, int N, int Nk, int T,
-                                 float scale, cudaStream_t s) {
+                                 int D, float scale, cudaStream_t s) {
   CUtensorMap mq, mk, mv, mkt, mvt;
   cudaError_t e;
-  if ((e = make_map(&mq, q, (int64_t)B * H * N, 128)) != cudaSuccess) return e;
-  if ((e = make_map(&mk, k, (int64_t)B * H * Nk, 128)) != cudaSuccess) return e;
-  if ((e = make_map(&mv, v, (int64_t)B * H * Nk, 128)) != cudaSuccess) return e;
+  if ((e = make_map(&mq, q, (int64_t)B * H * N, 128, D)) != cudaSuccess) return e;
+  if ((e = make_map(&mk, k, (int64_t)B * H * Nk, 128, D)) != cudaSuccess) return e;
+  if ((e = make_map(&mv, v, (int64_t)B * H * Nk, 128, D)) != cudaSuccess) return e;
   if (T > 0) {
-    if ((e = make_map(&mkt, kt, (int64_t)B * H * T, 128)) != cudaSuccess) return e;
-    if ((e = make_map(&mvt, vt, (int64_t)B * H * T, 128)) != cudaSuccess) return e;
+    if ((e = make_map(&mkt, kt, (int64_t)B * H * T, 128, D)) != cudaSuccess) return e;
+    if ((e = make_map(&mvt, vt, (int64_t)B * H * T, 128, D)) != cudaSuccess) return e;
   } else {
     mkt = mk;   // never read without text keys
     mvt = mv;
@@ -1168,7 +1203,9 @@ cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, co
   prm.da = DenseArgs{B, H, N, Nk, (N + 255) / 256};
   prm.num_units = B * H * prm.da.units_per_head;
   prm.o = static_cast<__nv_bfloat16*>(o);
-  return launch_tc<false, false>(mq, mk, mv, mk, mv, mkt, mvt, prm, s);   // no patch maps in dense mode
+  // no patch maps in dense mode
+  if (D == 64) return launch_tc<false, false, 64>(mq, mk, mv, mk, mv, mkt, mvt, prm, s);
+  return launch_tc<false, false, 128>(mq, mk, mv, mk, mv, mkt, mvt, prm, s);
 }
 
 int64_t window_ws_bytes(const PlanLayout& L, int H, int D) {
@@ -1178,19 +1215,19 @@ int64_t window_ws_bytes(const PlanLayout& L, int H, int D) {
 cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, const void* kt,
                                   const void* vt, int T, const int* cand, int R,
                                   const PlanLayout& L, const void* plan, void* o, void* ws,
-                                  int H, float scale, cudaStream_t s) {
+                                  int H, int D, float scale, cudaStream_t s) {
   CUtensorMap mq, mk, mv, mkt, mvt;
   cudaError_t e;
   const int64_t rows = L.B * H * L.N;
-  if ((e = make_map(&mq, q, rows, 1)) != cudaSuccess) return e;
-  if ((e = make_map(&mk, k, rows, 1)) != cudaSuccess) return e;
-  if ((e = make_map(&mv, v, rows, 1)) != cudaSuccess) return e;
+  if ((e = make_map(&mq, q, rows, 1, D)) != cudaSuccess) return e;
+  if ((e = make_map(&mk, k, rows, 1, D)) != cudaSuccess) return e;
+  if ((e = make_map(&mv, v, rows, 1, D)) != cudaSuccess) return e;
   CUtensorMap mkp, mvp;
-  if ((e = make_map_patch(&mkp, k, L.B * H * L.Hg, (int)L.Wg)) != cudaSuccess) return e;
-  if ((e = make_map_patch(&mvp, v, L.B * H * L.Hg, (int)L.Wg)) != cudaSuccess) return e;
+  if ((e = make_map_patch(&mkp, k, L.B * H * L.Hg, (int)L.Wg, D)) != cudaSuccess) return e;
+  if ((e = make_map_patch(&mvp, v, L.B * H * L.Hg, (int)L.Wg, D)) != cudaSuccess) return e;
   if (T > 0) {
-    if ((e = make_map(&mkt, kt, L.B * H * T, 128)) != cudaSuccess) return e;
-    if ((e = make_map(&mvt, vt, L.B * H * T, 128)) != cudaSuccess) return e;
+    if ((e = make_map(&mkt, kt, L.B * H * T, 128, D)) != cudaSuccess) return e;
+    if ((e = make_map(&mvt, vt, L.B * H * T, 128, D)) != cudaSuccess) return e;
   } else {
     mkt = mq;   // never read without text keys
     mvt = mq;
@@ -1210,8 +1247,12 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, c
   prm.n_ov = L.n_ov;
   // unit counter and class completion counters start at zero
   if ((e = cudaMemsetAsync(ws, 0, kWsHeaderBytes, s)) != cudaSuccess) return e;
-  if (cand) return launch_tc<true, true>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
-  return launch_tc<true, false>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
+  if (D == 64) {
+    if (cand) return launch_tc<true, true, 64>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
+    return launch_tc<true, false, 64>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
+  }
+  if (cand) return launch_tc<true, true, 128>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
+  return launch_tc<true, false, 128>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
 }
 
 }  // namespace area

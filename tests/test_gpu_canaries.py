@@ -42,6 +42,7 @@ def _rand(shape, dtype, seed):
     (1, 2, 34, 18, 9, 1, 7, 128, torch.bfloat16),    # ragged tiling, odd window side
     (2, 1, 40, 28, 12, 3, 130, 128, torch.bfloat16),  # global list over two key tiles
     (1, 2, 24, 40, 12, 2, 17, 64, torch.float32),     # CUDA-core path, head_dim 64
+    (2, 3, 26, 34, 10, 2, 21, 64, torch.bfloat16),    # tensor cores, head_dim 64, overlaps
 ])
 def test_phase2_outputs_stay_in_bounds(B, H, Hg, Wg, w, h, G, D, dt):
     N = Hg * Wg

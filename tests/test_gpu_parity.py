@@ -455,7 +455,7 @@ def test_window_attn_bridge(data):
     (1, 1, 1, 1, 128, "bf16"),          # degenerate single query / key
     (2, 3, 1000, 300, 128, "bf16"),     # ragged query and key tails
     (1, 2, 257, 4097, 128, "bf16"),     # key count one past a tile
-    (1, 2, 300, 200, 64, "bf16"),       # head_dim 64 (CUDA-core path)
+    (1, 2, 300, 200, 64, "bf16"),       # head_dim 64 on the tensor cores
     (2, 2, 333, 129, 64, "fp32"),
     (1, 2, 130, 70, 128, "fp32"),
 ])
@@ -479,7 +479,8 @@ def test_dense_attn_ragged(B, H, N, Nk, D, dtype):
     (16, 16, 7, 2, 5, 128, "bf16", 2),     # unequal quadrants, ragged query tiles
     (12, 20, 64, 0, 3, 128, "bf16", 1),    # one window = full attention
     (10, 14, 4, 1, 0, 128, "bf16", 2),     # no global KV
-    (24, 40, 12, 3, 17, 64, "bf16", 2),    # head_dim 64
+    (24, 40, 12, 3, 17, 64, "bf16", 2),    # head_dim 64 on the tensor cores
+    (26, 34, 10, 2, 130, 64, "bf16", 3),   # head_dim 64, global list over two key tiles
     (20, 12, 6, 1, 9, 128, "fp32", 2),     # fp32 head_dim 128
     (64, 48, 24, 4, 130, 128, "bf16", 3),  # global list spans two key tiles
 ])
