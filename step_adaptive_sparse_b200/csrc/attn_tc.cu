@@ -403,7 +403,7 @@ struct UnitRec {
   int ncx;            // window: patches per row of the Halo rectangle
   int nt;             // all key tiles of the unit, text tiles included
   int cls;            // window: parity class of the base window
-  int pad;
+  int one;            // 1: at most 128 valid queries, only query tile 0 runs
   int4 win, ext;      // window: the window and its Halo rectangle (y0, x0, hy, wx)
   int4 my, mx;        // window: merge geometry of the base window per axis (axis_merge)
   long long glist;    // window: element offset of the global list in the plan or cand
@@ -438,7 +438,7 @@ __device__ __forceinline__ int window_query_token(const int4& win, int nq, int p
 template <bool WINDOW>
 __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
   r.valid = 1;
-  r.pad = 0;
+  r.one = 0;
   r.cls = 0;
   r.glist = 0;
   r.ntr = r.ncx = 0;
@@ -449,6 +449,7 @@ __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
     r.b = r.bh / prm.da.H;
     r.q0 = (u % prm.da.units_per_head) * 256;
     r.nq = prm.da.N;
+    r.one = r.nq - r.q0 <= 128;
     r.nkv = prm.da.Nk;
     r.ngt = (prm.da.Nk + 127) / 128;
     r.nt = r.ngt + (prm.T + 127) / 128;
@@ -479,6 +480,7 @@ __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
       r.mx = axis_merge(parent % P.nbx, P.nbx, P.Wg, P.wx, P.sx);
       r.q0 = it.y * 256;
       r.nq = r.win.z * r.win.w;
+      r.one = r.nq - r.q0 <= 128;
       r.nkv = prm.cand ? prm.R : P.gcount[wo];
       r.ngt = (r.nkv + 127) / 128;
       r.ncx = (r.ext.w + kPW - 1) / kPW;
@@ -599,17 +601,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const UnitRec& R = s_rec[unit_count % kRecSlots];
       if (!R.valid) break;
       if (!warp_wait0(bar(BAR_Q_EMPTY), (unit_count & 1u) ^ 1u, abort_flag)) break;
-      if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL), 2 * G::kTileBytes);
+      const int nqt = R.one ? 1 : 2;          // query tiles of this unit
+      if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL), nqt * G::kTileBytes);
       __syncwarp();
       if constexpr (!WINDOW) {
         if (lane == 0) {
-          for (int t = 0; t < 2; ++t)
+          for (int t = 0; t < nqt; ++t)
             for (int hf = 0; hf < G::kHalves; ++hf)
               tma_load_2d(sbase + G::kSmemQ + t * G::kTileBytes + hf * kHalfBytes, &tm_q,
                           bar(BAR_Q_FULL), hf * 64, R.bh * Ntok + R.q0 + t * 128);
         }
       } else {
-        for (int t = 0; t < 2; ++t) {
+        for (int t = 0; t < nqt; ++t) {
           int r[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i)
@@ -732,6 +735,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (!(ok = mbar_wait(bar(BAR_REC_FULL + slot), (unit_count / kRecSlots) & 1u, abort_flag)))
           break;
         const int valid = s_rec[slot].valid, nt = s_rec[slot].nt;
+        const bool two = s_rec[slot].one == 0;   // query tile 1 runs too
         mbar_arrive(bar(BAR_REC_EMPTY + slot));
         if (!valid) break;
         if (!(ok = mbar_wait(bar(BAR_Q_FULL), unit_count & 1u, abort_flag))) break;
@@ -742,8 +746,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc_fence_after();
         qk(tS0, q0s, kv_addr(k0));
         mma_commit(bar(BAR_S_FULL0));
-        qk(tS1, q1s, kv_addr(k0));
-        mma_commit(bar(BAR_S_FULL1));
+        if (two) {
+          qk(tS1, q1s, kv_addr(k0));
+          mma_commit(bar(BAR_S_FULL1));
+        }
         mma_commit(bar(BAR_KV_EMPTY + k0 % kStages));
         if (nt == 1) mma_commit(bar(BAR_Q_EMPTY));
         for (int j = 0; j < nt && ok; ++j) {
@@ -762,13 +768,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tc_fence_after();
             qk(tS0, q0s, kv_addr(kn));
             mma_commit(bar(BAR_S_FULL0));
+            if (!two) {                          // K(j+1) is done with after QK0
+              mma_commit(bar(BAR_KV_EMPTY + kn % kStages));
+              if (j + 2 == nt) mma_commit(bar(BAR_Q_EMPTY));
+            }
           }
-          if (!(ok = pv_parts(tO1, tS1, kv_addr(vi), j == 0, BAR_P_PART1, BAR_P_FULL1, p_cnt1)))
-            break;
-          ++p_cnt1;
-          if (j == nt - 1) mma_commit(bar(BAR_O_FULL1));
+          if (two) {
+            if (!(ok = pv_parts(tO1, tS1, kv_addr(vi), j == 0, BAR_P_PART1, BAR_P_FULL1, p_cnt1)))
+              break;
+            ++p_cnt1;
+            if (j == nt - 1) mma_commit(bar(BAR_O_FULL1));
+          }
           mma_commit(bar(BAR_KV_EMPTY + vi % kStages));
-          if (j + 1 < nt) {
+          if (two && j + 1 < nt) {
             qk(tS1, q1s, kv_addr(kn));
             mma_commit(bar(BAR_S_FULL1));
             mma_commit(bar(BAR_KV_EMPTY + kn % kStages));
@@ -808,6 +820,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         break;
       const UnitRec& R = s_rec[slot];
       if (!R.valid) break;
+      if (qt == 1 && R.one) {
+        // at most 128 valid queries: query tile 1 does not run; its warps
+        // only sign the unit off (completion count and record slot)
+        if (WINDOW && lane == 0) atomicAdd(prm.counters + kWsClassDone + R.cls, 1u);
+        if (lane == 0) mbar_arrive(bar(BAR_REC_EMPTY + slot));
+        ++unit_count;
+        continue;
+      }
       const int nkv = R.nkv, nt = R.nt, ngt = R.ngt, ntr = R.ntr, ncx = R.ncx;
       const int nti = ngt + ntr;
       const int ew = R.ext.w, eh = R.ext.z;
