@@ -325,13 +325,15 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // [-0.5, 0.5]; 2^f by a cubic fitted in this project by the Remez exchange on
 // relative error over [-0.5, 0.5] (maximum relative error 7.5e-5 in fp32,
 // below the 2^-9 rounding of the bf16 probabilities it feeds); 2^n applied by
-// adding n to the exponent field.  Arguments below -126 are raised to -126,
-// so a masked key (x = -inf) gets 2^-126 instead of 0.
+// adding n to the exponent field.  Arguments below -125 are raised to -125
+// (so 2^n stays a normal number: at n = -126 the sum of exponents would reach
+// the subnormal range and drop the implicit bit of the mantissa), so a masked
+// key (x = -inf) gets 2^-125 instead of 0.
 constexpr float kExp2C0 = 0.9999280571937561f, kExp2C1 = 0.6932609677314758f,
                 kExp2C2 = 0.2426111251115799f, kExp2C3 = 0.0551716685295105f;
 __device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
-  x0 = fmaxf(x0, -126.f);
-  x1 = fmaxf(x1, -126.f);
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
   float t0, t1, p0, p1;
   asm("{\n\t.reg .b64 px, pm, pt, pn, pf, pp, c;\n\t"
       "mov.b64 px, {%4, %5};\n\t"

@@ -65,7 +65,9 @@ def _check_items(got, want, b=0):
     assert len(items) == len(expect) and set(map(tuple, items.tolist())) == expect
     # grouped by the parity class of the base window (row and column index of
     # the base tiling); within a class unsplit windows first
-    nbx = int(np.sum(want.base[:, 0] == want.base[0, 0]))
+    # base windows per row: the oracle's column tiling under the plan's shift
+    # (with a shift, two rows may both start at y = 0, so y0 cannot tell rows apart)
+    nbx = len(ora.tile_windows(want.Wg, want.w, int(got["shift"][1])))
     parent = want.parent[items[:, 0]]
     cls = ((parent // nbx) % 2) * 2 + (parent % nbx) % 2
     split = want.split[parent].astype(int)
