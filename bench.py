@@ -439,11 +439,14 @@ def schedule_graph_leg(cfg, st, stream, full_ms, steps=28, shift=3.0, sigma_star
     kp = torch.empty((cfg.B, cfg.H, nk_max, cfg.D), dtype=st.q.dtype, device=dev)
     vp = torch.empty_like(kp)
     plans = {}
+    wsb = 0
     for w in sorted(set(ws_sides)):
         pc = area.make_cfg(cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
         nb = area.area_window_plan_bytes(pc)
-        assert area.area_window_attn_ws_bytes(pc, cfg.H, cfg.D) <= st.ws_bytes
+        wsb = max(wsb, area.area_window_attn_ws_bytes(pc, cfg.H, cfg.D))
         plans[w] = (pc, torch.empty(nb, dtype=torch.uint8, device=dev), nb)
+    # the run's window sides overlap differently from the step's: own workspace
+    ws = torch.empty(wsb // 4, dtype=torch.float32, device=dev)
 
     def run():
         for kd, p in sched:
@@ -457,7 +460,7 @@ def schedule_graph_leg(cfg, st, stream, full_ms, steps=28, shift=3.0, sigma_star
                 pc, plan, nb = plans[p]
                 area.area_dwt_window_plan(st.src, st.dt, cfg.C, area.AREA_DETAIL_HH, st.energy,
                                           pc, plan, nb, stream)
-                area.area_window_attn(st.q, st.k, st.v, pc, plan, nb, st.o2, st.ws, st.ws_bytes,
+                area.area_window_attn(st.q, st.k, st.v, pc, plan, nb, st.o2, ws, wsb,
                                       cfg.H, cfg.D, cfg.scale, st.dt, stream)
 
     with torch.cuda.stream(stream):
@@ -547,9 +550,10 @@ def profile_pass(args) -> int:
     """Every kernel of the path, twice, on one configuration: the input of the
     per-kernel ncu captures (a capture selects the second launch of a kernel
     with -s/-c).  Sequence per pass: pool_kv, coarse attention, the detail
-    map, the separate planner, the one-launch planner, window attention at
-    schedule step --profile-step, bridge selection and bridged window
-    attention.  Nothing is timed."""
+    map, the separate planner, the one-launch planner (once per window step),
+    window attention at schedule step --profile-step (or one call per step of
+    --profile-steps), bridge selection and bridged window attention.  Nothing
+    is timed."""
     import torch
 
     import step_adaptive_sparse_b200 as area
@@ -561,7 +565,9 @@ def profile_pass(args) -> int:
     src = torch.from_numpy(make_detail_source(cfg)).to(dev).to(tdt)
     stream = torch.cuda.Stream(device=dev)
     st = AreaStep(cfg, q, k, v, src, stream)
-    i = args.profile_step % len(cfg.schedule)
+    steps = ([int(x) % len(cfg.schedule) for x in args.profile_steps.split(",")]
+             if args.profile_steps else [args.profile_step % len(cfg.schedule)])
+    i = steps[-1]
     w = cfg.schedule[i]
     ry, rx = area.area_bridge_lattice(w, cfg.Hg, cfg.Wg)
     cand = torch.empty((cfg.B, cfg.H, ry * rx), dtype=torch.int32, device=dev)
@@ -577,10 +583,12 @@ def profile_pass(args) -> int:
             area.area_dwt_detail(src, st.dt, cfg.C, st.energy, cfg.B, cfg.Hg, cfg.Wg,
                                  area.AREA_DETAIL_HH, s)
             area.area_window_plan(st.energy, st.pcfg[i], st.plan[i], st.plan_bytes[i], s)
-            area.area_dwt_window_plan(src, st.dt, cfg.C, area.AREA_DETAIL_HH, st.energy,
-                                      st.pcfg[i], st.plan[i], st.plan_bytes[i], s)
-            area.area_window_attn(q, k, v, st.pcfg[i], st.plan[i], st.plan_bytes[i], st.o2, st.ws,
-                                  st.ws_bytes, cfg.H, cfg.D, cfg.scale, st.dt, s)
+            for si in steps:
+                area.area_dwt_window_plan(src, st.dt, cfg.C, area.AREA_DETAIL_HH, st.energy,
+                                          st.pcfg[si], st.plan[si], st.plan_bytes[si], s)
+            for si in steps:
+                area.area_window_attn(q, k, v, st.pcfg[si], st.plan[si], st.plan_bytes[si], st.o2,
+                                      st.ws, st.ws_bytes, cfg.H, cfg.D, cfg.scale, st.dt, s)
             area.area_bridge_select(k, st.dt, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, ry, rx, cand,
                                     mws, mws.numel() * 4, s)
             area.area_window_attn_bridge(q, k, v, cand, ry * rx, st.pcfg[i], st.plan[i],
@@ -588,7 +596,8 @@ def profile_pass(args) -> int:
                                          cfg.D, cfg.scale, st.dt, s)
     torch.cuda.synchronize()
     err = area.area_kernel_error()
-    print(json.dumps({"profile_pass": cfg.name, "window_side": w, "kernel_error": err}))
+    print(json.dumps({"profile_pass": cfg.name, "window_sides": [cfg.schedule[si] for si in steps],
+                      "kernel_error": err}))
     return 0 if err == 0 else 1
 
 
@@ -970,6 +979,9 @@ def main(argv=None):
                          "input of the per-kernel ncu captures)")
     ap.add_argument("--profile-step", type=int, default=-1,
                     help="schedule step of the window calls in --profile-pass")
+    ap.add_argument("--profile-steps", default="",
+                    help="comma-separated schedule steps: one window call each per pass "
+                         "(overrides --profile-step)")
     args = ap.parse_args(argv)
     if args.profile_pass:
         return profile_pass(args)
