@@ -176,6 +176,27 @@ def test_plain_c_consumer(tmp_path):
     assert "C-ABI host checks passed" in r.stdout
 
 
+def test_merge_geometry_host_check(tmp_path):
+    # The window kernels' merge geometry (which windows share a token, which
+    # of them stores first and which normalises last, the token's accumulator
+    # row) is plain integer arithmetic in area_internal.cuh.  Compile it on
+    # the host and check every token of many tilings, with border shifts.
+    import shutil
+    import subprocess
+    from step_adaptive_sparse_b200 import build as b
+    nvcc = b.nvcc()
+    if shutil.which(nvcc) is None and not os.path.exists(nvcc):
+        pytest.skip("nvcc is not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    exe = str(tmp_path / "merge_geometry_check")
+    subprocess.run([nvcc, "-O2", "-std=c++17", "-Wno-deprecated-gpu-targets", "-I",
+                    os.path.join(root, "include"), "-I", b.CSRC,
+                    os.path.join(root, "tests", "merge_geometry_check.cu"), "-o", exe], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert "tilings checked" in r.stdout
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     # no fallback: without the built library every call raises
     from step_adaptive_sparse_b200 import binding
