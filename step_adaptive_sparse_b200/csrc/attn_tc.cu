@@ -72,7 +72,10 @@ constexpr int kThreads = kSoftWarp0 * 32 + 256;
 constexpr int kRegsLow = 56, kRegsHigh = 208;
 constexpr int kPolyPer8 = AREA_EXP2_POLY_PER8;
 static_assert(kPolyPer8 >= 0 && kPolyPer8 <= 8, "polynomial share");
-constexpr int kStages = 4;              // K/V ring stages of 32 KB
+#ifndef AREA_TC_STAGES
+#define AREA_TC_STAGES 4
+#endif
+constexpr int kStages = AREA_TC_STAGES;  // K/V ring stages (32 KB each at head_dim 128)
 constexpr int kHalfBytes = 128 * 128;   // 128 rows x 64 bf16: one 128B-swizzled half tile
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
@@ -97,6 +100,7 @@ struct Geo {
   static constexpr int kSmemKV = 2 * kTileBytes;
   static constexpr int kSmemBar = kSmemKV + kStages * kTileBytes;
   static constexpr int kSmemBytes = kSmemBar + 256 + 1024;   // barriers + alignment slack
+  static_assert(kSmemBytes + 1024 <= 227 * 1024, "shared memory of one CTA");
 };
 
 // barrier indices
