@@ -444,17 +444,6 @@ int area_test_plan_barrier_expiry(const void* src, int src_dtype, int C,
                                   void* plan, size_t plan_bytes,
                                   cudaStream_t stream);
 
-/*
- * area_test_exp2_poly -- TEST HOOK, not part of the method (the pages have no
- * counterpart).  y[i] = 2^x[i] by the polynomial exponent the attention
- * softmax uses for part of its keys: Cody-Waite range reduction to
- * f in [-0.5, 0.5] and a cubic fitted in this project by the Remez exchange
- * (relative error below 7.5e-5 for -125 <= x <= 0; arguments below -125
- * give 2^-125).  x, y: device fp32 arrays of n elements.
- * Errors: AREA_EINVAL, AREA_ECUDA.
- */
-int area_test_exp2_poly(const float* x, float* y, long long n, cudaStream_t stream);
-
 /* ---- schedule (host functions: no device memory, no stream) ------------ */
 
 /*

@@ -35,8 +35,7 @@ EXPORTED = ("area_status_string", "area_last_cuda_error", "area_version", "area_
             "area_schedule",
             "area_coarse_attn", "area_full_attn", "area_dwt_detail", "area_window_plan_bytes",
             "area_window_plan", "area_window_attn_ws_bytes", "area_window_attn",
-            "area_window_attn_noalloc", "area_test_plan_barrier_expiry",
-            "area_test_exp2_poly")
+            "area_window_attn_noalloc", "area_test_plan_barrier_expiry")
 
 
 class AreaError(RuntimeError):
@@ -82,7 +81,6 @@ _SIGS = {
                                   _P]),
     "area_test_plan_barrier_expiry": (_I, [_P, _I, _I, _P, ctypes.POINTER(area_plan_cfg), _P,
                                            _SZ, _P]),
-    "area_test_exp2_poly": (_I, [_P, _P, ctypes.c_longlong, _P]),
     "area_pool_ramp": (_I, [_I, _I, _I, _I, _I, _P]),
     "area_window_sides": (_I, [_I, _I, _I, _P]),
     "area_bridge_lattice": (_I, [_I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
@@ -218,13 +216,6 @@ def area_test_plan_barrier_expiry(src, src_dtype, C, energy, cfg: area_plan_cfg,
                                                 ctypes.byref(cfg), _ptr(plan), plan_bytes,
                                                 _stream(stream)),
            "area_test_plan_barrier_expiry")
-
-
-def area_test_exp2_poly(x, y, n, stream=None) -> None:
-    """Test hook: the softmax's polynomial 2^x over n fp32 values (see
-    include/area.h)."""
-    _check(_lib().area_test_exp2_poly(_ptr(x), _ptr(y), n, _stream(stream)),
-           "area_test_exp2_poly")
 
 
 def area_window_attn_ws_bytes(cfg: area_plan_cfg, H: int, D: int) -> int:

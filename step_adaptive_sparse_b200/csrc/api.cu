@@ -190,12 +190,6 @@ int area_test_plan_barrier_expiry(const void* src, int src_dtype, int C, float* 
                                              plan, stream, 1u, 1000000ull));
 }
 
-int area_test_exp2_poly(const float* x, float* y, long long n, cudaStream_t stream) {
-  if (!x || !y || n < 0 || n > (1ll << 40)) return AREA_EINVAL;
-  if (n == 0) return AREA_OK;
-  return finish(area::launch_exp2_poly(x, y, (int64_t)n, stream));
-}
-
 int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D, size_t* ws_bytes) {
   if (!ws_bytes || H < 1 || D < 1) return AREA_EINVAL;
   area::PlanLayout L;

@@ -221,8 +221,6 @@ cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, co
                                  const void* vt, void* o, int B, int H, int N, int Nk, int T,
                                  int D, float scale, cudaStream_t s);
 cudaError_t read_and_clear_tc_error(int* code);
-// The softmax's polynomial 2^x (exp2_poly2) over an array, for its accuracy test.
-cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s);
 // cand (may be null): per-head bridge candidates [B*H][R]; when given they
 // replace the plan's global-KV lists, candidates inside a window's Halo
 // rectangle are skipped.

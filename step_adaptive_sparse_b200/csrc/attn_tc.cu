@@ -47,35 +47,9 @@ __device__ int g_tc_error = 0;   // set on a bounded-wait expiry; read by tests
 
 namespace {
 
-// Warp roles.  By default warp 0 is the producer, warp 1 the MMA issuer and
-// warps 2-9 the softmax (320 threads, every thread capped at 168 registers).
-// With AREA_TC_WG_SPLIT the CTA has three warpgroups (384 threads launched at
-// 168 registers each): warpgroup 0 (producer, MMA issuer, two idle warps)
-// gives registers back with setmaxnreg and the two softmax warpgroups take
-// them, 56 + 2 x 224 = 3 x 168 per lane of a warpgroup, the block's whole
-// launch allocation.
-#ifndef AREA_TC_WG_SPLIT
-#define AREA_TC_WG_SPLIT 0
-#endif
-// Exponentials of every 8 key pairs computed on the FMA pipe instead of the
-// MUFU unit (0..8); see exp2_poly2.
-#ifndef AREA_EXP2_POLY_PER8
-#define AREA_EXP2_POLY_PER8 0
-#endif
-constexpr bool kWgSplit = AREA_TC_WG_SPLIT != 0;
-constexpr int kSoftWarp0 = kWgSplit ? 4 : 2;          // first softmax warp
-constexpr int kThreads = kSoftWarp0 * 32 + 256;
-// The split is sized for the registers the kernel is compiled to start with
-// (ptxas, no launch bound: the setmaxnreg regions may not exceed a bound).
-// The host refuses the launch unless warpgroup 0's release covers the softmax
-// warpgroups' increase: kRegsLow * 128 + kRegsHigh * 256 <= entry * 384.
-constexpr int kRegsLow = 56, kRegsHigh = 208;
-constexpr int kPolyPer8 = AREA_EXP2_POLY_PER8;
-static_assert(kPolyPer8 >= 0 && kPolyPer8 <= 8, "polynomial share");
-#ifndef AREA_TC_STAGES
-#define AREA_TC_STAGES 4
-#endif
-constexpr int kStages = AREA_TC_STAGES;  // K/V ring stages (32 KB each at head_dim 128)
+constexpr int kThreads = 320;     // producer, MMA issuer, 8 softmax warps
+constexpr int kSoftWarp0 = 2;     // first softmax warp
+constexpr int kStages = 4;               // K/V ring stages (32 KB each at head_dim 128)
 constexpr int kHalfBytes = 128 * 128;   // 128 rows x 64 bf16: one 128B-swizzled half tile
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
@@ -323,45 +297,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x for two arguments on the FMA pipe (packed f32x2 arithmetic), for
-// x <= 0 as in the softmax.  Method: Cody-Waite range reduction
-// x = n + f with n = round(x) (the 1.5 * 2^23 rounding constant), f in
-// [-0.5, 0.5]; 2^f by a cubic fitted in this project by the Remez exchange on
-// relative error over [-0.5, 0.5] (maximum relative error 7.5e-5 in fp32,
-// below the 2^-9 rounding of the bf16 probabilities it feeds); 2^n applied by
-// adding n to the exponent field.  Arguments below -125 are raised to -125
-// (so 2^n stays a normal number: at n = -126 the sum of exponents would reach
-// the subnormal range and drop the implicit bit of the mantissa), so a masked
-// key (x = -inf) gets 2^-125 instead of 0.
-constexpr float kExp2C0 = 0.9999280571937561f, kExp2C1 = 0.6932609677314758f,
-                kExp2C2 = 0.2426111251115799f, kExp2C3 = 0.0551716685295105f;
-__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
-  x0 = fmaxf(x0, -125.f);
-  x1 = fmaxf(x1, -125.f);
-  float t0, t1, p0, p1;
-  asm("{\n\t.reg .b64 px, pm, pt, pn, pf, pp, c;\n\t"
-      "mov.b64 px, {%4, %5};\n\t"
-      "mov.b64 pm, {%6, %6};\n\t"
-      "add.rn.f32x2 pt, px, pm;\n\t"          // t = x + 1.5 * 2^23: round to integer
-      "sub.rn.f32x2 pn, pt, pm;\n\t"          // n = round(x)
-      "sub.rn.f32x2 pf, px, pn;\n\t"          // f = x - n
-      "mov.b64 c, {%10, %10};\n\t"
-      "mov.b64 pp, {%9, %9};\n\t"
-      "fma.rn.f32x2 pp, c, pf, pp;\n\t"       // c3 f + c2
-      "mov.b64 c, {%8, %8};\n\t"
-      "fma.rn.f32x2 pp, pp, pf, c;\n\t"       // (..) f + c1
-      "mov.b64 c, {%7, %7};\n\t"
-      "fma.rn.f32x2 pp, pp, pf, c;\n\t"       // (..) f + c0
-      "mov.b64 {%0, %1}, pt;\n\t"
-      "mov.b64 {%2, %3}, pp;\n\t}"
-      : "=f"(t0), "=f"(t1), "=f"(p0), "=f"(p1)
-      : "f"(x0), "f"(x1), "f"(12582912.0f), "f"(kExp2C0), "f"(kExp2C1), "f"(kExp2C2),
-        "f"(kExp2C3));
-  // the low mantissa bits of t hold n: shifted into the exponent field
-  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
 // Packed fp32 pair arithmetic of sm_100 (one instruction for two lanes of work).
 __device__ __forceinline__ void fma2(float& y0, float& y1, float a0, float a1, float b, float c) {
   asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\t"
@@ -499,14 +434,9 @@ __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
   return false;
 }
 
-#if AREA_TC_WG_SPLIT
-#define AREA_TC_BOUNDS
-#else
-#define AREA_TC_BOUNDS __launch_bounds__(kThreads, 1)
-#endif
 
 template <bool WINDOW, bool BRIDGE, int D>
-__global__ void AREA_TC_BOUNDS
+__global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
                const __grid_constant__ CUtensorMap tm_vp, const __grid_constant__ CUtensorMap tm_kt,
@@ -524,12 +454,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if constexpr (kWgSplit) {
-    // first thing: warpgroup 0 gives registers back, the softmax warpgroups
-    // take them (so almost no code runs at the entry allocation)
-    if (warp < kSoftWarp0) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
-    else asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
-  }
 
   if (threadIdx.x == 0) {
     s_abort = 0;
@@ -925,13 +849,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           for (int i = kKeys * h; i < kKeys * h + kKeys; i += 2) {
             float x0, x1;
             fma2(x0, x1, __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]), sl2, negm);
-            float p0, p1;
-            if (kPolyPer8 > 0 && ((i >> 1) & 7) < kPolyPer8) {
-              exp2_poly2(p0, p1, x0, x1);
-            } else {
-              p0 = fast_exp2(x0);
-              p1 = fast_exp2(x1);
-            }
+            const float p0 = fast_exp2(x0);
+            const float p1 = fast_exp2(x1);
             if ((i >> 1) & 1) add2(ls[2], ls[3], p0, p1); else add2(ls[0], ls[1], p0, p1);
             sr[i >> 1] = pack_bf16(p0, p1);
           }
@@ -1159,44 +1078,12 @@ cudaError_t launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
   auto fn = attn_tc_kernel<WINDOW, BRIDGE, D>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  if constexpr (kWgSplit) {
-    // setmaxnreg.inc waits until registers are free: launch only when the
-    // registers warpgroup 0 gives back cover what the softmax warpgroups take
-    // (entry count rounded up to the allocation unit of 8 per thread)
-    cudaFuncAttributes fa;
-    if ((e = cudaFuncGetAttributes(&fa, fn)) != cudaSuccess) return e;
-    const int entry = (fa.numRegs + 7) & ~7;
-    if (entry < kRegsLow || entry > kRegsHigh ||
-        (entry - kRegsLow) * 128 < (kRegsHigh - entry) * 256)
-      return cudaErrorInvalidConfiguration;
-  }
   const int grid = prm.num_units < num_sms() ? prm.num_units : num_sms();
   fn<<<grid > 0 ? grid : 1, kThreads, kSmemBytes, s>>>(mq, mk, mv, mkp, mvp, mkt, mvt, prm);
   return cudaGetLastError();
 }
 
 }  // namespace
-
-namespace {
-// exp2_poly2 over an array (the accuracy test of the polynomial exponent)
-__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
-  const int64_t i = 2 * (blockIdx.x * (int64_t)blockDim.x + threadIdx.x);
-  if (i + 1 < n) {
-    exp2_poly2(y[i], y[i + 1], x[i], x[i + 1]);
-  } else if (i < n) {
-    float a, b;
-    exp2_poly2(a, b, x[i], 0.f);
-    y[i] = a;
-  }
-}
-}  // namespace
-
-cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s) {
-  const int64_t pairs = (n + 1) / 2;
-  const int64_t blocks = (pairs + 255) / 256;
-  exp2_poly_kernel<<<(unsigned)(blocks > 0 ? blocks : 1), 256, 0, s>>>(x, y, n);
-  return cudaGetLastError();
-}
 
 cudaError_t read_and_clear_tc_error(int* code) {
   cudaError_t e = cudaDeviceSynchronize();
