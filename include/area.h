@@ -32,8 +32,9 @@
  *     grid barriers; and the window-attention calls on the tensor cores,
  *     where a CTA about to add a later parity class of windows into an
  *     overlapped token's accumulator row waits until every unit of the
- *     earlier classes has completed (units are claimed in class order by
- *     running CTAs, so every unit waited on is held by a running CTA).  The return value
+ *     earlier classes of the same head has completed (a head's units are
+ *     claimed in class order by running CTAs, so every unit waited on is
+ *     held by a running CTA).  The return value
  *     reports argument validation and launch errors only; AREA_ECUDA carries
  *     the CUDA error, see area_status_string.  The schedule functions at the
  *     end are host arithmetic (no device memory, no stream).
@@ -294,14 +295,16 @@ int area_dwt_window_plan(const void* src, int src_dtype, int C, int mode,
 
 /*
  * area_window_attn_ws_bytes -- workspace for area_window_attn (host only):
- * 256 bytes of counters, then one fp32 row of D values per (batch element,
- * head, token covered by more than one base window):
- *   256 + B * H * n_ov * D * 4 bytes,
+ * a header of 1 + 4 * B * H uint32 counters (the unit counter and one
+ * completion counter per batch element, head and parity class) rounded up
+ * to 256 bytes, then one fp32 row of D values per (batch element, head,
+ * token covered by more than one base window):
+ *   hdr + B * H * n_ov * D * 4 bytes, hdr = ceil256(4 * (1 + 4 * B * H)),
  * n_ov = ny2 * Wg + (Hg - ny2) * nx2, where ny2 (nx2) counts the rows
  * (columns) of the grid that two base windows share along that axis under
  * the plan's border shift.  Windows that tile an axis exactly share nothing
  * (e.g. 64-token windows on a 384-token axis), and then the workspace is the
- * 256-byte header alone.
+ * header alone.
  */
 int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D,
                               size_t* ws_bytes);
@@ -315,11 +318,12 @@ int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D,
  *   cfg, plan  : the configuration and buffer given to area_window_plan
  *   ws         : workspace of ws_bytes >= area_window_attn_ws_bytes(),
  *                16-byte aligned; contents on entry are ignored, on exit
- *                unspecified.  The call resets its 256-byte header (a memset
+ *                unspecified.  The call resets its counter header (a memset
  *                on the stream) before the kernel.
  * Merge order: a token covered by several windows is summed over them in a
- * fixed order (by the parity class of the base window, see the plan's ITEMS),
- * so the output is bit-identical from run to run and in CUDA-graph replays.
+ * fixed order (by the parity class of the base window, see the plan's ITEMS;
+ * the units of one head run class by class), so the output is bit-identical
+ * from run to run and in CUDA-graph replays.
  * Errors: AREA_EINVAL, AREA_EUNSUPPORTED (D, dtype), AREA_ENOSPACE.
  */
 int area_window_attn(const void* q, const void* k, const void* v,

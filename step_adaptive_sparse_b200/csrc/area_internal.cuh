@@ -168,11 +168,14 @@ __host__ __device__ inline MergeRole merge_role(int y, int x, int cls, int4 my, 
   return r;
 }
 
-// Window-attention workspace: a 256-byte header of counters (the dynamic
-// unit counter, then one completion counter per parity class), then one fp32
-// accumulator row per (element, head, overlapped token).
-constexpr int kWsHeaderBytes = 256;
+// Window-attention workspace: a header of uint32 counters (the dynamic unit
+// counter, then one completion counter per (element, head, parity class)),
+// rounded up to 256 bytes, then one fp32 accumulator row per (element, head,
+// overlapped token).
 constexpr int kWsUnitCounter = 0, kWsClassDone = 1;
+__host__ __device__ inline int64_t window_ws_header_bytes(int64_t B, int64_t H) {
+  return ((4 * (1 + 4 * B * H)) + 255) & ~int64_t(255);
+}
 
 // Counter-based draws: output number (stream * 2^32 + index) of the SplitMix64
 // sequence (Steele, Lea, Flood 2014) seeded with `seed`.

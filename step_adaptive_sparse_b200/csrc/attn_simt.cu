@@ -238,7 +238,8 @@ cudaError_t launch_window_attn_simt(const void* q, const void* k, const void* v,
                                     const PlanLayout& L, const void* plan, void* o, void* ws,
                                     int H, int D, float scale, int dtype, cudaStream_t s) {
   PlanView P = plan_view(L, const_cast<void*>(plan));
-  const MergeArgs ma{reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeaderBytes),
+  const MergeArgs ma{reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                              window_ws_header_bytes(L.B, H)),
                      (int)L.nx2, (long long)L.n_ov};
   dim3 grid((unsigned)(L.nitem_max * (kQTile / kSimtQ)), H, (unsigned)L.B);
   DenseRows dr{(int)L.N, (int)L.N};

@@ -374,8 +374,10 @@ __device__ __forceinline__ int window_query_token(const int4& win, int nq, int p
 }
 
 // Decode unit u into a record (producer lane 0).  Dense: (b*H + h, 256-query
-// block), head-major.  Window: by parity class, then batch element, then
-// head, then the class's work items in plan order.
+// block), head-major.  Window: by batch element, then head, then the work
+// items in plan order, which run class by class: a head's four parity
+// classes follow one another, so its accumulator rows are re-read while they
+// are still in L2.
 template <bool WINDOW>
 __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
   r.valid = 1;
@@ -398,38 +400,34 @@ __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
   }
   const PlanView& P = prm.P;
   int rem = u;
-  for (int c = 0; c < 4; ++c) {
-    for (int b = 0; b < P.B; ++b) {
-      const int n = P.nclass[b * 4 + c];
-      const int cnt = n * prm.H;
-      if (rem >= cnt) {
-        rem -= cnt;
-        continue;
-      }
-      int coff = 0;
-      for (int c2 = 0; c2 < c; ++c2) coff += P.nclass[b * 4 + c2];
-      const int h = rem / n;
-      const int2 it = P.items[(int64_t)b * P.nitem_max + coff + rem % n];
-      const int64_t wo = (int64_t)b * P.nw + it.x;
-      r.b = b;
-      r.bh = b * prm.H + h;
-      r.win = P.win[wo];
-      r.ext = P.ext[wo];
-      const int parent = P.parent[wo];
-      r.cls = window_class(parent, P.nbx);
-      r.my = axis_merge(parent / P.nbx, P.nby, P.Hg, P.hy, P.sy);
-      r.mx = axis_merge(parent % P.nbx, P.nbx, P.Wg, P.wx, P.sx);
-      r.q0 = it.y * 256;
-      r.nq = r.win.z * r.win.w;
-      r.one = r.nq - r.q0 <= 128;
-      r.nkv = prm.cand ? prm.R : P.gcount[wo];
-      r.ngt = (r.nkv + 127) / 128;
-      r.ncx = (r.ext.w + kPW - 1) / kPW;
-      r.ntr = r.ncx * ((r.ext.z + kPH - 1) / kPH);
-      r.nt = r.ngt + r.ntr + (prm.T + 127) / 128;
-      r.glist = prm.cand ? (long long)r.bh * prm.R : (long long)wo * P.G;
-      return true;
+  for (int b = 0; b < P.B; ++b) {
+    const int n = P.nitem[b];
+    const int cnt = n * prm.H;
+    if (rem >= cnt) {
+      rem -= cnt;
+      continue;
     }
+    const int h = rem / n;
+    const int2 it = P.items[(int64_t)b * P.nitem_max + rem % n];
+    const int64_t wo = (int64_t)b * P.nw + it.x;
+    r.b = b;
+    r.bh = b * prm.H + h;
+    r.win = P.win[wo];
+    r.ext = P.ext[wo];
+    const int parent = P.parent[wo];
+    r.cls = window_class(parent, P.nbx);
+    r.my = axis_merge(parent / P.nbx, P.nby, P.Hg, P.hy, P.sy);
+    r.mx = axis_merge(parent % P.nbx, P.nbx, P.Wg, P.wx, P.sx);
+    r.q0 = it.y * 256;
+    r.nq = r.win.z * r.win.w;
+    r.one = r.nq - r.q0 <= 128;
+    r.nkv = prm.cand ? prm.R : P.gcount[wo];
+    r.ngt = (r.nkv + 127) / 128;
+    r.ncx = (r.ext.w + kPW - 1) / kPW;
+    r.ntr = r.ncx * ((r.ext.z + kPH - 1) / kPH);
+    r.nt = r.ngt + r.ntr + (prm.T + 127) / 128;
+    r.glist = prm.cand ? (long long)r.bh * prm.R : (long long)wo * P.G;
+    return true;
   }
   return false;
 }
@@ -753,7 +751,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (qt == 1 && R.one) {
         // at most 128 valid queries: query tile 1 does not run; its warps
         // only sign the unit off (completion count and record slot)
-        if (WINDOW && lane == 0) atomicAdd(prm.counters + kWsClassDone + R.cls, 1u);
+        if (WINDOW && lane == 0) atomicAdd(prm.counters + kWsClassDone + R.bh * 4 + R.cls, 1u);
         if (lane == 0) mbar_arrive(bar(BAR_REC_EMPTY + slot));
         ++unit_count;
         continue;
@@ -930,13 +928,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           if (lane == 0) {
             const uint64_t t0 = global_ns();
             for (int c = 0; c < cls && wok; ++c) {
-              // completions class c needs: 8 warps per unit, H units per item
-              const unsigned target = 8u * (unsigned)prm.H * (unsigned)prm.P.nclass[prm.P.B * 4 + c];
+              // completions class c of this (element, head) needs: 8 warps per unit
+              const unsigned target = 8u * (unsigned)prm.P.nclass[R.b * 4 + c];
+              const unsigned* ctr = prm.counters + kWsClassDone + bh * 4 + c;
               uint32_t it = 0;
               for (;;) {
                 unsigned v;
                 asm volatile("ld.acquire.gpu.global.u32 %0, [%1];"
-                             : "=r"(v) : "l"(prm.counters + kWsClassDone + c) : "memory");
+                             : "=r"(v) : "l"(ctr) : "memory");
                 if (v >= target) break;
                 if ((++it & 63u) == 0) {
                   if (*(volatile int*)abort_flag) { wok = 0; break; }
@@ -1003,7 +1002,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // this warp's rows of the unit are complete
         __threadfence();
         __syncwarp();
-        if (lane == 0) atomicAdd(prm.counters + kWsClassDone + cls, 1u);
+        if (lane == 0) atomicAdd(prm.counters + kWsClassDone + bh * 4 + cls, 1u);
       }
       tc_fence_before();
       if (lane == 0) mbar_arrive(bar(BAR_REC_EMPTY + slot));
@@ -1122,7 +1121,7 @@ cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, co
 }
 
 int64_t window_ws_bytes(const PlanLayout& L, int H, int D) {
-  return kWsHeaderBytes + L.B * H * L.n_ov * D * 4;
+  return window_ws_header_bytes(L.B, H) + L.B * H * L.n_ov * D * 4;
 }
 
 cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, const void* kt,
@@ -1155,11 +1154,12 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, c
   prm.num_units = (int)(L.nitem_max * L.B * H);
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.counters = static_cast<unsigned*>(ws);
-  prm.acc = reinterpret_cast<float*>(static_cast<char*>(ws) + kWsHeaderBytes);
+  const int64_t hdr = window_ws_header_bytes(L.B, H);
+  prm.acc = reinterpret_cast<float*>(static_cast<char*>(ws) + hdr);
   prm.nx2 = (int)L.nx2;
   prm.n_ov = L.n_ov;
   // unit counter and class completion counters start at zero
-  if ((e = cudaMemsetAsync(ws, 0, kWsHeaderBytes, s)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(ws, 0, (size_t)hdr, s)) != cudaSuccess) return e;
   if (D == 64) {
     if (cand) return launch_tc<true, true, 64>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
     return launch_tc<true, false, 64>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);

@@ -14,15 +14,16 @@ int main(void) {
   area_plan_cfg cfg = {1, 256, 256, 64, 4, 512, 0.4f, 0ull};
   size_t nb = 0;
   if (area_window_plan_bytes(&cfg, &nb) != AREA_OK || nb == 0 || nb % 256 != 0) return 3;
-  /* merge workspace: a 256-byte header plus one fp32 row per overlapped
-   * token; 64-token windows tile 256 exactly (no overlap), 80-token windows
+  /* merge workspace: a header of 1 + 4 * B * H counters (4 * 97 bytes for
+   * 24 heads, rounded up to 512) plus one fp32 row per overlapped token and
+   * head; 64-token windows tile 256 exactly (no overlap), 80-token windows
    * (starts 0, 58, 117, 176) overlap on 64 positions per axis, so on
    * 64 * 256 + 192 * 64 = 28672 tokens */
   size_t ws = 0;
-  if (area_window_attn_ws_bytes(&cfg, 24, 128, &ws) != AREA_OK || ws != 256) return 4;
+  if (area_window_attn_ws_bytes(&cfg, 24, 128, &ws) != AREA_OK || ws != 512) return 4;
   area_plan_cfg cfg80 = {1, 256, 256, 80, 4, 512, 0.4f, 0ull};
   if (area_window_attn_ws_bytes(&cfg80, 24, 128, &ws) != AREA_OK ||
-      ws != (size_t)256 + (size_t)24 * 28672 * 128 * 4)
+      ws != (size_t)512 + (size_t)24 * 28672 * 128 * 4)
     return 4;
 
   /* the printed pooling ramp at a 256 x 256 grid */

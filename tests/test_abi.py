@@ -106,7 +106,9 @@ def test_plan_config_validation_and_sizes(area):
     assert area.area_window_plan_bytes(area.make_cfg(1, 256, 256, 32, 4, 512, 0.4)) > n
     assert area.area_window_plan_bytes(area.make_cfg(2, 256, 256, 64, 4, 512, 0.4)) > n
     # 64-token windows tile 256 exactly: no overlap, only the counter header
-    assert area.area_window_attn_ws_bytes(good, 24, 128) == 256
+    # (1 + 4 * B * H uint32 counters, rounded up to 256 bytes)
+    assert area.area_window_attn_ws_bytes(good, 24, 128) == 512
+    assert area.area_window_attn_ws_bytes(good, 1, 128) == 256
     for bad in [area.make_cfg(0, 256, 256, 64, 4, 512, 0.4),
                 area.make_cfg(1, 255, 256, 64, 4, 512, 0.4),
                 area.make_cfg(1, 256, 256, 0, 4, 512, 0.4),
@@ -243,8 +245,9 @@ def test_noalloc_rejects_bad_input_with_the_status_of_area_window_attn(area):
 
 
 def test_window_ws_bytes_count_the_overlapped_tokens(area):
-    # Workspace = 256-byte counter header + one fp32 row of D per (element,
-    # head, token covered by more than one base window).  The overlapped
+    # Workspace = counter header (1 + 4 * B * H uint32, rounded up to 256
+    # bytes) + one fp32 row of D per (element, head, token covered by more
+    # than one base window).  The overlapped
     # tokens are counted here by brute force over the oracle's base tiling
     # (with the border shift the seed draws).
     from oracle import area_oracle as ora
@@ -263,4 +266,5 @@ def test_window_ws_bytes_count_the_overlapped_tokens(area):
         n_ov = int(((cy[:, None] * cx[None, :]) > 1).sum())
         for H, D in [(1, 64), (24, 128)]:
             cfg = area.make_cfg(B, Hg, Wg, w, 4, 16, 0.1, seed)
-            assert area.area_window_attn_ws_bytes(cfg, H, D) == 256 + B * H * n_ov * D * 4
+            hdr = (4 * (1 + 4 * B * H) + 255) // 256 * 256
+            assert area.area_window_attn_ws_bytes(cfg, H, D) == hdr + B * H * n_ov * D * 4
