@@ -15,11 +15,12 @@
 //               ring read by the other roles, and issues the TMA loads: Q
 //               tiles once per unit, then a ring of K and V tiles (128 keys x
 //               128 dims, 128B-swizzled, 32 KB each).  Dense rows use tiled
-//               2-D loads.  Window keys are the global-KV list first (gather4,
-//               4 rows per lane), then the Halo rectangle covered by 16x8-token
-//               patches (one 3-D tiled box each, masked at the rectangle's
-//               right and bottom edges); window queries (the rectangle
-//               enumerated row-major) use gather4.
+//               2-D loads.  Window keys are the global-KV list first (rows
+//               copied with 16-byte cp.async by the 32 producer lanes), then
+//               the Halo rectangle covered by 16x8-token patches (one 3-D
+//               tiled box each, masked at the rectangle's right and bottom
+//               edges); window queries (the rectangle enumerated row-major)
+//               are copied row by row with cp.async too.
 //   warp 1      TMEM allocator and the single MMA-issuing thread.
 //   warps 2-5   softmax of query tile 0, warps 6-9 of query tile 1: each
 //               thread owns one query row (TMEM lane 32*(warp mod 4) + lane).
@@ -183,14 +184,20 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int c0, int r0, int r1, int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
-      "r"(r3)
-      : "memory");
+// 16 bytes global -> shared, asynchronous (L2 only), and the arrive-on of an
+// mbarrier when all of the thread's earlier cp.async copies have landed (the
+// barrier's pending count is raised by one at once, so the phase cannot
+// complete before the copies).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+// Shared-memory writes of the generic proxy (cp.async) made visible to the
+// async proxy (tcgen05.mma operands).
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // UMMA shared-memory descriptor, 128-byte swizzle, sm_100 version field.
@@ -361,6 +368,7 @@ struct TcParams {
   DenseArgs da;
   PlanView P;
   __nv_bfloat16* o;   // output
+  const __nv_bfloat16 *q, *k, *v;   // window: the inputs, for rows copied with cp.async
   unsigned* counters; // window: workspace header (unit counter, per-class completions)
   float* acc;         // window: fp32 accumulator rows [B*H][n_ov][128]
   int nx2;            // window: columns covered by two base windows
@@ -373,11 +381,47 @@ __device__ __forceinline__ int window_query_token(const int4& win, int nq, int p
   return (win.x + p / win.w) * Wg + win.y + p % win.w;
 }
 
+// One 128-row tile of D bf16 copied row by row with cp.async by the 32 lanes
+// of a warp into the 128B-swizzled K-major layout that TMA's 128-byte swizzle
+// produces (and UMMA reads): in each 64-column half, row R at R * 128 bytes,
+// its 16-byte chunk c at ((c ^ (R mod 8)) * 16).  Lane l holds the source
+// rows of tile rows 4l .. 4l + 3 in r[0..3] (row indices of `base`).  Each
+// warp instruction copies whole rows (256 or 128 contiguous bytes per row).
+// Gathered rows go this way rather than through tile::gather4, whose issue
+// rate (about 7 bytes per clock per SM, measured) made them the window
+// kernel's largest fixed cost.
+template <int D>
+__device__ __forceinline__ void cp_async_rows(uint32_t dst, const __nv_bfloat16* base,
+                                              const int (&r)[4], int lane) {
+  constexpr int kChunks = D / 8;              // 16-byte chunks per row: 16 or 8
+  constexpr int kRowsPerIt = 32 / kChunks;    // rows per warp instruction: 2 or 4
+  const int q = lane % kChunks, sub = lane / kChunks;
+  const uint32_t half = (uint32_t)((q >> 3) * kHalfBytes);
+  const int c = q & 7;
+#pragma unroll 4
+  for (int o = 0; o < 32; ++o) {              // the four rows held by lane o
+    const int t0 = __shfl_sync(0xffffffffu, r[0], o), t1 = __shfl_sync(0xffffffffu, r[1], o);
+    const int t2 = __shfl_sync(0xffffffffu, r[2], o), t3 = __shfl_sync(0xffffffffu, r[3], o);
+#pragma unroll
+    for (int k = 0; k < 4 / kRowsPerIt; ++k) {
+      const int e = k * kRowsPerIt + sub;     // which of the four
+      const int tok = e == 0 ? t0 : e == 1 ? t1 : e == 2 ? t2 : t3;
+      const int R = o * 4 + e;
+      cp_async16(dst + half + (uint32_t)(R * 128 + ((c ^ (R & 7)) << 4)),
+                 base + (int64_t)tok * D + q * 8);
+    }
+  }
+}
+
 // Decode unit u into a record (producer lane 0).  Dense: (b*H + h, 256-query
-// block), head-major.  Window: by batch element, then head, then the work
-// items in plan order, which run class by class: a head's four parity
-// classes follow one another, so its accumulator rows are re-read while they
-// are still in L2.
+// block), head-major.  Window: per batch element, the (head, parity class)
+// groups of work items run skewed: at step t = 0, 1, ... come head t's
+// class 0, head t-1's class 1, head t-2's class 2 and head t-3's class 3,
+// each group's items in plan order.  A head's classes thus run in order, its
+// accumulator rows are re-read a few groups after they were written (still
+// in L2), and three other groups lie between a class and the next class of
+// the same head, so the units of the earlier class have usually completed
+// by the time the later class needs them.
 template <bool WINDOW>
 __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
   r.valid = 1;
@@ -401,14 +445,30 @@ __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
   const PlanView& P = prm.P;
   int rem = u;
   for (int b = 0; b < P.B; ++b) {
-    const int n = P.nitem[b];
-    const int cnt = n * prm.H;
+    const int cnt = P.nitem[b] * prm.H;
     if (rem >= cnt) {
       rem -= cnt;
       continue;
     }
-    const int h = rem / n;
-    const int2 it = P.items[(int64_t)b * P.nitem_max + rem % n];
+    // items per class; the items are stored class by class
+    const int n0 = P.nclass[b * 4 + 0], n1 = P.nclass[b * 4 + 1];
+    const int n2 = P.nclass[b * 4 + 2], n3 = P.nclass[b * 4 + 3];
+    int h = -1, idx = 0;
+    for (int t = 0; t < prm.H + 3 && h < 0; ++t) {
+      for (int c = 0; c < 4; ++c) {
+        const int hh = t - c;
+        if (hh < 0 || hh >= prm.H) continue;
+        const int nc = c == 0 ? n0 : c == 1 ? n1 : c == 2 ? n2 : n3;
+        if (rem < nc) {
+          h = hh;
+          idx = rem + (c > 0 ? n0 : 0) + (c > 1 ? n1 : 0) + (c > 2 ? n2 : 0);
+          break;
+        }
+        rem -= nc;
+      }
+    }
+    if (h < 0) return false;
+    const int2 it = P.items[(int64_t)b * P.nitem_max + idx];
     const int64_t wo = (int64_t)b * P.nw + it.x;
     r.b = b;
     r.bh = b * prm.H + h;
@@ -530,25 +590,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (!R.valid) break;
       if (!warp_wait0(bar(BAR_Q_EMPTY), (unit_count & 1u) ^ 1u, abort_flag)) break;
       const int nqt = R.one ? 1 : 2;          // query tiles of this unit
-      if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL), nqt * G::kTileBytes);
-      __syncwarp();
       if constexpr (!WINDOW) {
         if (lane == 0) {
+          mbar_arrive_tx(bar(BAR_Q_FULL), nqt * G::kTileBytes);
           for (int t = 0; t < nqt; ++t)
             for (int hf = 0; hf < G::kHalves; ++hf)
               tma_load_2d(sbase + G::kSmemQ + t * G::kTileBytes + hf * kHalfBytes, &tm_q,
                           bar(BAR_Q_FULL), hf * 64, R.bh * Ntok + R.q0 + t * 128);
         }
+        __syncwarp();
       } else {
+        // window queries: the rectangle enumerated row-major, copied row by row
         for (int t = 0; t < nqt; ++t) {
           int r[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             r[i] = R.bh * Ntok + window_query_token(R.win, R.nq, R.q0 + t * 128 + lane * 4 + i, Wg);
-          for (int hf = 0; hf < G::kHalves; ++hf)
-            tma_gather4(sbase + G::kSmemQ + t * G::kTileBytes + hf * kHalfBytes + lane * 512, &tm_q,
-                        bar(BAR_Q_FULL), hf * 64, r[0], r[1], r[2], r[3]);
+          cp_async_rows<D>(sbase + G::kSmemQ + t * G::kTileBytes, prm.q, r, lane);
         }
+        cp_async_arrive(bar(BAR_Q_FULL));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_Q_FULL));
       }
       const int nt = R.nt, ngt = R.ngt, ntr = R.ntr, ncx = R.ncx, nkv = R.nkv;
       const int nti = ngt + ntr;
@@ -568,10 +630,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ok = false;
             break;
           }
-          if (lane == 0) mbar_arrive_tx(bar(BAR_KV_FULL + s), G::kTileBytes);
-          __syncwarp();
           const CUtensorMap* tm = kv ? &tm_v : &tm_k;
           const uint32_t dst = sbase + G::kSmemKV + s * G::kTileBytes;
+          if (WINDOW && j < ngt) {
+            // global-KV list (or bridge candidates), copied row by row
+            const int g0 = j * 128 + lane * 4;
+            int r[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int p = g0 + i < nkv ? g0 + i : nkv - 1;
+              r[i] = bh * Nkrows + glist[p];
+            }
+            cp_async_rows<D>(dst, kv ? prm.v : prm.k, r, lane);
+            cp_async_arrive(bar(BAR_KV_FULL + s));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(BAR_KV_FULL + s));
+            ++kv_it;
+            continue;
+          }
+          if (lane == 0) mbar_arrive_tx(bar(BAR_KV_FULL + s), G::kTileBytes);
+          __syncwarp();
           if (j >= nti) {
             // text keys: rows of the [B*H*T, 128] text tensors
             if (lane == 0) {
@@ -585,18 +663,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               for (int hf = 0; hf < G::kHalves; ++hf)
                 tma_load_2d(dst + hf * kHalfBytes, tm, bar(BAR_KV_FULL + s), hf * 64,
                             bh * Nkrows + j * 128);
-          } else if (j < ngt) {
-            // global-KV list (or bridge candidates), gathered 4 rows per lane
-            const int g0 = j * 128 + lane * 4;
-            int r[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int p = g0 + i < nkv ? g0 + i : nkv - 1;
-              r[i] = bh * Nkrows + glist[p];
-            }
-            for (int hf = 0; hf < G::kHalves; ++hf)
-              tma_gather4(dst + hf * kHalfBytes + lane * 512, tm, bar(BAR_KV_FULL + s), hf * 64,
-                          r[0], r[1], r[2], r[3]);
           } else {
             // patch (px, py) of the Halo rectangle: kPH grid rows of kPW tokens
             if (lane == 0) {
@@ -616,12 +682,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (!published && !(ok = publish(unit_count + 1))) break;
       ++unit_count;
     }
-    // Drain: the most recent load of every stage has landed (bounded wait).
+    // Drain: the most recent load of every stage has landed (bounded wait),
+    // and no cp.async copy of this warp is still in flight.
     int drain_abort = 0;
     for (uint32_t k = 0; k < kStages && k < kv_it; ++k) {
       const uint32_t it = kv_it - 1 - k;
       warp_wait0(bar(BAR_KV_FULL + it % kStages), (it / kStages) & 1u, &drain_abort);
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -671,6 +739,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t k0 = kv_it;
         if (!(ok = mbar_wait(bar(BAR_KV_FULL + k0 % kStages), (k0 / kStages) & 1u, abort_flag)))
           break;
+        if (WINDOW) fence_proxy_async();        // queries and global-KV rows came by cp.async
         tc_fence_after();
         qk(tS0, q0s, kv_addr(k0));
         mma_commit(bar(BAR_S_FULL0));
@@ -685,6 +754,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const uint32_t kn = kv_it + 2 * j + 2;
           if (!(ok = mbar_wait(bar(BAR_KV_FULL + vi % kStages), (vi / kStages) & 1u, abort_flag)))
             break;
+          if (WINDOW) fence_proxy_async();
           if (!(ok = pv_parts(tO0, tS0, kv_addr(vi), j == 0, BAR_P_PART0, BAR_P_FULL0, p_cnt0)))
             break;
           ++p_cnt0;
@@ -693,6 +763,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (!(ok = mbar_wait(bar(BAR_KV_FULL + kn % kStages), (kn / kStages) & 1u,
                                  abort_flag)))
               break;
+            if (WINDOW) fence_proxy_async();
             tc_fence_after();
             qk(tS0, q0s, kv_addr(kn));
             mma_commit(bar(BAR_S_FULL0));
@@ -1153,6 +1224,9 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, c
   prm.R = R;
   prm.num_units = (int)(L.nitem_max * L.B * H);
   prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.k = static_cast<const __nv_bfloat16*>(k);
+  prm.v = static_cast<const __nv_bfloat16*>(v);
   prm.counters = static_cast<unsigned*>(ws);
   const int64_t hdr = window_ws_header_bytes(L.B, H);
   prm.acc = reinterpret_cast<float*>(static_cast<char*>(ws) + hdr);
