@@ -50,7 +50,8 @@ namespace {
 
 constexpr int kThreads = 320;     // producer, MMA issuer, 8 softmax warps
 constexpr int kSoftWarp0 = 2;     // first softmax warp
-constexpr int kStages = 4;               // K/V ring stages (32 KB each at head_dim 128)
+constexpr int kStages = 3;               // K/V ring stages (32 KB each at head_dim 128)
+constexpr int kQSlots = 2;               // query buffers: the next unit's loads during this one
 constexpr int kHalfBytes = 128 * 128;   // 128 rows x 64 bf16: one 128B-swizzled half tile
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
@@ -71,8 +72,8 @@ struct Geo {
   static_assert(D == 64 || D == 128, "head_dim");
   static constexpr int kHalves = D / 64;
   static constexpr int kTileBytes = kHalves * kHalfBytes;
-  static constexpr int kSmemQ = 0;
-  static constexpr int kSmemKV = 2 * kTileBytes;
+  static constexpr int kSmemQ = 0;                            // kQSlots x 2 query tiles
+  static constexpr int kSmemKV = kQSlots * 2 * kTileBytes;
   static constexpr int kSmemBar = kSmemKV + kStages * kTileBytes;
   static constexpr int kSmemBytes = kSmemBar + 256 + 1024;   // barriers + alignment slack
   static_assert(kSmemBytes + 1024 <= 227 * 1024, "shared memory of one CTA");
@@ -80,9 +81,9 @@ struct Geo {
 
 // barrier indices
 enum {
-  BAR_Q_FULL = 0,
-  BAR_Q_EMPTY,
-  BAR_S_FULL0, BAR_S_FULL1,
+  BAR_Q_FULL = 0,                    // kQSlots of them
+  BAR_Q_EMPTY = BAR_Q_FULL + kQSlots,
+  BAR_S_FULL0 = BAR_Q_EMPTY + kQSlots, BAR_S_FULL1,
   BAR_P_FULL0, BAR_P_FULL1,
   BAR_O_FULL0, BAR_O_FULL1,
   BAR_P_PART0,                       // kPParts - 1 per query tile: leading parts of P stored
@@ -181,6 +182,17 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// Four rows (of a 2-D map) gathered into consecutive rows of shared memory.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
+      "r"(r3)
       : "memory");
 }
 
@@ -515,8 +527,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
   if (threadIdx.x == 0) {
     s_abort = 0;
-    mbar_init(bar(BAR_Q_FULL), 1);
-    mbar_init(bar(BAR_Q_EMPTY), 1);
+    for (int q = 0; q < kQSlots; ++q) {
+      mbar_init(bar(BAR_Q_FULL + q), 1);
+      mbar_init(bar(BAR_Q_EMPTY + q), 1);
+    }
     mbar_init(bar(BAR_S_FULL0), 1);
     mbar_init(bar(BAR_S_FULL1), 1);
     mbar_init(bar(BAR_P_FULL0), 128);
@@ -584,34 +598,44 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       __syncwarp();
       return true;
     };
-    ok = publish(0);
-    while (ok) {
-      const UnitRec& R = s_rec[unit_count % kRecSlots];
-      if (!R.valid) break;
-      if (!warp_wait0(bar(BAR_Q_EMPTY), (unit_count & 1u) ^ 1u, abort_flag)) break;
-      const int nqt = R.one ? 1 : 2;          // query tiles of this unit
+    // Queries of this CTA's k-th unit into query slot k mod 2: issued while
+    // the previous unit still computes, so they are in place when it ends.
+    // Window queries (the rectangle enumerated row-major) come from DRAM
+    // once per unit: TMA gather4 keeps enough of them in flight, which a
+    // warp's cp.async stream does not.
+    auto load_q = [&](uint32_t k) -> bool {
+      const UnitRec& Rq = s_rec[k % kRecSlots];
+      if (!Rq.valid) return true;
+      const uint32_t qs = k % kQSlots;
+      if (!warp_wait0(bar(BAR_Q_EMPTY + qs), ((k / kQSlots) & 1u) ^ 1u, abort_flag)) return false;
+      const uint32_t qbase = sbase + G::kSmemQ + qs * 2 * G::kTileBytes;
+      const int nqt = Rq.one ? 1 : 2;
+      if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL + qs), nqt * G::kTileBytes);
+      __syncwarp();
       if constexpr (!WINDOW) {
-        if (lane == 0) {
-          mbar_arrive_tx(bar(BAR_Q_FULL), nqt * G::kTileBytes);
+        if (lane == 0)
           for (int t = 0; t < nqt; ++t)
             for (int hf = 0; hf < G::kHalves; ++hf)
-              tma_load_2d(sbase + G::kSmemQ + t * G::kTileBytes + hf * kHalfBytes, &tm_q,
-                          bar(BAR_Q_FULL), hf * 64, R.bh * Ntok + R.q0 + t * 128);
-        }
-        __syncwarp();
+              tma_load_2d(qbase + t * G::kTileBytes + hf * kHalfBytes, &tm_q, bar(BAR_Q_FULL + qs),
+                          hf * 64, Rq.bh * Ntok + Rq.q0 + t * 128);
       } else {
-        // window queries: the rectangle enumerated row-major, copied row by row
         for (int t = 0; t < nqt; ++t) {
           int r[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            r[i] = R.bh * Ntok + window_query_token(R.win, R.nq, R.q0 + t * 128 + lane * 4 + i, Wg);
-          cp_async_rows<D>(sbase + G::kSmemQ + t * G::kTileBytes, prm.q, r, lane);
+            r[i] = Rq.bh * Ntok +
+                   window_query_token(Rq.win, Rq.nq, Rq.q0 + t * 128 + lane * 4 + i, Wg);
+          for (int hf = 0; hf < G::kHalves; ++hf)
+            tma_gather4(qbase + t * G::kTileBytes + hf * kHalfBytes + lane * 512, &tm_q,
+                        bar(BAR_Q_FULL + qs), hf * 64, r[0], r[1], r[2], r[3]);
         }
-        cp_async_arrive(bar(BAR_Q_FULL));
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_Q_FULL));
       }
+      return true;
+    };
+    ok = publish(0) && load_q(0);
+    while (ok) {
+      const UnitRec& R = s_rec[unit_count % kRecSlots];
+      if (!R.valid) break;
       const int nt = R.nt, ngt = R.ngt, ntr = R.ntr, ncx = R.ncx, nkv = R.nkv;
       const int nti = ngt + ntr;
       const int bh = R.bh;
@@ -622,7 +646,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       for (int j = 0; j < nt && ok; ++j) {
         if (j == jn) {
           published = true;
-          if (!(ok = publish(unit_count + 1))) break;
+          if (!(ok = publish(unit_count + 1) && load_q(unit_count + 1))) break;
         }
         for (int kv = 0; kv < 2; ++kv) {       // K then V
           const int s = (int)(kv_it % kStages);
@@ -679,7 +703,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
       }
       if (!ok) break;
-      if (!published && !(ok = publish(unit_count + 1))) break;
+      if (!published && !(ok = publish(unit_count + 1) && load_q(unit_count + 1))) break;
       ++unit_count;
     }
     // Drain: the most recent load of every stage has landed (bounded wait),
@@ -696,7 +720,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       uint32_t kv_it = 0, unit_count = 0;
       uint32_t p_cnt0 = 0, p_cnt1 = 0;
       const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
-      const uint32_t q0s = sbase + G::kSmemQ, q1s = sbase + G::kSmemQ + G::kTileBytes;
+
       bool ok = true;
       auto kv_addr = [&](uint32_t it) { return sbase + G::kSmemKV + (it % kStages) * G::kTileBytes; };
       auto qk = [&](uint32_t d, uint32_t qs, uint32_t ks) {
@@ -734,7 +758,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const bool two = s_rec[slot].one == 0;   // query tile 1 runs too
         mbar_arrive(bar(BAR_REC_EMPTY + slot));
         if (!valid) break;
-        if (!(ok = mbar_wait(bar(BAR_Q_FULL), unit_count & 1u, abort_flag))) break;
+        const uint32_t qs = unit_count % kQSlots;
+        const uint32_t q0s = sbase + G::kSmemQ + qs * 2 * G::kTileBytes;
+        const uint32_t q1s = q0s + G::kTileBytes;
+        const uint32_t bQe = bar(BAR_Q_EMPTY + qs);
+        if (!(ok = mbar_wait(bar(BAR_Q_FULL + qs), (unit_count / kQSlots) & 1u, abort_flag))) break;
         // prologue: S(0)
         const uint32_t k0 = kv_it;
         if (!(ok = mbar_wait(bar(BAR_KV_FULL + k0 % kStages), (k0 / kStages) & 1u, abort_flag)))
@@ -748,7 +776,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           mma_commit(bar(BAR_S_FULL1));
         }
         mma_commit(bar(BAR_KV_EMPTY + k0 % kStages));
-        if (nt == 1) mma_commit(bar(BAR_Q_EMPTY));
+        if (nt == 1) mma_commit(bQe);
         for (int j = 0; j < nt && ok; ++j) {
           const uint32_t vi = kv_it + 2 * j + 1;
           const uint32_t kn = kv_it + 2 * j + 2;
@@ -769,7 +797,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mma_commit(bar(BAR_S_FULL0));
             if (!two) {                          // K(j+1) is done with after QK0
               mma_commit(bar(BAR_KV_EMPTY + kn % kStages));
-              if (j + 2 == nt) mma_commit(bar(BAR_Q_EMPTY));
+              if (j + 2 == nt) mma_commit(bQe);
             }
           }
           if (two) {
@@ -783,7 +811,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             qk(tS1, q1s, kv_addr(kn));
             mma_commit(bar(BAR_S_FULL1));
             mma_commit(bar(BAR_KV_EMPTY + kn % kStages));
-            if (j + 2 == nt) mma_commit(bar(BAR_Q_EMPTY));
+            if (j + 2 == nt) mma_commit(bQe);
           }
         }
         kv_it += 2 * nt;
