@@ -50,8 +50,8 @@ namespace {
 
 constexpr int kThreads = 320;     // producer, MMA issuer, 8 softmax warps
 constexpr int kSoftWarp0 = 2;     // first softmax warp
-constexpr int kStages = 3;               // K/V ring stages (32 KB each at head_dim 128)
-constexpr int kQSlots = 2;               // query buffers: the next unit's loads during this one
+constexpr int kStages = 4;               // K/V ring stages (32 KB each at head_dim 128)
+constexpr int kQSlots = 1;               // query buffers (a second one would cost a K/V stage)
 constexpr int kHalfBytes = 128 * 128;   // 128 rows x 64 bf16: one 128B-swizzled half tile
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
@@ -185,15 +185,10 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Four rows (of a 2-D map) gathered into consecutive rows of shared memory.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int c0, int r0, int r1, int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
-      "r"(r3)
-      : "memory");
+// Bulk prefetch of `bytes` contiguous bytes (a multiple of 16, 16-byte
+// aligned) from global memory into L2.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // 16 bytes global -> shared, asynchronous (L2 only), and the arrive-on of an
@@ -401,7 +396,8 @@ __device__ __forceinline__ int window_query_token(const int4& win, int nq, int p
 // warp instruction copies whole rows (256 or 128 contiguous bytes per row).
 // Gathered rows go this way rather than through tile::gather4, whose issue
 // rate (about 7 bytes per clock per SM, measured) made them the window
-// kernel's largest fixed cost.
+// kernel's largest fixed cost; rows not yet in L2 are prefetched first (a
+// warp's cp.async stream keeps too few DRAM reads in flight).
 template <int D>
 __device__ __forceinline__ void cp_async_rows(uint32_t dst, const __nv_bfloat16* base,
                                               const int (&r)[4], int lane) {
@@ -598,11 +594,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       __syncwarp();
       return true;
     };
-    // Queries of this CTA's k-th unit into query slot k mod 2: issued while
-    // the previous unit still computes, so they are in place when it ends.
-    // Window queries (the rectangle enumerated row-major) come from DRAM
-    // once per unit: TMA gather4 keeps enough of them in flight, which a
-    // warp's cp.async stream does not.
+    // Window queries of this CTA's k-th unit pulled into L2 ahead of time
+    // (issued when its record is published, a unit before it runs): one bulk
+    // prefetch per grid row of the window that its 256 queries touch.
+    auto prefetch_q = [&](uint32_t k) {
+      if constexpr (WINDOW) {
+        const UnitRec& Rq = s_rec[k % kRecSlots];
+        if (!Rq.valid) return;
+        const int wx = Rq.win.w;
+        const int p0 = Rq.q0, p1 = min(Rq.q0 + 256, Rq.nq) - 1;   // positions of the unit
+        const int r0 = p0 / wx, r1 = p1 / wx;
+        for (int r = r0 + lane; r <= r1; r += 32) {
+          const int xa = r == r0 ? p0 % wx : 0, xb = r == r1 ? p1 % wx : wx - 1;
+          const int64_t tok = (int64_t)Rq.bh * Ntok + (int64_t)(Rq.win.x + r) * Wg + Rq.win.y + xa;
+          prefetch_l2(prm.q + tok * D, (uint32_t)((xb - xa + 1) * D * 2));
+        }
+      }
+    };
+    // Queries of this CTA's k-th unit, once the previous unit's last QK has
+    // read the buffer.  Window queries (the rectangle enumerated row-major)
+    // are copied row by row with cp.async from L2, where prefetch_q put them.
     auto load_q = [&](uint32_t k) -> bool {
       const UnitRec& Rq = s_rec[k % kRecSlots];
       if (!Rq.valid) return true;
@@ -610,14 +621,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (!warp_wait0(bar(BAR_Q_EMPTY + qs), ((k / kQSlots) & 1u) ^ 1u, abort_flag)) return false;
       const uint32_t qbase = sbase + G::kSmemQ + qs * 2 * G::kTileBytes;
       const int nqt = Rq.one ? 1 : 2;
-      if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL + qs), nqt * G::kTileBytes);
-      __syncwarp();
       if constexpr (!WINDOW) {
-        if (lane == 0)
+        if (lane == 0) {
+          mbar_arrive_tx(bar(BAR_Q_FULL + qs), nqt * G::kTileBytes);
           for (int t = 0; t < nqt; ++t)
             for (int hf = 0; hf < G::kHalves; ++hf)
               tma_load_2d(qbase + t * G::kTileBytes + hf * kHalfBytes, &tm_q, bar(BAR_Q_FULL + qs),
                           hf * 64, Rq.bh * Ntok + Rq.q0 + t * 128);
+        }
+        __syncwarp();
       } else {
         for (int t = 0; t < nqt; ++t) {
           int r[4];
@@ -625,17 +637,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           for (int i = 0; i < 4; ++i)
             r[i] = Rq.bh * Ntok +
                    window_query_token(Rq.win, Rq.nq, Rq.q0 + t * 128 + lane * 4 + i, Wg);
-          for (int hf = 0; hf < G::kHalves; ++hf)
-            tma_gather4(qbase + t * G::kTileBytes + hf * kHalfBytes + lane * 512, &tm_q,
-                        bar(BAR_Q_FULL + qs), hf * 64, r[0], r[1], r[2], r[3]);
+          cp_async_rows<D>(qbase + t * G::kTileBytes, prm.q, r, lane);
         }
+        cp_async_arrive(bar(BAR_Q_FULL + qs));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_Q_FULL + qs));
       }
       return true;
     };
-    ok = publish(0) && load_q(0);
+    ok = publish(0);
+    if (ok) prefetch_q(0);
     while (ok) {
       const UnitRec& R = s_rec[unit_count % kRecSlots];
       if (!R.valid) break;
+      if (!(ok = load_q(unit_count))) break;
       const int nt = R.nt, ngt = R.ngt, ntr = R.ntr, ncx = R.ncx, nkv = R.nkv;
       const int nti = ngt + ntr;
       const int bh = R.bh;
@@ -646,7 +661,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       for (int j = 0; j < nt && ok; ++j) {
         if (j == jn) {
           published = true;
-          if (!(ok = publish(unit_count + 1) && load_q(unit_count + 1))) break;
+          if (!(ok = publish(unit_count + 1))) break;
+          prefetch_q(unit_count + 1);
         }
         for (int kv = 0; kv < 2; ++kv) {       // K then V
           const int s = (int)(kv_it % kStages);
@@ -703,7 +719,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
       }
       if (!ok) break;
-      if (!published && !(ok = publish(unit_count + 1) && load_q(unit_count + 1))) break;
+      if (!published) {
+        if (!(ok = publish(unit_count + 1))) break;
+        prefetch_q(unit_count + 1);
+      }
       ++unit_count;
     }
     // Drain: the most recent load of every stage has landed (bounded wait),
