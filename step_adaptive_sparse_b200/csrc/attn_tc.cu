@@ -50,6 +50,15 @@ namespace {
 
 constexpr int kThreads = 320;     // producer, MMA issuer, 8 softmax warps
 constexpr int kSoftWarp0 = 2;     // first softmax warp
+#ifndef AREA_Q_GATHER4
+#define AREA_Q_GATHER4 0
+#endif
+#ifndef AREA_G_GATHER4
+#define AREA_G_GATHER4 0
+#endif
+#ifndef AREA_ORDER
+#define AREA_ORDER 2
+#endif
 constexpr int kStages = 4;               // K/V ring stages (32 KB each at head_dim 128)
 constexpr int kQSlots = 1;               // query buffers (a second one would cost a K/V stage)
 constexpr int kHalfBytes = 128 * 128;   // 128 rows x 64 bf16: one 128B-swizzled half tile
@@ -182,6 +191,17 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// Four rows (of a 2-D map) gathered into consecutive rows of shared memory.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int r0, int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
+      "r"(r3)
       : "memory");
 }
 
@@ -421,6 +441,8 @@ __device__ __forceinline__ void cp_async_rows(uint32_t dst, const __nv_bfloat16*
   }
 }
 
+__device__ bool fill_window_unit(int b, int h, int idx, const TcParams& prm, UnitRec& r);
+
 // Decode unit u into a record (producer lane 0).  Dense: (b*H + h, 256-query
 // block), head-major.  Window: per batch element, the (head, parity class)
 // groups of work items run skewed: at step t = 0, 1, ... come head t's
@@ -452,6 +474,31 @@ __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
   }
   const PlanView& P = prm.P;
   int rem = u;
+  if (AREA_ORDER == 0) {      // class-major over all heads
+    for (int c = 0; c < 4; ++c)
+      for (int b = 0; b < P.B; ++b) {
+        const int n = P.nclass[b * 4 + c];
+        if (rem >= n * prm.H) {
+          rem -= n * prm.H;
+          continue;
+        }
+        int coff = 0;
+        for (int c2 = 0; c2 < c; ++c2) coff += P.nclass[b * 4 + c2];
+        return fill_window_unit(b, rem / n, coff + rem % n, prm, r);
+      }
+    return false;
+  }
+  if (AREA_ORDER == 1) {      // head-major, a head's classes back to back
+    for (int b = 0; b < P.B; ++b) {
+      const int n = P.nitem[b];
+      if (rem >= n * prm.H) {
+        rem -= n * prm.H;
+        continue;
+      }
+      return fill_window_unit(b, rem / n, rem % n, prm, r);
+    }
+    return false;
+  }
   for (int b = 0; b < P.B; ++b) {
     const int cnt = P.nitem[b] * prm.H;
     if (rem >= cnt) {
@@ -476,6 +523,15 @@ __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
       }
     }
     if (h < 0) return false;
+    return fill_window_unit(b, h, idx, prm, r);
+  }
+  return false;
+}
+
+// The record of work item idx of batch element b for head h.
+__device__ bool fill_window_unit(int b, int h, int idx, const TcParams& prm, UnitRec& r) {
+  const PlanView& P = prm.P;
+  {
     const int2 it = P.items[(int64_t)b * P.nitem_max + idx];
     const int64_t wo = (int64_t)b * P.nw + it.x;
     r.b = b;
@@ -598,7 +654,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // (issued when its record is published, a unit before it runs): one bulk
     // prefetch per grid row of the window that its 256 queries touch.
     auto prefetch_q = [&](uint32_t k) {
-      if constexpr (WINDOW) {
+      if constexpr (WINDOW && !AREA_Q_GATHER4) {
         const UnitRec& Rq = s_rec[k % kRecSlots];
         if (!Rq.valid) return;
         const int wx = Rq.win.w;
@@ -630,6 +686,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                           hf * 64, Rq.bh * Ntok + Rq.q0 + t * 128);
         }
         __syncwarp();
+      } else if (AREA_Q_GATHER4) {
+        if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL + qs), nqt * G::kTileBytes);
+        __syncwarp();
+        for (int t = 0; t < nqt; ++t) {
+          int r[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            r[i] = Rq.bh * Ntok +
+                   window_query_token(Rq.win, Rq.nq, Rq.q0 + t * 128 + lane * 4 + i, Wg);
+          for (int hf = 0; hf < G::kHalves; ++hf)
+            tma_gather4(qbase + t * G::kTileBytes + hf * kHalfBytes + lane * 512, &tm_q,
+                        bar(BAR_Q_FULL + qs), hf * 64, r[0], r[1], r[2], r[3]);
+        }
       } else {
         for (int t = 0; t < nqt; ++t) {
           int r[4];
@@ -672,6 +741,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
           const CUtensorMap* tm = kv ? &tm_v : &tm_k;
           const uint32_t dst = sbase + G::kSmemKV + s * G::kTileBytes;
+          if (WINDOW && j < ngt && AREA_G_GATHER4) {
+            const int g0 = j * 128 + lane * 4;
+            int r[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int p = g0 + i < nkv ? g0 + i : nkv - 1;
+              r[i] = bh * Nkrows + glist[p];
+            }
+            if (lane == 0) mbar_arrive_tx(bar(BAR_KV_FULL + s), G::kTileBytes);
+            __syncwarp();
+            for (int hf = 0; hf < G::kHalves; ++hf)
+              tma_gather4(dst + hf * kHalfBytes + lane * 512, tm, bar(BAR_KV_FULL + s), hf * 64,
+                          r[0], r[1], r[2], r[3]);
+            ++kv_it;
+            continue;
+          }
           if (WINDOW && j < ngt) {
             // global-KV list (or bridge candidates), copied row by row
             const int g0 = j * 128 + lane * 4;
