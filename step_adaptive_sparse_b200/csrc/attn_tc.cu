@@ -50,15 +50,6 @@ namespace {
 
 constexpr int kThreads = 320;     // producer, MMA issuer, 8 softmax warps
 constexpr int kSoftWarp0 = 2;     // first softmax warp
-#ifndef AREA_Q_GATHER4
-#define AREA_Q_GATHER4 0
-#endif
-#ifndef AREA_G_GATHER4
-#define AREA_G_GATHER4 0
-#endif
-#ifndef AREA_ORDER
-#define AREA_ORDER 2
-#endif
 constexpr int kStages = 4;               // K/V ring stages (32 KB each at head_dim 128)
 constexpr int kQSlots = 1;               // query buffers (a second one would cost a K/V stage)
 constexpr int kHalfBytes = 128 * 128;   // 128 rows x 64 bf16: one 128B-swizzled half tile
@@ -203,12 +194,6 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2),
       "r"(r3)
       : "memory");
-}
-
-// Bulk prefetch of `bytes` contiguous bytes (a multiple of 16, 16-byte
-// aligned) from global memory into L2.
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // 16 bytes global -> shared, asynchronous (L2 only), and the arrive-on of an
@@ -395,7 +380,7 @@ struct TcParams {
   DenseArgs da;
   PlanView P;
   __nv_bfloat16* o;   // output
-  const __nv_bfloat16 *q, *k, *v;   // window: the inputs, for rows copied with cp.async
+  const __nv_bfloat16 *k, *v;       // window: keys and values, for rows copied with cp.async
   unsigned* counters; // window: workspace header (unit counter, per-class completions)
   float* acc;         // window: fp32 accumulator rows [B*H][n_ov][128]
   int nx2;            // window: columns covered by two base windows
@@ -414,10 +399,11 @@ __device__ __forceinline__ int window_query_token(const int4& win, int nq, int p
 // its 16-byte chunk c at ((c ^ (R mod 8)) * 16).  Lane l holds the source
 // rows of tile rows 4l .. 4l + 3 in r[0..3] (row indices of `base`).  Each
 // warp instruction copies whole rows (256 or 128 contiguous bytes per row).
-// Gathered rows go this way rather than through tile::gather4, whose issue
-// rate (about 7 bytes per clock per SM, measured) made them the window
-// kernel's largest fixed cost; rows not yet in L2 are prefetched first (a
-// warp's cp.async stream keeps too few DRAM reads in flight).
+// Gathered global-KV rows go this way rather than through tile::gather4,
+// whose issue rate (about 7 bytes per clock per SM, measured) made them the
+// window kernel's largest fixed cost.  Used for rows that are mostly in L2
+// (the global-KV lists); for rows read from DRAM a warp's cp.async stream
+// keeps too few reads in flight, and TMA gather4 does better.
 template <int D>
 __device__ __forceinline__ void cp_async_rows(uint32_t dst, const __nv_bfloat16* base,
                                               const int (&r)[4], int lane) {
@@ -441,17 +427,37 @@ __device__ __forceinline__ void cp_async_rows(uint32_t dst, const __nv_bfloat16*
   }
 }
 
-__device__ bool fill_window_unit(int b, int h, int idx, const TcParams& prm, UnitRec& r);
+// The record of work item idx of batch element b for head h.
+__device__ void fill_window_unit(int b, int h, int idx, const TcParams& prm, UnitRec& r) {
+  const PlanView& P = prm.P;
+  const int2 it = P.items[(int64_t)b * P.nitem_max + idx];
+  const int64_t wo = (int64_t)b * P.nw + it.x;
+  r.b = b;
+  r.bh = b * prm.H + h;
+  r.win = P.win[wo];
+  r.ext = P.ext[wo];
+  const int parent = P.parent[wo];
+  r.cls = window_class(parent, P.nbx);
+  r.my = axis_merge(parent / P.nbx, P.nby, P.Hg, P.hy, P.sy);
+  r.mx = axis_merge(parent % P.nbx, P.nbx, P.Wg, P.wx, P.sx);
+  r.q0 = it.y * 256;
+  r.nq = r.win.z * r.win.w;
+  r.one = r.nq - r.q0 <= 128;
+  r.nkv = prm.cand ? prm.R : P.gcount[wo];
+  r.ngt = (r.nkv + 127) / 128;
+  r.ncx = (r.ext.w + kPW - 1) / kPW;
+  r.ntr = r.ncx * ((r.ext.z + kPH - 1) / kPH);
+  r.nt = r.ngt + r.ntr + (prm.T + 127) / 128;
+  r.glist = prm.cand ? (long long)r.bh * prm.R : (long long)wo * P.G;
+}
 
 // Decode unit u into a record (producer lane 0).  Dense: (b*H + h, 256-query
-// block), head-major.  Window: per batch element, the (head, parity class)
-// groups of work items run skewed: at step t = 0, 1, ... come head t's
-// class 0, head t-1's class 1, head t-2's class 2 and head t-3's class 3,
-// each group's items in plan order.  A head's classes thus run in order, its
-// accumulator rows are re-read a few groups after they were written (still
-// in L2), and three other groups lie between a class and the next class of
-// the same head, so the units of the earlier class have usually completed
-// by the time the later class needs them.
+// block), head-major.  Window: by parity class, then batch element, then
+// head, then the class's work items in plan order (unsplit windows first,
+// costliest first).  A class's units all come before the next class's, so a
+// unit merging into an overlapped token rarely waits for the earlier class;
+// with few units per head a head-by-head order made the classes wait on each
+// other (measured), so the order is class-major over all heads.
 template <bool WINDOW>
 __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
   r.valid = 1;
@@ -474,88 +480,20 @@ __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
   }
   const PlanView& P = prm.P;
   int rem = u;
-  if (AREA_ORDER == 0) {      // class-major over all heads
-    for (int c = 0; c < 4; ++c)
-      for (int b = 0; b < P.B; ++b) {
-        const int n = P.nclass[b * 4 + c];
-        if (rem >= n * prm.H) {
-          rem -= n * prm.H;
-          continue;
-        }
-        int coff = 0;
-        for (int c2 = 0; c2 < c; ++c2) coff += P.nclass[b * 4 + c2];
-        return fill_window_unit(b, rem / n, coff + rem % n, prm, r);
-      }
-    return false;
-  }
-  if (AREA_ORDER == 1) {      // head-major, a head's classes back to back
+  for (int c = 0; c < 4; ++c)
     for (int b = 0; b < P.B; ++b) {
-      const int n = P.nitem[b];
+      const int n = P.nclass[b * 4 + c];
       if (rem >= n * prm.H) {
         rem -= n * prm.H;
         continue;
       }
-      return fill_window_unit(b, rem / n, rem % n, prm, r);
+      int coff = 0;                          // the class's first item (items are class by class)
+      for (int c2 = 0; c2 < c; ++c2) coff += P.nclass[b * 4 + c2];
+      fill_window_unit(b, rem / n, coff + rem % n, prm, r);
+      return true;
     }
-    return false;
-  }
-  for (int b = 0; b < P.B; ++b) {
-    const int cnt = P.nitem[b] * prm.H;
-    if (rem >= cnt) {
-      rem -= cnt;
-      continue;
-    }
-    // items per class; the items are stored class by class
-    const int n0 = P.nclass[b * 4 + 0], n1 = P.nclass[b * 4 + 1];
-    const int n2 = P.nclass[b * 4 + 2], n3 = P.nclass[b * 4 + 3];
-    int h = -1, idx = 0;
-    for (int t = 0; t < prm.H + 3 && h < 0; ++t) {
-      for (int c = 0; c < 4; ++c) {
-        const int hh = t - c;
-        if (hh < 0 || hh >= prm.H) continue;
-        const int nc = c == 0 ? n0 : c == 1 ? n1 : c == 2 ? n2 : n3;
-        if (rem < nc) {
-          h = hh;
-          idx = rem + (c > 0 ? n0 : 0) + (c > 1 ? n1 : 0) + (c > 2 ? n2 : 0);
-          break;
-        }
-        rem -= nc;
-      }
-    }
-    if (h < 0) return false;
-    return fill_window_unit(b, h, idx, prm, r);
-  }
   return false;
 }
-
-// The record of work item idx of batch element b for head h.
-__device__ bool fill_window_unit(int b, int h, int idx, const TcParams& prm, UnitRec& r) {
-  const PlanView& P = prm.P;
-  {
-    const int2 it = P.items[(int64_t)b * P.nitem_max + idx];
-    const int64_t wo = (int64_t)b * P.nw + it.x;
-    r.b = b;
-    r.bh = b * prm.H + h;
-    r.win = P.win[wo];
-    r.ext = P.ext[wo];
-    const int parent = P.parent[wo];
-    r.cls = window_class(parent, P.nbx);
-    r.my = axis_merge(parent / P.nbx, P.nby, P.Hg, P.hy, P.sy);
-    r.mx = axis_merge(parent % P.nbx, P.nbx, P.Wg, P.wx, P.sx);
-    r.q0 = it.y * 256;
-    r.nq = r.win.z * r.win.w;
-    r.one = r.nq - r.q0 <= 128;
-    r.nkv = prm.cand ? prm.R : P.gcount[wo];
-    r.ngt = (r.nkv + 127) / 128;
-    r.ncx = (r.ext.w + kPW - 1) / kPW;
-    r.ntr = r.ncx * ((r.ext.z + kPH - 1) / kPH);
-    r.nt = r.ngt + r.ntr + (prm.T + 127) / 128;
-    r.glist = prm.cand ? (long long)r.bh * prm.R : (long long)wo * P.G;
-    return true;
-  }
-  return false;
-}
-
 
 template <bool WINDOW, bool BRIDGE, int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -650,26 +588,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       __syncwarp();
       return true;
     };
-    // Window queries of this CTA's k-th unit pulled into L2 ahead of time
-    // (issued when its record is published, a unit before it runs): one bulk
-    // prefetch per grid row of the window that its 256 queries touch.
-    auto prefetch_q = [&](uint32_t k) {
-      if constexpr (WINDOW && !AREA_Q_GATHER4) {
-        const UnitRec& Rq = s_rec[k % kRecSlots];
-        if (!Rq.valid) return;
-        const int wx = Rq.win.w;
-        const int p0 = Rq.q0, p1 = min(Rq.q0 + 256, Rq.nq) - 1;   // positions of the unit
-        const int r0 = p0 / wx, r1 = p1 / wx;
-        for (int r = r0 + lane; r <= r1; r += 32) {
-          const int xa = r == r0 ? p0 % wx : 0, xb = r == r1 ? p1 % wx : wx - 1;
-          const int64_t tok = (int64_t)Rq.bh * Ntok + (int64_t)(Rq.win.x + r) * Wg + Rq.win.y + xa;
-          prefetch_l2(prm.q + tok * D, (uint32_t)((xb - xa + 1) * D * 2));
-        }
-      }
-    };
     // Queries of this CTA's k-th unit, once the previous unit's last QK has
-    // read the buffer.  Window queries (the rectangle enumerated row-major)
-    // are copied row by row with cp.async from L2, where prefetch_q put them.
+    // read the buffer.  Window queries (the rectangle enumerated row-major,
+    // read from DRAM once per unit) are gathered by TMA, 4 rows per lane:
+    // a warp's cp.async stream issued them about 7x slower (measured).
     auto load_q = [&](uint32_t k) -> bool {
       const UnitRec& Rq = s_rec[k % kRecSlots];
       if (!Rq.valid) return true;
@@ -686,7 +608,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                           hf * 64, Rq.bh * Ntok + Rq.q0 + t * 128);
         }
         __syncwarp();
-      } else if (AREA_Q_GATHER4) {
+      } else {
         if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL + qs), nqt * G::kTileBytes);
         __syncwarp();
         for (int t = 0; t < nqt; ++t) {
@@ -699,23 +621,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tma_gather4(qbase + t * G::kTileBytes + hf * kHalfBytes + lane * 512, &tm_q,
                         bar(BAR_Q_FULL + qs), hf * 64, r[0], r[1], r[2], r[3]);
         }
-      } else {
-        for (int t = 0; t < nqt; ++t) {
-          int r[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            r[i] = Rq.bh * Ntok +
-                   window_query_token(Rq.win, Rq.nq, Rq.q0 + t * 128 + lane * 4 + i, Wg);
-          cp_async_rows<D>(qbase + t * G::kTileBytes, prm.q, r, lane);
-        }
-        cp_async_arrive(bar(BAR_Q_FULL + qs));
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_Q_FULL + qs));
       }
       return true;
     };
     ok = publish(0);
-    if (ok) prefetch_q(0);
     while (ok) {
       const UnitRec& R = s_rec[unit_count % kRecSlots];
       if (!R.valid) break;
@@ -731,7 +640,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (j == jn) {
           published = true;
           if (!(ok = publish(unit_count + 1))) break;
-          prefetch_q(unit_count + 1);
         }
         for (int kv = 0; kv < 2; ++kv) {       // K then V
           const int s = (int)(kv_it % kStages);
@@ -741,24 +649,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
           const CUtensorMap* tm = kv ? &tm_v : &tm_k;
           const uint32_t dst = sbase + G::kSmemKV + s * G::kTileBytes;
-          if (WINDOW && j < ngt && AREA_G_GATHER4) {
-            const int g0 = j * 128 + lane * 4;
-            int r[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int p = g0 + i < nkv ? g0 + i : nkv - 1;
-              r[i] = bh * Nkrows + glist[p];
-            }
-            if (lane == 0) mbar_arrive_tx(bar(BAR_KV_FULL + s), G::kTileBytes);
-            __syncwarp();
-            for (int hf = 0; hf < G::kHalves; ++hf)
-              tma_gather4(dst + hf * kHalfBytes + lane * 512, tm, bar(BAR_KV_FULL + s), hf * 64,
-                          r[0], r[1], r[2], r[3]);
-            ++kv_it;
-            continue;
-          }
           if (WINDOW && j < ngt) {
-            // global-KV list (or bridge candidates), copied row by row
+            // global-KV list (or bridge candidates), copied row by row: the
+            // rows of a head's list serve all its windows and sit in L2, and
+            // from L2 cp.async beats TMA gather4 by about 4x (measured)
             const int g0 = j * 128 + lane * 4;
             int r[4];
 #pragma unroll
@@ -804,10 +698,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
       }
       if (!ok) break;
-      if (!published) {
-        if (!(ok = publish(unit_count + 1))) break;
-        prefetch_q(unit_count + 1);
-      }
+      if (!published && !(ok = publish(unit_count + 1))) break;
       ++unit_count;
     }
     // Drain: the most recent load of every stage has landed (bounded wait),
@@ -1356,7 +1247,6 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, c
   prm.R = R;
   prm.num_units = (int)(L.nitem_max * L.B * H);
   prm.o = static_cast<__nv_bfloat16*>(o);
-  prm.q = static_cast<const __nv_bfloat16*>(q);
   prm.k = static_cast<const __nv_bfloat16*>(k);
   prm.v = static_cast<const __nv_bfloat16*>(v);
   prm.counters = static_cast<unsigned*>(ws);
