@@ -36,7 +36,7 @@ if ROOT not in sys.path:
 
 METRIC = "AReA attention TFLOP/s per schedule step (bf16, 1 B200)"
 # Bumped whenever attn_tc.cu changes, so that stale DRAM counters are not reported.
-KERNEL_REVISION = "attn_tc r10 (unit records in a shared-memory ring, dynamic window units in parity-class order, global-KV tiles first, merge in class order without atomics)"
+KERNEL_REVISION = "attn_tc v11 (class-major dynamic window units, window queries by TMA gather4, global-KV rows by cp.async, per-(b,h,class) merge counters, single-tile units)"
 DEFAULT_CONFIG = "flux6144"
 
 
