@@ -38,7 +38,8 @@
  *     reports argument validation and launch errors only; AREA_ECUDA carries
  *     the CUDA error, see area_status_string.  The schedule functions at the
  *     end are host arithmetic (no device memory, no stream).
- *   - Device pointers passed to the attention calls must be 16-byte aligned.
+ *   - Device pointers passed to the attention calls must be 16-byte aligned;
+ *     their outputs (o) and the window workspace (ws) 32-byte aligned.
  */
 #ifndef AREA_H_
 #define AREA_H_
@@ -317,7 +318,7 @@ int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D,
  *   q, k, v, o : [B, H, Hg*Wg, D] (dtype)
  *   cfg, plan  : the configuration and buffer given to area_window_plan
  *   ws         : workspace of ws_bytes >= area_window_attn_ws_bytes(),
- *                16-byte aligned; contents on entry are ignored, on exit
+ *                32-byte aligned; contents on entry are ignored, on exit
  *                unspecified.  The call resets its counter header (a memset
  *                on the stream) before the kernel.
  * Merge order: a token covered by several windows is summed over them in a

@@ -22,6 +22,9 @@ using area::fail_cuda;
 int finish(cudaError_t e) { return e == cudaSuccess ? AREA_OK : fail_cuda(e); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+// outputs and the merge workspace are written 32 bytes (one L2 sector) per
+// thread and instruction
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31) == 0; }
 
 bool valid_dtype(int dtype) { return dtype == AREA_DTYPE_F32 || dtype == AREA_DTYPE_BF16; }
 
@@ -32,7 +35,7 @@ int check_attn(const void* q, const void* k, const void* v, const void* o, int B
   if (B < 1 || H < 1 || N < 1 || Nk < 1) return AREA_EINVAL;
   if (!valid_dtype(dtype)) return AREA_EUNSUPPORTED;
   if (D != 64 && D != 128) return AREA_EUNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return AREA_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned32(o)) return AREA_EINVAL;
   if ((int64_t)B * H > 65535 * 64) return AREA_EINVAL;
   return AREA_OK;
 }
@@ -64,7 +67,7 @@ int window_attn(const void* q, const void* k, const void* v, const void* kt, con
   if (cand && R < 1) return AREA_EINVAL;
   if (plan_bytes < (size_t)L.total) return AREA_ENOSPACE;
   if (ws_bytes < (size_t)area::window_ws_bytes(L, H, D)) return AREA_ENOSPACE;
-  if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(plan) & 255) != 0) return AREA_EINVAL;
+  if (!aligned32(ws) || (reinterpret_cast<uintptr_t>(plan) & 255) != 0) return AREA_EINVAL;
   if (H > 65535 || L.B > 65535) return AREA_EINVAL;
   if (dtype == AREA_DTYPE_BF16)       // tensor cores, head_dim 64 or 128
     return finish(area::launch_window_attn_tc(q, k, v, kt, vt, T, cand, R, L, plan, o, ws, H, D,

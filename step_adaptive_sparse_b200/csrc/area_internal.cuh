@@ -168,6 +168,73 @@ __host__ __device__ inline MergeRole merge_role(int y, int x, int cls, int4 my, 
   return r;
 }
 
+// Window keys: the Halo rectangle is covered by full patches of kPW x kPH
+// grid tokens (one 128-key tile, one 3-D tiled TMA box per 64-column half),
+// and its right and bottom strips left over by the patches by cells of
+// kCW x kCH tokens, kCells cells per tile, one box each (the tokens of one
+// grid row are contiguous).  Only the last tile of a rectangle whose sides
+// are multiples of 4 has unused rows.  Patches alone (16 x 8, masked at the
+// edges) computed 6% more (query, key) pairs than valid ones over the
+// FLUX-shaped 6144^2 schedule and 21% more at 2048^2; cells alone cost TMA
+// throughput (8 boxes per half tile: 11% slower tiles on a 256 x 256 window,
+// measured).  Queries of a window whose sides are multiples of 4 come in
+// cells too; other windows' queries are gathered row by row.  The global-KV
+// list is copied row by row.
+constexpr int kPW = 16, kPH = 8;
+constexpr int kCW = 4, kCH = 4;
+constexpr int kCellKeys = kCW * kCH;         // rows of one cell
+constexpr int kCells = 128 / kCellKeys;      // cells per tile
+static_assert(kPW * kPH == 128 && kPW % kCW == 0 && kPH % kCH == 0, "patch of whole cells");
+
+// Tiling of a Halo rectangle of eh x ew tokens: npx x npy patches (row-major),
+// then the cells of the right strip (x >= kPW * npx, all rows; c1x per row)
+// and of the bottom strip (x < kPW * npx, y >= kPH * npy; c2x per row).
+struct RectTiling {
+  int npx, npy, npatch;   // patches per row, patch rows, patches (= patch tiles)
+  int c1x, n1;            // right strip: cells per row, cells
+  int c2x;                // bottom strip: cells per row
+  int ncell;              // cells of both strips
+};
+__host__ __device__ __forceinline__ RectTiling rect_tiling(int eh, int ew) {
+  RectTiling t;
+  t.npx = ew / kPW;
+  t.npy = eh / kPH;
+  t.npatch = t.npx * t.npy;
+  t.c1x = (ew - kPW * t.npx + kCW - 1) / kCW;
+  t.n1 = t.c1x * ((eh + kCH - 1) / kCH);
+  t.c2x = kPW * t.npx / kCW;
+  t.ncell = t.n1 + t.c2x * ((eh - kPH * t.npy + kCH - 1) / kCH);
+  return t;
+}
+// Rectangle tiles: the patches, then the cells kCells by kCells.
+__host__ __device__ __forceinline__ int rect_tiles(const RectTiling& t) {
+  return t.npatch + (t.ncell + kCells - 1) / kCells;
+}
+// Offset (y, x) inside the rectangle of the top-left token of strip cell c.
+__host__ __device__ __forceinline__ int2 strip_cell(const RectTiling& t, int c) {
+  if (c < t.n1) return make_int2((c / t.c1x) * kCH, kPW * t.npx + (c % t.c1x) * kCW);
+  c -= t.n1;
+  return make_int2(kPH * t.npy + (c / t.c2x) * kCH, (c % t.c2x) * kCW);
+}
+
+// Cells per row of a window (y0, x0, hy, wx) whose queries are taken in cells
+// (both sides multiples of the cell's), else 0: its queries are row-major.
+__host__ __device__ __forceinline__ int query_cells_per_row(int4 win) {
+  return (win.z % kCH == 0 && win.w % kCW == 0) ? win.w / kCW : 0;
+}
+// Query token of position p of a window (positions past nq read position 0).
+// With qcx > 0 the window is enumerated cell by cell (cells row-major, qcx per
+// row; inside a cell row-major), else row-major.
+__host__ __device__ __forceinline__ int window_query_token(const int4& win, int qcx, int nq, int p,
+                                                  int Wg) {
+  if (p >= nq) p = 0;
+  if (qcx > 0) {
+    const int c = p / kCellKeys, k = p % kCellKeys;
+    return (win.x + (c / qcx) * kCH + k / kCW) * Wg + win.y + (c % qcx) * kCW + k % kCW;
+  }
+  return (win.x + p / win.w) * Wg + win.y + p % win.w;
+}
+
 // Window-attention workspace: a header of uint32 counters (the dynamic unit
 // counter, then one completion counter per (element, head, parity class)),
 // rounded up to 256 bytes, then one fp32 accumulator row per (element, head,

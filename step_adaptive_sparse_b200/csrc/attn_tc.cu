@@ -17,10 +17,10 @@
 //               128 dims, 128B-swizzled, 32 KB each).  Dense rows use tiled
 //               2-D loads.  Window keys are the global-KV list first (rows
 //               copied with 16-byte cp.async by the 32 producer lanes), then
-//               the Halo rectangle covered by 16x8-token patches (one 3-D
-//               tiled box each, masked at the rectangle's right and bottom
-//               edges); window queries (the rectangle enumerated row-major)
-//               are copied row by row with cp.async too.
+//               the Halo rectangle in 4x4-token cells (one 3-D tiled box per
+//               cell, 8 cells per tile, loaded by 8 lanes); window queries
+//               come in cells too when the window's sides are multiples of 4,
+//               else row by row by TMA gather4.
 //   warp 1      TMEM allocator and the single MMA-issuing thread.
 //   warps 2-5   softmax of query tile 0, warps 6-9 of query tile 1: each
 //               thread owns one query row (TMEM lane 32*(warp mod 4) + lane).
@@ -57,10 +57,11 @@ constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr int kMaxChains = 8;                // independent partial maxima of a score row
 constexpr int kPParts = 2;                   // P handed to the PV product in this many parts
-// Window keys: the Halo rectangle is covered by patches of kPW x kPH tokens,
-// one 128-key tile each, loaded by a 3-D tiled TMA box (tokens of one grid
-// row are contiguous).  Only the global-KV list is gathered row by row.
-constexpr int kPW = 16, kPH = 8;
+// Window keys and queries: patches and cells of the token grid (kPW x kPH,
+// kCW x kCH; rect_tiling and window_query_token in area_internal.cuh).  A
+// cell of one 64-column half takes kCellBytes of shared memory.
+constexpr int kCellBytes = kCellKeys * 128;
+static_assert(kCells <= 32 && kCellBytes % 1024 == 0, "cells: one lane each, whole swizzle atoms");
 constexpr int kRecSlots = 3;                 // unit records in flight (shared-memory ring)
 
 // Tile geometry for head_dim D (64 or 128): a tile is 128 rows of D bf16,
@@ -202,6 +203,25 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map
 // complete before the copies).
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// 32-byte global accesses (sm_100): a thread moves one whole L2 sector per
+// instruction.  The addresses must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]),
+               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+__device__ __forceinline__ void st_global_v8f(float* p, const float* f) {
+  asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "f"(f[0]),
+               "f"(f[1]), "f"(f[2]), "f"(f[3]), "f"(f[4]), "f"(f[5]), "f"(f[6]), "f"(f[7])
+               : "memory");
+}
+__device__ __forceinline__ void ld_global_v8f(const float* p, float* f) {
+  asm volatile("ld.global.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3]), "=f"(f[4]), "=f"(f[5]),
+                 "=f"(f[6]), "=f"(f[7])
+               : "l"(p)
+               : "memory");
 }
 __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
@@ -353,22 +373,33 @@ struct DenseArgs {
 };
 
 struct UnitRec {
+  int4 win, ext;      // window: the window and its Halo rectangle (y0, x0, hy, wx)
+  int4 my, mx;        // window: merge geometry of the base window per axis (axis_merge)
+  long long glist;    // window: element offset of the global list in the plan or cand
   int valid;          // 0: no more work for this CTA
   int bh, b;
   int q0;             // first query position of tile 0 (tile 1 = q0 + 128)
   int nq;             // valid query positions (dense: N; window: its area)
   int nkv;            // keys of the leading list tiles (dense keys, or global-KV count)
   int ngt;            // leading list tiles (dense key tiles, or global-KV tiles)
-  int ntr;            // window: Halo-rectangle patch tiles, after the list tiles
-  int ncx;            // window: patches per row of the Halo rectangle
+  int ntr;            // window: Halo-rectangle tiles, after the list tiles
+  int qcx;            // window: cells per row of the window when its queries come
+                      // in cells (sides multiples of kCH, kCW), else 0
   int nt;             // all key tiles of the unit, text tiles included
   int cls;            // window: parity class of the base window
   int one;            // 1: at most 128 valid queries, only query tile 0 runs
-  int4 win, ext;      // window: the window and its Halo rectangle (y0, x0, hy, wx)
-  int4 my, mx;        // window: merge geometry of the base window per axis (axis_merge)
-  long long glist;    // window: element offset of the global list in the plan or cand
 };
 static_assert(sizeof(UnitRec) <= 128, "unit record");
+
+// Tensor maps of one launch (bf16, 128B swizzle, boxes of 64 head dims).
+struct TcMaps {
+  CUtensorMap q;        // queries [rows, D]: 128-row box (dense), 1-row box (window gather4)
+  CUtensorMap qc;       // window queries [B*H*Hg, Wg, D]: one cell
+  CUtensorMap k, v;     // dense keys and values [rows, D]: 128-row box
+  CUtensorMap kp, vp;   // window keys and values [B*H*Hg, Wg, D]: one patch
+  CUtensorMap kc, vc;   // window keys and values [B*H*Hg, Wg, D]: one cell
+  CUtensorMap kt, vt;   // text keys and values [B*H*T, D]: 128-row box
+};
 
 struct TcParams {
   float scale_log2;
@@ -387,11 +418,6 @@ struct TcParams {
   long long n_ov;     // window: overlapped tokens per element
 };
 
-// Query token of position p of a window enumerated row-major (clamped).
-__device__ __forceinline__ int window_query_token(const int4& win, int nq, int p, int Wg) {
-  if (p >= nq) p = 0;
-  return (win.x + p / win.w) * Wg + win.y + p % win.w;
-}
 
 // One 128-row tile of D bf16 copied row by row with cp.async by the 32 lanes
 // of a warp into the 128B-swizzled K-major layout that TMA's 128-byte swizzle
@@ -445,8 +471,8 @@ __device__ void fill_window_unit(int b, int h, int idx, const TcParams& prm, Uni
   r.one = r.nq - r.q0 <= 128;
   r.nkv = prm.cand ? prm.R : P.gcount[wo];
   r.ngt = (r.nkv + 127) / 128;
-  r.ncx = (r.ext.w + kPW - 1) / kPW;
-  r.ntr = r.ncx * ((r.ext.z + kPH - 1) / kPH);
+  r.ntr = rect_tiles(rect_tiling(r.ext.z, r.ext.w));
+  r.qcx = query_cells_per_row(r.win);
   r.nt = r.ngt + r.ntr + (prm.T + 127) / 128;
   r.glist = prm.cand ? (long long)r.bh * prm.R : (long long)wo * P.G;
 }
@@ -464,7 +490,7 @@ __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
   r.one = 0;
   r.cls = 0;
   r.glist = 0;
-  r.ntr = r.ncx = 0;
+  r.ntr = r.qcx = 0;
   r.win = r.ext = r.my = r.mx = make_int4(0, 0, 0, 0);
   if (!WINDOW) {
     if (u >= prm.num_units) return false;
@@ -497,10 +523,7 @@ __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
 
 template <bool WINDOW, bool BRIDGE, int D>
 __global__ void __launch_bounds__(kThreads, 1)
-attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
-               const __grid_constant__ CUtensorMap tm_vp, const __grid_constant__ CUtensorMap tm_kt,
-               const __grid_constant__ CUtensorMap tm_vt, const TcParams prm) {
+attn_tc_kernel(const __grid_constant__ TcMaps tm, const TcParams prm) {
   using G = Geo<D>;
   constexpr uint32_t kIdescPV = idesc(D, true);
   extern __shared__ uint8_t smem_raw[];
@@ -589,9 +612,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       return true;
     };
     // Queries of this CTA's k-th unit, once the previous unit's last QK has
-    // read the buffer.  Window queries (the rectangle enumerated row-major,
-    // read from DRAM once per unit) are gathered by TMA, 4 rows per lane:
-    // a warp's cp.async stream issued them about 7x slower (measured).
+    // read the buffer.  Window queries are read from DRAM once per unit: in
+    // cells of kCW x kCH tokens (one tiled box per lane) when the window's
+    // sides allow, else row by row with TMA gather4, 4 rows per lane (a warp's
+    // cp.async stream issued those about 7x slower, measured; gather4 itself
+    // moves about 7 bytes per clock per SM against about 37 for tiled boxes).
     auto load_q = [&](uint32_t k) -> bool {
       const UnitRec& Rq = s_rec[k % kRecSlots];
       if (!Rq.valid) return true;
@@ -604,8 +629,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           mbar_arrive_tx(bar(BAR_Q_FULL + qs), nqt * G::kTileBytes);
           for (int t = 0; t < nqt; ++t)
             for (int hf = 0; hf < G::kHalves; ++hf)
-              tma_load_2d(qbase + t * G::kTileBytes + hf * kHalfBytes, &tm_q, bar(BAR_Q_FULL + qs),
+              tma_load_2d(qbase + t * G::kTileBytes + hf * kHalfBytes, &tm.q, bar(BAR_Q_FULL + qs),
                           hf * 64, Rq.bh * Ntok + Rq.q0 + t * 128);
+        }
+        __syncwarp();
+      } else if (Rq.qcx > 0) {
+        if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL + qs), nqt * G::kTileBytes);
+        __syncwarp();
+        if (lane < kCells) {
+          // cell q0 / kCellKeys + t * kCells + lane (clamped to the last one;
+          // the rows past nq are computed and not stored)
+          const int ncq = Rq.nq / kCellKeys;
+          for (int t = 0; t < nqt; ++t) {
+            int c = Rq.q0 / kCellKeys + t * kCells + lane;
+            if (c > ncq - 1) c = ncq - 1;
+            const int cx = Rq.win.y + (c % Rq.qcx) * kCW;
+            const int cy = Rq.bh * prm.P.Hg + Rq.win.x + (c / Rq.qcx) * kCH;
+            for (int hf = 0; hf < G::kHalves; ++hf)
+              tma_load_3d(qbase + t * G::kTileBytes + hf * kHalfBytes + lane * kCellBytes, &tm.qc,
+                          bar(BAR_Q_FULL + qs), hf * 64, cx, cy);
+          }
         }
         __syncwarp();
       } else {
@@ -616,9 +659,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             r[i] = Rq.bh * Ntok +
-                   window_query_token(Rq.win, Rq.nq, Rq.q0 + t * 128 + lane * 4 + i, Wg);
+                   window_query_token(Rq.win, 0, Rq.nq, Rq.q0 + t * 128 + lane * 4 + i, Wg);
           for (int hf = 0; hf < G::kHalves; ++hf)
-            tma_gather4(qbase + t * G::kTileBytes + hf * kHalfBytes + lane * 512, &tm_q,
+            tma_gather4(qbase + t * G::kTileBytes + hf * kHalfBytes + lane * 512, &tm.q,
                         bar(BAR_Q_FULL + qs), hf * 64, r[0], r[1], r[2], r[3]);
         }
       }
@@ -629,10 +672,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const UnitRec& R = s_rec[unit_count % kRecSlots];
       if (!R.valid) break;
       if (!(ok = load_q(unit_count))) break;
-      const int nt = R.nt, ngt = R.ngt, ntr = R.ntr, ncx = R.ncx, nkv = R.nkv;
+      const int nt = R.nt, ngt = R.ngt, ntr = R.ntr, nkv = R.nkv;
       const int nti = ngt + ntr;
       const int bh = R.bh;
       const int4 ext = R.ext;
+      const RectTiling rt = rect_tiling(ext.z, ext.w);
       const int* glist = (BRIDGE ? prm.cand : prm.P.gidx) + R.glist;
       const int jn = nt < 2 ? nt : 2;         // the next record is published before tile jn
       bool published = false;
@@ -647,7 +691,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ok = false;
             break;
           }
-          const CUtensorMap* tm = kv ? &tm_v : &tm_k;
+          const CUtensorMap* tmd = kv ? &tm.v : &tm.k;
           const uint32_t dst = sbase + G::kSmemKV + s * G::kTileBytes;
           if (WINDOW && j < ngt) {
             // global-KV list (or bridge candidates), copied row by row: the
@@ -672,7 +716,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           if (j >= nti) {
             // text keys: rows of the [B*H*T, 128] text tensors
             if (lane == 0) {
-              const CUtensorMap* tt = kv ? &tm_vt : &tm_kt;
+              const CUtensorMap* tt = kv ? &tm.vt : &tm.kt;
               for (int hf = 0; hf < G::kHalves; ++hf)
                 tma_load_2d(dst + hf * kHalfBytes, tt, bar(BAR_KV_FULL + s), hf * 64,
                             bh * prm.T + (j - nti) * 128);
@@ -680,19 +724,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           } else if (!WINDOW) {
             if (lane == 0)
               for (int hf = 0; hf < G::kHalves; ++hf)
-                tma_load_2d(dst + hf * kHalfBytes, tm, bar(BAR_KV_FULL + s), hf * 64,
+                tma_load_2d(dst + hf * kHalfBytes, tmd, bar(BAR_KV_FULL + s), hf * 64,
                             bh * Nkrows + j * 128);
           } else {
-            // patch (px, py) of the Halo rectangle: kPH grid rows of kPW tokens
-            if (lane == 0) {
-              const CUtensorMap* tp = kv ? &tm_vp : &tm_kp;
-              const int jj = j - ngt;
-              const int px = jj % ncx, py = jj / ncx;
-              const int cx = ext.y + px * kPW;
-              const int cy = bh * prm.P.Hg + ext.x + py * kPH;
+            // Halo rectangle: patch j - ngt, or kCells strip cells, one per
+            // lane (past the last cell the last one is loaded again: finite
+            // values under masked keys)
+            const int jj = j - ngt;
+            if (jj < rt.npatch) {
+              if (lane == 0) {
+                const CUtensorMap* tp = kv ? &tm.vp : &tm.kp;
+                const int cx = ext.y + (jj % rt.npx) * kPW;
+                const int cy = bh * prm.P.Hg + ext.x + (jj / rt.npx) * kPH;
+                for (int hf = 0; hf < G::kHalves; ++hf)
+                  tma_load_3d(dst + hf * kHalfBytes, tp, bar(BAR_KV_FULL + s), hf * 64, cx, cy);
+              }
+            } else if (lane < kCells) {
+              const CUtensorMap* tc = kv ? &tm.vc : &tm.kc;
+              int c = (jj - rt.npatch) * kCells + lane;
+              if (c > rt.ncell - 1) c = rt.ncell - 1;
+              const int2 o = strip_cell(rt, c);
+              const int cx = ext.y + o.y;
+              const int cy = bh * prm.P.Hg + ext.x + o.x;
               for (int hf = 0; hf < G::kHalves; ++hf)
-                tma_load_3d(dst + hf * kHalfBytes, tp, bar(BAR_KV_FULL + s), hf * 64, cx, cy);
+                tma_load_3d(dst + hf * kHalfBytes + lane * kCellBytes, tc, bar(BAR_KV_FULL + s),
+                            hf * 64, cx, cy);
             }
+            __syncwarp();
           }
           ++kv_it;
         }
@@ -750,6 +808,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (!(ok = mbar_wait(bar(BAR_REC_FULL + slot), (unit_count / kRecSlots) & 1u, abort_flag)))
           break;
         const int valid = s_rec[slot].valid, nt = s_rec[slot].nt;
+        const int ngt = WINDOW ? s_rec[slot].ngt : 0;   // leading tiles copied by cp.async
         const bool two = s_rec[slot].one == 0;   // query tile 1 runs too
         mbar_arrive(bar(BAR_REC_EMPTY + slot));
         if (!valid) break;
@@ -762,7 +821,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t k0 = kv_it;
         if (!(ok = mbar_wait(bar(BAR_KV_FULL + k0 % kStages), (k0 / kStages) & 1u, abort_flag)))
           break;
-        if (WINDOW) fence_proxy_async();        // queries and global-KV rows came by cp.async
+        if (ngt > 0) fence_proxy_async();       // global-KV rows came by cp.async
         tc_fence_after();
         qk(tS0, q0s, kv_addr(k0));
         mma_commit(bar(BAR_S_FULL0));
@@ -777,7 +836,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const uint32_t kn = kv_it + 2 * j + 2;
           if (!(ok = mbar_wait(bar(BAR_KV_FULL + vi % kStages), (vi / kStages) & 1u, abort_flag)))
             break;
-          if (WINDOW) fence_proxy_async();
+          if (j < ngt) fence_proxy_async();
           if (!(ok = pv_parts(tO0, tS0, kv_addr(vi), j == 0, BAR_P_PART0, BAR_P_FULL0, p_cnt0)))
             break;
           ++p_cnt0;
@@ -786,7 +845,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (!(ok = mbar_wait(bar(BAR_KV_FULL + kn % kStages), (kn / kStages) & 1u,
                                  abort_flag)))
               break;
-            if (WINDOW) fence_proxy_async();
+            if (j + 1 < ngt) fence_proxy_async();
             tc_fence_after();
             qk(tS0, q0s, kv_addr(kn));
             mma_commit(bar(BAR_S_FULL0));
@@ -850,29 +909,52 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ++unit_count;
         continue;
       }
-      const int nkv = R.nkv, nt = R.nt, ngt = R.ngt, ntr = R.ntr, ncx = R.ncx;
+      const int nkv = R.nkv, nt = R.nt, ngt = R.ngt, ntr = R.ntr;
       const int nti = ngt + ntr;
       const int ew = R.ext.w, eh = R.ext.z;
+      int ncb, ncell;                                // first strip-cell tile, strip cells
+      {
+        const RectTiling rt = rect_tiling(eh, ew);
+        ncb = ngt + rt.npatch;
+        ncell = rt.ncell;
+      }
+      // a Halo rectangle whose sides are multiples of the cell's has full
+      // cells only: its cell tiles hold a prefix of valid keys
+      const bool ragged = WINDOW && (ew % kCW != 0 || eh % kCH != 0);
       float m = -INFINITY, l = 0.f;
-      int pcx = 0, pcy = 0;                          // patch of tile j in the Halo rectangle
       for (int j = 0; j < nt; ++j) {
         // Bridge candidates: drop those past the list or inside the Halo
         // rectangle; lane l tests keys 4l..4l+3 and ballots the result.  This
         // does not depend on S, so it is done before waiting for S (the loads
-        // overlap the wait) and before S occupies 128 registers.
+        // overlap the wait) and before S occupies 128 registers.  Keys of a
+        // ragged rectangle's cells are tested the same way.
         const bool bridge_tile = BRIDGE && j < ngt;
+        const bool ragged_tile = ragged && j >= ncb && j < nti;
         uint32_t keep[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-        if (bridge_tile) {
-          const int* cl = prm.cand + R.glist;
+        if (bridge_tile || ragged_tile) {
           const int4 ex = R.ext;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const int p = j * 128 + lane * 4 + i;
-            bool in = p < nkv;
-            if (in) {
-              const int tok = cl[p];
-              const int ty = tok / prm.P.Wg, tx = tok % prm.P.Wg;
-              in = !(ty >= ex.x && ty < ex.x + eh && tx >= ex.y && tx < ex.y + ew);
+            const int kk = lane * 4 + i;
+            bool in;
+            if (bridge_tile) {
+              const int p = j * 128 + kk;
+              in = p < nkv;
+              if (in) {
+                const int tok = prm.cand[R.glist + p];
+                const int ty = tok / prm.P.Wg, tx = tok % prm.P.Wg;
+                in = !(ty >= ex.x && ty < ex.x + ex.z && tx >= ex.y && tx < ex.y + ex.w);
+              }
+            } else {
+              // the tiling is recomputed from the record here (a shared-memory
+              // read the compiler cannot hoist past the loop's barrier waits)
+              // rather than kept in registers through the whole tile loop
+              const int c = (j - ncb) * kCells + kk / kCellKeys, e = kk % kCellKeys;
+              in = c < ncell;
+              if (in) {
+                const int2 o = strip_cell(rect_tiling(ex.z, ex.w), c);
+                in = o.y + e % kCW < ex.w && o.x + e / kCW < ex.z;
+              }
             }
             keep[i] = __ballot_sync(0xffffffffu, in);
           }
@@ -880,28 +962,37 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (!(ok = warp_wait_all(bS, s_cnt & 1u, abort_flag))) break;
         ++s_cnt;
         tc_fence_after();
+        // Key validity (warp-uniform): bridge and ragged-rectangle tiles
+        // follow their ballots (key k in bit k / 4 of keep[k % 4]), applied
+        // to S in TMEM 32 columns at a time, so the ballots are not held
+        // with the whole score row; list, text and rectangle tiles are a
+        // prefix of `valid` keys.
+        if (bridge_tile || ragged_tile) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t t[32];
+            tmem_ld32(tS + c * 32, t);
+            const uint32_t k0 = keep[0], k1 = keep[1], k2 = keep[2], k3 = keep[3];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const uint32_t kw = (i & 3) == 0 ? k0 : (i & 3) == 1 ? k1 : (i & 3) == 2 ? k2 : k3;
+              if (!((kw >> (c * 8 + (i >> 2))) & 1u)) t[i] = 0xff800000u;
+            }
+            tmem_st32(tS + c * 32, t);
+          }
+          tmem_wait_st();
+        }
         uint32_t sr[128];
         tmem_ld128(tS, sr);
-        // Key validity (warp-uniform): list and text tiles are a prefix of
-        // `valid` keys; a rectangle patch keeps columns dx < rem_x of rows
-        // dy < rem_y (key k = dy * kPW + dx).
-        if (bridge_tile) {
-#pragma unroll
-          for (int i = 0; i < 128; ++i)
-            if (!((keep[i & 3] >> (i >> 2)) & 1u)) sr[i] = 0xff800000u;
-        } else if (!WINDOW || j < ngt || j >= nti) {
-          const int valid = j < ngt ? min(128, nkv - j * 128) : min(128, prm.T - (j - nti) * 128);
+        if (!(bridge_tile || ragged_tile)) {
+          const int valid = j < ngt    ? min(128, nkv - j * 128)
+                            : j < ncb  ? 128
+                            : j < nti  ? min(128, (ncell - (j - ncb) * kCells) * kCellKeys)
+                                       : min(128, prm.T - (j - nti) * 128);
           if (valid < 128) {
 #pragma unroll
             for (int i = 0; i < 128; ++i)
               if (i >= valid) sr[i] = 0xff800000u;        // -inf: no weight
-          }
-        } else {
-          const int rem_x = ew - pcx * kPW, rem_y = eh - pcy * kPH;
-          if (rem_x < kPW || rem_y < kPH) {
-#pragma unroll
-            for (int i = 0; i < 128; ++i)
-              if ((i % kPW) >= rem_x || (i / kPW) >= rem_y) sr[i] = 0xff800000u;
           }
         }
         // row maximum: kMaxChains independent partial maxima, then a tree
@@ -963,10 +1054,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           mbar_arrive(h + 1 < kPParts ? bar(bPpart + h) : bP);
         }
         l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-        if (WINDOW && j >= ngt && j < nti && ++pcx == ncx) {
-          pcx = 0;
-          ++pcy;
-        }
       }
       if (!ok) break;
       // ---- epilogue
@@ -984,15 +1071,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           uint32_t orr[32];
           tmem_ld32(tO + c * 32, orr);
           if (qvalid) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) {
-              uint4 w;
-              w.x = pack_bf16(__uint_as_float(orr[8 * v4 + 0]) * inv, __uint_as_float(orr[8 * v4 + 1]) * inv);
-              w.y = pack_bf16(__uint_as_float(orr[8 * v4 + 2]) * inv, __uint_as_float(orr[8 * v4 + 3]) * inv);
-              w.z = pack_bf16(__uint_as_float(orr[8 * v4 + 4]) * inv, __uint_as_float(orr[8 * v4 + 5]) * inv);
-              w.w = pack_bf16(__uint_as_float(orr[8 * v4 + 6]) * inv, __uint_as_float(orr[8 * v4 + 7]) * inv);
-              d4[v4] = w;
+            for (int h = 0; h < 2; ++h) {
+              uint32_t w[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                w[i] = pack_bf16(__uint_as_float(orr[16 * h + 2 * i]) * inv,
+                                 __uint_as_float(orr[16 * h + 2 * i + 1]) * inv);
+              st_global_v8(dst + c * 32 + h * 16, w);
             }
           }
         }
@@ -1004,7 +1090,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // of one class never overlap, and a class adds only after every unit
         // of the lower classes has completed (a bounded wait on their
         // completion counters), so the sum runs in a fixed order.
-        const int tok = window_query_token(R.win, R.nq, qpos, Wg);
+        const int tok = window_query_token(R.win, R.qcx, R.nq, qpos, Wg);
         const int y = tok / Wg, x = tok % Wg;
         const MergeRole mr = merge_role(y, x, R.cls, R.my, R.mx, Wg, prm.nx2);
         const bool rmw = qvalid && mr.ov;
@@ -1061,36 +1147,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
           for (int i = 0; i < 32; ++i) vals[i] = __uint_as_float(orr[i]) * sc;
           if (rmw) {
-            float4* a4 = reinterpret_cast<float4*>(acc + c * 32);
+            float* a = acc + c * 32;
             if (!mr.first) {
 #pragma unroll
-              for (int v4 = 0; v4 < 8; ++v4) {
-                const float4 a = a4[v4];
-                vals[4 * v4 + 0] += a.x;
-                vals[4 * v4 + 1] += a.y;
-                vals[4 * v4 + 2] += a.z;
-                vals[4 * v4 + 3] += a.w;
+              for (int v = 0; v < 4; ++v) {
+                float t[8];
+                ld_global_v8f(a + 8 * v, t);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) vals[8 * v + i] += t[i];
               }
             }
             if (!mr.last) {
 #pragma unroll
-              for (int v4 = 0; v4 < 8; ++v4)
-                a4[v4] = make_float4(vals[4 * v4], vals[4 * v4 + 1], vals[4 * v4 + 2],
-                                     vals[4 * v4 + 3]);
+              for (int v = 0; v < 4; ++v) st_global_v8f(a + 8 * v, vals + 8 * v);
               continue;
             }
 #pragma unroll
             for (int i = 0; i < 32; ++i) vals[i] *= winv;
           }
-          uint4* d4 = reinterpret_cast<uint4*>(dsto + c * 32);
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            uint4 w;
-            w.x = pack_bf16(vals[8 * v4 + 0], vals[8 * v4 + 1]);
-            w.y = pack_bf16(vals[8 * v4 + 2], vals[8 * v4 + 3]);
-            w.z = pack_bf16(vals[8 * v4 + 4], vals[8 * v4 + 5]);
-            w.w = pack_bf16(vals[8 * v4 + 6], vals[8 * v4 + 7]);
-            d4[v4] = w;
+          for (int h = 0; h < 2; ++h) {
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[i] = pack_bf16(vals[16 * h + 2 * i], vals[16 * h + 2 * i + 1]);
+            st_global_v8(dsto + c * 32 + h * 16, w);
           }
         }
         // this warp's rows of the unit are complete
@@ -1142,13 +1222,14 @@ cudaError_t make_map(CUtensorMap* m, const void* base, int64_t rows, int box_row
 }
 
 // 3-D bf16 map over [rows_y, Wg, D] (token-grid rows of all (b, h), grid
-// columns, head dims) with a box of 64 dims x kPW tokens x kPH grid rows.
-cudaError_t make_map_patch(CUtensorMap* m, const void* base, int64_t rows_y, int Wg, int D) {
+// columns, head dims) with a box of 64 dims x bw tokens x bh grid rows.
+cudaError_t make_map_grid(CUtensorMap* m, const void* base, int64_t rows_y, int Wg, int D, int bw,
+                          int bh) {
   auto enc = get_encode();
   if (!enc) return cudaErrorNotSupported;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Wg, (cuuint64_t)rows_y};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Wg * D * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)kPW, (cuuint32_t)kPH};
+  cuuint32_t box[3] = {64, (cuuint32_t)bw, (cuuint32_t)bh};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1164,15 +1245,13 @@ int num_sms() {
 }
 
 template <bool WINDOW, bool BRIDGE, int D>
-cudaError_t launch_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                      const CUtensorMap& mkp, const CUtensorMap& mvp, const CUtensorMap& mkt,
-                      const CUtensorMap& mvt, const TcParams& prm, cudaStream_t s) {
+cudaError_t launch_tc(const TcMaps& maps, const TcParams& prm, cudaStream_t s) {
   constexpr int kSmemBytes = Geo<D>::kSmemBytes;
   auto fn = attn_tc_kernel<WINDOW, BRIDGE, D>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int grid = prm.num_units < num_sms() ? prm.num_units : num_sms();
-  fn<<<grid > 0 ? grid : 1, kThreads, kSmemBytes, s>>>(mq, mk, mv, mkp, mvp, mkt, mvt, prm);
+  fn<<<grid > 0 ? grid : 1, kThreads, kSmemBytes, s>>>(maps, prm);
   return cudaGetLastError();
 }
 
@@ -1190,18 +1269,19 @@ cudaError_t read_and_clear_tc_error(int* code) {
 cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, const void* kt,
                                  const void* vt, void* o, int B, int H, int N, int Nk, int T,
                                  int D, float scale, cudaStream_t s) {
-  CUtensorMap mq, mk, mv, mkt, mvt;
+  TcMaps m;
   cudaError_t e;
-  if ((e = make_map(&mq, q, (int64_t)B * H * N, 128, D)) != cudaSuccess) return e;
-  if ((e = make_map(&mk, k, (int64_t)B * H * Nk, 128, D)) != cudaSuccess) return e;
-  if ((e = make_map(&mv, v, (int64_t)B * H * Nk, 128, D)) != cudaSuccess) return e;
+  if ((e = make_map(&m.q, q, (int64_t)B * H * N, 128, D)) != cudaSuccess) return e;
+  if ((e = make_map(&m.k, k, (int64_t)B * H * Nk, 128, D)) != cudaSuccess) return e;
+  if ((e = make_map(&m.v, v, (int64_t)B * H * Nk, 128, D)) != cudaSuccess) return e;
   if (T > 0) {
-    if ((e = make_map(&mkt, kt, (int64_t)B * H * T, 128, D)) != cudaSuccess) return e;
-    if ((e = make_map(&mvt, vt, (int64_t)B * H * T, 128, D)) != cudaSuccess) return e;
+    if ((e = make_map(&m.kt, kt, (int64_t)B * H * T, 128, D)) != cudaSuccess) return e;
+    if ((e = make_map(&m.vt, vt, (int64_t)B * H * T, 128, D)) != cudaSuccess) return e;
   } else {
-    mkt = mk;   // never read without text keys
-    mvt = mv;
+    m.kt = m.k;   // never read without text keys
+    m.vt = m.v;
   }
+  m.qc = m.kp = m.vp = m.kc = m.vc = m.q;   // window maps: never read in dense mode
   TcParams prm{};
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.H = H;
@@ -1209,9 +1289,8 @@ cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, co
   prm.da = DenseArgs{B, H, N, Nk, (N + 255) / 256};
   prm.num_units = B * H * prm.da.units_per_head;
   prm.o = static_cast<__nv_bfloat16*>(o);
-  // no patch maps in dense mode
-  if (D == 64) return launch_tc<false, false, 64>(mq, mk, mv, mk, mv, mkt, mvt, prm, s);
-  return launch_tc<false, false, 128>(mq, mk, mv, mk, mv, mkt, mvt, prm, s);
+  if (D == 64) return launch_tc<false, false, 64>(m, prm, s);
+  return launch_tc<false, false, 128>(m, prm, s);
 }
 
 int64_t window_ws_bytes(const PlanLayout& L, int H, int D) {
@@ -1222,21 +1301,24 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, c
                                   const void* vt, int T, const int* cand, int R,
                                   const PlanLayout& L, const void* plan, void* o, void* ws,
                                   int H, int D, float scale, cudaStream_t s) {
-  CUtensorMap mq, mk, mv, mkt, mvt;
+  TcMaps m;
   cudaError_t e;
-  const int64_t rows = L.B * H * L.N;
-  if ((e = make_map(&mq, q, rows, 1, D)) != cudaSuccess) return e;
-  if ((e = make_map(&mk, k, rows, 1, D)) != cudaSuccess) return e;
-  if ((e = make_map(&mv, v, rows, 1, D)) != cudaSuccess) return e;
-  CUtensorMap mkp, mvp;
-  if ((e = make_map_patch(&mkp, k, L.B * H * L.Hg, (int)L.Wg, D)) != cudaSuccess) return e;
-  if ((e = make_map_patch(&mvp, v, L.B * H * L.Hg, (int)L.Wg, D)) != cudaSuccess) return e;
+  const int64_t rows = L.B * H * L.N, rows_y = L.B * H * L.Hg;
+  const int Wg = (int)L.Wg;
+  if ((e = make_map(&m.q, q, rows, 1, D)) != cudaSuccess) return e;
+  if ((e = make_map_grid(&m.qc, q, rows_y, Wg, D, kCW, kCH)) != cudaSuccess) return e;
+  if ((e = make_map_grid(&m.kp, k, rows_y, Wg, D, kPW, kPH)) != cudaSuccess) return e;
+  if ((e = make_map_grid(&m.vp, v, rows_y, Wg, D, kPW, kPH)) != cudaSuccess) return e;
+  if ((e = make_map_grid(&m.kc, k, rows_y, Wg, D, kCW, kCH)) != cudaSuccess) return e;
+  if ((e = make_map_grid(&m.vc, v, rows_y, Wg, D, kCW, kCH)) != cudaSuccess) return e;
+  m.k = m.kp;   // global-KV rows are copied with cp.async: no row map
+  m.v = m.vp;
   if (T > 0) {
-    if ((e = make_map(&mkt, kt, L.B * H * T, 128, D)) != cudaSuccess) return e;
-    if ((e = make_map(&mvt, vt, L.B * H * T, 128, D)) != cudaSuccess) return e;
+    if ((e = make_map(&m.kt, kt, L.B * H * T, 128, D)) != cudaSuccess) return e;
+    if ((e = make_map(&m.vt, vt, L.B * H * T, 128, D)) != cudaSuccess) return e;
   } else {
-    mkt = mq;   // never read without text keys
-    mvt = mq;
+    m.kt = m.q;   // never read without text keys
+    m.vt = m.q;
   }
   TcParams prm{};
   prm.scale_log2 = scale * 1.4426950408889634f;
@@ -1257,11 +1339,11 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, c
   // unit counter and class completion counters start at zero
   if ((e = cudaMemsetAsync(ws, 0, (size_t)hdr, s)) != cudaSuccess) return e;
   if (D == 64) {
-    if (cand) return launch_tc<true, true, 64>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
-    return launch_tc<true, false, 64>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
+    if (cand) return launch_tc<true, true, 64>(m, prm, s);
+    return launch_tc<true, false, 64>(m, prm, s);
   }
-  if (cand) return launch_tc<true, true, 128>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
-  return launch_tc<true, false, 128>(mq, mk, mv, mkp, mvp, mkt, mvt, prm, s);
+  if (cand) return launch_tc<true, true, 128>(m, prm, s);
+  return launch_tc<true, false, 128>(m, prm, s);
 }
 
 }  // namespace area

@@ -144,6 +144,15 @@ def test_window_calls_reject_small_buffers_on_host(area):
     with pytest.raises(area.AreaError) as e:
         area.area_window_attn(fake, fake, fake, cfg, fake + 16, need, fake, fake, ws, 2, 64, 0.125, 0)
     assert e.value.status == area.AREA_EINVAL
+    # outputs and the workspace are written 32 bytes per thread: 16-byte
+    # aligned ones are refused
+    for o, w in ((fake + 16, fake), (fake, fake + 16)):
+        with pytest.raises(area.AreaError) as e:
+            area.area_window_attn(fake, fake, fake, cfg, fake, need, o, w, ws, 2, 64, 0.125, 1)
+        assert e.value.status == area.AREA_EINVAL
+    with pytest.raises(area.AreaError) as e:
+        area.area_coarse_attn(fake, fake, fake, fake + 16, 1, 1, 16, 4, 128, 1.0, 1)
+    assert e.value.status == area.AREA_EINVAL
 
 
 def test_binding_has_no_oracle_dependency():
@@ -197,6 +206,29 @@ def test_merge_geometry_host_check(tmp_path):
     r = subprocess.run([exe], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
     assert "tilings checked" in r.stdout
+
+
+def test_rect_tiling_host_check(tmp_path):
+    # The tensor-core window kernel loads a Halo rectangle as full 16 x 8
+    # patches plus 4 x 4 cells of its right and bottom strips, and a window's
+    # queries in 4 x 4 cells: integer arithmetic in area_internal.cuh.  Check
+    # on the host that every key of every rectangle up to 72 x 72 (and some
+    # large ones) lands in exactly one tile row and that the query positions
+    # enumerate each window's tokens once.
+    import shutil
+    import subprocess
+    from step_adaptive_sparse_b200 import build as b
+    nvcc = b.nvcc()
+    if shutil.which(nvcc) is None and not os.path.exists(nvcc):
+        pytest.skip("nvcc is not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    exe = str(tmp_path / "rect_tiling_check")
+    subprocess.run([nvcc, "-O2", "-std=c++17", "-Wno-deprecated-gpu-targets", "-I",
+                    os.path.join(root, "include"), "-I", b.CSRC,
+                    os.path.join(root, "tests", "rect_tiling_check.cu"), "-o", exe], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert "rectangles and" in r.stdout
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
