@@ -36,7 +36,7 @@ if ROOT not in sys.path:
 
 METRIC = "AReA attention TFLOP/s per schedule step (bf16, 1 B200)"
 # Bumped whenever attn_tc.cu changes, so that stale DRAM counters are not reported.
-KERNEL_REVISION = "attn_tc v11 (class-major dynamic window units, window queries by TMA gather4, global-KV rows by cp.async, per-(b,h,class) merge counters, single-tile units)"
+KERNEL_REVISION = "attn_tc v12 (Halo rectangles as 16x8 patches plus 4x4 strip cells, window queries in 4x4 cells or gather4, global-KV rows by cp.async, class-major dynamic units, 32-byte epilogue stores)"
 DEFAULT_CONFIG = "flux6144"
 
 
