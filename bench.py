@@ -36,7 +36,7 @@ if ROOT not in sys.path:
 
 METRIC = "AReA attention TFLOP/s per schedule step (bf16, 1 B200)"
 # Bumped whenever attn_tc.cu changes, so that stale DRAM counters are not reported.
-KERNEL_REVISION = "attn_tc v12 (Halo rectangles as 16x8 patches plus 4x4 strip cells, window queries in 4x4 cells or gather4, global-KV rows by cp.async, class-major dynamic units, 32-byte epilogue stores)"
+KERNEL_REVISION = "attn_tc v13 (v12 plus whole global-KV tiles staged per call by stage_list_kernel and loaded as tiles)"
 DEFAULT_CONFIG = "flux6144"
 
 
@@ -81,10 +81,11 @@ def plan_launches(B: int) -> int:
     return 5 + 13 * B
 
 
-# kernels of one area_window_attn call on the tensor-core path (the merge runs
-# inside the attention kernel; a 256-byte memset of the workspace counters
-# precedes it)
-WINDOW_LAUNCHES = 1
+# kernels of one area_window_attn call on the tensor-core path with the
+# staging area in the workspace: the copy of the windows' global-KV rows, then
+# the attention kernel (the merge runs inside it); a 256-byte memset of the
+# workspace counters precedes both
+WINDOW_LAUNCHES = 2
 
 
 # ---------------------------------------------------------------------------
@@ -234,7 +235,9 @@ class AreaStep:
             self.pcfg.append(pc)
             self.plan.append(torch.empty(nb, dtype=torch.uint8, device=dev))
             self.plan_bytes.append(nb)
-            wsb = max(wsb, area.area_window_attn_ws_bytes(pc, cfg.H, cfg.D))
+            # the minimum plus the staging area of the global-KV rows (fast path)
+            wsb = max(wsb, area.area_window_attn_ws_bytes(pc, cfg.H, cfg.D)
+                      + area.area_window_attn_stage_bytes(pc, cfg.H, cfg.D))
         self.ws = torch.empty(wsb // 4, dtype=torch.float32, device=dev)
         self.ws_bytes = wsb
         self.n_phase1 = len(cfg.schedule)
@@ -443,7 +446,8 @@ def schedule_graph_leg(cfg, st, stream, full_ms, steps=28, shift=3.0, sigma_star
     for w in sorted(set(ws_sides)):
         pc = area.make_cfg(cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
         nb = area.area_window_plan_bytes(pc)
-        wsb = max(wsb, area.area_window_attn_ws_bytes(pc, cfg.H, cfg.D))
+        wsb = max(wsb, area.area_window_attn_ws_bytes(pc, cfg.H, cfg.D)
+                  + area.area_window_attn_stage_bytes(pc, cfg.H, cfg.D))
         plans[w] = (pc, torch.empty(nb, dtype=torch.uint8, device=dev), nb)
     # the run's window sides overlap differently from the step's: own workspace
     ws = torch.empty(wsb // 4, dtype=torch.float32, device=dev)
@@ -886,7 +890,7 @@ def run_area(args):
     if t_window >= t_coarse:
         dom, dom_flops, dom_ms, dom_launches = ("window_attn", win_flops / len(cfg.schedule),
                                                 t_window / len(cfg.schedule),
-                                                "1 launch after a 256-byte memset")
+                                                "the global-KV staging copy and the attention kernel, after a 256-byte memset; timed together")
     else:
         dom, dom_flops, dom_ms, dom_launches = ("coarse_attn", phase1_flops(cfg), coarse_ms,
                                                 "1 launch")

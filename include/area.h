@@ -311,6 +311,21 @@ int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D,
                               size_t* ws_bytes);
 
 /*
+ * area_window_attn_stage_bytes -- optional extra workspace (host only): when
+ * the ws given to area_window_attn (or _text) holds at least
+ * area_window_attn_ws_bytes() + stage_bytes, the bf16 tensor-core path first
+ * copies each window's global-KV rows that fill whole 128-row tiles into it
+ * (one launch on the stream), as [B][H][nw][G][D] K then V with nw the
+ * plan's final-window capacity, and the attention kernel then loads them as
+ * tiles instead of gathering them row by row in every work unit.  The result
+ * is the same (the same keys in the same order).  stage_bytes =
+ * 2 * B * H * nw * G * D * 2; 0 when G = 0.  The fp32 path and the bridged
+ * calls do not use it.
+ */
+int area_window_attn_stage_bytes(const area_plan_cfg* cfg, int H, int D,
+                                 size_t* stage_bytes);
+
+/*
  * area_window_attn -- Phase II windowed attention and centre-weighted merge
  * ([ai] Phase II).  For every final window W of the plan:
  *   O_W(q) = softmax(scale * q K_S^T) V_S,  S = ext(W) followed by G_W,
@@ -320,7 +335,9 @@ int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D,
  *   ws         : workspace of ws_bytes >= area_window_attn_ws_bytes(),
  *                32-byte aligned; contents on entry are ignored, on exit
  *                unspecified.  The call resets its counter header (a memset
- *                on the stream) before the kernel.
+ *                on the stream) before the kernel.  With ws_bytes >=
+ *                area_window_attn_ws_bytes() + area_window_attn_stage_bytes()
+ *                the global-KV rows are staged first (faster, same result).
  * Merge order: a token covered by several windows is summed over them in a
  * fixed order (by the parity class of the base window, see the plan's ITEMS;
  * the units of one head run class by class), so the output is bit-identical

@@ -34,7 +34,8 @@ EXPORTED = ("area_status_string", "area_last_cuda_error", "area_version", "area_
             "area_dwt_window_plan", "area_pool_ramp", "area_window_sides", "area_bridge_lattice", "area_phase_switch",
             "area_schedule",
             "area_coarse_attn", "area_full_attn", "area_dwt_detail", "area_window_plan_bytes",
-            "area_window_plan", "area_window_attn_ws_bytes", "area_window_attn",
+            "area_window_plan", "area_window_attn_ws_bytes", "area_window_attn_stage_bytes",
+            "area_window_attn",
             "area_window_attn_noalloc", "area_test_plan_barrier_expiry")
 
 
@@ -73,6 +74,8 @@ _SIGS = {
     "area_window_plan_bytes": (_I, [ctypes.POINTER(area_plan_cfg), ctypes.POINTER(_SZ)]),
     "area_window_plan": (_I, [_P, ctypes.POINTER(area_plan_cfg), _P, _SZ, _P]),
     "area_window_attn_ws_bytes": (_I, [ctypes.POINTER(area_plan_cfg), _I, _I, ctypes.POINTER(_SZ)]),
+    "area_window_attn_stage_bytes": (_I, [ctypes.POINTER(area_plan_cfg), _I, _I,
+                                          ctypes.POINTER(_SZ)]),
     "area_window_attn": (_I, [_P, _P, _P, ctypes.POINTER(area_plan_cfg), _P, _SZ, _P, _P, _SZ,
                               _I, _I, _F, _I, _P]),
     "area_window_attn_noalloc": (_I, [_P, _P, _P, ctypes.POINTER(area_plan_cfg), _P, _SZ, _P,
@@ -222,6 +225,13 @@ def area_window_attn_ws_bytes(cfg: area_plan_cfg, H: int, D: int) -> int:
     out = _SZ(0)
     _check(_lib().area_window_attn_ws_bytes(ctypes.byref(cfg), H, D, ctypes.byref(out)),
            "area_window_attn_ws_bytes")
+    return int(out.value)
+
+
+def area_window_attn_stage_bytes(cfg: area_plan_cfg, H: int, D: int) -> int:
+    out = _SZ(0)
+    _check(_lib().area_window_attn_stage_bytes(ctypes.byref(cfg), H, D, ctypes.byref(out)),
+           "area_window_attn_stage_bytes")
     return int(out.value)
 
 

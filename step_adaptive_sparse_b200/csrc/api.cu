@@ -66,12 +66,17 @@ int window_attn(const void* q, const void* k, const void* v, const void* kt, con
   if (T < 0 || (T > 0 && (!kt || !vt || !aligned16(kt) || !aligned16(vt)))) return AREA_EINVAL;
   if (cand && R < 1) return AREA_EINVAL;
   if (plan_bytes < (size_t)L.total) return AREA_ENOSPACE;
-  if (ws_bytes < (size_t)area::window_ws_bytes(L, H, D)) return AREA_ENOSPACE;
+  const size_t ws_need = (size_t)area::window_ws_bytes(L, H, D);
+  if (ws_bytes < ws_need) return AREA_ENOSPACE;
+  // room for the staging area: the plan's global-KV rows are copied once per
+  // call and loaded as tiles (tensor-core path, plan lists only)
+  const bool staged = dtype == AREA_DTYPE_BF16 && !cand && L.G > 0 && L.B * H <= 65535 &&
+                      ws_bytes >= ws_need + (size_t)area::window_stage_bytes(L, H, D);
   if (!aligned32(ws) || (reinterpret_cast<uintptr_t>(plan) & 255) != 0) return AREA_EINVAL;
   if (H > 65535 || L.B > 65535) return AREA_EINVAL;
   if (dtype == AREA_DTYPE_BF16)       // tensor cores, head_dim 64 or 128
-    return finish(area::launch_window_attn_tc(q, k, v, kt, vt, T, cand, R, L, plan, o, ws, H, D,
-                                              scale, stream));
+    return finish(area::launch_window_attn_tc(q, k, v, kt, vt, T, cand, R, L, plan, o, ws,
+                                              staged, H, D, scale, stream));
   return finish(area::launch_window_attn_simt(q, k, v, kt, vt, T, cand, R, L, plan, o, ws, H, D,
                                               scale, dtype, stream));
 }
@@ -199,6 +204,15 @@ int area_window_attn_ws_bytes(const area_plan_cfg* cfg, int H, int D, size_t* ws
   const int st = area::plan_layout(cfg, &L);
   if (st != AREA_OK) return st;
   *ws_bytes = (size_t)area::window_ws_bytes(L, H, D);
+  return AREA_OK;
+}
+
+int area_window_attn_stage_bytes(const area_plan_cfg* cfg, int H, int D, size_t* stage_bytes) {
+  if (!stage_bytes || H < 1 || D < 1) return AREA_EINVAL;
+  area::PlanLayout L;
+  const int st = area::plan_layout(cfg, &L);
+  if (st != AREA_OK) return st;
+  *stage_bytes = (size_t)area::window_stage_bytes(L, H, D);
   return AREA_OK;
 }
 

@@ -294,12 +294,18 @@ cudaError_t read_and_clear_tc_error(int* code);
 // cand (may be null): per-head bridge candidates [B*H][R]; when given they
 // replace the plan's global-KV lists, candidates inside a window's Halo
 // rectangle are skipped.
+// staged: the workspace extends window_stage_bytes past window_ws_bytes, and
+// the global-KV rows of each window are first copied there (one launch) so
+// that the attention kernel loads whole list tiles with tiled TMA.
 cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, const void* kt,
                                   const void* vt, int T, const int* cand, int R,
                                   const PlanLayout& L, const void* plan, void* o, void* ws,
-                                  int H, int D, float scale, cudaStream_t s);
+                                  bool staged, int H, int D, float scale, cudaStream_t s);
 // Bytes of the window workspace for H heads of head_dim D.
 int64_t window_ws_bytes(const PlanLayout& L, int H, int D);
+// Bytes of the optional staging area of the global-KV rows (bf16 K then V,
+// [B][H][nw][G][D] each), appended to the workspace.
+int64_t window_stage_bytes(const PlanLayout& L, int H, int D);
 // Detail map and planner in one cooperative launch (one memset of the
 // barrier words first); a barrier timeout raises the planner error flag.
 // target_extra (0 in every product call) raises each grid-barrier target so

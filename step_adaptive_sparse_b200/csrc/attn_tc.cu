@@ -399,6 +399,7 @@ struct TcMaps {
   CUtensorMap kp, vp;   // window keys and values [B*H*Hg, Wg, D]: one patch
   CUtensorMap kc, vc;   // window keys and values [B*H*Hg, Wg, D]: one cell
   CUtensorMap kt, vt;   // text keys and values [B*H*T, D]: 128-row box
+  CUtensorMap ks, vs;   // staged global-KV rows [B*H*nw*G, D]: 128-row box
 };
 
 struct TcParams {
@@ -416,6 +417,7 @@ struct TcParams {
   float* acc;         // window: fp32 accumulator rows [B*H][n_ov][128]
   int nx2;            // window: columns covered by two base windows
   long long n_ov;     // window: overlapped tokens per element
+  int staged;         // window: whole global-KV tiles come from the staging area
 };
 
 
@@ -693,6 +695,22 @@ attn_tc_kernel(const __grid_constant__ TcMaps tm, const TcParams prm) {
           }
           const CUtensorMap* tmd = kv ? &tm.v : &tm.k;
           const uint32_t dst = sbase + G::kSmemKV + s * G::kTileBytes;
+          if (WINDOW && !BRIDGE && j < ngt && prm.staged && (j + 1) * 128 <= nkv) {
+            // a whole tile of the window's global-KV rows, staged in the
+            // workspace by this call's copy launch: one tiled load
+            if (lane == 0) {
+              mbar_arrive_tx(bar(BAR_KV_FULL + s), G::kTileBytes);
+              // staging row of the window: ((b * H + h) * nw + w) * G, and
+              // R.glist = (b * nw + w) * G
+              const long long srow = R.glist + (long long)(bh - R.b) * prm.P.nw * prm.P.G;
+              for (int hf = 0; hf < G::kHalves; ++hf)
+                tma_load_2d(dst + hf * kHalfBytes, kv ? &tm.vs : &tm.ks, bar(BAR_KV_FULL + s),
+                            hf * 64, (int)(srow + j * 128));
+            }
+            __syncwarp();
+            ++kv_it;
+            continue;
+          }
           if (WINDOW && j < ngt) {
             // global-KV list (or bridge candidates), copied row by row: the
             // rows of a head's list serve all its windows and sit in L2, and
@@ -808,7 +826,10 @@ attn_tc_kernel(const __grid_constant__ TcMaps tm, const TcParams prm) {
         if (!(ok = mbar_wait(bar(BAR_REC_FULL + slot), (unit_count / kRecSlots) & 1u, abort_flag)))
           break;
         const int valid = s_rec[slot].valid, nt = s_rec[slot].nt;
-        const int ngt = WINDOW ? s_rec[slot].ngt : 0;   // leading tiles copied by cp.async
+        // leading list tiles copied by cp.async (not the staged whole ones)
+        const int ngt = WINDOW ? s_rec[slot].ngt : 0;
+        const int ncp = !WINDOW ? 0 : (!BRIDGE && prm.staged) ? ngt - s_rec[slot].nkv / 128 : ngt;
+        auto copied = [&](int j) { return j < ngt && j >= ngt - ncp; };
         const bool two = s_rec[slot].one == 0;   // query tile 1 runs too
         mbar_arrive(bar(BAR_REC_EMPTY + slot));
         if (!valid) break;
@@ -821,7 +842,7 @@ attn_tc_kernel(const __grid_constant__ TcMaps tm, const TcParams prm) {
         const uint32_t k0 = kv_it;
         if (!(ok = mbar_wait(bar(BAR_KV_FULL + k0 % kStages), (k0 / kStages) & 1u, abort_flag)))
           break;
-        if (ngt > 0) fence_proxy_async();       // global-KV rows came by cp.async
+        if (copied(0)) fence_proxy_async();     // rows copied by cp.async
         tc_fence_after();
         qk(tS0, q0s, kv_addr(k0));
         mma_commit(bar(BAR_S_FULL0));
@@ -836,7 +857,7 @@ attn_tc_kernel(const __grid_constant__ TcMaps tm, const TcParams prm) {
           const uint32_t kn = kv_it + 2 * j + 2;
           if (!(ok = mbar_wait(bar(BAR_KV_FULL + vi % kStages), (vi / kStages) & 1u, abort_flag)))
             break;
-          if (j < ngt) fence_proxy_async();
+          if (copied(j)) fence_proxy_async();
           if (!(ok = pv_parts(tO0, tS0, kv_addr(vi), j == 0, BAR_P_PART0, BAR_P_FULL0, p_cnt0)))
             break;
           ++p_cnt0;
@@ -845,7 +866,7 @@ attn_tc_kernel(const __grid_constant__ TcMaps tm, const TcParams prm) {
             if (!(ok = mbar_wait(bar(BAR_KV_FULL + kn % kStages), (kn / kStages) & 1u,
                                  abort_flag)))
               break;
-            if (j + 1 < ngt) fence_proxy_async();
+            if (copied(j + 1)) fence_proxy_async();
             tc_fence_after();
             qk(tS0, q0s, kv_addr(kn));
             mma_commit(bar(BAR_S_FULL0));
@@ -1191,6 +1212,31 @@ attn_tc_kernel(const __grid_constant__ TcMaps tm, const TcParams prm) {
   }
 }
 
+// One CTA per (window slot, element x head): copies the window's global-KV
+// rows that fill whole 128-row tiles, K then V, to the staging area
+// [B*H][nw][G][D] (rows past those tiles, and windows past the plan's count,
+// are skipped: the attention kernel gathers a partial last tile itself).
+template <int D>
+__global__ void __launch_bounds__(256) stage_list_kernel(const __nv_bfloat16* __restrict__ k,
+                                                         const __nv_bfloat16* __restrict__ v,
+                                                         const PlanView P, int H,
+                                                         __nv_bfloat16* __restrict__ sk,
+                                                         __nv_bfloat16* __restrict__ sv) {
+  const int w = blockIdx.x, bh = blockIdx.y, b = bh / H;
+  if (w >= P.nwin[b]) return;
+  const int64_t wo = (int64_t)b * P.nw + w;
+  const int nrow = P.gcount[wo] / 128 * 128;
+  const int* gl = P.gidx + wo * P.G;
+  const int64_t src0 = (int64_t)bh * P.N, dst0 = ((int64_t)bh * P.nw + w) * P.G;
+  constexpr int kChunks = D / 8;               // 16-byte chunks per row
+  for (int i = threadIdx.x; i < nrow * kChunks; i += blockDim.x) {
+    const int r = i / kChunks, c = i % kChunks;
+    const int64_t src = (src0 + gl[r]) * D + c * 8, dst = (dst0 + r) * D + c * 8;
+    *reinterpret_cast<uint4*>(sk + dst) = *reinterpret_cast<const uint4*>(k + src);
+    *reinterpret_cast<uint4*>(sv + dst) = *reinterpret_cast<const uint4*>(v + src);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -1281,7 +1327,7 @@ cudaError_t launch_dense_attn_tc(const void* q, const void* k, const void* v, co
     m.kt = m.k;   // never read without text keys
     m.vt = m.v;
   }
-  m.qc = m.kp = m.vp = m.kc = m.vc = m.q;   // window maps: never read in dense mode
+  m.qc = m.kp = m.vp = m.kc = m.vc = m.ks = m.vs = m.q;   // window maps: never read in dense mode
   TcParams prm{};
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.H = H;
@@ -1297,10 +1343,14 @@ int64_t window_ws_bytes(const PlanLayout& L, int H, int D) {
   return window_ws_header_bytes(L.B, H) + L.B * H * L.n_ov * D * 4;
 }
 
+int64_t window_stage_bytes(const PlanLayout& L, int H, int D) {
+  return 2 * L.B * H * L.nw * L.G * D * 2;
+}
+
 cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, const void* kt,
                                   const void* vt, int T, const int* cand, int R,
                                   const PlanLayout& L, const void* plan, void* o, void* ws,
-                                  int H, int D, float scale, cudaStream_t s) {
+                                  bool staged, int H, int D, float scale, cudaStream_t s) {
   TcMaps m;
   cudaError_t e;
   const int64_t rows = L.B * H * L.N, rows_y = L.B * H * L.Hg;
@@ -1311,8 +1361,21 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, c
   if ((e = make_map_grid(&m.vp, v, rows_y, Wg, D, kPW, kPH)) != cudaSuccess) return e;
   if ((e = make_map_grid(&m.kc, k, rows_y, Wg, D, kCW, kCH)) != cudaSuccess) return e;
   if ((e = make_map_grid(&m.vc, v, rows_y, Wg, D, kCW, kCH)) != cudaSuccess) return e;
-  m.k = m.kp;   // global-KV rows are copied with cp.async: no row map
+  m.k = m.kp;   // partial global-KV tiles are copied with cp.async: no row map
   m.v = m.vp;
+  // whole global-KV tiles: staged rows [B*H*nw*G, D] after the workspace
+  const int64_t nstage = L.B * H * L.nw * L.G;
+  __nv_bfloat16* sk = nullptr;
+  __nv_bfloat16* sv = nullptr;
+  if (staged && !cand && nstage > 0 && nstage < (int64_t(1) << 31)) {
+    sk = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + window_ws_bytes(L, H, D));
+    sv = sk + nstage * D;
+    if ((e = make_map(&m.ks, sk, nstage, 128, D)) != cudaSuccess) return e;
+    if ((e = make_map(&m.vs, sv, nstage, 128, D)) != cudaSuccess) return e;
+  } else {
+    staged = false;
+    m.ks = m.vs = m.q;   // never read
+  }
   if (T > 0) {
     if ((e = make_map(&m.kt, kt, L.B * H * T, 128, D)) != cudaSuccess) return e;
     if ((e = make_map(&m.vt, vt, L.B * H * T, 128, D)) != cudaSuccess) return e;
@@ -1336,8 +1399,17 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, c
   prm.acc = reinterpret_cast<float*>(static_cast<char*>(ws) + hdr);
   prm.nx2 = (int)L.nx2;
   prm.n_ov = L.n_ov;
+  prm.staged = staged ? 1 : 0;
   // unit counter and class completion counters start at zero
   if ((e = cudaMemsetAsync(ws, 0, (size_t)hdr, s)) != cudaSuccess) return e;
+  if (staged) {
+    const dim3 grid((unsigned)L.nw, (unsigned)(L.B * H));
+    const auto* kb = static_cast<const __nv_bfloat16*>(k);
+    const auto* vb = static_cast<const __nv_bfloat16*>(v);
+    if (D == 64) stage_list_kernel<64><<<grid, 256, 0, s>>>(kb, vb, prm.P, H, sk, sv);
+    else stage_list_kernel<128><<<grid, 256, 0, s>>>(kb, vb, prm.P, H, sk, sv);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   if (D == 64) {
     if (cand) return launch_tc<true, true, 64>(m, prm, s);
     return launch_tc<true, false, 64>(m, prm, s);

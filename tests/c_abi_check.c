@@ -25,6 +25,12 @@ int main(void) {
   if (area_window_attn_ws_bytes(&cfg80, 24, 128, &ws) != AREA_OK ||
       ws != (size_t)512 + (size_t)24 * 28672 * 128 * 4)
     return 4;
+  /* staging area of the global-KV rows: K and V, [B][H][nw][G][D] bf16 each,
+   * nw = 4 final windows per base window = 4 * 16 at w = 64 */
+  size_t sb = 0;
+  if (area_window_attn_stage_bytes(&cfg, 24, 128, &sb) != AREA_OK ||
+      sb != (size_t)2 * 24 * 64 * 512 * 128 * 2)
+    return 13;
 
   /* the printed pooling ramp at a 256 x 256 grid */
   const int want[8] = {4, 4, 4, 4, 2, 2, 2, 2};

@@ -106,9 +106,16 @@ def gpu_plan(energy, B, Hg, Wg, w, halo, G, thr):
     return cfg, plan, nbytes
 
 
-def gpu_window(q, k, v, cfg, plan, nbytes, H, D, scale, dtype):
-    o = torch.empty_like(q)
+def window_ws_bytes(cfg, H, D, staged=True):
+    """Workspace bytes of a window call: the minimum, plus the staging area of
+    the global-KV rows (the bf16 fast path) when `staged`."""
     wsb = area.area_window_attn_ws_bytes(cfg, H, D)
+    return wsb + area.area_window_attn_stage_bytes(cfg, H, D) if staged else wsb
+
+
+def gpu_window(q, k, v, cfg, plan, nbytes, H, D, scale, dtype, staged=True):
+    o = torch.empty_like(q)
+    wsb = window_ws_bytes(cfg, H, D, staged)
     ws = torch.empty(wsb // 4, dtype=torch.float32, device="cuda")
     area.area_window_attn(q, k, v, cfg, plan, nbytes, o, ws, wsb, H, D, scale, area_dtype(dtype))
     return o

@@ -120,6 +120,21 @@ def test_plan_config_validation_and_sizes(area):
         assert e.value.status == area.AREA_EINVAL
 
 
+def test_stage_bytes(area):
+    # K and V rows of every window slot: 2 * B * H * nw * G * D * 2 bytes with
+    # nw = 4 quadrants per base-window slot (16 slots at w = 64 on 256; 25
+    # when a seed may shift the tiling by up to one window per axis)
+    unit = 2 * 24 * 512 * 128 * 2
+    assert area.area_window_attn_stage_bytes(area.make_cfg(1, 256, 256, 64, 4, 512, 0.4), 24,
+                                             128) == 64 * unit
+    assert area.area_window_attn_stage_bytes(area.make_cfg(1, 256, 256, 64, 4, 512, 0.4, 99), 24,
+                                             128) == 100 * unit
+    assert area.area_window_attn_stage_bytes(area.make_cfg(2, 256, 256, 64, 4, 512, 0.4), 12,
+                                             64) == 64 * unit // 2
+    assert area.area_window_attn_stage_bytes(area.make_cfg(1, 256, 256, 64, 4, 0, 0.4), 24,
+                                             128) == 0
+
+
 def test_plan_size_with_seed_covers_every_shift(area):
     # a seeded plan may hold one more base window per axis
     base = area.area_window_plan_bytes(area.make_cfg(1, 384, 384, 72, 4, 512, 0.4))

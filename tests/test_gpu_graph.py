@@ -43,7 +43,8 @@ def test_schedule_step_graph_replay_matches_eager(name):
         pc = area.make_cfg(cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
         nb = area.area_window_plan_bytes(pc)
         plans.append((pc, torch.empty(nb, dtype=torch.uint8, device="cuda"), nb))
-        wsb = max(wsb, area.area_window_attn_ws_bytes(pc, cfg.H, cfg.D))
+        wsb = max(wsb, area.area_window_attn_ws_bytes(pc, cfg.H, cfg.D)
+                  + area.area_window_attn_stage_bytes(pc, cfg.H, cfg.D))
     ws = torch.empty(wsb // 4, dtype=torch.float32, device="cuda")
     o1 = torch.empty_like(q)
     o2 = [torch.empty_like(q) for _ in cfg.schedule]
@@ -143,7 +144,8 @@ def test_whole_sampling_run_in_one_graph():
         pc = area.make_cfg(cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G, cfg.split_thr)
         nb = area.area_window_plan_bytes(pc)
         plans[w] = (pc, torch.empty(nb, dtype=torch.uint8, device="cuda"), nb)
-        wsb = max(wsb, area.area_window_attn_ws_bytes(pc, cfg.H, cfg.D))
+        wsb = max(wsb, area.area_window_attn_ws_bytes(pc, cfg.H, cfg.D)
+                  + area.area_window_attn_stage_bytes(pc, cfg.H, cfg.D))
     ws = torch.empty(wsb // 4, dtype=torch.float32, device="cuda")
     o1, o2 = torch.empty_like(q), torch.empty_like(q)
     outs1, outs2 = [], []

@@ -343,7 +343,7 @@ def test_window_attn_text(data, which):
     pcfg, plan, nbytes = gr.gpu_plan(energy, cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, cfg.G,
                                      cfg.split_thr)
     o = torch.empty_like(data.dq)
-    wsb = gr.area.area_window_attn_ws_bytes(pcfg, cfg.H, cfg.D)
+    wsb = gr.window_ws_bytes(pcfg, cfg.H, cfg.D)
     ws = torch.empty(wsb // 4, dtype=torch.float32, device="cuda")
     gr.area.area_window_attn_text(data.dq, data.dk, data.dv, dkt, dvt, T, pcfg, plan, nbytes, o,
                                   ws, wsb, cfg.H, cfg.D, cfg.scale, gr.area_dtype(cfg.dtype))
@@ -504,6 +504,34 @@ def test_window_attn_edge_cases(Hg, Wg, w, h, G, D, dtype, H):
     for b in range(B):
         want = ora.window_attn(q[b:b + 1], k[b:b + 1], v[b:b + 1], [plans[b]], scale)
         gr.assert_close(gr.to_host(o[b:b + 1]), want, dtype, "window edge")
+
+
+@pytest.mark.parametrize("Hg,Wg,w,h,G,D,H", [
+    (64, 48, 24, 4, 130, 128, 3),   # one whole staged tile, a gathered partial one
+    (64, 64, 24, 4, 512, 128, 2),   # four whole staged tiles
+    (26, 34, 10, 2, 256, 64, 3),    # head_dim 64, two whole tiles
+    (16, 16, 7, 2, 5, 128, 2),      # no whole tile: nothing staged
+])
+def test_window_attn_staged_equals_gathered(Hg, Wg, w, h, G, D, H):
+    # With room for the staging area the whole global-KV tiles are copied
+    # once per call and loaded as tiles; the keys of every tile and their
+    # order are the same as when each unit gathers them, so the outputs are
+    # identical to the bit.
+    rng = np.random.default_rng(Hg * 7 + G)
+    B = 2
+    N = Hg * Wg
+    dq, dk, dv = (gr.to_dev(rng.standard_normal((B, H, N, D)).astype(np.float32), "bf16")
+                  for _ in range(3))
+    E = (rng.random((B, Hg // 2, Wg // 2)) ** 3).astype(np.float32)
+    pcfg, plan, nbytes = gr.gpu_plan(torch.from_numpy(E).cuda(), B, Hg, Wg, w, h, G,
+                                     float(np.median(E)))
+    scale = 1.0 / np.sqrt(D)
+    staged = gr.gpu_window(dq, dk, dv, pcfg, plan, nbytes, H, D, scale, "bf16", staged=True)
+    gathered = gr.gpu_window(dq, dk, dv, pcfg, plan, nbytes, H, D, scale, "bf16", staged=False)
+    torch.cuda.synchronize()
+    assert gr.area.area_window_attn_stage_bytes(pcfg, H, D) > 0
+    assert torch.equal(staged, gathered)
+    assert gr.area.area_kernel_error() == 0
 
 
 # ---------------------------------------------------------------------------
