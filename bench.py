@@ -38,6 +38,7 @@ METRIC = "AReA attention TFLOP/s per schedule step (bf16, 1 B200)"
 # Bumped whenever attn_tc.cu changes, so that stale DRAM counters are not reported.
 KERNEL_REVISION = "attn_tc v13 (v12 plus whole global-KV tiles staged per call by stage_list_kernel and loaded as tiles)"
 DEFAULT_CONFIG = "flux6144"
+PUBLISHED_BF16_TFLOPS = 2250.0   # B200 dense bf16 tensor rate, published (no sparsity)
 
 
 # ---------------------------------------------------------------------------
@@ -901,7 +902,9 @@ def run_area(args):
             "traffic": None if sharded else load_traffic(cfg.name, dom),
             "kernel": dom, "per_call": dom_launches,
             "peak_kind": f"bf16 dense, {peaks['source']} sustained",
-            "frac_of_burst_peak": achieved / peaks["bf16_tflops"]}
+            "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
+            # the B200's published dense bf16 rate (2.25 PFLOP/s), for reference
+            "frac_of_published_peak": achieved / PUBLISHED_BF16_TFLOPS}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
