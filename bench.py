@@ -342,6 +342,7 @@ def oracle_sample(cfg, q, k, v, src, budget_s: float = 15.0, rows_per_call: int 
     E = ora.dwt_detail(src, cfg.Hg, cfg.Wg)
     kp = ora.pool_kv(k[:, h:h + 1], cfg.Hg, cfg.Wg, cfg.f)
     vp = ora.pool_kv(v[:, h:h + 1], cfg.Hg, cfg.Wg, cfg.f)
+    rows_per_call = min(rows_per_call, cfg.N)
     rows = np.sort(rng.choice(cfg.N, size=rows_per_call, replace=False))
     ora.coarse_attn(q[:, h:h + 1], kp, vp, cfg.scale, rows=rows)
     flops += 4.0 * rows.size * cfg.Nk * cfg.D
@@ -908,7 +909,9 @@ def run_area(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        val, sec, desc, threads = oracle_sample(cfg, qh, kh, vh, srch, budget_s=args.ref_budget)
+        # about 10 s of the host's cores: 8192 query rows per sampled call
+        val, sec, desc, threads = oracle_sample(cfg, qh, kh, vh, srch, budget_s=args.ref_budget,
+                                                rows_per_call=8192)
         cpu = {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": desc, "seconds": sec}
 
