@@ -15,12 +15,14 @@
 //               ring read by the other roles, and issues the TMA loads: Q
 //               tiles once per unit, then a ring of K and V tiles (128 keys x
 //               128 dims, 128B-swizzled, 32 KB each).  Dense rows use tiled
-//               2-D loads.  Window keys are the global-KV list first (rows
-//               copied with 16-byte cp.async by the 32 producer lanes), then
-//               the Halo rectangle in 4x4-token cells (one 3-D tiled box per
-//               cell, 8 cells per tile, loaded by 8 lanes); window queries
-//               come in cells too when the window's sides are multiples of 4,
-//               else row by row by TMA gather4.
+//               2-D loads.  Window keys are the global-KV list first (whole
+//               tiles from the workspace's staging copy by one tiled load,
+//               else rows copied with 16-byte cp.async by the 32 producer
+//               lanes), then the Halo rectangle: 16x8-token patches (one 3-D
+//               tiled box each) and 4x4-token cells on the strips the
+//               patches leave (8 cells per tile, loaded by 8 lanes); window
+//               queries come in 4x4 cells when the window's sides are
+//               multiples of 4, else row by row by TMA gather4.
 //   warp 1      TMEM allocator and the single MMA-issuing thread.
 //   warps 2-5   softmax of query tile 0, warps 6-9 of query tile 1: each
 //               thread owns one query row (TMEM lane 32*(warp mod 4) + lane).
