@@ -405,8 +405,15 @@ int area_bridge_select(const void* k, int dtype, int B, int H, int Hg, int Wg,
  * area_bridge_select for (b, h) that lie outside ext(W), instead of the
  * plan's energy-ranked list (the plan's G is ignored; build it with G = 0).
  *   cand : int32 [B, H, R] from area_bridge_select (R = ry*rx)
+ *   ws   : as area_window_attn; with ws_bytes >= area_window_attn_ws_bytes()
+ *          + area_window_attn_bridge_stage_bytes() the bf16 tensor-core path
+ *          first copies each head's candidate rows that fill whole 128-row
+ *          tiles into it (one launch), and loads those tiles as tiles; the
+ *          result is the same.
  * Errors: as area_window_attn, and AREA_EINVAL for null cand or R < 1.
  */
+int area_window_attn_bridge_stage_bytes(int B, int H, int R, int D,
+                                        size_t* stage_bytes);   /* 2 * B * H * R * D * 2 */
 int area_window_attn_bridge(const void* q, const void* k, const void* v,
                             const int* cand, int R, const area_plan_cfg* cfg,
                             const void* plan, size_t plan_bytes, void* o,

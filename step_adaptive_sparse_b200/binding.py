@@ -35,6 +35,7 @@ EXPORTED = ("area_status_string", "area_last_cuda_error", "area_version", "area_
             "area_schedule",
             "area_coarse_attn", "area_full_attn", "area_dwt_detail", "area_window_plan_bytes",
             "area_window_plan", "area_window_attn_ws_bytes", "area_window_attn_stage_bytes",
+            "area_window_attn_bridge_stage_bytes",
             "area_window_attn",
             "area_window_attn_noalloc", "area_test_plan_barrier_expiry")
 
@@ -76,6 +77,7 @@ _SIGS = {
     "area_window_attn_ws_bytes": (_I, [ctypes.POINTER(area_plan_cfg), _I, _I, ctypes.POINTER(_SZ)]),
     "area_window_attn_stage_bytes": (_I, [ctypes.POINTER(area_plan_cfg), _I, _I,
                                           ctypes.POINTER(_SZ)]),
+    "area_window_attn_bridge_stage_bytes": (_I, [_I, _I, _I, _I, ctypes.POINTER(_SZ)]),
     "area_window_attn": (_I, [_P, _P, _P, ctypes.POINTER(area_plan_cfg), _P, _SZ, _P, _P, _SZ,
                               _I, _I, _F, _I, _P]),
     "area_window_attn_noalloc": (_I, [_P, _P, _P, ctypes.POINTER(area_plan_cfg), _P, _SZ, _P,
@@ -232,6 +234,13 @@ def area_window_attn_stage_bytes(cfg: area_plan_cfg, H: int, D: int) -> int:
     out = _SZ(0)
     _check(_lib().area_window_attn_stage_bytes(ctypes.byref(cfg), H, D, ctypes.byref(out)),
            "area_window_attn_stage_bytes")
+    return int(out.value)
+
+
+def area_window_attn_bridge_stage_bytes(B: int, H: int, R: int, D: int) -> int:
+    out = _SZ(0)
+    _check(_lib().area_window_attn_bridge_stage_bytes(B, H, R, D, ctypes.byref(out)),
+           "area_window_attn_bridge_stage_bytes")
     return int(out.value)
 
 

@@ -70,8 +70,11 @@ int window_attn(const void* q, const void* k, const void* v, const void* kt, con
   if (ws_bytes < ws_need) return AREA_ENOSPACE;
   // room for the staging area: the plan's global-KV rows are copied once per
   // call and loaded as tiles (tensor-core path, plan lists only)
-  const bool staged = dtype == AREA_DTYPE_BF16 && !cand && L.G > 0 && L.B * H <= 65535 &&
-                      ws_bytes >= ws_need + (size_t)area::window_stage_bytes(L, H, D);
+  // (the plan's lists, or the bridged call's per-head candidate rows)
+  const size_t stage_need = cand ? (size_t)4 * L.B * H * R * D
+                                 : (size_t)area::window_stage_bytes(L, H, D);
+  const bool staged = dtype == AREA_DTYPE_BF16 && (cand ? R >= 128 : L.G > 0) &&
+                      L.B * H <= 65535 && ws_bytes >= ws_need + stage_need;
   if (!aligned32(ws) || (reinterpret_cast<uintptr_t>(plan) & 255) != 0) return AREA_EINVAL;
   if (H > 65535 || L.B > 65535) return AREA_EINVAL;
   if (dtype == AREA_DTYPE_BF16)       // tensor cores, head_dim 64 or 128
@@ -253,6 +256,12 @@ int area_bridge_select(const void* k, int dtype, int B, int H, int Hg, int Wg, i
   if (!aligned16(k) || !aligned16(ws)) return AREA_EINVAL;
   return finish(area::launch_bridge_select(k, dtype, B, H, Hg, Wg, D, ry, rx, cand,
                                            static_cast<float*>(ws), stream));
+}
+
+int area_window_attn_bridge_stage_bytes(int B, int H, int R, int D, size_t* stage_bytes) {
+  if (!stage_bytes || B < 1 || H < 1 || R < 1 || D < 1) return AREA_EINVAL;
+  *stage_bytes = (size_t)4 * B * H * R * D;
+  return AREA_OK;
 }
 
 int area_window_attn_bridge(const void* q, const void* k, const void* v, const int* cand, int R,

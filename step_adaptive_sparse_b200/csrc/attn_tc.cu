@@ -697,14 +697,16 @@ attn_tc_kernel(const __grid_constant__ TcMaps tm, const TcParams prm) {
           }
           const CUtensorMap* tmd = kv ? &tm.v : &tm.k;
           const uint32_t dst = sbase + G::kSmemKV + s * G::kTileBytes;
-          if (WINDOW && !BRIDGE && j < ngt && prm.staged && (j + 1) * 128 <= nkv) {
-            // a whole tile of the window's global-KV rows, staged in the
-            // workspace by this call's copy launch: one tiled load
+          if (WINDOW && j < ngt && prm.staged && (j + 1) * 128 <= nkv) {
+            // a whole tile of the window's global-KV rows (or of the head's
+            // bridge candidates), staged in the workspace by this call's copy
+            // launch: one tiled load
             if (lane == 0) {
               mbar_arrive_tx(bar(BAR_KV_FULL + s), G::kTileBytes);
-              // staging row of the window: ((b * H + h) * nw + w) * G, and
-              // R.glist = (b * nw + w) * G
-              const long long srow = R.glist + (long long)(bh - R.b) * prm.P.nw * prm.P.G;
+              // staging row: plan lists ((b * H + h) * nw + w) * G with
+              // R.glist = (b * nw + w) * G; candidates (b * H + h) * R = R.glist
+              const long long srow =
+                  BRIDGE ? R.glist : R.glist + (long long)(bh - R.b) * prm.P.nw * prm.P.G;
               for (int hf = 0; hf < G::kHalves; ++hf)
                 tma_load_2d(dst + hf * kHalfBytes, kv ? &tm.vs : &tm.ks, bar(BAR_KV_FULL + s),
                             hf * 64, (int)(srow + j * 128));
@@ -830,7 +832,7 @@ attn_tc_kernel(const __grid_constant__ TcMaps tm, const TcParams prm) {
         const int valid = s_rec[slot].valid, nt = s_rec[slot].nt;
         // leading list tiles copied by cp.async (not the staged whole ones)
         const int ngt = WINDOW ? s_rec[slot].ngt : 0;
-        const int ncp = !WINDOW ? 0 : (!BRIDGE && prm.staged) ? ngt - s_rec[slot].nkv / 128 : ngt;
+        const int ncp = !WINDOW ? 0 : prm.staged ? ngt - s_rec[slot].nkv / 128 : ngt;
         auto copied = [&](int j) { return j < ngt && j >= ngt - ncp; };
         const bool two = s_rec[slot].one == 0;   // query tile 1 runs too
         mbar_arrive(bar(BAR_REC_EMPTY + slot));
@@ -1239,6 +1241,26 @@ __global__ void __launch_bounds__(256) stage_list_kernel(const __nv_bfloat16* __
   }
 }
 
+// One CTA per (128-row tile, element x head): copies the head's bridge
+// candidate rows of whole 128-row tiles, K then V, to [B*H][R][D].
+template <int D>
+__global__ void __launch_bounds__(256) stage_cand_kernel(const __nv_bfloat16* __restrict__ k,
+                                                         const __nv_bfloat16* __restrict__ v,
+                                                         const int* __restrict__ cand, int R,
+                                                         int N, __nv_bfloat16* __restrict__ sk,
+                                                         __nv_bfloat16* __restrict__ sv) {
+  const int t = blockIdx.x, bh = blockIdx.y;
+  const int* cl = cand + (int64_t)bh * R + t * 128;
+  const int64_t src0 = (int64_t)bh * N, dst0 = (int64_t)bh * R + t * 128;
+  constexpr int kChunks = D / 8;
+  for (int i = threadIdx.x; i < 128 * kChunks; i += blockDim.x) {
+    const int r = i / kChunks, c = i % kChunks;
+    const int64_t src = (src0 + cl[r]) * D + c * 8, dst = (dst0 + r) * D + c * 8;
+    *reinterpret_cast<uint4*>(sk + dst) = *reinterpret_cast<const uint4*>(k + src);
+    *reinterpret_cast<uint4*>(sv + dst) = *reinterpret_cast<const uint4*>(v + src);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -1365,11 +1387,12 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, c
   if ((e = make_map_grid(&m.vc, v, rows_y, Wg, D, kCW, kCH)) != cudaSuccess) return e;
   m.k = m.kp;   // partial global-KV tiles are copied with cp.async: no row map
   m.v = m.vp;
-  // whole global-KV tiles: staged rows [B*H*nw*G, D] after the workspace
-  const int64_t nstage = L.B * H * L.nw * L.G;
+  // whole global-KV tiles: staged rows after the workspace, [B*H*nw*G, D]
+  // (plan lists) or [B*H*R, D] (bridge candidates)
+  const int64_t nstage = cand ? L.B * H * R : L.B * H * L.nw * L.G;
   __nv_bfloat16* sk = nullptr;
   __nv_bfloat16* sv = nullptr;
-  if (staged && !cand && nstage > 0 && nstage < (int64_t(1) << 31)) {
+  if (staged && nstage > 0 && nstage < (int64_t(1) << 31)) {
     sk = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + window_ws_bytes(L, H, D));
     sv = sk + nstage * D;
     if ((e = make_map(&m.ks, sk, nstage, 128, D)) != cudaSuccess) return e;
@@ -1405,11 +1428,18 @@ cudaError_t launch_window_attn_tc(const void* q, const void* k, const void* v, c
   // unit counter and class completion counters start at zero
   if ((e = cudaMemsetAsync(ws, 0, (size_t)hdr, s)) != cudaSuccess) return e;
   if (staged) {
-    const dim3 grid((unsigned)L.nw, (unsigned)(L.B * H));
     const auto* kb = static_cast<const __nv_bfloat16*>(k);
     const auto* vb = static_cast<const __nv_bfloat16*>(v);
-    if (D == 64) stage_list_kernel<64><<<grid, 256, 0, s>>>(kb, vb, prm.P, H, sk, sv);
-    else stage_list_kernel<128><<<grid, 256, 0, s>>>(kb, vb, prm.P, H, sk, sv);
+    if (cand) {
+      const dim3 grid((unsigned)(R / 128), (unsigned)(L.B * H));
+      const int N = (int)L.N;
+      if (D == 64) stage_cand_kernel<64><<<grid, 256, 0, s>>>(kb, vb, cand, R, N, sk, sv);
+      else stage_cand_kernel<128><<<grid, 256, 0, s>>>(kb, vb, cand, R, N, sk, sv);
+    } else {
+      const dim3 grid((unsigned)L.nw, (unsigned)(L.B * H));
+      if (D == 64) stage_list_kernel<64><<<grid, 256, 0, s>>>(kb, vb, prm.P, H, sk, sv);
+      else stage_list_kernel<128><<<grid, 256, 0, s>>>(kb, vb, prm.P, H, sk, sv);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (D == 64) {

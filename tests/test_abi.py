@@ -135,6 +135,14 @@ def test_stage_bytes(area):
                                              128) == 0
 
 
+def test_bridge_stage_bytes(area):
+    # K and V rows of every head's candidates: 2 * B * H * R * D * 2 bytes
+    assert area.area_window_attn_bridge_stage_bytes(1, 24, 1024, 128) == 2 * 24 * 1024 * 128 * 2
+    assert area.area_window_attn_bridge_stage_bytes(2, 3, 240, 64) == 2 * 2 * 3 * 240 * 64 * 2
+    with pytest.raises(area.AreaError):
+        area.area_window_attn_bridge_stage_bytes(1, 24, 0, 128)
+
+
 def test_plan_size_with_seed_covers_every_shift(area):
     # a seeded plan may hold one more base window per axis
     base = area.area_window_plan_bytes(area.make_cfg(1, 384, 384, 72, 4, 512, 0.4))

@@ -430,7 +430,9 @@ def test_window_attn_bridge(data):
     energy = gr.gpu_dwt(data.dsrc, cfg.B, cfg.Hg, cfg.Wg, cfg.C, cfg.dtype)
     pcfg, plan, nbytes = gr.gpu_plan(energy, cfg.B, cfg.Hg, cfg.Wg, w, cfg.halo, 0, cfg.split_thr)
     o = torch.empty_like(data.dq)
-    wsb = gr.area.area_window_attn_ws_bytes(pcfg, cfg.H, cfg.D)
+    # with the staging area of the candidate rows (bf16: whole tiles as tiles)
+    wsb = (gr.area.area_window_attn_ws_bytes(pcfg, cfg.H, cfg.D)
+           + gr.area.area_window_attn_bridge_stage_bytes(cfg.B, cfg.H, ry * rx, cfg.D))
     ws = torch.empty(wsb // 4, dtype=torch.float32, device="cuda")
     gr.area.area_window_attn_bridge(data.dq, data.dk, data.dv, cand, ry * rx, pcfg, plan, nbytes,
                                     o, ws, wsb, cfg.H, cfg.D, cfg.scale, gr.area_dtype(cfg.dtype))
@@ -531,6 +533,35 @@ def test_window_attn_staged_equals_gathered(Hg, Wg, w, h, G, D, H):
     torch.cuda.synchronize()
     assert gr.area.area_window_attn_stage_bytes(pcfg, H, D) > 0
     assert torch.equal(staged, gathered)
+    assert gr.area.area_kernel_error() == 0
+
+
+@pytest.mark.parametrize("Hg,Wg,w,ry,rx,D,H", [
+    (64, 64, 16, 16, 16, 128, 2),   # 256 candidates: two whole staged tiles
+    (48, 64, 24, 12, 20, 64, 3),    # 240: one whole tile, a gathered partial one
+])
+def test_window_attn_bridge_staged_equals_gathered(Hg, Wg, w, ry, rx, D, H):
+    # the bridged call stages each head's candidate rows of whole tiles when
+    # the workspace has room; the outputs are identical to the bit
+    rng = np.random.default_rng(Hg + 3 * Wg + D)
+    B = 1
+    N = Hg * Wg
+    dq, dk, dv = (gr.to_dev(rng.standard_normal((B, H, N, D)).astype(np.float32), "bf16")
+                  for _ in range(3))
+    cand = torch.from_numpy(_gpu_bridge(dk, B, H, Hg, Wg, D, ry, rx, "bf16")).cuda()
+    E = (rng.random((B, Hg // 2, Wg // 2)) ** 3).astype(np.float32)
+    pcfg, plan, nbytes = gr.gpu_plan(torch.from_numpy(E).cuda(), B, Hg, Wg, w, 2, 0,
+                                     float(np.median(E)))
+    wmin = gr.area.area_window_attn_ws_bytes(pcfg, H, D)
+    outs = []
+    for wsb in (wmin + gr.area.area_window_attn_bridge_stage_bytes(B, H, ry * rx, D), wmin):
+        o = torch.empty_like(dq)
+        ws = torch.empty(wsb // 4, dtype=torch.float32, device="cuda")
+        gr.area.area_window_attn_bridge(dq, dk, dv, cand, ry * rx, pcfg, plan, nbytes, o, ws, wsb,
+                                        H, D, 1.0 / np.sqrt(D), gr.area.AREA_DTYPE_BF16)
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1])
     assert gr.area.area_kernel_error() == 0
 
 
