@@ -739,8 +739,9 @@ def run_area(args):
     ramp_out["total_ms"] = float(sum(ramp_out["ms"]))
     del kp_r, vp_r, o_r
 
-    # ---- the pages' own bridge rule on the last (smallest) window size,
-    # measured once: candidate selection plus window attention
+    # ---- the pages' own bridge rule on the last (smallest) window size:
+    # candidate selection plus window attention, median of 4 timed repetitions
+    # after one untimed
     w_b = cfg.schedule[-1]
     ry, rx = area.area_bridge_lattice(w_b, cfg.Hg, cfg.Wg)
     cand = torch.empty((cfg.B, cfg.H, ry * rx), dtype=torch.int32, device=dev)
@@ -754,7 +755,8 @@ def run_area(args):
         area.area_dwt_detail(src, st.dt, cfg.C, st.energy, cfg.B, cfg.Hg, cfg.Wg,
                              area.AREA_DETAIL_HH, stream)
         area.area_window_plan(st.energy, pc0, plan0, nb0, stream)
-        for rep in range(2):
+        bev = []
+        for rep in range(5):
             a, b2, c2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
             a.record(stream)
             area.area_bridge_select(k, st.dt, cfg.B, cfg.H, cfg.Hg, cfg.Wg, cfg.D, ry, rx, cand,
@@ -763,6 +765,8 @@ def run_area(args):
             area.area_window_attn_bridge(q, k, v, cand, ry * rx, pc0, plan0, nb0, st.o2, st.ws,
                                          st.ws_bytes, cfg.H, cfg.D, cfg.scale, st.dt, stream)
             c2.record(stream)
+            if rep > 0:
+                bev.append((a, b2, c2))
     torch.cuda.synchronize()
     d0 = area.parse_plan(plan0.cpu().numpy())
     cnd = cand.cpu().numpy().astype(np.int64)
@@ -775,8 +779,8 @@ def run_area(args):
         outside = ~((cy >= ey0) & (cy < ey0 + ehy) & (cx >= ex0) & (cx < ex0 + ewx))
         pairs += hy * wx * (ehy * ewx * cfg.H + float(outside.sum()))
     bflops = 4.0 * cfg.D * cfg.B * pairs
-    battn_ms = b2.elapsed_time(c2)
-    sel_ms = a.elapsed_time(b2)
+    battn_ms = float(np.median([b_.elapsed_time(c_) for a_, b_, c_ in bev]))
+    sel_ms = float(np.median([a_.elapsed_time(b_) for a_, b_, c_ in bev]))
     k_bytes = float(k.numel() * k.element_size())
     bridge_out = {"window": w_b, "lattice": [ry, rx], "select_ms": sel_ms,
                   "select_gbs": 2.0 * k_bytes / (sel_ms * 1e-3) / 1e9,
