@@ -66,6 +66,14 @@ def test_phase2_outputs_stay_in_bounds(B, H, Hg, Wg, w, h, G, D, dt):
     o = Guarded((B, H, N, D), dt)
     area.area_window_attn(q, k, v, cfg, plan.t, nb, o.t, ws.t, wsb, H, D, D ** -0.5, adt)
     assert o.intact() and ws.intact()
+    # the same call with the staging area of the global-KV rows: the staging
+    # copy and the tiled loads stay inside it, and the output is the same
+    wsb2 = wsb + area.area_window_attn_stage_bytes(cfg, H, D)
+    ws2 = Guarded((wsb2 // 4,), torch.float32)
+    o2 = Guarded((B, H, N, D), dt)
+    area.area_window_attn(q, k, v, cfg, plan.t, nb, o2.t, ws2.t, wsb2, H, D, D ** -0.5, adt)
+    assert o2.intact() and ws2.intact()
+    assert torch.equal(o2.t, o.t)
     assert area.area_kernel_error() == 0
 
 
@@ -98,4 +106,33 @@ def test_bridge_outputs_stay_in_bounds():
     ws = Guarded((wsb // 4,), torch.float32)
     area.area_bridge_select(k, area.AREA_DTYPE_BF16, B, H, Hg, Wg, D, ry, rx, cand.t, ws.t, wsb)
     assert cand.intact() and ws.intact()
+    assert area.area_kernel_error() == 0
+
+
+def test_bridged_window_outputs_stay_in_bounds():
+    # 16 x 16 = 256 candidates per head: two whole tiles staged per head
+    B, H, Hg, Wg, D, ry, rx, w = 1, 2, 40, 56, 128, 16, 16, 12
+    N = Hg * Wg
+    q, k, v = (_rand((B, H, N, D), torch.bfloat16, s) for s in (9, 10, 11))
+    cand = torch.empty((B, H, ry * rx), dtype=torch.int32, device="cuda")
+    swsb = area.area_bridge_select_ws_bytes(B, H, Hg, Wg, D)
+    sws = torch.empty(swsb // 4, dtype=torch.float32, device="cuda")
+    area.area_bridge_select(k, area.AREA_DTYPE_BF16, B, H, Hg, Wg, D, ry, rx, cand, sws, swsb)
+    src = _rand((B, N, 16), torch.bfloat16, 12)
+    energy = torch.empty((B, Hg // 2, Wg // 2), dtype=torch.float32, device="cuda")
+    area.area_dwt_detail(src, area.AREA_DTYPE_BF16, 16, energy, B, Hg, Wg, area.AREA_DETAIL_HH)
+    cfg = area.make_cfg(B, Hg, Wg, w, 2, 0, float(energy.mean()))
+    nb = area.area_window_plan_bytes(cfg)
+    plan = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    area.area_window_plan(energy, cfg, plan, nb)
+    outs = []
+    for extra in (area.area_window_attn_bridge_stage_bytes(B, H, ry * rx, D), 0):
+        wsb = area.area_window_attn_ws_bytes(cfg, H, D) + extra
+        ws = Guarded((wsb // 4,), torch.float32)
+        o = Guarded((B, H, N, D), torch.bfloat16)
+        area.area_window_attn_bridge(q, k, v, cand, ry * rx, cfg, plan, nb, o.t, ws.t, wsb, H, D,
+                                     D ** -0.5, area.AREA_DTYPE_BF16)
+        assert o.intact() and ws.intact()
+        outs.append(o.t.clone())
+    assert torch.equal(outs[0], outs[1])
     assert area.area_kernel_error() == 0
