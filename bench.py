@@ -36,7 +36,7 @@ if ROOT not in sys.path:
 
 METRIC = "AReA attention TFLOP/s per schedule step (bf16, 1 B200)"
 # Bumped whenever attn_tc.cu changes, so that stale DRAM counters are not reported.
-KERNEL_REVISION = "attn_tc v13 (v12 plus whole global-KV tiles staged per call by stage_list_kernel and loaded as tiles)"
+KERNEL_REVISION = "attn_tc v14 (v13 plus a 384-thread window kernel whose warpgroups split the registers 136 / 184 with setmaxnreg)"
 DEFAULT_CONFIG = "flux6144"
 PUBLISHED_BF16_TFLOPS = 2250.0   # B200 dense bf16 tensor rate, published (no sparsity)
 

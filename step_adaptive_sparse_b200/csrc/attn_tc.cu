@@ -8,7 +8,8 @@
 // Pages: ai.info "Methodology in Plain English" (Phase I, Phase II);
 // gpt-diffusion.com "Las dos fases de AReA".
 //
-// Design (one persistent CTA per SM, 320 threads):
+// Design (one persistent CTA per SM; 320 threads for dense calls, 384 for
+// window calls, whose warps 2-3 are idle and whose softmax warps are 4-11):
 //   warp 0      producer: claims work units (window mode: from a counter in
 //               the workspace, in the plan's parity-class order; dense mode:
 //               statically), publishes one record per unit in a shared-memory
@@ -26,6 +27,8 @@
 //   warp 1      TMEM allocator and the single MMA-issuing thread.
 //   warps 2-5   softmax of query tile 0, warps 6-9 of query tile 1: each
 //               thread owns one query row (TMEM lane 32*(warp mod 4) + lane).
+//               In window calls the warpgroups shift by two warps (4-7, 8-11)
+//               so that setmaxnreg can move registers from warpgroup 0 to them.
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.  P (bf16)
 // overwrites the first 64 columns of its S tile and feeds the PV MMA straight
 // from TMEM.  P is handed over in two parts of 64 keys, each with its own
@@ -50,8 +53,15 @@ __device__ int g_tc_error = 0;   // set on a bounded-wait expiry; read by tests
 
 namespace {
 
-constexpr int kThreads = 320;     // producer, MMA issuer, 8 softmax warps
-constexpr int kSoftWarp0 = 2;     // first softmax warp
+// Dense calls: 320 threads (producer, MMA issuer, 8 softmax warps), every
+// thread at the block's register cap.  Window calls: 384 threads, warpgroup 0
+// (producer, MMA issuer, two idle warps) drops to kRegsLow registers and the
+// two softmax warpgroups rise to kRegsHigh; the split uses exactly the
+// allocation of a 168-register launch (launch_tc checks it before launching).
+__host__ __device__ constexpr int tc_threads(bool window) { return window ? 384 : 320; }
+__host__ __device__ constexpr int tc_soft_warp0(bool window) { return window ? 4 : 2; }   // first softmax warp
+constexpr int kRegsLow = 136, kRegsHigh = 184;
+static_assert(128 * kRegsLow + 256 * kRegsHigh == 384 * 168, "register split");
 constexpr int kStages = 4;               // K/V ring stages (32 KB each at head_dim 128)
 constexpr int kQSlots = 1;               // query buffers (a second one would cost a K/V stage)
 constexpr int kHalfBytes = 128 * 128;   // 128 rows x 64 bf16: one 128B-swizzled half tile
@@ -526,9 +536,10 @@ __device__ bool decode_unit(int u, const TcParams& prm, UnitRec& r) {
 }
 
 template <bool WINDOW, bool BRIDGE, int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(tc_threads(WINDOW), 1)
 attn_tc_kernel(const __grid_constant__ TcMaps tm, const TcParams prm) {
   using G = Geo<D>;
+  constexpr int kSoftWarp0 = tc_soft_warp0(WINDOW);
   constexpr uint32_t kIdescPV = idesc(D, true);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -584,325 +595,330 @@ attn_tc_kernel(const __grid_constant__ TcMaps tm, const TcParams prm) {
   const int Ntok = WINDOW ? prm.P.N : prm.da.N;     // rows per (b, h) of Q
   const int Nkrows = WINDOW ? prm.P.N : prm.da.Nk;  // rows per (b, h) of K and V
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    // Units are claimed from a counter in the workspace (window mode) or
-    // statically (dense mode).  The record of the next unit is written while
-    // the current unit's first key tiles are in flight.
-    uint32_t kv_it = 0, unit_count = 0, claims = 0;
-    bool ok = true;
-    auto claim = [&]() -> int {
-      int u = 0;
-      if (lane == 0) {
-        if (WINDOW) u = (int)atomicAdd(prm.counters + kWsUnitCounter, 1u);
-        else u = blockIdx.x + (int)claims * gridDim.x;
-      }
-      ++claims;
-      return __shfl_sync(0xffffffffu, u, 0);
-    };
-    // Claim, decode and publish the record of this CTA's k-th unit.
-    auto publish = [&](uint32_t k) -> bool {
-      const int u = claim();
-      const uint32_t slot = k % kRecSlots;
-      if (!warp_wait0(bar(BAR_REC_EMPTY + slot), ((k / kRecSlots) & 1u) ^ 1u, abort_flag))
-        return false;
-      if (lane == 0) {
-        UnitRec r;
-        if (!decode_unit<WINDOW>(u, prm, r)) r.valid = 0;
-        s_rec[slot] = r;
-        mbar_arrive(bar(BAR_REC_FULL + slot));
-      }
-      __syncwarp();
-      return true;
-    };
-    // Queries of this CTA's k-th unit, once the previous unit's last QK has
-    // read the buffer.  Window queries are read from DRAM once per unit: in
-    // cells of kCW x kCH tokens (one tiled box per lane) when the window's
-    // sides allow, else row by row with TMA gather4, 4 rows per lane (a warp's
-    // cp.async stream issued those about 7x slower, measured; gather4 itself
-    // moves about 7 bytes per clock per SM against about 37 for tiled boxes).
-    auto load_q = [&](uint32_t k) -> bool {
-      const UnitRec& Rq = s_rec[k % kRecSlots];
-      if (!Rq.valid) return true;
-      const uint32_t qs = k % kQSlots;
-      if (!warp_wait0(bar(BAR_Q_EMPTY + qs), ((k / kQSlots) & 1u) ^ 1u, abort_flag)) return false;
-      const uint32_t qbase = sbase + G::kSmemQ + qs * 2 * G::kTileBytes;
-      const int nqt = Rq.one ? 1 : 2;
-      if constexpr (!WINDOW) {
-        if (lane == 0) {
-          mbar_arrive_tx(bar(BAR_Q_FULL + qs), nqt * G::kTileBytes);
-          for (int t = 0; t < nqt; ++t)
-            for (int hf = 0; hf < G::kHalves; ++hf)
-              tma_load_2d(qbase + t * G::kTileBytes + hf * kHalfBytes, &tm.q, bar(BAR_Q_FULL + qs),
-                          hf * 64, Rq.bh * Ntok + Rq.q0 + t * 128);
-        }
-        __syncwarp();
-      } else if (Rq.qcx > 0) {
-        if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL + qs), nqt * G::kTileBytes);
-        __syncwarp();
-        if (lane < kCells) {
-          // cell q0 / kCellKeys + t * kCells + lane (clamped to the last one;
-          // the rows past nq are computed and not stored)
-          const int ncq = Rq.nq / kCellKeys;
-          for (int t = 0; t < nqt; ++t) {
-            int c = Rq.q0 / kCellKeys + t * kCells + lane;
-            if (c > ncq - 1) c = ncq - 1;
-            const int cx = Rq.win.y + (c % Rq.qcx) * kCW;
-            const int cy = Rq.bh * prm.P.Hg + Rq.win.x + (c / Rq.qcx) * kCH;
-            for (int hf = 0; hf < G::kHalves; ++hf)
-              tma_load_3d(qbase + t * G::kTileBytes + hf * kHalfBytes + lane * kCellBytes, &tm.qc,
-                          bar(BAR_Q_FULL + qs), hf * 64, cx, cy);
-          }
-        }
-        __syncwarp();
-      } else {
-        if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL + qs), nqt * G::kTileBytes);
-        __syncwarp();
-        for (int t = 0; t < nqt; ++t) {
-          int r[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            r[i] = Rq.bh * Ntok +
-                   window_query_token(Rq.win, 0, Rq.nq, Rq.q0 + t * 128 + lane * 4 + i, Wg);
-          for (int hf = 0; hf < G::kHalves; ++hf)
-            tma_gather4(qbase + t * G::kTileBytes + hf * kHalfBytes + lane * 512, &tm.q,
-                        bar(BAR_Q_FULL + qs), hf * 64, r[0], r[1], r[2], r[3]);
-        }
-      }
-      return true;
-    };
-    ok = publish(0);
-    while (ok) {
-      const UnitRec& R = s_rec[unit_count % kRecSlots];
-      if (!R.valid) break;
-      if (!(ok = load_q(unit_count))) break;
-      const int nt = R.nt, ngt = R.ngt, ntr = R.ntr, nkv = R.nkv;
-      const int nti = ngt + ntr;
-      const int bh = R.bh;
-      const int4 ext = R.ext;
-      const RectTiling rt = rect_tiling(ext.z, ext.w);
-      const int* glist = (BRIDGE ? prm.cand : prm.P.gidx) + R.glist;
-      const int jn = nt < 2 ? nt : 2;         // the next record is published before tile jn
-      bool published = false;
-      for (int j = 0; j < nt && ok; ++j) {
-        if (j == jn) {
-          published = true;
-          if (!(ok = publish(unit_count + 1))) break;
-        }
-        for (int kv = 0; kv < 2; ++kv) {       // K then V
-          const int s = (int)(kv_it % kStages);
-          if (!warp_wait0(bar(BAR_KV_EMPTY + s), ((kv_it / kStages) & 1u) ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const CUtensorMap* tmd = kv ? &tm.v : &tm.k;
-          const uint32_t dst = sbase + G::kSmemKV + s * G::kTileBytes;
-          if (WINDOW && j < ngt && prm.staged && (j + 1) * 128 <= nkv) {
-            // a whole tile of the window's global-KV rows (or of the head's
-            // bridge candidates), staged in the workspace by this call's copy
-            // launch: one tiled load
-            if (lane == 0) {
-              mbar_arrive_tx(bar(BAR_KV_FULL + s), G::kTileBytes);
-              // staging row: plan lists ((b * H + h) * nw + w) * G with
-              // R.glist = (b * nw + w) * G; candidates (b * H + h) * R = R.glist
-              const long long srow =
-                  BRIDGE ? R.glist : R.glist + (long long)(bh - R.b) * prm.P.nw * prm.P.G;
-              for (int hf = 0; hf < G::kHalves; ++hf)
-                tma_load_2d(dst + hf * kHalfBytes, kv ? &tm.vs : &tm.ks, bar(BAR_KV_FULL + s),
-                            hf * 64, (int)(srow + j * 128));
-            }
-            __syncwarp();
-            ++kv_it;
-            continue;
-          }
-          if (WINDOW && j < ngt) {
-            // global-KV list (or bridge candidates), copied row by row: the
-            // rows of a head's list serve all its windows and sit in L2, and
-            // from L2 cp.async beats TMA gather4 by about 4x (measured)
-            const int g0 = j * 128 + lane * 4;
-            int r[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int p = g0 + i < nkv ? g0 + i : nkv - 1;
-              r[i] = bh * Nkrows + glist[p];
-            }
-            cp_async_rows<D>(dst, kv ? prm.v : prm.k, r, lane);
-            cp_async_arrive(bar(BAR_KV_FULL + s));
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(BAR_KV_FULL + s));
-            ++kv_it;
-            continue;
-          }
-          if (lane == 0) mbar_arrive_tx(bar(BAR_KV_FULL + s), G::kTileBytes);
-          __syncwarp();
-          if (j >= nti) {
-            // text keys: rows of the [B*H*T, 128] text tensors
-            if (lane == 0) {
-              const CUtensorMap* tt = kv ? &tm.vt : &tm.kt;
-              for (int hf = 0; hf < G::kHalves; ++hf)
-                tma_load_2d(dst + hf * kHalfBytes, tt, bar(BAR_KV_FULL + s), hf * 64,
-                            bh * prm.T + (j - nti) * 128);
-            }
-          } else if (!WINDOW) {
-            if (lane == 0)
-              for (int hf = 0; hf < G::kHalves; ++hf)
-                tma_load_2d(dst + hf * kHalfBytes, tmd, bar(BAR_KV_FULL + s), hf * 64,
-                            bh * Nkrows + j * 128);
-          } else {
-            // Halo rectangle: patch j - ngt, or kCells strip cells, one per
-            // lane (past the last cell the last one is loaded again: finite
-            // values under masked keys)
-            const int jj = j - ngt;
-            if (jj < rt.npatch) {
-              if (lane == 0) {
-                const CUtensorMap* tp = kv ? &tm.vp : &tm.kp;
-                const int cx = ext.y + (jj % rt.npx) * kPW;
-                const int cy = bh * prm.P.Hg + ext.x + (jj / rt.npx) * kPH;
-                for (int hf = 0; hf < G::kHalves; ++hf)
-                  tma_load_3d(dst + hf * kHalfBytes, tp, bar(BAR_KV_FULL + s), hf * 64, cx, cy);
-              }
-            } else if (lane < kCells) {
-              const CUtensorMap* tc = kv ? &tm.vc : &tm.kc;
-              int c = (jj - rt.npatch) * kCells + lane;
-              if (c > rt.ncell - 1) c = rt.ncell - 1;
-              const int2 o = strip_cell(rt, c);
-              const int cx = ext.y + o.y;
-              const int cy = bh * prm.P.Hg + ext.x + o.x;
-              for (int hf = 0; hf < G::kHalves; ++hf)
-                tma_load_3d(dst + hf * kHalfBytes + lane * kCellBytes, tc, bar(BAR_KV_FULL + s),
-                            hf * 64, cx, cy);
-            }
-            __syncwarp();
-          }
-          ++kv_it;
-        }
-      }
-      if (!ok) break;
-      if (!published && !(ok = publish(unit_count + 1))) break;
-      ++unit_count;
-    }
-    // Drain: the most recent load of every stage has landed (bounded wait),
-    // and no cp.async copy of this warp is still in flight.
-    int drain_abort = 0;
-    for (uint32_t k = 0; k < kStages && k < kv_it; ++k) {
-      const uint32_t it = kv_it - 1 - k;
-      warp_wait0(bar(BAR_KV_FULL + it % kStages), (it / kStages) & 1u, &drain_abort);
-    }
-    asm volatile("cp.async.wait_all;" ::: "memory");
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t kv_it = 0, unit_count = 0;
-      uint32_t p_cnt0 = 0, p_cnt1 = 0;
-      const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
-
+  if (warp < kSoftWarp0) {
+    // warpgroup 0 (window calls: producer, MMA issuer, two idle warps)
+    if constexpr (WINDOW) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow) : "memory");
+    if (warp == 0) {
+      // ------------------------------------------------------------ producer
+      // Units are claimed from a counter in the workspace (window mode) or
+      // statically (dense mode).  The record of the next unit is written while
+      // the current unit's first key tiles are in flight.
+      uint32_t kv_it = 0, unit_count = 0, claims = 0;
       bool ok = true;
-      auto kv_addr = [&](uint32_t it) { return sbase + G::kSmemKV + (it % kStages) * G::kTileBytes; };
-      auto qk = [&](uint32_t d, uint32_t qs, uint32_t ks) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          mma_ss(d, sdesc(qs + off, 16, 1024), sdesc(ks + off, 16, 1024), kIdescQK, kk > 0);
+      auto claim = [&]() -> int {
+        int u = 0;
+        if (lane == 0) {
+          if (WINDOW) u = (int)atomicAdd(prm.counters + kWsUnitCounter, 1u);
+          else u = blockIdx.x + (int)claims * gridDim.x;
         }
+        ++claims;
+        return __shfl_sync(0xffffffffu, u, 0);
       };
-      // PV over part h of the tile's keys (128 / kPParts keys, 16 per instruction)
-      auto pv_part = [&](uint32_t d, uint32_t p_tmem, uint32_t vs, bool first, int h) {
-        constexpr int kPer = 8 / kPParts;
-#pragma unroll
-        for (int kk = kPer * h; kk < kPer * h + kPer; ++kk)
-          mma_ts(d, p_tmem + kk * 8, sdesc(vs + kk * 2048, kHalfBytes, 1024), kIdescPV,
-                 (first && kk == 0) ? 0u : 1u);
+      // Claim, decode and publish the record of this CTA's k-th unit.
+      auto publish = [&](uint32_t k) -> bool {
+        const int u = claim();
+        const uint32_t slot = k % kRecSlots;
+        if (!warp_wait0(bar(BAR_REC_EMPTY + slot), ((k / kRecSlots) & 1u) ^ 1u, abort_flag))
+          return false;
+        if (lane == 0) {
+          UnitRec r;
+          if (!decode_unit<WINDOW>(u, prm, r)) r.valid = 0;
+          s_rec[slot] = r;
+          mbar_arrive(bar(BAR_REC_FULL + slot));
+        }
+        __syncwarp();
+        return true;
       };
-      // PV of one query tile, part by part as the softmax hands P over
-      auto pv_parts = [&](uint32_t d, uint32_t p_tmem, uint32_t vs, bool first, int bpart,
-                          int bfull, uint32_t cnt) {
-#pragma unroll
-        for (int h = 0; h < kPParts; ++h) {
-          const uint32_t b = h + 1 < kPParts ? bar(bpart + h) : bar(bfull);
-          if (!mbar_wait(b, cnt & 1u, abort_flag)) return false;
-          tc_fence_after();
-          pv_part(d, p_tmem, vs, first, h);
+      // Queries of this CTA's k-th unit, once the previous unit's last QK has
+      // read the buffer.  Window queries are read from DRAM once per unit: in
+      // cells of kCW x kCH tokens (one tiled box per lane) when the window's
+      // sides allow, else row by row with TMA gather4, 4 rows per lane (a warp's
+      // cp.async stream issued those about 7x slower, measured; gather4 itself
+      // moves about 7 bytes per clock per SM against about 37 for tiled boxes).
+      auto load_q = [&](uint32_t k) -> bool {
+        const UnitRec& Rq = s_rec[k % kRecSlots];
+        if (!Rq.valid) return true;
+        const uint32_t qs = k % kQSlots;
+        if (!warp_wait0(bar(BAR_Q_EMPTY + qs), ((k / kQSlots) & 1u) ^ 1u, abort_flag)) return false;
+        const uint32_t qbase = sbase + G::kSmemQ + qs * 2 * G::kTileBytes;
+        const int nqt = Rq.one ? 1 : 2;
+        if constexpr (!WINDOW) {
+          if (lane == 0) {
+            mbar_arrive_tx(bar(BAR_Q_FULL + qs), nqt * G::kTileBytes);
+            for (int t = 0; t < nqt; ++t)
+              for (int hf = 0; hf < G::kHalves; ++hf)
+                tma_load_2d(qbase + t * G::kTileBytes + hf * kHalfBytes, &tm.q, bar(BAR_Q_FULL + qs),
+                            hf * 64, Rq.bh * Ntok + Rq.q0 + t * 128);
+          }
+          __syncwarp();
+        } else if (Rq.qcx > 0) {
+          if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL + qs), nqt * G::kTileBytes);
+          __syncwarp();
+          if (lane < kCells) {
+            // cell q0 / kCellKeys + t * kCells + lane (clamped to the last one;
+            // the rows past nq are computed and not stored)
+            const int ncq = Rq.nq / kCellKeys;
+            for (int t = 0; t < nqt; ++t) {
+              int c = Rq.q0 / kCellKeys + t * kCells + lane;
+              if (c > ncq - 1) c = ncq - 1;
+              const int cx = Rq.win.y + (c % Rq.qcx) * kCW;
+              const int cy = Rq.bh * prm.P.Hg + Rq.win.x + (c / Rq.qcx) * kCH;
+              for (int hf = 0; hf < G::kHalves; ++hf)
+                tma_load_3d(qbase + t * G::kTileBytes + hf * kHalfBytes + lane * kCellBytes, &tm.qc,
+                            bar(BAR_Q_FULL + qs), hf * 64, cx, cy);
+            }
+          }
+          __syncwarp();
+        } else {
+          if (lane == 0) mbar_arrive_tx(bar(BAR_Q_FULL + qs), nqt * G::kTileBytes);
+          __syncwarp();
+          for (int t = 0; t < nqt; ++t) {
+            int r[4];
+  #pragma unroll
+            for (int i = 0; i < 4; ++i)
+              r[i] = Rq.bh * Ntok +
+                     window_query_token(Rq.win, 0, Rq.nq, Rq.q0 + t * 128 + lane * 4 + i, Wg);
+            for (int hf = 0; hf < G::kHalves; ++hf)
+              tma_gather4(qbase + t * G::kTileBytes + hf * kHalfBytes + lane * 512, &tm.q,
+                          bar(BAR_Q_FULL + qs), hf * 64, r[0], r[1], r[2], r[3]);
+          }
         }
         return true;
       };
+      ok = publish(0);
       while (ok) {
-        const uint32_t slot = unit_count % kRecSlots;
-        if (!(ok = mbar_wait(bar(BAR_REC_FULL + slot), (unit_count / kRecSlots) & 1u, abort_flag)))
-          break;
-        const int valid = s_rec[slot].valid, nt = s_rec[slot].nt;
-        // leading list tiles copied by cp.async (not the staged whole ones)
-        const int ngt = WINDOW ? s_rec[slot].ngt : 0;
-        const int ncp = !WINDOW ? 0 : prm.staged ? ngt - s_rec[slot].nkv / 128 : ngt;
-        auto copied = [&](int j) { return j < ngt && j >= ngt - ncp; };
-        const bool two = s_rec[slot].one == 0;   // query tile 1 runs too
-        mbar_arrive(bar(BAR_REC_EMPTY + slot));
-        if (!valid) break;
-        const uint32_t qs = unit_count % kQSlots;
-        const uint32_t q0s = sbase + G::kSmemQ + qs * 2 * G::kTileBytes;
-        const uint32_t q1s = q0s + G::kTileBytes;
-        const uint32_t bQe = bar(BAR_Q_EMPTY + qs);
-        if (!(ok = mbar_wait(bar(BAR_Q_FULL + qs), (unit_count / kQSlots) & 1u, abort_flag))) break;
-        // prologue: S(0)
-        const uint32_t k0 = kv_it;
-        if (!(ok = mbar_wait(bar(BAR_KV_FULL + k0 % kStages), (k0 / kStages) & 1u, abort_flag)))
-          break;
-        if (copied(0)) fence_proxy_async();     // rows copied by cp.async
-        tc_fence_after();
-        qk(tS0, q0s, kv_addr(k0));
-        mma_commit(bar(BAR_S_FULL0));
-        if (two) {
-          qk(tS1, q1s, kv_addr(k0));
-          mma_commit(bar(BAR_S_FULL1));
-        }
-        mma_commit(bar(BAR_KV_EMPTY + k0 % kStages));
-        if (nt == 1) mma_commit(bQe);
+        const UnitRec& R = s_rec[unit_count % kRecSlots];
+        if (!R.valid) break;
+        if (!(ok = load_q(unit_count))) break;
+        const int nt = R.nt, ngt = R.ngt, ntr = R.ntr, nkv = R.nkv;
+        const int nti = ngt + ntr;
+        const int bh = R.bh;
+        const int4 ext = R.ext;
+        const RectTiling rt = rect_tiling(ext.z, ext.w);
+        const int* glist = (BRIDGE ? prm.cand : prm.P.gidx) + R.glist;
+        const int jn = nt < 2 ? nt : 2;         // the next record is published before tile jn
+        bool published = false;
         for (int j = 0; j < nt && ok; ++j) {
-          const uint32_t vi = kv_it + 2 * j + 1;
-          const uint32_t kn = kv_it + 2 * j + 2;
-          if (!(ok = mbar_wait(bar(BAR_KV_FULL + vi % kStages), (vi / kStages) & 1u, abort_flag)))
-            break;
-          if (copied(j)) fence_proxy_async();
-          if (!(ok = pv_parts(tO0, tS0, kv_addr(vi), j == 0, BAR_P_PART0, BAR_P_FULL0, p_cnt0)))
-            break;
-          ++p_cnt0;
-          if (j == nt - 1) mma_commit(bar(BAR_O_FULL0));
-          if (j + 1 < nt) {
-            if (!(ok = mbar_wait(bar(BAR_KV_FULL + kn % kStages), (kn / kStages) & 1u,
-                                 abort_flag)))
+          if (j == jn) {
+            published = true;
+            if (!(ok = publish(unit_count + 1))) break;
+          }
+          for (int kv = 0; kv < 2; ++kv) {       // K then V
+            const int s = (int)(kv_it % kStages);
+            if (!warp_wait0(bar(BAR_KV_EMPTY + s), ((kv_it / kStages) & 1u) ^ 1u, abort_flag)) {
+              ok = false;
               break;
-            if (copied(j + 1)) fence_proxy_async();
+            }
+            const CUtensorMap* tmd = kv ? &tm.v : &tm.k;
+            const uint32_t dst = sbase + G::kSmemKV + s * G::kTileBytes;
+            if (WINDOW && j < ngt && prm.staged && (j + 1) * 128 <= nkv) {
+              // a whole tile of the window's global-KV rows (or of the head's
+              // bridge candidates), staged in the workspace by this call's copy
+              // launch: one tiled load
+              if (lane == 0) {
+                mbar_arrive_tx(bar(BAR_KV_FULL + s), G::kTileBytes);
+                // staging row: plan lists ((b * H + h) * nw + w) * G with
+                // R.glist = (b * nw + w) * G; candidates (b * H + h) * R = R.glist
+                const long long srow =
+                    BRIDGE ? R.glist : R.glist + (long long)(bh - R.b) * prm.P.nw * prm.P.G;
+                for (int hf = 0; hf < G::kHalves; ++hf)
+                  tma_load_2d(dst + hf * kHalfBytes, kv ? &tm.vs : &tm.ks, bar(BAR_KV_FULL + s),
+                              hf * 64, (int)(srow + j * 128));
+              }
+              __syncwarp();
+              ++kv_it;
+              continue;
+            }
+            if (WINDOW && j < ngt) {
+              // global-KV list (or bridge candidates), copied row by row: the
+              // rows of a head's list serve all its windows and sit in L2, and
+              // from L2 cp.async beats TMA gather4 by about 4x (measured)
+              const int g0 = j * 128 + lane * 4;
+              int r[4];
+  #pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int p = g0 + i < nkv ? g0 + i : nkv - 1;
+                r[i] = bh * Nkrows + glist[p];
+              }
+              cp_async_rows<D>(dst, kv ? prm.v : prm.k, r, lane);
+              cp_async_arrive(bar(BAR_KV_FULL + s));
+              __syncwarp();
+              if (lane == 0) mbar_arrive(bar(BAR_KV_FULL + s));
+              ++kv_it;
+              continue;
+            }
+            if (lane == 0) mbar_arrive_tx(bar(BAR_KV_FULL + s), G::kTileBytes);
+            __syncwarp();
+            if (j >= nti) {
+              // text keys: rows of the [B*H*T, 128] text tensors
+              if (lane == 0) {
+                const CUtensorMap* tt = kv ? &tm.vt : &tm.kt;
+                for (int hf = 0; hf < G::kHalves; ++hf)
+                  tma_load_2d(dst + hf * kHalfBytes, tt, bar(BAR_KV_FULL + s), hf * 64,
+                              bh * prm.T + (j - nti) * 128);
+              }
+            } else if (!WINDOW) {
+              if (lane == 0)
+                for (int hf = 0; hf < G::kHalves; ++hf)
+                  tma_load_2d(dst + hf * kHalfBytes, tmd, bar(BAR_KV_FULL + s), hf * 64,
+                              bh * Nkrows + j * 128);
+            } else {
+              // Halo rectangle: patch j - ngt, or kCells strip cells, one per
+              // lane (past the last cell the last one is loaded again: finite
+              // values under masked keys)
+              const int jj = j - ngt;
+              if (jj < rt.npatch) {
+                if (lane == 0) {
+                  const CUtensorMap* tp = kv ? &tm.vp : &tm.kp;
+                  const int cx = ext.y + (jj % rt.npx) * kPW;
+                  const int cy = bh * prm.P.Hg + ext.x + (jj / rt.npx) * kPH;
+                  for (int hf = 0; hf < G::kHalves; ++hf)
+                    tma_load_3d(dst + hf * kHalfBytes, tp, bar(BAR_KV_FULL + s), hf * 64, cx, cy);
+                }
+              } else if (lane < kCells) {
+                const CUtensorMap* tc = kv ? &tm.vc : &tm.kc;
+                int c = (jj - rt.npatch) * kCells + lane;
+                if (c > rt.ncell - 1) c = rt.ncell - 1;
+                const int2 o = strip_cell(rt, c);
+                const int cx = ext.y + o.y;
+                const int cy = bh * prm.P.Hg + ext.x + o.x;
+                for (int hf = 0; hf < G::kHalves; ++hf)
+                  tma_load_3d(dst + hf * kHalfBytes + lane * kCellBytes, tc, bar(BAR_KV_FULL + s),
+                              hf * 64, cx, cy);
+              }
+              __syncwarp();
+            }
+            ++kv_it;
+          }
+        }
+        if (!ok) break;
+        if (!published && !(ok = publish(unit_count + 1))) break;
+        ++unit_count;
+      }
+      // Drain: the most recent load of every stage has landed (bounded wait),
+      // and no cp.async copy of this warp is still in flight.
+      int drain_abort = 0;
+      for (uint32_t k = 0; k < kStages && k < kv_it; ++k) {
+        const uint32_t it = kv_it - 1 - k;
+        warp_wait0(bar(BAR_KV_FULL + it % kStages), (it / kStages) & 1u, &drain_abort);
+      }
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        uint32_t kv_it = 0, unit_count = 0;
+        uint32_t p_cnt0 = 0, p_cnt1 = 0;
+        const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
+
+        bool ok = true;
+        auto kv_addr = [&](uint32_t it) { return sbase + G::kSmemKV + (it % kStages) * G::kTileBytes; };
+        auto qk = [&](uint32_t d, uint32_t qs, uint32_t ks) {
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+            mma_ss(d, sdesc(qs + off, 16, 1024), sdesc(ks + off, 16, 1024), kIdescQK, kk > 0);
+          }
+        };
+        // PV over part h of the tile's keys (128 / kPParts keys, 16 per instruction)
+        auto pv_part = [&](uint32_t d, uint32_t p_tmem, uint32_t vs, bool first, int h) {
+          constexpr int kPer = 8 / kPParts;
+  #pragma unroll
+          for (int kk = kPer * h; kk < kPer * h + kPer; ++kk)
+            mma_ts(d, p_tmem + kk * 8, sdesc(vs + kk * 2048, kHalfBytes, 1024), kIdescPV,
+                   (first && kk == 0) ? 0u : 1u);
+        };
+        // PV of one query tile, part by part as the softmax hands P over
+        auto pv_parts = [&](uint32_t d, uint32_t p_tmem, uint32_t vs, bool first, int bpart,
+                            int bfull, uint32_t cnt) {
+  #pragma unroll
+          for (int h = 0; h < kPParts; ++h) {
+            const uint32_t b = h + 1 < kPParts ? bar(bpart + h) : bar(bfull);
+            if (!mbar_wait(b, cnt & 1u, abort_flag)) return false;
             tc_fence_after();
-            qk(tS0, q0s, kv_addr(kn));
-            mma_commit(bar(BAR_S_FULL0));
-            if (!two) {                          // K(j+1) is done with after QK0
+            pv_part(d, p_tmem, vs, first, h);
+          }
+          return true;
+        };
+        while (ok) {
+          const uint32_t slot = unit_count % kRecSlots;
+          if (!(ok = mbar_wait(bar(BAR_REC_FULL + slot), (unit_count / kRecSlots) & 1u, abort_flag)))
+            break;
+          const int valid = s_rec[slot].valid, nt = s_rec[slot].nt;
+          // leading list tiles copied by cp.async (not the staged whole ones)
+          const int ngt = WINDOW ? s_rec[slot].ngt : 0;
+          const int ncp = !WINDOW ? 0 : prm.staged ? ngt - s_rec[slot].nkv / 128 : ngt;
+          auto copied = [&](int j) { return j < ngt && j >= ngt - ncp; };
+          const bool two = s_rec[slot].one == 0;   // query tile 1 runs too
+          mbar_arrive(bar(BAR_REC_EMPTY + slot));
+          if (!valid) break;
+          const uint32_t qs = unit_count % kQSlots;
+          const uint32_t q0s = sbase + G::kSmemQ + qs * 2 * G::kTileBytes;
+          const uint32_t q1s = q0s + G::kTileBytes;
+          const uint32_t bQe = bar(BAR_Q_EMPTY + qs);
+          if (!(ok = mbar_wait(bar(BAR_Q_FULL + qs), (unit_count / kQSlots) & 1u, abort_flag))) break;
+          // prologue: S(0)
+          const uint32_t k0 = kv_it;
+          if (!(ok = mbar_wait(bar(BAR_KV_FULL + k0 % kStages), (k0 / kStages) & 1u, abort_flag)))
+            break;
+          if (copied(0)) fence_proxy_async();     // rows copied by cp.async
+          tc_fence_after();
+          qk(tS0, q0s, kv_addr(k0));
+          mma_commit(bar(BAR_S_FULL0));
+          if (two) {
+            qk(tS1, q1s, kv_addr(k0));
+            mma_commit(bar(BAR_S_FULL1));
+          }
+          mma_commit(bar(BAR_KV_EMPTY + k0 % kStages));
+          if (nt == 1) mma_commit(bQe);
+          for (int j = 0; j < nt && ok; ++j) {
+            const uint32_t vi = kv_it + 2 * j + 1;
+            const uint32_t kn = kv_it + 2 * j + 2;
+            if (!(ok = mbar_wait(bar(BAR_KV_FULL + vi % kStages), (vi / kStages) & 1u, abort_flag)))
+              break;
+            if (copied(j)) fence_proxy_async();
+            if (!(ok = pv_parts(tO0, tS0, kv_addr(vi), j == 0, BAR_P_PART0, BAR_P_FULL0, p_cnt0)))
+              break;
+            ++p_cnt0;
+            if (j == nt - 1) mma_commit(bar(BAR_O_FULL0));
+            if (j + 1 < nt) {
+              if (!(ok = mbar_wait(bar(BAR_KV_FULL + kn % kStages), (kn / kStages) & 1u,
+                                   abort_flag)))
+                break;
+              if (copied(j + 1)) fence_proxy_async();
+              tc_fence_after();
+              qk(tS0, q0s, kv_addr(kn));
+              mma_commit(bar(BAR_S_FULL0));
+              if (!two) {                          // K(j+1) is done with after QK0
+                mma_commit(bar(BAR_KV_EMPTY + kn % kStages));
+                if (j + 2 == nt) mma_commit(bQe);
+              }
+            }
+            if (two) {
+              if (!(ok = pv_parts(tO1, tS1, kv_addr(vi), j == 0, BAR_P_PART1, BAR_P_FULL1, p_cnt1)))
+                break;
+              ++p_cnt1;
+              if (j == nt - 1) mma_commit(bar(BAR_O_FULL1));
+            }
+            mma_commit(bar(BAR_KV_EMPTY + vi % kStages));
+            if (two && j + 1 < nt) {
+              qk(tS1, q1s, kv_addr(kn));
+              mma_commit(bar(BAR_S_FULL1));
               mma_commit(bar(BAR_KV_EMPTY + kn % kStages));
               if (j + 2 == nt) mma_commit(bQe);
             }
           }
-          if (two) {
-            if (!(ok = pv_parts(tO1, tS1, kv_addr(vi), j == 0, BAR_P_PART1, BAR_P_FULL1, p_cnt1)))
-              break;
-            ++p_cnt1;
-            if (j == nt - 1) mma_commit(bar(BAR_O_FULL1));
-          }
-          mma_commit(bar(BAR_KV_EMPTY + vi % kStages));
-          if (two && j + 1 < nt) {
-            qk(tS1, q1s, kv_addr(kn));
-            mma_commit(bar(BAR_S_FULL1));
-            mma_commit(bar(BAR_KV_EMPTY + kn % kStages));
-            if (j + 2 == nt) mma_commit(bQe);
-          }
+          kv_it += 2 * nt;
+          ++unit_count;
         }
-        kv_it += 2 * nt;
-        ++unit_count;
+        // Drain: every MMA issued by this thread has completed (bounded wait).
+        int drain_abort = 0;
+        mma_commit(bar(BAR_DRAIN));
+        mbar_wait(bar(BAR_DRAIN), 0, &drain_abort);
       }
-      // Drain: every MMA issued by this thread has completed (bounded wait).
-      int drain_abort = 0;
-      mma_commit(bar(BAR_DRAIN));
-      mbar_wait(bar(BAR_DRAIN), 0, &drain_abort);
+      __syncwarp();
     }
-    __syncwarp();
-  } else if (warp >= kSoftWarp0) {
+  } else {
+    if constexpr (WINDOW) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh) : "memory");
     // ------------------------------------------------------------ softmax / epilogue
     // The first four softmax warps own query tile 0, the next four query
     // tile 1.  A warp may only touch the TMEM lane quarter (warp id mod 4),
@@ -1317,7 +1333,18 @@ int num_sms() {
 template <bool WINDOW, bool BRIDGE, int D>
 cudaError_t launch_tc(const TcMaps& maps, const TcParams& prm, cudaStream_t s) {
   constexpr int kSmemBytes = Geo<D>::kSmemBytes;
+  constexpr int kThreads = tc_threads(WINDOW);
   auto fn = attn_tc_kernel<WINDOW, BRIDGE, D>;
+  if constexpr (WINDOW) {
+    // setmaxnreg.inc waits until the registers it asks for are free, so the
+    // split must fit in what the launch allocates (registers per thread,
+    // rounded down to the allocation unit of 8, times the block's threads)
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+    if (e != cudaSuccess) return e;
+    if (kThreads * (fa.numRegs / 8 * 8) < 128 * kRegsLow + 256 * kRegsHigh)
+      return cudaErrorInvalidConfiguration;
+  }
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const int grid = prm.num_units < num_sms() ? prm.num_units : num_sms();
