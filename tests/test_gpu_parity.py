@@ -476,6 +476,57 @@ def test_dense_attn_ragged(B, H, N, Nk, D, dtype):
 
 
 # ---------------------------------------------------------------------------
+# Online softmax: score maxima that grow past the rescale threshold from one
+# key tile to the next (O rescaled in TMEM) or fall (the running maximum
+# stays ahead of every later tile)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("growing", [True, False])
+@pytest.mark.parametrize("D", [128, 64])
+def test_dense_attn_rescaled_maxima(growing, D):
+    rng = np.random.default_rng(7 + D + growing)
+    B, H, N, Nk = 1, 2, 300, 1000
+    q = rng.standard_normal((B, H, N, D)).astype(np.float32)
+    k = rng.standard_normal((B, H, Nk, D)).astype(np.float32)
+    v = rng.standard_normal((B, H, Nk, D)).astype(np.float32)
+    # key tile t (128 keys) scaled by 1 + 4t (or the reverse): its row maxima
+    # differ from the previous tile's by far more than 2^8 in exp2 units
+    t = np.arange(Nk) // 128
+    f = 1.0 + 4.0 * (t if growing else t.max() - t)
+    k *= f[None, None, :, None].astype(np.float32)
+    dq, dk, dv = gr.to_dev(q, "bf16"), gr.to_dev(k, "bf16"), gr.to_dev(v, "bf16")
+    q, k, v = gr.to_host(dq), gr.to_host(dk), gr.to_host(dv)
+    scale = 1.0 / np.sqrt(D)
+    o = gr.gpu_dense(dq, dk, dv, B, H, N, Nk, D, scale, "bf16")
+    gr.assert_close(gr.to_host(o), ora.coarse_attn(q, k, v, scale), "bf16", "dense rescaled maxima")
+
+
+@pytest.mark.parametrize("growing", [True, False])
+def test_window_attn_rescaled_maxima(growing):
+    rng = np.random.default_rng(11 + growing)
+    B, H, Hg, Wg, w, h, G, D = 1, 2, 64, 48, 24, 4, 130, 128
+    N = Hg * Wg
+    q = rng.standard_normal((B, H, N, D)).astype(np.float32)
+    k = rng.standard_normal((B, H, N, D)).astype(np.float32)
+    v = rng.standard_normal((B, H, N, D)).astype(np.float32)
+    # keys scaled by grid row: the Halo rectangle's 16x8 patches come in row
+    # order, so each band of 8 rows raises (or lowers) the row maxima by far
+    # more than 2^8 in exp2 units; the global-KV tiles come first
+    y = np.arange(N) // Wg
+    f = 1.0 + 0.5 * (y if growing else (Hg - 1) - y)
+    k *= f[None, None, :, None].astype(np.float32)
+    dq, dk, dv = gr.to_dev(q, "bf16"), gr.to_dev(k, "bf16"), gr.to_dev(v, "bf16")
+    q, k, v = gr.to_host(dq), gr.to_host(dk), gr.to_host(dv)
+    E = (rng.random((B, Hg // 2, Wg // 2)) ** 3).astype(np.float32)
+    thr = float(np.median(E))
+    pcfg, plan, nbytes = gr.gpu_plan(torch.from_numpy(E).cuda(), B, Hg, Wg, w, h, G, thr)
+    scale = 1.0 / np.sqrt(D)
+    o = gr.gpu_window(dq, dk, dv, pcfg, plan, nbytes, H, D, scale, "bf16")
+    want = ora.window_attn(q, k, v, [ora.window_plan(E[0], Hg, Wg, w, h, G, thr)], scale)
+    gr.assert_close(gr.to_host(o), want, "bf16", "window rescaled maxima")
+
+
+# ---------------------------------------------------------------------------
 # Phase II edge cases
 # ---------------------------------------------------------------------------
 
