@@ -616,6 +616,40 @@ def test_window_attn_bridge_staged_equals_gathered(Hg, Wg, w, ry, rx, D, H):
     assert gr.area.area_kernel_error() == 0
 
 
+@pytest.mark.parametrize("Hg,Wg,w,ry,rx,D,H", [
+    (32, 32, 32, 16, 16, 128, 2),   # one window = the grid: every candidate tile masked
+    (64, 32, 32, 16, 16, 128, 2),   # two windows: one candidate tile masked, one in part
+    (64, 32, 32, 16, 16, 64, 3),    # the same at head_dim 64
+])
+def test_window_attn_bridge_masked_tiles(Hg, Wg, w, ry, rx, D, H):
+    # The candidates come in lattice-cell order, 128 to a tile; a tile whose
+    # candidates all lie inside the window's Halo rectangle is masked
+    # entirely, so the rows start with a running maximum of -inf and take
+    # their first weights from a later tile.
+    rng = np.random.default_rng(Hg * 7 + Wg + D)
+    B, halo = 1, 2
+    N = Hg * Wg
+    q, k, v = (rng.standard_normal((B, H, N, D)).astype(np.float32) for _ in range(3))
+    dq, dk, dv = gr.to_dev(q, "bf16"), gr.to_dev(k, "bf16"), gr.to_dev(v, "bf16")
+    q, k, v = gr.to_host(dq), gr.to_host(dk), gr.to_host(dv)
+    cand = torch.from_numpy(_gpu_bridge(dk, B, H, Hg, Wg, D, ry, rx, "bf16")).cuda()
+    E = (rng.random((B, Hg // 2, Wg // 2)) ** 3).astype(np.float32)
+    thr = 0.0                                  # no window splits
+    pcfg, plan, nbytes = gr.gpu_plan(torch.from_numpy(E).cuda(), B, Hg, Wg, w, halo, 0, thr)
+    wsb = (gr.area.area_window_attn_ws_bytes(pcfg, H, D)
+           + gr.area.area_window_attn_bridge_stage_bytes(B, H, ry * rx, D))
+    ws = torch.empty(wsb // 4, dtype=torch.float32, device="cuda")
+    o = torch.empty_like(dq)
+    scale = 1.0 / np.sqrt(D)
+    gr.area.area_window_attn_bridge(dq, dk, dv, cand, ry * rx, pcfg, plan, nbytes, o, ws, wsb,
+                                    H, D, scale, gr.area.AREA_DTYPE_BF16)
+    oplan = ora.window_plan(E[0], Hg, Wg, w, halo, 0, thr)
+    ocand = np.stack([ora.bridge_candidates(k[0, h], Hg, Wg, ry, rx) for h in range(H)])[None]
+    want = ora.window_attn(q, k, v, [oplan], scale, bridge=ocand)
+    gr.assert_close(gr.to_host(o), want, "bf16", "window bridge, masked candidate tiles")
+    assert gr.area.area_kernel_error() == 0
+
+
 # ---------------------------------------------------------------------------
 # the pages' bridge: edge cases of the candidate selection (bit-exact)
 # ---------------------------------------------------------------------------
